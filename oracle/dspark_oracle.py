@@ -1,0 +1,353 @@
+"""CPU oracle of the DSpark draft/verify round (test infrastructure).
+
+This is a plain, slow, float64 NumPy restatement of what the round computes.
+It is test infrastructure: only the tests, the package smoke check and the
+benchmark's CPU-baseline leg may import it.  It shares no code with the CUDA
+path and never takes an input or an expected value from it.
+
+Sources (three public web pages on DSpark):
+  [P1] "大模型推理加速的系统级工程：DeepSeek V4-Pro DSpark 推测解码方案深度解析与开源工具链 DeepSpec"
+       (austery.github.io write-up of a Best Partners TV video)
+  [P2] "DeepSeek 开源 DSpark，一个可将大语言模型推理速度提升高达 85% 的新框架"
+       (Chinese translation of a VentureBeat article)
+  [P3] "DSpark Speculative Decoding" (lukebest.github.io concept note)
+
+What each function follows:
+  * draft      -- P3 §Semi-Autoregressive Generation: p_k(v) ∝ exp(U_k(v) + B_k(v)),
+                  Markov head B(x_{k-1}, ·) = W1[x_{k-1}] W2 of low rank r;
+                  P1 §"DSpark 架构设计：半自回归生成与马尔可夫修正" (one previous
+                  token only, positions filled left to right).
+  * verify     -- P1 §"大模型推理的显存瓶颈与推测解码的演进逻辑" (rejection
+                  sampling: accept the longest prefix, resample at the first
+                  rejection, drop the rest) and P3 opening paragraph (longest
+                  consistent prefix plus a bonus token).
+  * tv_labels  -- P3 §Confidence-Scheduled Verification: c*_k = 1 - ½‖p_d - p_t‖₁;
+                  P1 §"硬件感知与置信度自适应调度机制" (label = analytic acceptance rate).
+  * prefix_survival -- P3 §Confidence-Scheduled Verification: a_{r,j} = ∏_{i≤j} c_{r,i}.
+  * prefix_schedule -- P3 §Confidence-Scheduled Verification (Algorithm 1,
+                  Θ = τ·SPS(B)); P1 §"硬件感知与置信度自适应调度机制" (sort all
+                  candidate tokens by survival, add them one at a time, evaluate
+                  expected throughput, stop when it falls; global search on the GPU).
+
+Readings where the pages leave a step open (each is listed in the design doc):
+  * temperature: p ∝ exp(ℓ/T) on both draft and target; the scaling is an fp32
+    multiply of the fp32 logits by fl32(1/T), so that both sides take every
+    sampling and acceptance decision from the same fp32 scaled logits; all
+    later arithmetic is fp64.  T = 0 means greedy (argmax, lowest index).
+  * the draft logits ℓ_d = U + bias are stored as fp32; sampling uses the
+    stored values.
+  * acceptance is strict: accept iff u·p_d(x) < p_t(x) (u in [0, 1)).
+  * inverse CDF in vocabulary order: the first v with F_v > u; if rounding
+    leaves u ≥ F_{V-1}, the last v with positive mass.
+  * a zero residual after a rejection (only possible through rounding) falls
+    back to sampling the target row.
+  * one uniform u_res per request serves whichever of residual or bonus
+    sample happens; the bonus uses target row L+1 (1-based).
+  * Θ(D) = (B + S(D))·sps[D]: τ counts the always-emitted residual/bonus
+    token of every request plus the expected accepted drafts S(D), the sum
+    of the D largest survivals; sps is indexed by D.
+  * ties in the survival sort: survival descending, then request, then position.
+  * ARGMAX mode takes the smallest D attaining max Θ (global search);
+    EARLY_STOP takes the first D with Θ(D+1) ≤ Θ(D).
+  * near-ties: a decision closer than 1e-6 (|u - F|, |u - p_t/p_d|, a greedy
+    top-2 gap of 1e-6·max(1,|z|)) or than 1e-12 relative (scheduler Θ) is
+    reported together with every outcome that is valid within that window.
+"""
+
+from __future__ import annotations
+
+import itertools
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+NEAR_TIE = 1e-6
+THETA_NEAR_TIE = 1e-12
+
+SCHED_ARGMAX = 0
+SCHED_EARLY_STOP = 1
+
+
+# --------------------------------------------------------------------------- shared definitions
+
+def scaled_logits(logits, T: float) -> np.ndarray:
+    """z = ℓ / T as the fp32 product ℓ · fl32(1/T) (reading of the temperature)."""
+    l32 = np.asarray(logits, dtype=np.float32)
+    inv_t = np.float32(1.0) / np.float32(T)
+    return (l32 * inv_t).astype(np.float32)
+
+
+def softmax(logits, T: float) -> np.ndarray:
+    """p ∝ exp(ℓ/T) over the last axis, fp64 (P3 §Semi-Autoregressive Generation)."""
+    z = scaled_logits(logits, T).astype(np.float64)
+    m = np.max(z, axis=-1, keepdims=True)
+    e = np.exp(z - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def greedy_choice(logits) -> Tuple[int, List[int]]:
+    """argmax with the lowest index on ties, plus every index within the near-tie gap."""
+    z = np.asarray(logits, dtype=np.float32).astype(np.float64)
+    x = int(np.argmax(z))
+    gap = NEAR_TIE * max(1.0, abs(z[x]))
+    alts = [int(v) for v in np.nonzero(z >= z[x] - gap)[0]]
+    return x, alts
+
+
+def inverse_cdf(p: np.ndarray, u: float) -> Tuple[int, List[int]]:
+    """Sample index v = min{v : F_v > u}, F the running sum of p in vocabulary order.
+
+    Returns the index and every index whose CDF interval lies within NEAR_TIE of u.
+    """
+    p = np.asarray(p, dtype=np.float64)
+    F = np.cumsum(p)
+    u = float(u)
+    v = int(np.searchsorted(F, u, side="right"))
+    if v >= p.shape[0]:
+        v = int(np.nonzero(p > 0)[0][-1])
+    lo = np.concatenate([[0.0], F[:-1]])
+    near = (p > 0) & (lo - NEAR_TIE <= u) & (u < F + NEAR_TIE)
+    alts = sorted(set(int(i) for i in np.nonzero(near)[0]) | {v})
+    return v, alts
+
+
+# --------------------------------------------------------------------------- draft (Markov head)
+
+def markov_bias(W1, W2, prev) -> np.ndarray:
+    """B(x_{k-1}, ·) = W1[x_{k-1}] · W2 in fp64 from the stored weights (P3 §Semi-Autoregressive Generation)."""
+    W1 = np.asarray(W1)
+    W2 = np.asarray(W2)
+    g = W1[np.asarray(prev)].astype(np.float64)
+    return g @ W2.astype(np.float64)
+
+
+def draft_step(U_k, W1, W2, prev, u, T: float, W2_64: Optional[np.ndarray] = None):
+    """One sequential step for one request: ℓ_d = U_k + W1[prev]·W2, then x ~ softmax(ℓ_d/T).
+
+    Returns (x, ld32 [V], alternatives).  ld32 is ℓ_d rounded to fp32 (its stored type).
+    """
+    g = np.asarray(W1)[int(prev)].astype(np.float64)
+    bias = g @ (W2_64 if W2_64 is not None else np.asarray(W2).astype(np.float64))
+    ld32 = (np.asarray(U_k, dtype=np.float32).astype(np.float64) + bias).astype(np.float32)
+    if T == 0.0:
+        x, alts = greedy_choice(ld32)
+    else:
+        x, alts = inverse_cdf(softmax(ld32, T), u)
+    return x, ld32, alts
+
+
+def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None):
+    """The γ sequential Markov-head steps for every request.
+
+    U [B, γ, V] fp32, x0 [B], u_draft [B, γ].  Step k uses the token chosen at
+    step k-1 (x0 for the first step).  Returns (x [B, γ] int32,
+    ld [B, γ, V] fp32, alts) where alts[(b, k)] lists the valid tokens at a
+    near-tie.  `follow` maps (b, k) to a token that must be one of the valid
+    alternatives at that step; the chain then continues from it (used to
+    follow one branch of a near-tie).
+    """
+    U = np.asarray(U, dtype=np.float32)
+    B, G, V = U.shape
+    W1 = np.asarray(W1)
+    W2_64 = np.asarray(W2).astype(np.float64)
+    x = np.zeros((B, G), dtype=np.int32)
+    ld = np.zeros((B, G, V), dtype=np.float32)
+    alts = {}
+    prev = np.asarray(x0, dtype=np.int64).copy()
+    for k in range(G):
+        bias = markov_bias(W1, W2_64, prev)                      # [B, V] fp64
+        ld[:, k] = (U[:, k].astype(np.float64) + bias).astype(np.float32)
+        for b in range(B):
+            if T == 0.0:
+                xk, a = greedy_choice(ld[b, k])
+            else:
+                xk, a = inverse_cdf(softmax(ld[b, k], T), u_draft[b, k])
+            if len(a) > 1:
+                alts[(b, k)] = a
+            if follow is not None and (b, k) in follow:
+                f = int(follow[(b, k)])
+                if f not in a:
+                    raise ValueError(f"token {f} is not a valid outcome at {(b, k)}: {a}")
+                xk = f
+            x[b, k] = xk
+        prev = x[:, k].astype(np.int64)
+    return x, ld, alts
+
+
+# --------------------------------------------------------------------------- verification
+
+def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
+                   force_accept: Optional[Dict[int, bool]] = None, force_token: Optional[int] = None):
+    """Rejection-sampling verification of one request's block.
+
+    ld_b [γ, V] draft logits, lt_b [≥L+1, V] target logits, x_b [γ] drafted
+    tokens, L the number of positions to verify.  Positions k = 0..L-1 are
+    accepted while u·p_d(x_k) < p_t(x_k); at the first rejection one token is
+    drawn from norm(max(0, p_t - p_d)); if all L survive, a bonus token is
+    drawn from the target row L.
+
+    Returns a dict with n (accepted count), y [γ+1] (x_0..x_{n-1}, the
+    resampled/bonus token, then -1), accept_ties (positions whose decision is
+    a near-tie), sample_alts (valid tokens for the last emitted one),
+    residual_mass (Z when a residual was drawn) and kind ('residual'/'bonus').
+    `force_accept`/`force_token` pin a near-tie outcome to one of its valid values.
+    """
+    G = len(x_b)
+    V = np.asarray(lt_b).shape[-1]
+    y = np.full(G + 1, -1, dtype=np.int32)
+    accept_ties = []
+    n = 0
+    for k in range(L):
+        xk = int(x_b[k])
+        if T == 0.0:
+            acc = (0 <= xk < V) and xk == int(np.argmax(np.asarray(lt_b[k], dtype=np.float32)))
+        else:
+            if not (0 <= xk < V):
+                acc = False
+            else:
+                pd = softmax(ld_b[k], T)[xk]
+                pt = softmax(lt_b[k], T)[xk]
+                u = float(u_acc_b[k])
+                acc = u * pd < pt
+                if pd > 0 and abs(u - pt / pd) < NEAR_TIE:
+                    accept_ties.append(k)
+        if force_accept is not None and k in force_accept:
+            if k not in accept_ties and force_accept[k] != acc:
+                raise ValueError(f"position {k} is not a near-tie")
+            acc = force_accept[k]
+        if not acc:
+            break
+        y[k] = xk
+        n += 1
+    residual_mass = None
+    if T == 0.0:
+        tok, alts = greedy_choice(lt_b[n])
+        kind = "residual" if n < L else "bonus"
+    elif n < L:
+        q = np.maximum(0.0, softmax(lt_b[n], T) - softmax(ld_b[n], T))
+        Z = float(np.sum(q))
+        residual_mass = Z
+        kind = "residual"
+        if Z > 0.0:
+            tok, alts = inverse_cdf(q / Z, u_res)
+        else:
+            tok, alts = inverse_cdf(softmax(lt_b[n], T), u_res)
+    else:
+        kind = "bonus"
+        tok, alts = inverse_cdf(softmax(lt_b[L], T), u_res)
+    if force_token is not None:
+        if force_token not in alts:
+            raise ValueError(f"token {force_token} is not a valid outcome: {alts}")
+        tok = force_token
+    y[n] = tok
+    return dict(n=n, y=y, accept_ties=accept_ties, sample_alts=alts, residual_mass=residual_mass, kind=kind)
+
+
+def verify(ld, lt, x, L, u_acc, u_res, T: float):
+    """Verify every request; returns (n_acc [B], y [B, γ+1], per-request detail dicts)."""
+    ld = np.asarray(ld, dtype=np.float32)
+    lt = np.asarray(lt, dtype=np.float32)
+    B, G = np.asarray(x).shape
+    n_acc = np.zeros(B, dtype=np.int32)
+    y = np.full((B, G + 1), -1, dtype=np.int32)
+    detail = []
+    for b in range(B):
+        Lb = G if L is None else int(L[b])
+        r = verify_request(ld[b], lt[b], x[b], Lb, u_acc[b], u_res[b], T)
+        n_acc[b], y[b] = r["n"], r["y"]
+        detail.append(r)
+    return n_acc, y, detail
+
+
+# --------------------------------------------------------------------------- TV confidence labels
+
+def tv_labels(ld, lt, T: float) -> np.ndarray:
+    """c*_k = 1 - ½ Σ_v |p_d,k(v) - p_t,k(v)| for every drafted position (fp64 [B, γ]).
+
+    Greedy (T = 0): the distributions are one-hot at the argmax, so c* is 1 when
+    the argmaxes agree and 0 otherwise.
+    """
+    ld = np.asarray(ld, dtype=np.float32)
+    lt = np.asarray(lt, dtype=np.float32)
+    B, G, V = ld.shape
+    out = np.zeros((B, G), dtype=np.float64)
+    for b in range(B):
+        for k in range(G):
+            if T == 0.0:
+                out[b, k] = 1.0 if int(np.argmax(ld[b, k])) == int(np.argmax(lt[b, k])) else 0.0
+            else:
+                out[b, k] = 1.0 - 0.5 * float(np.sum(np.abs(softmax(ld[b, k], T) - softmax(lt[b, k], T))))
+    return out
+
+
+# --------------------------------------------------------------------------- prefix survival + scheduler
+
+def prefix_survival(c) -> np.ndarray:
+    """a_{b,j} = ∏_{i≤j} c_{b,i}, multiplied left to right in fp32."""
+    c = np.asarray(c, dtype=np.float32)
+    return np.cumprod(c, axis=1, dtype=np.float32)
+
+
+def schedule_order(a) -> np.ndarray:
+    """Item order (flat index b*γ + j): survival descending, then request, then position."""
+    a = np.asarray(a, dtype=np.float32)
+    key = -a.reshape(-1).astype(np.float64)
+    key[np.isnan(key)] = np.inf
+    return np.argsort(key, kind="stable")
+
+
+def prefix_schedule(c, sps, D_max: int, mode: int = SCHED_ARGMAX):
+    """Greedy hardware-aware prefix scheduler.
+
+    All B·γ candidate tokens are ranked by prefix survival; adding them one at a
+    time, the expected throughput after D additions is
+    Θ(D) = (B + S(D)) · sps[D], with S(D) the sum of the D best survivals.
+    ARGMAX keeps the best D over 0..D_max; EARLY_STOP keeps the first D after
+    which Θ no longer rises.  L_b is the number of request b's tokens kept.
+
+    Returns dict(L [B] int32, a [B, γ] fp32, theta (Θ at D*), D, thetas, near_tie).
+    """
+    a = prefix_survival(c)
+    B, G = a.shape
+    D_max = int(min(D_max, B * G))
+    sps = np.asarray(sps, dtype=np.float64)
+    order = schedule_order(a)
+    a_sorted = a.reshape(-1)[order].astype(np.float64)
+    S = np.concatenate([[0.0], np.cumsum(a_sorted[:D_max])])
+    theta = (B + S) * sps[: D_max + 1]
+    if mode == SCHED_ARGMAX:
+        D = int(np.argmax(theta))
+        others = np.delete(theta, D)
+        near = bool(others.size and np.any(np.abs(others - theta[D]) <= THETA_NEAR_TIE * abs(theta[D])))
+    elif mode == SCHED_EARLY_STOP:
+        D = D_max
+        near = False
+        for d in range(D_max):
+            if abs(theta[d + 1] - theta[d]) <= THETA_NEAR_TIE * abs(theta[d]):
+                near = True
+            if theta[d + 1] <= theta[d]:
+                D = d
+                break
+    else:
+        raise ValueError(mode)
+    L = np.bincount(order[:D] // G, minlength=B).astype(np.int32)
+    return dict(L=L, a=a, theta=float(theta[D]), D=D, thetas=theta, near_tie=near)
+
+
+def exhaustive_schedule(c, sps, D_max: int):
+    """Brute force over every length vector L ∈ {0..γ}^B with Σ L ≤ D_max.
+
+    Θ(L) = (B + Σ_b Σ_{j<L_b} a_{b,j}) · sps[Σ L].  Returns (best Θ, list of the
+    L attaining it within 1e-12 relative).  Only for tiny B and γ.
+    """
+    a = prefix_survival(c).astype(np.float64)
+    B, G = a.shape
+    cands = []
+    for Ls in itertools.product(range(G + 1), repeat=B):
+        D = sum(Ls)
+        if D > D_max:
+            continue
+        tau = B + sum(float(np.sum(a[b, :Ls[b]])) for b in range(B))
+        cands.append((tau * float(sps[D]), tuple(Ls)))
+    best = max(t for t, _ in cands)
+    return best, [Ls for t, Ls in cands if abs(t - best) <= THETA_NEAR_TIE * abs(best)]
