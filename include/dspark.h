@@ -1,0 +1,208 @@
+/*
+ * dspark.h -- C ABI of libdspark.so: the data-parallel hot path of one DSpark
+ * speculative-decoding round (Markov-head draft, rejection-sampling verify,
+ * TV confidence labels, prefix survival, hardware-aware prefix scheduler) as
+ * CUDA kernels for one NVIDIA B200 (sm_100a).
+ *
+ * Sources (three public web pages on DSpark):
+ *   [P1] "大模型推理加速的系统级工程：DeepSeek V4-Pro DSpark 推测解码方案深度解析与开源工具链 DeepSpec"
+ *        (austery.github.io)
+ *   [P3] "DSpark Speculative Decoding" (lukebest.github.io concept note)
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
+ *     never allocates, frees or keeps device memory between calls.
+ *   - All tensors are dense and row-major (C order), with the shapes given.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL means the legacy default stream).  Outputs are valid once the stream
+ *     has reached the call.
+ *   - The return value is a dspark_status.  Argument errors are found on the
+ *     host before anything is launched (DSPARK_EINVAL, nothing written).  A
+ *     failed launch returns DSPARK_ECUDA.
+ *   - Problems found in the DATA on the device never stop a call: they set bits
+ *     in the per-request word flags[b] (bits below), which the caller zeroes
+ *     before the round; calls OR their bits in.  Device-side waits are bounded;
+ *     a wait that gives up sets DSPARK_FLAG_DEVICE_TIMEOUT in every flags word
+ *     the kernel could reach and, where a workspace is passed, DSPARK_ETIMEOUT
+ *     in its status word (dspark_workspace_status).
+ *   - Scaled logits z = l * (1/T) are formed as the fp32 product of the fp32
+ *     logit and the fp32 reciprocal of T; T == 0 selects greedy decoding
+ *     (argmax, lowest index on ties).
+ *   - Random numbers are inputs: uniforms in [0, 1) passed as fp32 tensors.
+ */
+#ifndef DSPARK_H_
+#define DSPARK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSPARK_OK = 0,
+  DSPARK_EINVAL = 1,    /* bad argument (null, size <= 0, gamma > 64, T < 0, bad dtype, workspace too small) */
+  DSPARK_ECUDA = 2,     /* a CUDA launch or driver call failed */
+  DSPARK_ENOTIMPL = 3,  /* shape outside what the kernels support (message in dspark_last_error) */
+  DSPARK_ETIMEOUT = 4   /* a bounded device wait gave up (read through dspark_workspace_status) */
+} dspark_status;
+
+/* weight dtypes */
+enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 };
+
+/* scheduler modes */
+enum { DSPARK_SCHED_ARGMAX = 0, DSPARK_SCHED_EARLY_STOP = 1 };
+
+/* workspace kinds for dspark_workspace_size */
+enum { DSPARK_WS_DRAFT = 0, DSPARK_WS_VERIFY = 1, DSPARK_WS_SCHEDULE = 2 };
+
+/* bits of flags[b] */
+#define DSPARK_FLAG_DRAFT_NEAR_TIE    (1u << 0) /* |u - F| < 1e-6 at the drafted token, or greedy top-2 gap <= 1e-6*max(1,|z|) */
+#define DSPARK_FLAG_ACCEPT_NEAR_TIE   (1u << 1) /* |u - p_t/p_d| < 1e-6 at a verified position */
+#define DSPARK_FLAG_SAMPLE_NEAR_TIE   (1u << 2) /* |u - F| < 1e-6 at the residual or bonus token */
+#define DSPARK_FLAG_SMALL_RESIDUAL    (1u << 3) /* residual mass < 1e-3 at the first rejection */
+#define DSPARK_FLAG_NONFINITE         (1u << 4) /* NaN or Inf among the logits */
+#define DSPARK_FLAG_TOKEN_RANGE       (1u << 5) /* a token id outside [0, V) */
+#define DSPARK_FLAG_CONF_RANGE        (1u << 6) /* a confidence outside [0, 1] */
+#define DSPARK_FLAG_SCHED_NEAR_TIE    (1u << 7) /* the chosen D is within 1e-12 (relative) of another */
+#define DSPARK_FLAG_DEVICE_TIMEOUT    (1u << 31)
+
+/* Human-readable name of a status code. */
+const char* dspark_status_string(int status);
+
+/* Text of the last host-side error of this thread ("" if none). */
+const char* dspark_last_error(void);
+
+/* Tuning knobs (process-wide, host side; no effect on results beyond the choice of kernel):
+ *   "draft_tc_min_b"  bf16 drafts with B >= value use the tensor-core main pass (default 9)
+ *   "draft_path"      0 automatic, 1 always the CUDA-core GEMV pass, 2 always tensor cores
+ *   "draft_pdl"       1 (default) chain draft kernels with programmatic dependent launch
+ *   "verify_cluster"  0 automatic, else the cluster size of the verify kernel (1..16, power of 2)
+ *   "sm_count"        0 query the device, else the SM count used to size persistent grids
+ * Returns DSPARK_EINVAL for an unknown key. */
+int dspark_set_option(const char* key, long value);
+
+/* Device workspace bytes an entry point needs for the given sizes (r is used by
+ * DSPARK_WS_DRAFT only).  Returns 0 for an unknown kind.  The workspace holds
+ * per-call scratch only: its contents need not be preserved between calls. */
+size_t dspark_workspace_size(int which, int B, int gamma, int V, int r);
+
+/* Read the status word of a workspace after the stream has reached the call
+ * that used it (synchronous copy).  Returns DSPARK_OK or DSPARK_ETIMEOUT. */
+int dspark_workspace_status(const void* ws, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_markov_draft -- the Markov-head sequential draft stage.
+ *
+ * [P3 §Semi-Autoregressive Generation] p_k(v) ∝ exp(U_k(v) + B_k(v)) with the
+ * low-rank Markov bias B_k = W1[x_{k-1}] · W2 (rank r); [P1 §"DSpark 架构设计：
+ * 半自回归生成与马尔可夫修正"] the head only looks at the previous sampled token and
+ * fills the block left to right.  For each request b and k = 1..gamma:
+ *     l_d[b,k,:] = U[b,k,:] + W1[x_{k-1}, :] · W2        (x_0 = x0[b])
+ *     x_k        = min{ v : sum_{w<=v} exp(z_w - max z) > u_draft[b,k] * sum_w exp(z_w - max z) },
+ *                  z = l_d[b,k,:] * (1/T)              (T > 0)
+ *     x_k        = argmax_v l_d[b,k,v], lowest index    (T == 0)
+ *
+ * U        [B, gamma, V] fp32   base logits of the parallel stage.
+ * W1       [V, r]  and  W2 [r, V]   Markov-head factors, dtype w_dtype
+ *          (DSPARK_BF16 or DSPARK_F32), fp32 accumulation.
+ * x0       [B] int32    last committed token of each request (must be in [0, V)).
+ * u_draft  [B, gamma] fp32 uniforms in [0, 1) (ignored when T == 0).
+ * x_out    [B, gamma] int32   drafted tokens.
+ * ld_out   [B, gamma, V] fp32 raw draft logits l_d (U + bias), kept for verify.
+ * flags    [B] uint32   OR'ed with DRAFT_NEAR_TIE / NONFINITE / TOKEN_RANGE.
+ * ws       workspace of at least dspark_workspace_size(DSPARK_WS_DRAFT, B, gamma, V, r) bytes.
+ * Limits: 1 <= gamma <= 64, B >= 1, V >= 2, r >= 1, T >= 0.
+ * -------------------------------------------------------------------------- */
+int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dtype,
+                        const int32_t* x0, const float* u_draft,
+                        int B, int gamma, int V, int r, float T,
+                        int32_t* x_out, float* ld_out, uint32_t* flags,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_verify -- lossless rejection-sampling verification of the drafted block.
+ *
+ * [P1 §"大模型推理的显存瓶颈与推测解码的演进逻辑"] the target checks the drafted tokens
+ * left to right, keeps the longest prefix that passes the rejection-sampling
+ * test, resamples one token at the first failure and drops the rest;
+ * [P3, opening paragraph] longest consistent prefix plus a bonus token.
+ * For each request b with L = L[b] (gamma when L is NULL):
+ *     p_d,k = softmax(l_d[b,k] / T),  p_t,k = softmax(l_t[b,k] / T)
+ *     accept position k (k = 0..L-1, in order) iff u_acc[b,k] * p_d,k(x_k) < p_t,k(x_k)
+ *     n = number of leading accepted positions
+ *     n < L : y_n ~ max(0, p_t,n - p_d,n) / Z   (inverse CDF with u_res[b];
+ *             Z == 0 falls back to p_t,n)
+ *     n == L: y_L ~ p_t,L (the bonus row)       (inverse CDF with u_res[b])
+ *     T == 0: accept iff x_k == argmax l_t,k; the resampled/bonus token is argmax l_t,n.
+ *
+ * ld     [B, gamma, V] fp32 draft logits (dspark_markov_draft's ld_out).
+ * lt     [B, gamma+1, V] fp32 target logits (row gamma = bonus position).
+ * x      [B, gamma] int32 drafted tokens.
+ * L      [B] int32 verify lengths in [0, gamma] (e.g. from dspark_prefix_schedule), or NULL.
+ * u_acc  [B, gamma] fp32, u_res [B] fp32 uniforms in [0, 1).
+ * n_acc  [B] int32 accepted count n.
+ * y_out  [B, gamma+1] int32: y[0..n-1] = x[0..n-1], y[n] = resampled/bonus token, rest -1.
+ * c_star [B, gamma] fp32 TV labels of every position (as dspark_tv_labels), or NULL.
+ * flags  [B] uint32 OR'ed with ACCEPT_NEAR_TIE / SAMPLE_NEAR_TIE / SMALL_RESIDUAL /
+ *        NONFINITE / TOKEN_RANGE.
+ * ws     workspace of at least dspark_workspace_size(DSPARK_WS_VERIFY, B, gamma, V, 0) bytes.
+ * Rows of l_t beyond L[b] (and rows of l_d at or beyond L[b]) are not read
+ * unless c_star is requested.
+ * -------------------------------------------------------------------------- */
+int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int32_t* L,
+                  const float* u_acc, const float* u_res,
+                  int B, int gamma, int V, float T,
+                  int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_tv_labels -- confidence-head supervision labels.
+ *
+ * [P3 §Confidence-Scheduled Verification] c*_k = 1 - ½ ‖p_d,k - p_t,k‖₁;
+ * [P1 §"硬件感知与置信度自适应调度机制"] the label is the analytic acceptance rate
+ * obtained from the total-variation distance.  For every b and k = 0..gamma-1.
+ * T == 0: c* = 1 if the argmaxes agree, else 0.
+ *
+ * ld      [B, gamma, V] fp32.
+ * lt      [B, lt_rows, V] fp32, lt_rows = gamma or gamma+1 (row stride of lt);
+ *         only the first gamma rows of each request are read.
+ * c_star  [B, gamma] fp32.
+ * No workspace.
+ * -------------------------------------------------------------------------- */
+int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, int lt_rows,
+                     float T, float* c_star, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_prefix_schedule -- prefix survival + greedy hardware-aware prefix scheduler.
+ *
+ * [P3 §Confidence-Scheduled Verification] a_{b,j} = ∏_{i<=j} c_{b,i} and
+ * Algorithm 1, maximise Θ = τ · SPS(B); [P1 §"硬件感知与置信度自适应调度机制"] all
+ * candidate tokens are sorted by survival and added one at a time while the
+ * expected throughput rises; the global search runs on the GPU.
+ *     a     = running product of c along each request, fp32, left to right
+ *     order = all B*gamma items by (a descending, b ascending, j ascending)
+ *     S(D)  = sum of the first D survivals in that order (fp64)
+ *     Θ(D)  = (B + S(D)) * sps[D],  D = 0..D_max
+ *     D*    = ARGMAX: the smallest D attaining max Θ;
+ *             EARLY_STOP: the first D with Θ(D+1) <= Θ(D), else D_max
+ *     L[b]  = number of request b's items among the first D*.
+ *
+ * c          [B, gamma] fp32 confidences (conditional pass probabilities).
+ * sps        [D_max+1] fp64 steps/s of the verify forward with D scheduled drafts.
+ * D_max      token budget, 0 <= D_max <= B*gamma.
+ * L_out      [B] int32.   a_out [B, gamma] fp32 or NULL.   theta_out [1] fp64 (Θ(D*)).
+ * flags      [B] uint32 or NULL: CONF_RANGE for requests with c outside [0, 1];
+ *            SCHED_NEAR_TIE in every word when the decision is within 1e-12.
+ * Limits: B*gamma <= 16384.  No workspace (ws may be NULL, ws_bytes 0).
+ * -------------------------------------------------------------------------- */
+int dspark_prefix_schedule(const float* c, const double* sps, int B, int gamma, int D_max, int mode,
+                           int32_t* L_out, float* a_out, double* theta_out, uint32_t* flags,
+                           void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_H_ */

@@ -200,7 +200,10 @@ def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
     for k in range(L):
         xk = int(x_b[k])
         if T == 0.0:
-            acc = (0 <= xk < V) and xk == int(np.argmax(np.asarray(lt_b[k], dtype=np.float32)))
+            tk, talts = greedy_choice(lt_b[k])
+            acc = (0 <= xk < V) and xk == tk
+            if len(talts) > 1 and (xk in talts):
+                accept_ties.append(k)
         else:
             if not (0 <= xk < V):
                 acc = False

@@ -1,0 +1,157 @@
+// C ABI of libdspark.so: host-side argument checks and dispatch to the kernel launchers.
+// Every entry point validates its arguments before anything is launched and returns a
+// dspark_status; nothing here allocates device memory.
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+
+namespace dspark {
+
+static thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+Options& options() {
+  static Options o;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    if (const char* e = std::getenv("DSPARK_DRAFT_TC_MIN_B")) o.draft_tc_min_b = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_DRAFT_PATH")) o.draft_force_path = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_DRAFT_PDL")) o.draft_pdl = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_VERIFY_CLUSTER")) o.verify_cluster = std::atoi(e);
+  });
+  return o;
+}
+
+int device_sm_count() {
+  if (options().sm_count > 0) return options().sm_count;
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+static dspark_status einval(const std::string& msg) {
+  set_error(msg);
+  return DSPARK_EINVAL;
+}
+
+}  // namespace dspark
+
+using namespace dspark;
+
+extern "C" {
+
+const char* dspark_status_string(int status) {
+  switch (status) {
+    case DSPARK_OK: return "DSPARK_OK";
+    case DSPARK_EINVAL: return "DSPARK_EINVAL";
+    case DSPARK_ECUDA: return "DSPARK_ECUDA";
+    case DSPARK_ENOTIMPL: return "DSPARK_ENOTIMPL";
+    case DSPARK_ETIMEOUT: return "DSPARK_ETIMEOUT";
+    default: return "DSPARK_UNKNOWN";
+  }
+}
+
+const char* dspark_last_error(void) { return g_last_error.c_str(); }
+
+int dspark_set_option(const char* key, long value) {
+  if (!key) return einval("dspark_set_option: null key");
+  Options& o = options();
+  if (!std::strcmp(key, "draft_tc_min_b")) o.draft_tc_min_b = (int)value;
+  else if (!std::strcmp(key, "draft_path")) o.draft_force_path = (int)value;
+  else if (!std::strcmp(key, "draft_pdl")) o.draft_pdl = (int)value;
+  else if (!std::strcmp(key, "verify_cluster")) o.verify_cluster = (int)value;
+  else if (!std::strcmp(key, "sm_count")) o.sm_count = (int)value;
+  else return einval(std::string("dspark_set_option: unknown key ") + key);
+  return DSPARK_OK;
+}
+
+size_t dspark_workspace_size(int which, int B, int gamma, int V, int r) {
+  if (B <= 0 || gamma <= 0 || V <= 0) return 0;
+  switch (which) {
+    case DSPARK_WS_DRAFT: return draft_workspace_bytes(B, gamma, V, r);
+    case DSPARK_WS_VERIFY: return verify_workspace_bytes(B, gamma, V);
+    case DSPARK_WS_SCHEDULE: return 0;
+    default: return 0;
+  }
+}
+
+int dspark_workspace_status(const void* ws, void* stream) {
+  if (!ws) return einval("dspark_workspace_status: null workspace");
+  uint32_t st = 0;
+  cudaError_t rc = cudaMemcpyAsync(&st, ws, sizeof(st), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (rc == cudaSuccess) rc = cudaStreamSynchronize((cudaStream_t)stream);
+  if (rc != cudaSuccess) {
+    set_error(std::string("dspark_workspace_status: ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
+  }
+  return st ? DSPARK_ETIMEOUT : DSPARK_OK;
+}
+
+int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dtype, const int32_t* x0,
+                        const float* u_draft, int B, int gamma, int V, int r, float T, int32_t* x_out,
+                        float* ld_out, uint32_t* flags, void* ws, size_t ws_bytes, void* stream) {
+  if (!U || !W1 || !W2 || !x0 || !x_out || !ld_out || !flags || !ws) return einval("dspark_markov_draft: null pointer");
+  if (T != 0.f && !u_draft) return einval("dspark_markov_draft: u_draft is required when T > 0");
+  if (B <= 0 || V < 2 || r <= 0) return einval("dspark_markov_draft: B, r must be >= 1 and V >= 2");
+  if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_markov_draft: gamma must be in [1, 64]");
+  if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_markov_draft: T must be finite and >= 0");
+  if (w_dtype != DSPARK_BF16 && w_dtype != DSPARK_F32) return einval("dspark_markov_draft: w_dtype must be DSPARK_BF16 or DSPARK_F32");
+  if ((long long)B * gamma * V >= (1ll << 40)) return einval("dspark_markov_draft: tensor too large");
+  if (ws_bytes < draft_workspace_bytes(B, gamma, V, r)) return einval("dspark_markov_draft: workspace too small");
+  if ((uintptr_t)ws % 256) return einval("dspark_markov_draft: workspace must be 256-byte aligned");
+  DraftCall c{U, W1, W2, w_dtype, x0, u_draft, B, gamma, V, r, T, x_out, ld_out, flags, ws, ws_bytes,
+              (cudaStream_t)stream};
+  return launch_draft(c);
+}
+
+int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int32_t* L, const float* u_acc,
+                  const float* u_res, int B, int gamma, int V, float T, int32_t* n_acc, int32_t* y_out,
+                  float* c_star, uint32_t* flags, void* ws, size_t ws_bytes, void* stream) {
+  if (!ld || !lt || !x || !n_acc || !y_out || !flags || !ws) return einval("dspark_verify: null pointer");
+  if (T != 0.f && (!u_acc || !u_res)) return einval("dspark_verify: u_acc and u_res are required when T > 0");
+  if (B <= 0 || V < 2) return einval("dspark_verify: B must be >= 1 and V >= 2");
+  if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_verify: gamma must be in [1, 64]");
+  if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_verify: T must be finite and >= 0");
+  if (ws_bytes < verify_workspace_bytes(B, gamma, V)) return einval("dspark_verify: workspace too small");
+  if ((uintptr_t)ws % 256) return einval("dspark_verify: workspace must be 256-byte aligned");
+  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, 1, n_acc, y_out, c_star, flags, ws, ws_bytes,
+               (cudaStream_t)stream};
+  return launch_verify(c);
+}
+
+int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, int lt_rows, float T, float* c_star,
+                     void* stream) {
+  if (!ld || !lt || !c_star) return einval("dspark_tv_labels: null pointer");
+  if (B <= 0 || V < 2) return einval("dspark_tv_labels: B must be >= 1 and V >= 2");
+  if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_tv_labels: gamma must be in [1, 64]");
+  if (lt_rows != gamma && lt_rows != gamma + 1) return einval("dspark_tv_labels: lt_rows must be gamma or gamma+1");
+  if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_tv_labels: T must be finite and >= 0");
+  VerifyCall c{ld, lt, nullptr, nullptr, nullptr, nullptr, B, gamma, V, lt_rows, T, 0, nullptr, nullptr, c_star,
+               nullptr, nullptr, 0, (cudaStream_t)stream};
+  return launch_verify(c);
+}
+
+int dspark_prefix_schedule(const float* c, const double* sps, int B, int gamma, int D_max, int mode, int32_t* L_out,
+                           float* a_out, double* theta_out, uint32_t* flags, void* ws, size_t ws_bytes,
+                           void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!c || !sps || !L_out || !theta_out) return einval("dspark_prefix_schedule: null pointer");
+  if (B <= 0 || gamma < 1 || gamma > kMaxGamma) return einval("dspark_prefix_schedule: B >= 1, gamma in [1, 64]");
+  if ((long long)B * gamma > kMaxScheduleItems) return einval("dspark_prefix_schedule: B*gamma must be <= 16384");
+  if (D_max < 0 || D_max > B * gamma) return einval("dspark_prefix_schedule: D_max must be in [0, B*gamma]");
+  if (mode != DSPARK_SCHED_ARGMAX && mode != DSPARK_SCHED_EARLY_STOP) return einval("dspark_prefix_schedule: bad mode");
+  ScheduleCall s{c, sps, B, gamma, D_max, mode, L_out, a_out, theta_out, flags, (cudaStream_t)stream};
+  return launch_schedule(s);
+}
+
+}  // extern "C"

@@ -1,0 +1,87 @@
+// Host-side interface between the C ABI (api.cu) and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+void set_error(const std::string& msg);
+
+struct Options {
+  int draft_tc_min_b = 9;        // bf16 drafts with at least this many requests use the tensor-core path
+  int draft_force_path = 0;      // 0 auto, 1 CUDA-core GEMV, 2 tensor cores
+  int draft_pdl = 1;             // chain the draft kernels with programmatic dependent launch
+  int verify_cluster = 0;        // 0 auto, else the cluster size (1, 2, 4, 8, 16)
+  int sm_count = 0;              // 0: query the device
+};
+Options& options();
+
+int device_sm_count();
+
+struct DraftCall {
+  const float* U;
+  const void* W1;
+  const void* W2;
+  int w_dtype;
+  const int32_t* x0;
+  const float* u_draft;
+  int B, gamma, V, r;
+  float T;
+  int32_t* x_out;
+  float* ld_out;
+  uint32_t* flags;
+  void* ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+};
+
+struct VerifyCall {
+  const float* ld;
+  const float* lt;
+  const int32_t* x;
+  const int32_t* L;
+  const float* u_acc;
+  const float* u_res;
+  int B, gamma, V, lt_rows;
+  float T;
+  int do_verify;
+  int32_t* n_acc;
+  int32_t* y_out;
+  float* c_star;
+  uint32_t* flags;
+  void* ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+};
+
+struct ScheduleCall {
+  const float* c;
+  const double* sps;
+  int B, gamma, D_max, mode;
+  int32_t* L_out;
+  float* a_out;
+  double* theta_out;
+  uint32_t* flags;
+  cudaStream_t stream;
+};
+
+size_t draft_workspace_bytes(int B, int gamma, int V, int r);
+size_t verify_workspace_bytes(int B, int gamma, int V);
+
+dspark_status launch_draft(const DraftCall& c);
+dspark_status launch_verify(const VerifyCall& c);
+dspark_status launch_schedule(const ScheduleCall& c);
+
+constexpr int kMaxGamma = 64;
+constexpr int kMaxScheduleItems = 16384;
+constexpr size_t kWsHeader = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace dspark

@@ -1,0 +1,278 @@
+// Prefix survival and the greedy hardware-aware prefix scheduler.
+//
+// [P3 "DSpark Speculative Decoding" §Confidence-Scheduled Verification: a_{r,j} = ∏_{i≤j} c_{r,i};
+//  Algorithm 1 maximises Θ = τ·SPS(B) by extending verify lengths greedily along a]
+// [P1 "DeepSeek V4-Pro DSpark 推测解码方案深度解析" §硬件感知与置信度自适应调度机制: every candidate
+//  token of the batch is ranked by cumulative survival and added one at a time while expected
+//  accepted tokens x hardware speed keeps rising; the global search runs on the GPU]
+//
+// One CTA of 1024 threads: running products per request (fp32, left to right), 64-bit keys
+// (survival descending, then flat index b*gamma + j) sorted bitonically in shared memory with
+// warp shuffles for the short strides, an fp64 block scan of the sorted survivals giving
+// Θ(D) = (B + S(D)) * sps[D] for D = 0..D_max, the ARGMAX / EARLY_STOP choice, and per-request
+// counts of the kept items.
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dspark {
+
+constexpr int kSchedThreads = 1024;
+constexpr int kSchedWarps = kSchedThreads / 32;
+
+struct SchedArgs {
+  const float* c;
+  const double* sps;
+  int B, gamma, D_max, mode, P;
+  int32_t* L_out;
+  float* a_out;
+  double* theta_out;
+  uint32_t* flags;
+};
+
+// Survival descending -> ascending 32-bit key; -0 ranks as +0, NaN ranks last.
+__device__ __forceinline__ uint32_t desc_key(float a) {
+  if (isnan(a)) return 0xFFFFFFFFu;
+  if (a == 0.f) a = 0.f;
+  const uint32_t u = __float_as_uint(a);
+  const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ~ord;
+}
+
+__device__ __forceinline__ float key_value(uint64_t key) {
+  const uint32_t ord = ~(uint32_t)(key >> 32);
+  const uint32_t u = (ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord;
+  return __uint_as_float(u);
+}
+
+__global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s) {
+  extern __shared__ __align__(16) uint64_t keys[];
+  int* cnt = reinterpret_cast<int*>(keys + s.P);
+  __shared__ double sh_w[kSchedWarps];
+  __shared__ double sh_best[kSchedWarps];
+  __shared__ int sh_bestD[kSchedWarps];
+  __shared__ int sh_stop[kSchedWarps];
+  __shared__ int sh_tie[kSchedWarps];
+  __shared__ int s_D;
+  __shared__ double s_theta;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int B = s.B, G = s.gamma, N = B * G, P = s.P, Dm = s.D_max;
+
+  // ---------------------------------------------------------------- survival and keys
+  for (int b = tid; b < B; b += kSchedThreads) {
+    float prod = 1.f;
+    bool bad = false;
+    for (int j = 0; j < G; ++j) {
+      const float cj = s.c[(size_t)b * G + j];
+      bad |= !(cj >= 0.f && cj <= 1.f);
+      prod = (j == 0) ? cj : __fmul_rn(prod, cj);
+      if (s.a_out) s.a_out[(size_t)b * G + j] = prod;
+      keys[b * G + j] = ((uint64_t)desc_key(prod) << 32) | (uint32_t)(b * G + j);
+    }
+    if (bad && s.flags) atomicOr(s.flags + b, DSPARK_FLAG_CONF_RANGE);
+    cnt[b] = 0;
+  }
+  for (int i = N + tid; i < P; i += kSchedThreads) keys[i] = ~0ull;
+  __syncthreads();
+
+  // ---------------------------------------------------------------- bitonic sort (ascending)
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32 || P < 64) {
+        for (int i = tid; i < P; i += kSchedThreads) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const uint64_t x = keys[i], y = keys[ixj];
+            const bool up = (i & k) == 0;
+            if ((x > y) == up) {
+              keys[i] = y;
+              keys[ixj] = x;
+            }
+          }
+        }
+        __syncthreads();
+      } else {
+        // strides 16..1 stay inside a warp: 32 consecutive keys per warp pass
+        for (int base = warp * 32; base < P; base += kSchedThreads) {
+          const int i = base + lane;
+          uint64_t x = keys[i];
+          for (int jj = j; jj > 0; jj >>= 1) {
+            const uint64_t y = __shfl_xor_sync(0xffffffffu, x, jj);
+            const bool up = (i & k) == 0;
+            const bool lower = (lane & jj) == 0;
+            const uint64_t mn = x < y ? x : y, mx = x < y ? y : x;
+            x = (lower == up) ? mn : mx;
+          }
+          keys[i] = x;
+        }
+        __syncthreads();
+        break;  // all strides below 32 handled
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- Θ pass (twice: choose, then tie check)
+  // The sorted survivals are scanned in chunks of kSchedThreads items; item i moves D from
+  // i to i+1, so the thread owning it sees Θ(i) and Θ(i+1).
+  const double theta0 = (double)B * s.sps[0];
+  double best = theta0;
+  int bestD = 0;
+  int stop = Dm;  // EARLY_STOP: first d with Θ(d+1) <= Θ(d)
+  for (int pass = 0; pass < 2; ++pass) {
+    int tie = 0;
+    double carry = 0.0;
+    const int Dstar = pass ? s_D : 0;
+    const double th_star = pass ? s_theta : 0.0;
+    for (int base = 0; base < Dm; base += kSchedThreads) {
+      const int i = base + tid;
+      const double ai = (i < Dm) ? (double)key_value(keys[i]) : 0.0;
+      const double incl = warp_incl_scan_d(ai);
+      double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+      if (lane == 0) excl = 0.0;
+      if (lane == 31) sh_w[warp] = incl;
+      __syncthreads();
+      double wpre = carry;
+      for (int w = 0; w < warp; ++w) wpre += sh_w[w];
+      double tot = carry;
+      for (int w = 0; w < kSchedWarps; ++w) tot += sh_w[w];
+      __syncthreads();
+      carry = tot;
+      if (i < Dm) {
+        const double th_lo = ((double)B + (wpre + excl)) * s.sps[i];      // Θ(i)
+        const double th_hi = ((double)B + (wpre + incl)) * s.sps[i + 1];  // Θ(i+1)
+        if (pass == 0) {
+          if (th_hi > best) {
+            best = th_hi;
+            bestD = i + 1;
+          }
+          if (th_hi <= th_lo && i < stop) stop = i;
+        } else if (s.mode == DSPARK_SCHED_ARGMAX) {
+          if (i + 1 != Dstar && fabs(th_hi - th_star) <= 1e-12 * fabs(th_star)) tie = 1;
+        } else {
+          if (i <= Dstar && i < Dm && fabs(th_hi - th_lo) <= 1e-12 * fabs(th_lo)) tie = 1;
+        }
+      }
+    }
+    if (pass == 0) {
+      // argmax with the smallest D among equal Θ; first stop index
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int od = __shfl_xor_sync(0xffffffffu, bestD, o);
+        if (ob > best || (ob == best && od < bestD)) {
+          best = ob;
+          bestD = od;
+        }
+        stop = min(stop, __shfl_xor_sync(0xffffffffu, stop, o));
+      }
+      if (lane == 0) {
+        sh_best[warp] = best;
+        sh_bestD[warp] = bestD;
+        sh_stop[warp] = stop;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        double bb = sh_best[0];
+        int bd = sh_bestD[0], sp = sh_stop[0];
+        for (int w = 1; w < kSchedWarps; ++w) {
+          if (sh_best[w] > bb || (sh_best[w] == bb && sh_bestD[w] < bd)) {
+            bb = sh_best[w];
+            bd = sh_bestD[w];
+          }
+          sp = min(sp, sh_stop[w]);
+        }
+        if (s.mode == DSPARK_SCHED_ARGMAX) {
+          s_D = bd;
+          s_theta = bb;
+        } else {
+          s_D = sp;
+          s_theta = 0.0;  // filled in below
+        }
+      }
+      __syncthreads();
+      if (s.mode != DSPARK_SCHED_ARGMAX) {
+        // Θ(D*) for EARLY_STOP: recompute S(D*) serially from the sorted keys is O(D); use the
+        // scan instead: the thread owning item D*-1 knows Θ(D*).
+        const int Ds = s_D;
+        double carry2 = 0.0;
+        for (int base = 0; base < max(Ds, 1); base += kSchedThreads) {
+          const int i = base + tid;
+          const double ai = (i < Ds) ? (double)key_value(keys[i]) : 0.0;
+          const double incl = warp_incl_scan_d(ai);
+          if (lane == 31) sh_w[warp] = incl;
+          __syncthreads();
+          double wpre = carry2;
+          for (int w = 0; w < warp; ++w) wpre += sh_w[w];
+          double tot = carry2;
+          for (int w = 0; w < kSchedWarps; ++w) tot += sh_w[w];
+          __syncthreads();
+          carry2 = tot;
+          if (i == Ds - 1) s_theta = ((double)B + (wpre + incl)) * s.sps[Ds];
+        }
+        if (Ds == 0 && tid == 0) s_theta = theta0;
+        __syncthreads();
+      }
+    } else {
+      const int any = __any_sync(0xffffffffu, tie);
+      if (lane == 0) sh_tie[warp] = any;
+      __syncthreads();
+      if (tid == 0) {
+        int t = 0;
+        for (int w = 0; w < kSchedWarps; ++w) t |= sh_tie[w];
+        if (s.mode == DSPARK_SCHED_ARGMAX && s_D != 0 && fabs(theta0 - s_theta) <= 1e-12 * fabs(s_theta)) t = 1;
+        sh_tie[0] = t;
+      }
+      __syncthreads();
+    }
+  }
+
+  // ---------------------------------------------------------------- counts and outputs
+  const int Ds = s_D;
+  for (int i = tid; i < Ds; i += kSchedThreads) atomicAdd(&cnt[(int)(uint32_t)keys[i] / G], 1);
+  __syncthreads();
+  const bool near = sh_tie[0] != 0;
+  for (int b = tid; b < B; b += kSchedThreads) {
+    s.L_out[b] = cnt[b];
+    if (near && s.flags) atomicOr(s.flags + b, DSPARK_FLAG_SCHED_NEAR_TIE);
+  }
+  if (tid == 0) s.theta_out[0] = s_theta;
+}
+
+dspark_status launch_schedule(const ScheduleCall& c) {
+  SchedArgs s{};
+  s.c = c.c;
+  s.sps = c.sps;
+  s.B = c.B;
+  s.gamma = c.gamma;
+  s.D_max = c.D_max;
+  s.mode = c.mode;
+  int P = 64;
+  while (P < c.B * c.gamma) P <<= 1;
+  s.P = P;
+  s.L_out = c.L_out;
+  s.a_out = c.a_out;
+  s.theta_out = c.theta_out;
+  s.flags = c.flags;
+  const size_t smem = (size_t)P * 8 + align_up((size_t)c.B * 4, 16);
+  static size_t attr_smem = 0;
+  cudaError_t rc;
+  if (smem > 48 * 1024 && smem > attr_smem) {
+    rc = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (rc != cudaSuccess) {
+      set_error(std::string("cudaFuncSetAttribute(schedule_kernel): ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
+    }
+    attr_smem = smem;
+  }
+  schedule_kernel<<<1, kSchedThreads, smem, c.stream>>>(s);
+  rc = cudaGetLastError();
+  if (rc != cudaSuccess) {
+    set_error(std::string("schedule launch: ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
+  }
+  return DSPARK_OK;
+}
+
+}  // namespace dspark

@@ -1,0 +1,617 @@
+// Fused rejection-sampling verification and TV confidence labels.
+//
+// [P1 "DeepSeek V4-Pro DSpark 推测解码方案深度解析" §大模型推理的显存瓶颈与推测解码的演进逻辑:
+//  the target checks the drafted tokens left to right with rejection sampling, keeps the
+//  longest passing prefix, resamples one token at the first failure and drops the rest]
+// [P3 "DSpark Speculative Decoding", opening paragraph: longest consistent prefix + bonus token;
+//  §Confidence-Scheduled Verification: label c*_k = 1 - ½‖p_d - p_t‖₁]
+//
+// One thread-block cluster per (request, block position) row.  The CS CTAs of a cluster
+// split the vocabulary; each holds its slice of the draft row and of the target row in
+// shared memory (one bulk copy each), so both tensors are read from HBM exactly once.
+// Partial statistics cross the cluster through distributed shared memory:
+//   A  max of z = l / T (or greedy top-2)            -> cluster max
+//   B  e = exp(z - max) in place, sums               -> normalisers S_d, S_t, e at x_k
+//   C  p = e / S, sum min(p_d, p_t), sum max(0, p_t - p_d)  -> c*, residual mass Z
+//   D  the CTA whose slice holds u_res * W (W = Z for a residual row, S_t for the bonus
+//      row) finds the token by an fp64 segment scan of its slice.
+// Every row that may be the first rejection samples its residual speculatively; the last
+// row of a request to finish (atomic counter) assembles n and y.
+
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace dspark {
+
+struct VerifyArgs {
+  const float* ld;
+  const float* lt;
+  const int32_t* x;
+  const int32_t* L;
+  const float* u_acc;
+  const float* u_res;
+  int B, gamma, V, lt_rows, rows_per_req;
+  float inv_T;
+  int greedy;
+  int do_verify;
+  float* c_star;
+  int32_t* n_acc;
+  int32_t* y_out;
+  uint32_t* flags;
+  uint32_t* status;
+  int32_t* row_acc;
+  int32_t* row_cand;
+  uint32_t* row_fl;
+  int32_t* counter;
+  int Vc;
+  int bulk;
+};
+
+struct __align__(16) Slot {
+  float md, mt;
+  Top2 gd, gt;
+  double sd, st;
+  float ed_x, et_x;
+  int has_x;
+  int pad0;
+  double smin, sq;
+  int cand;
+  uint32_t cand_fl;
+  uint32_t data_fl;
+  int pad1;
+};
+
+constexpr int kMaxWarps = 16;
+
+// exp(z - m) as 2^((z - m) log2 e); z and m are already-rounded fp32 values
+__device__ __forceinline__ float vex(float z, float m) { return exp2f(__fmul_rn(__fsub_rn(z, m), kLog2e)); }
+
+__device__ float block_max(float v, float* sh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  v = warp_max(v);
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  float r = sh[0];
+  for (int w = 1; w < nw; ++w) r = fmaxf(r, sh[w]);
+  __syncthreads();
+  return r;
+}
+
+__device__ double2 block_sum2(double a, double b, double2* sh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  a = warp_sum_d(a);
+  b = warp_sum_d(b);
+  if (lane == 0) sh[warp] = make_double2(a, b);
+  __syncthreads();
+  double2 r = sh[0];
+  for (int w = 1; w < nw; ++w) {
+    r.x += sh[w].x;
+    r.y += sh[w].y;
+  }
+  __syncthreads();
+  return r;
+}
+
+__device__ Top2 block_top2(Top2 t, Top2* sh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t = top2_merge(t, top2_shfl_xor(t, o));
+  if (lane == 0) sh[warp] = t;
+  __syncthreads();
+  Top2 r = sh[0];
+  for (int w = 1; w < nw; ++w) r = top2_merge(r, sh[w]);
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ void top2_push(Top2& t, float x, int idx) {
+  if (t.idx < 0 || x > t.best) {
+    t.second = fmaxf(t.second, t.best);
+    t.best = x;
+    t.idx = idx;
+  } else {
+    t.second = fmaxf(t.second, x);
+  }
+}
+
+// Assemble n_acc / y for request b once every one of its rows has reported.
+__device__ void finalize_request(const VerifyArgs& a, int b, int Lb) {
+  const int R = a.gamma + 1;
+  const int32_t* acc = a.row_acc + (size_t)b * R;
+  const int32_t* cand = a.row_cand + (size_t)b * R;
+  const uint32_t* rfl = a.row_fl + (size_t)b * R;
+  int n = 0;
+  while (n < Lb && __ldcg(acc + n)) ++n;
+  uint32_t fl = 0;
+  for (int j = 0; j <= n && j < Lb; ++j) fl |= __ldcg(rfl + j) & DSPARK_FLAG_ACCEPT_NEAR_TIE;
+  fl |= __ldcg(rfl + n) & (DSPARK_FLAG_SAMPLE_NEAR_TIE | DSPARK_FLAG_SMALL_RESIDUAL);
+  int32_t* y = a.y_out + (size_t)b * R;
+  for (int j = 0; j < R; ++j) y[j] = (j < n) ? a.x[(size_t)b * a.gamma + j] : (j == n ? __ldcg(cand + n) : -1);
+  a.n_acc[b] = n;
+  if (fl && a.flags) atomicOr(a.flags + b, fl);
+}
+
+__device__ void row_done(const VerifyArgs& a, int b, int Lb) {
+  __threadfence();
+  const int old = atomicAdd(a.counter + b, 1);
+  if (old == a.rows_per_req - 1) {
+    __threadfence();
+    finalize_request(a, b, Lb);
+  }
+}
+
+__global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CS = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int row = blockIdx.x / CS;
+  const int b = row / a.rows_per_req, kk = row - b * a.rows_per_req;
+  const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
+
+  extern __shared__ __align__(16) float vsm[];
+  float* sd = vsm;
+  float* st = vsm + a.Vc;
+  __shared__ Slot slot;
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ float sh_f[kMaxWarps];
+  __shared__ double2 sh_d[kMaxWarps];
+  __shared__ Top2 sh_t[kMaxWarps];
+  __shared__ double sh_w[kMaxWarps];
+  __shared__ int s_pick;
+  __shared__ double s_lo, s_hi;
+
+  int Lb = a.gamma;
+  if (a.do_verify && a.L) Lb = min(max(a.L[b], 0), a.gamma);
+  const bool need_cstar = (a.c_star != nullptr) && kk < a.gamma;
+  const bool need_acc = a.do_verify && kk < Lb;
+  const bool need_bonus = a.do_verify && kk == Lb;
+  const bool need_d = need_cstar || need_acc;
+  const bool need_t = need_d || need_bonus;
+
+  if (!need_t) {  // uniform over the cluster: nothing of this row is needed
+    if (a.do_verify && rank == 0 && tid == 0) row_done(a, b, Lb);
+    return;
+  }
+
+  const int v_beg = rank * a.Vc;
+  const int n = max(0, min(a.V, v_beg + a.Vc) - v_beg);
+  const size_t rowd = ((size_t)b * a.gamma + kk) * a.V + v_beg;
+  const size_t rowt = ((size_t)b * a.lt_rows + kk) * a.V + v_beg;
+  bool timed_out = false;
+
+  if (tid == 0) {
+    slot.cand = -1;
+    slot.cand_fl = 0;
+    slot.data_fl = 0;
+    slot.has_x = 0;
+  }
+  // ------------------------------------------------------------------ load the slices
+  if (a.bulk) {
+    if (tid == 0) {
+      mbar_init(&bar, 1);
+      fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0 && n > 0) {
+      const uint32_t bytes = (uint32_t)n * 4u;
+      mbar_arrive_expect_tx(&bar, need_d ? 2u * bytes : bytes);
+      if (need_d) bulk_g2s(sd, a.ld + rowd, bytes, &bar);
+      bulk_g2s(st, a.lt + rowt, bytes, &bar);
+    }
+    if (n > 0) timed_out = !mbar_wait(&bar, 0);
+  } else {
+    for (int i = tid; i < n; i += nthr) {
+      sd[i] = need_d ? a.ld[rowd + i] : 0.f;
+      st[i] = a.lt[rowt + i];
+    }
+    __syncthreads();
+  }
+  if (timed_out && a.status) atomicOr(a.status, (uint32_t)DSPARK_ETIMEOUT);
+
+  // ------------------------------------------------------------------ phase A: maxima
+  const float inv_T = a.inv_T;
+  const int n4 = n >> 2;
+  bool nonfin = false;
+  if (a.greedy) {
+    Top2 gd{-INFINITY, -1, -INFINITY}, gt{-INFINITY, -1, -INFINITY};
+    for (int i = tid; i < n; i += nthr) {
+      const float lt_ = st[i];
+      nonfin |= !isfinite(lt_);
+      top2_push(gt, lt_, v_beg + i);
+      if (need_d) {
+        const float ld_ = sd[i];
+        nonfin |= !isfinite(ld_);
+        top2_push(gd, ld_, v_beg + i);
+      }
+    }
+    gd = block_top2(gd, sh_t);
+    gt = block_top2(gt, sh_t);
+    if (nonfin) atomicOr(&slot.data_fl, DSPARK_FLAG_NONFINITE);
+    if (tid == 0) {
+      slot.gd = gd;
+      slot.gt = gt;
+    }
+    cluster.sync();
+    if (rank == 0 && tid == 0) {
+      Top2 GD{-INFINITY, -1, -INFINITY}, GT{-INFINITY, -1, -INFINITY};
+      uint32_t dfl = 0;
+      for (int r = 0; r < CS; ++r) {
+        const Slot* p = cluster.map_shared_rank(&slot, r);
+        GD = top2_merge(GD, p->gd);
+        GT = top2_merge(GT, p->gt);
+        dfl |= p->data_fl;
+      }
+      const int argt = min(max(GT.idx, 0), a.V - 1);
+      const bool ttie = GT.best - GT.second <= 1e-6f * fmaxf(1.f, fabsf(GT.best));
+      if (need_cstar) a.c_star[(size_t)b * a.gamma + kk] = (GD.idx == GT.idx) ? 1.f : 0.f;
+      const size_t ri = (size_t)b * (a.gamma + 1) + kk;
+      if (need_acc) {
+        const int xk = a.x[(size_t)b * a.gamma + kk];
+        if ((unsigned)xk >= (unsigned)a.V) dfl |= DSPARK_FLAG_TOKEN_RANGE;
+        a.row_acc[ri] = (xk == GT.idx) ? 1 : 0;
+      }
+      if (need_acc || need_bonus) {
+        a.row_cand[ri] = argt;
+        a.row_fl[ri] = ttie ? (DSPARK_FLAG_ACCEPT_NEAR_TIE | DSPARK_FLAG_SAMPLE_NEAR_TIE) : 0u;
+      }
+      if (timed_out) dfl |= DSPARK_FLAG_DEVICE_TIMEOUT;
+      if (dfl && a.flags) atomicOr(a.flags + b, dfl);
+    }
+    cluster.sync();
+    if (a.do_verify && rank == 0 && tid == 0) row_done(a, b, Lb);
+    return;
+  }
+
+  float md = -INFINITY, mt = -INFINITY;
+  {
+    const float4* sd4 = reinterpret_cast<const float4*>(sd);
+    const float4* st4 = reinterpret_cast<const float4*>(st);
+    for (int i = tid; i < n4; i += nthr) {
+      const float4 t4 = st4[i];
+      nonfin |= !(isfinite(t4.x) && isfinite(t4.y) && isfinite(t4.z) && isfinite(t4.w));
+      mt = fmaxf(mt, fmaxf(fmaxf(__fmul_rn(t4.x, inv_T), __fmul_rn(t4.y, inv_T)), fmaxf(__fmul_rn(t4.z, inv_T), __fmul_rn(t4.w, inv_T))));
+      if (need_d) {
+        const float4 d4 = sd4[i];
+        nonfin |= !(isfinite(d4.x) && isfinite(d4.y) && isfinite(d4.z) && isfinite(d4.w));
+        md = fmaxf(md, fmaxf(fmaxf(__fmul_rn(d4.x, inv_T), __fmul_rn(d4.y, inv_T)), fmaxf(__fmul_rn(d4.z, inv_T), __fmul_rn(d4.w, inv_T))));
+      }
+    }
+    for (int i = 4 * n4 + tid; i < n; i += nthr) {
+      nonfin |= !isfinite(st[i]);
+      mt = fmaxf(mt, __fmul_rn(st[i], inv_T));
+      if (need_d) {
+        nonfin |= !isfinite(sd[i]);
+        md = fmaxf(md, __fmul_rn(sd[i], inv_T));
+      }
+    }
+  }
+  md = block_max(md, sh_f);
+  mt = block_max(mt, sh_f);
+  if (nonfin) atomicOr(&slot.data_fl, DSPARK_FLAG_NONFINITE);
+  if (tid == 0) {
+    slot.md = md;
+    slot.mt = mt;
+  }
+  cluster.sync();
+  float Md = -INFINITY, Mt = -INFINITY;
+  for (int r = 0; r < CS; ++r) {
+    const Slot* p = cluster.map_shared_rank(&slot, r);
+    Md = fmaxf(Md, p->md);
+    Mt = fmaxf(Mt, p->mt);
+  }
+
+  // ------------------------------------------------------------------ phase B: exponentials, normalisers
+  {
+    float4* sd4 = reinterpret_cast<float4*>(sd);
+    float4* st4 = reinterpret_cast<float4*>(st);
+    float ad = 0.f, at = 0.f;
+    for (int i = tid; i < n4; i += nthr) {
+      float4 t4 = st4[i];
+      t4.x = vex(__fmul_rn(t4.x, inv_T), Mt);
+      t4.y = vex(__fmul_rn(t4.y, inv_T), Mt);
+      t4.z = vex(__fmul_rn(t4.z, inv_T), Mt);
+      t4.w = vex(__fmul_rn(t4.w, inv_T), Mt);
+      st4[i] = t4;
+      at += (t4.x + t4.y) + (t4.z + t4.w);
+      if (need_d) {
+        float4 d4 = sd4[i];
+        d4.x = vex(__fmul_rn(d4.x, inv_T), Md);
+        d4.y = vex(__fmul_rn(d4.y, inv_T), Md);
+        d4.z = vex(__fmul_rn(d4.z, inv_T), Md);
+        d4.w = vex(__fmul_rn(d4.w, inv_T), Md);
+        sd4[i] = d4;
+        ad += (d4.x + d4.y) + (d4.z + d4.w);
+      }
+    }
+    for (int i = 4 * n4 + tid; i < n; i += nthr) {
+      st[i] = vex(__fmul_rn(st[i], inv_T), Mt);
+      at += st[i];
+      if (need_d) {
+        sd[i] = vex(__fmul_rn(sd[i], inv_T), Md);
+        ad += sd[i];
+      }
+    }
+    const double2 s2 = block_sum2((double)ad, (double)at, sh_d);
+    if (tid == 0) {
+      slot.sd = s2.x;
+      slot.st = s2.y;
+      if (need_acc) {
+        const int xk = a.x[(size_t)b * a.gamma + kk];
+        if (xk >= v_beg && xk < v_beg + n) {
+          slot.ed_x = sd[xk - v_beg];
+          slot.et_x = st[xk - v_beg];
+          slot.has_x = 1;
+        }
+      }
+    }
+  }
+  cluster.sync();
+  double Sd = 0.0, St = 0.0, Wt[16];
+  float ed_x = 0.f, et_x = 0.f;
+  int x_found = 0;
+  for (int r = 0; r < CS; ++r) {
+    const Slot* p = cluster.map_shared_rank(&slot, r);
+    Sd += p->sd;
+    St += p->st;
+    Wt[r] = p->st;
+    if (p->has_x) {
+      ed_x = p->ed_x;
+      et_x = p->et_x;
+      x_found = 1;
+    }
+  }
+
+  // ------------------------------------------------------------------ phase C: TV and residual mass
+  const float iSd = (float)(1.0 / Sd), iSt = (float)(1.0 / St);
+  double Smin = 0.0, Z = 0.0, Wq[16];
+  const bool phase_c = need_cstar || need_acc;
+  if (phase_c) {
+    float amin = 0.f, aq = 0.f;
+    for (int i = tid; i < n; i += nthr) {
+      const float pd = __fmul_rn(sd[i], iSd), pt = __fmul_rn(st[i], iSt);
+      amin += fminf(pd, pt);
+      aq += fmaxf(pt - pd, 0.f);
+    }
+    const double2 s2 = block_sum2((double)amin, (double)aq, sh_d);
+    if (tid == 0) {
+      slot.smin = s2.x;
+      slot.sq = s2.y;
+    }
+    cluster.sync();
+    for (int r = 0; r < CS; ++r) {
+      const Slot* p = cluster.map_shared_rank(&slot, r);
+      Smin += p->smin;
+      Z += p->sq;
+      Wq[r] = p->sq;
+    }
+  }
+
+  // ------------------------------------------------------------------ phase D: residual / bonus sample
+  if (need_acc || need_bonus) {
+    const bool use_q = need_acc && Z > 0.0;
+    const double Wtot = use_q ? Z : St;
+    const double t = (double)a.u_res[b] * Wtot;
+    double P = 0.0;
+    for (int r = 0; r < rank; ++r) P += use_q ? Wq[r] : Wt[r];
+    const double Wr = use_q ? Wq[rank] : Wt[rank];
+    const double Pn = P + Wr;
+    int last_nz = -1;
+    for (int r = 0; r < CS; ++r)
+      if ((use_q ? Wq[r] : Wt[r]) > 0.0) last_nz = r;
+    const bool cross = (Wr > 0.0) && (P <= t) && (t < Pn || rank == last_nz);
+    if (cross) {  // uniform over the CTA
+      const int seg = (n + nthr - 1) / nthr;
+      const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
+      double tsum = 0.0;
+      for (int i = i0; i < i1; ++i)
+        tsum += use_q ? (double)fmaxf(__fmul_rn(st[i], iSt) - __fmul_rn(sd[i], iSd), 0.f) : (double)st[i];
+      const double incl = warp_incl_scan_d(tsum);
+      double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+      if (lane == 0) excl = 0.0;
+      if (lane == 31) sh_w[warp] = incl;
+      if (tid == 0) s_pick = -1;
+      __syncthreads();
+      double wpre = P;
+      for (int w = 0; w < warp; ++w) wpre += sh_w[w];
+      const double pre = wpre + excl, nxt = wpre + incl;
+      const bool last_nonempty = (i0 < i1) && (i1 == n);
+      if (i0 < i1 && pre <= t && (t < nxt || last_nonempty)) {
+        double R = pre, Rlast = pre, wlast = 0.0;
+        int pick = -1, last = -1;
+        double lo = 0.0, hi = 0.0;
+        for (int i = i0; i < i1; ++i) {
+          const double w = use_q ? (double)fmaxf(__fmul_rn(st[i], iSt) - __fmul_rn(sd[i], iSd), 0.f) : (double)st[i];
+          if (w > 0.0) {
+            last = i;
+            Rlast = R;
+            wlast = w;
+            if (t < R + w) {
+              pick = i;
+              lo = R;
+              hi = R + w;
+              break;
+            }
+          }
+          R += w;
+        }
+        if (pick < 0 && last >= 0) {
+          pick = last;
+          lo = Rlast;
+          hi = Rlast + wlast;
+        }
+        if (pick >= 0) {
+          s_pick = pick;
+          s_lo = lo;
+          s_hi = hi;
+        }
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int pick = s_pick;
+        double lo = s_lo, hi = s_hi;
+        if (pick < 0) {  // rounding left the threshold past every positive weight of the slice
+          for (int i = n - 1; i >= 0; --i) {
+            const double w = use_q ? (double)fmaxf(__fmul_rn(st[i], iSt) - __fmul_rn(sd[i], iSd), 0.f) : (double)st[i];
+            if (w > 0.0) {
+              pick = i;
+              lo = hi = t;
+              break;
+            }
+          }
+        }
+        uint32_t fl = 0;
+        if ((t - lo) < 1e-6 * Wtot || (hi - t) < 1e-6 * Wtot) fl |= DSPARK_FLAG_SAMPLE_NEAR_TIE;
+        if (need_acc && Z < 1e-3) fl |= DSPARK_FLAG_SMALL_RESIDUAL;
+        Slot* s0 = cluster.map_shared_rank(&slot, 0);
+        s0->cand = pick >= 0 ? v_beg + pick : -1;
+        s0->cand_fl = fl;
+      }
+    }
+  }
+  cluster.sync();
+
+  // ------------------------------------------------------------------ row results (rank 0)
+  if (rank == 0 && tid == 0) {
+    uint32_t dfl = 0;
+    for (int r = 0; r < CS; ++r) dfl |= cluster.map_shared_rank(&slot, r)->data_fl;
+    if (timed_out) dfl |= DSPARK_FLAG_DEVICE_TIMEOUT;
+    if (need_cstar) {
+      const double cs = (Z <= 0.5) ? 1.0 - Z : Smin;
+      a.c_star[(size_t)b * a.gamma + kk] = (float)cs;
+    }
+    if (need_acc || need_bonus) {
+      const size_t ri = (size_t)b * (a.gamma + 1) + kk;
+      uint32_t rfl = slot.cand_fl;
+      if (need_acc) {
+        const int xk = a.x[(size_t)b * a.gamma + kk];
+        int acc = 0;
+        if ((unsigned)xk >= (unsigned)a.V || !x_found) {
+          dfl |= DSPARK_FLAG_TOKEN_RANGE;
+        } else {
+          const double pd = (double)ed_x / Sd, pt = (double)et_x / St;
+          const double u = (double)a.u_acc[(size_t)b * a.gamma + kk];
+          acc = (u * pd < pt) ? 1 : 0;
+          if (pd > 0.0 && fabs(u - pt / pd) < 1e-6) rfl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
+        }
+        a.row_acc[ri] = acc;
+      }
+      int cand = slot.cand;
+      if (cand < 0 || cand >= a.V) {
+        dfl |= DSPARK_FLAG_NONFINITE;
+        cand = min(max(cand, 0), a.V - 1);
+      }
+      a.row_cand[ri] = cand;
+      a.row_fl[ri] = rfl;
+    }
+    if (dfl && a.flags) atomicOr(a.flags + b, dfl);
+    if (a.do_verify) row_done(a, b, Lb);
+  }
+}
+
+// ============================================================================ host side
+
+size_t verify_workspace_bytes(int B, int gamma, int V) {
+  (void)V;
+  const size_t rows = (size_t)B * (gamma + 1);
+  return kWsHeader + 3 * align_up(rows * 4, 256) + align_up((size_t)B * 4, 256);
+}
+
+static int pick_cluster(int V, int requested) {
+  if (requested == 1 || requested == 2 || requested == 4 || requested == 8 || requested == 16) return requested;
+  const size_t budget = 80 * 1024;
+  int cs = 1;
+  while (cs < 16) {
+    const size_t vc = align_up((size_t)(V + cs - 1) / cs, 4);
+    if (8 * vc <= budget) break;
+    cs *= 2;
+  }
+  return cs;
+}
+
+dspark_status launch_verify(const VerifyCall& c) {
+  VerifyArgs a{};
+  a.ld = c.ld;
+  a.lt = c.lt;
+  a.x = c.x;
+  a.L = c.L;
+  a.u_acc = c.u_acc;
+  a.u_res = c.u_res;
+  a.B = c.B;
+  a.gamma = c.gamma;
+  a.V = c.V;
+  a.lt_rows = c.lt_rows;
+  a.rows_per_req = c.do_verify ? c.gamma + 1 : c.gamma;
+  a.greedy = (c.T == 0.f) ? 1 : 0;
+  a.inv_T = a.greedy ? 1.f : 1.f / c.T;
+  a.do_verify = c.do_verify;
+  a.c_star = c.c_star;
+  a.n_acc = c.n_acc;
+  a.y_out = c.y_out;
+  a.flags = c.flags;
+  cudaError_t rc;
+  if (c.do_verify) {
+    uint8_t* ws = static_cast<uint8_t*>(c.ws);
+    const size_t rows = (size_t)c.B * (c.gamma + 1);
+    a.status = reinterpret_cast<uint32_t*>(ws);
+    a.row_acc = reinterpret_cast<int32_t*>(ws + kWsHeader);
+    a.row_cand = reinterpret_cast<int32_t*>(ws + kWsHeader + align_up(rows * 4, 256));
+    a.row_fl = reinterpret_cast<uint32_t*>(ws + kWsHeader + 2 * align_up(rows * 4, 256));
+    a.counter = reinterpret_cast<int32_t*>(ws + kWsHeader + 3 * align_up(rows * 4, 256));
+    rc = cudaMemsetAsync(ws, 0, kWsHeader, c.stream);
+    if (rc == cudaSuccess) rc = cudaMemsetAsync(a.counter, 0, (size_t)c.B * 4, c.stream);
+    if (rc != cudaSuccess) {
+      set_error(std::string("cudaMemsetAsync: ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
+    }
+  }
+  const int cs = pick_cluster(c.V, options().verify_cluster);
+  a.Vc = (int)align_up((size_t)(c.V + cs - 1) / cs, 4);
+  a.bulk = (c.V % 4 == 0) && ((uintptr_t)c.lt % 16 == 0) && ((uintptr_t)c.ld % 16 == 0);
+  const int nthr = a.Vc >= 4096 ? 512 : (a.Vc >= 1024 ? 256 : 128);
+  const size_t smem = (size_t)8 * a.Vc;
+  static size_t attr_smem = 0;
+  static bool np_set = false;
+  if (smem > attr_smem) {
+    rc = cudaFuncSetAttribute(verify_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (rc != cudaSuccess) {
+      set_error(std::string("cudaFuncSetAttribute(verify_rows, smem): ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
+    }
+    attr_smem = smem;
+  }
+  if (cs > 8 && !np_set) {
+    rc = cudaFuncSetAttribute(verify_rows, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (rc != cudaSuccess) {
+      set_error(std::string("cudaFuncSetAttribute(verify_rows, cluster 16): ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
+    }
+    np_set = true;
+  }
+  const long long nrows = (long long)c.B * a.rows_per_req;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nrows * cs));
+  cfg.blockDim = dim3(nthr);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  rc = cudaLaunchKernelEx(&cfg, verify_rows, a);
+  if (rc != cudaSuccess) {
+    set_error(std::string("verify launch (cluster ") + std::to_string(cs) + "): " + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
+  }
+  return DSPARK_OK;
+}
+
+}  // namespace dspark

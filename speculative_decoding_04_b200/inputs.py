@@ -208,3 +208,30 @@ def full_inputs(wl: Workload) -> dict:
     u_draft, u_acc, u_res = uniforms(wl)
     return dict(U=U, lt=lt, W1=W1, W2=W2, x0=tokens(wl), u_draft=u_draft, u_acc=u_acc,
                 u_res=u_res, c=confidences(wl), sps=sps_table(wl))
+
+
+def device_logits(wl: Workload, device, requests=None):
+    """(U [n, gamma, V], lt [n, gamma+1, V]) fp32 drawn on `device` with a seeded torch generator.
+
+    Same shapes and value recipe as `logits`, for workloads too large to draw on
+    the host (the vocabulary sweep); the values differ from `logits` but are
+    reproducible for a given workload.  Rows of a request are a function of
+    (seed, request) only, so any subset can be regenerated.
+    """
+    import torch
+
+    reqs = list(range(wl.B)) if requests is None else list(requests)
+    G, V = wl.gamma, wl.V
+    prior = torch.from_numpy(logzipf_prior(wl)).to(device) if wl.logits == "logzipf" else None
+    sig = torch.from_numpy(target_sigmas(wl)).to(device)[:, None]
+    U = torch.empty((len(reqs), G, V), dtype=torch.float32, device=device)
+    lt = torch.empty((len(reqs), G + 1, V), dtype=torch.float32, device=device)
+    g = torch.Generator(device=device)
+    for i, b in enumerate(reqs):
+        g.manual_seed(wl.seed * 1_000_003 + b)
+        u_ext = torch.randn((G + 1, V), generator=g, device=device) * wl.u_sigma
+        if prior is not None:
+            u_ext += prior
+        U[i] = u_ext[:G]
+        lt[i] = u_ext + torch.randn((G + 1, V), generator=g, device=device) * sig
+    return U, lt

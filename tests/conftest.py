@@ -11,3 +11,18 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU case")
+    # the C-ABI library is built in-tree (no-op when it is up to date)
+    from speculative_decoding_04_b200 import build
+    build.build()
+
+
+@pytest.fixture(autouse=True)
+def _default_options():
+    yield
+    import torch
+    if torch.cuda.is_available():
+        from speculative_decoding_04_b200 import dspark as D
+        D.set_option("draft_path", 0)
+        D.set_option("draft_tc_min_b", 9)
+        D.set_option("verify_cluster", 0)
+        D.set_option("draft_pdl", 1)
