@@ -83,6 +83,21 @@ __device__ float block_max(float v, float* sh) {
   return r;
 }
 
+__device__ float2 block_max2(float2 v, float2* sh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  v.x = warp_max(v.x);
+  v.y = warp_max(v.y);
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  float2 r = sh[0];
+  for (int w = 1; w < nw; ++w) {
+    r.x = fmaxf(r.x, sh[w].x);
+    r.y = fmaxf(r.y, sh[w].y);
+  }
+  __syncthreads();
+  return r;
+}
+
 __device__ double2 block_sum2(double a, double b, double2* sh) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   a = warp_sum_d(a);
@@ -163,6 +178,12 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
   __shared__ double2 sh_d[kMaxWarps];
   __shared__ Top2 sh_t[kMaxWarps];
   __shared__ double sh_w[kMaxWarps];
+  __shared__ float2 sh_f2[kMaxWarps];
+  __shared__ double sh_wt[16], sh_wq[16];
+  __shared__ double s_Sd, s_St, s_ft, s_pdx, s_ptx, s_Smin, s_Z;
+  __shared__ float s_cd, s_ct;
+  __shared__ int s_xfound;
+  __shared__ uint32_t s_dfl;
   __shared__ int s_pick;
   __shared__ double s_lo, s_hi;
 
@@ -268,6 +289,7 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
     return;
   }
 
+  // ------------------------------------------------------------------ pass 1: CTA maxima of z = l * (1/T)
   float md = -INFINITY, mt = -INFINITY;
   {
     const float4* sd4 = reinterpret_cast<const float4*>(sd);
@@ -275,11 +297,13 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
     for (int i = tid; i < n4; i += nthr) {
       const float4 t4 = st4[i];
       nonfin |= !(isfinite(t4.x) && isfinite(t4.y) && isfinite(t4.z) && isfinite(t4.w));
-      mt = fmaxf(mt, fmaxf(fmaxf(__fmul_rn(t4.x, inv_T), __fmul_rn(t4.y, inv_T)), fmaxf(__fmul_rn(t4.z, inv_T), __fmul_rn(t4.w, inv_T))));
+      mt = fmaxf(mt, fmaxf(fmaxf(__fmul_rn(t4.x, inv_T), __fmul_rn(t4.y, inv_T)),
+                           fmaxf(__fmul_rn(t4.z, inv_T), __fmul_rn(t4.w, inv_T))));
       if (need_d) {
         const float4 d4 = sd4[i];
         nonfin |= !(isfinite(d4.x) && isfinite(d4.y) && isfinite(d4.z) && isfinite(d4.w));
-        md = fmaxf(md, fmaxf(fmaxf(__fmul_rn(d4.x, inv_T), __fmul_rn(d4.y, inv_T)), fmaxf(__fmul_rn(d4.z, inv_T), __fmul_rn(d4.w, inv_T))));
+        md = fmaxf(md, fmaxf(fmaxf(__fmul_rn(d4.x, inv_T), __fmul_rn(d4.y, inv_T)),
+                             fmaxf(__fmul_rn(d4.z, inv_T), __fmul_rn(d4.w, inv_T))));
       }
     }
     for (int i = 4 * n4 + tid; i < n; i += nthr) {
@@ -291,54 +315,48 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
       }
     }
   }
-  md = block_max(md, sh_f);
-  mt = block_max(mt, sh_f);
   if (nonfin) atomicOr(&slot.data_fl, DSPARK_FLAG_NONFINITE);
-  if (tid == 0) {
-    slot.md = md;
-    slot.mt = mt;
-  }
-  cluster.sync();
-  float Md = -INFINITY, Mt = -INFINITY;
-  for (int r = 0; r < CS; ++r) {
-    const Slot* p = cluster.map_shared_rank(&slot, r);
-    Md = fmaxf(Md, p->md);
-    Mt = fmaxf(Mt, p->mt);
+  {
+    const float2 m2 = block_max2(make_float2(md, mt), sh_f2);
+    md = m2.x;
+    mt = m2.y;
   }
 
-  // ------------------------------------------------------------------ phase B: exponentials, normalisers
+  // ------------------------------------------------------------------ pass 2: e = exp(z - m_cta) in place, CTA sums
   {
     float4* sd4 = reinterpret_cast<float4*>(sd);
     float4* st4 = reinterpret_cast<float4*>(st);
     float ad = 0.f, at = 0.f;
     for (int i = tid; i < n4; i += nthr) {
       float4 t4 = st4[i];
-      t4.x = vex(__fmul_rn(t4.x, inv_T), Mt);
-      t4.y = vex(__fmul_rn(t4.y, inv_T), Mt);
-      t4.z = vex(__fmul_rn(t4.z, inv_T), Mt);
-      t4.w = vex(__fmul_rn(t4.w, inv_T), Mt);
+      t4.x = vex(__fmul_rn(t4.x, inv_T), mt);
+      t4.y = vex(__fmul_rn(t4.y, inv_T), mt);
+      t4.z = vex(__fmul_rn(t4.z, inv_T), mt);
+      t4.w = vex(__fmul_rn(t4.w, inv_T), mt);
       st4[i] = t4;
       at += (t4.x + t4.y) + (t4.z + t4.w);
       if (need_d) {
         float4 d4 = sd4[i];
-        d4.x = vex(__fmul_rn(d4.x, inv_T), Md);
-        d4.y = vex(__fmul_rn(d4.y, inv_T), Md);
-        d4.z = vex(__fmul_rn(d4.z, inv_T), Md);
-        d4.w = vex(__fmul_rn(d4.w, inv_T), Md);
+        d4.x = vex(__fmul_rn(d4.x, inv_T), md);
+        d4.y = vex(__fmul_rn(d4.y, inv_T), md);
+        d4.z = vex(__fmul_rn(d4.z, inv_T), md);
+        d4.w = vex(__fmul_rn(d4.w, inv_T), md);
         sd4[i] = d4;
         ad += (d4.x + d4.y) + (d4.z + d4.w);
       }
     }
     for (int i = 4 * n4 + tid; i < n; i += nthr) {
-      st[i] = vex(__fmul_rn(st[i], inv_T), Mt);
+      st[i] = vex(__fmul_rn(st[i], inv_T), mt);
       at += st[i];
       if (need_d) {
-        sd[i] = vex(__fmul_rn(sd[i], inv_T), Md);
+        sd[i] = vex(__fmul_rn(sd[i], inv_T), md);
         ad += sd[i];
       }
     }
     const double2 s2 = block_sum2((double)ad, (double)at, sh_d);
     if (tid == 0) {
+      slot.md = md;
+      slot.mt = mt;
       slot.sd = s2.x;
       slot.st = s2.y;
       if (need_acc) {
@@ -351,30 +369,52 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
       }
     }
   }
-  cluster.sync();
-  double Sd = 0.0, St = 0.0, Wt[16];
-  float ed_x = 0.f, et_x = 0.f;
-  int x_found = 0;
-  for (int r = 0; r < CS; ++r) {
-    const Slot* p = cluster.map_shared_rank(&slot, r);
-    Sd += p->sd;
-    St += p->st;
-    Wt[r] = p->st;
-    if (p->has_x) {
-      ed_x = p->ed_x;
-      et_x = p->et_x;
-      x_found = 1;
+  cluster.sync();  // (1) every CTA's (max, sum) pair is visible
+
+  // warp 0 combines the CS pairs: lane r reads rank r; totals in rank order via a fixed scan
+  if (warp == 0) {
+    const bool live = lane < CS;
+    const Slot* p = cluster.map_shared_rank(&slot, live ? lane : 0);
+    const float pmd = live ? p->md : -INFINITY, pmt = live ? p->mt : -INFINITY;
+    const double psd = live ? p->sd : 0.0, pst = live ? p->st : 0.0;
+    const uint32_t pfl = live ? p->data_fl : 0u;
+    const int phx = live ? p->has_x : 0;
+    const float pedx = live ? p->ed_x : 0.f, petx = live ? p->et_x : 0.f;
+    const float Md = warp_max(pmd), Mt = warp_max(pmt);
+    const double fd = live ? exp((double)pmd - (double)Md) : 0.0;  // exp(m_r - M): rank weight factor
+    const double ft = live ? exp((double)pmt - (double)Mt) : 0.0;
+    const double wd = live ? psd * fd : 0.0, wt = live ? pst * ft : 0.0;
+    const double Sd = __shfl_sync(0xffffffffu, warp_incl_scan_d(wd), 31);
+    const double St = __shfl_sync(0xffffffffu, warp_incl_scan_d(wt), 31);
+    const uint32_t fl = __reduce_or_sync(0xffffffffu, pfl);
+    const unsigned xm = __ballot_sync(0xffffffffu, phx != 0);
+    const int owner = xm ? __ffs(xm) - 1 : 0;
+    const double pdx = __shfl_sync(0xffffffffu, (double)pedx * fd, owner) / Sd;
+    const double ptx = __shfl_sync(0xffffffffu, (double)petx * ft, owner) / St;
+    const double own_fd = __shfl_sync(0xffffffffu, fd, rank), own_ft = __shfl_sync(0xffffffffu, ft, rank);
+    if (live) sh_wt[lane] = wt;
+    if (lane == 0) {
+      s_Sd = Sd;
+      s_St = St;
+      s_ft = own_ft;
+      s_cd = (float)(own_fd / Sd);
+      s_ct = (float)(own_ft / St);
+      s_pdx = pdx;
+      s_ptx = ptx;
+      s_xfound = xm != 0;
+      s_dfl = fl;
     }
   }
+  __syncthreads();
 
-  // ------------------------------------------------------------------ phase C: TV and residual mass
-  const float iSd = (float)(1.0 / Sd), iSt = (float)(1.0 / St);
-  double Smin = 0.0, Z = 0.0, Wq[16];
+  // ------------------------------------------------------------------ pass 3: TV and residual mass
+  double Smin = 0.0, Z = 0.0;
   const bool phase_c = need_cstar || need_acc;
+  const float cd = s_cd, ct = s_ct;
   if (phase_c) {
     float amin = 0.f, aq = 0.f;
     for (int i = tid; i < n; i += nthr) {
-      const float pd = __fmul_rn(sd[i], iSd), pt = __fmul_rn(st[i], iSt);
+      const float pd = __fmul_rn(sd[i], cd), pt = __fmul_rn(st[i], ct);
       amin += fminf(pd, pt);
       aq += fmaxf(pt - pd, 0.f);
     }
@@ -383,34 +423,44 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
       slot.smin = s2.x;
       slot.sq = s2.y;
     }
-    cluster.sync();
-    for (int r = 0; r < CS; ++r) {
-      const Slot* p = cluster.map_shared_rank(&slot, r);
-      Smin += p->smin;
-      Z += p->sq;
-      Wq[r] = p->sq;
+    cluster.sync();  // (2) every CTA's (sum min, residual mass) is visible
+    if (warp == 0) {
+      const bool live = lane < CS;
+      const Slot* p = cluster.map_shared_rank(&slot, live ? lane : 0);
+      const double pm = live ? p->smin : 0.0, pq = live ? p->sq : 0.0;
+      const double tm = __shfl_sync(0xffffffffu, warp_incl_scan_d(pm), 31);
+      const double tq = __shfl_sync(0xffffffffu, warp_incl_scan_d(pq), 31);
+      if (live) sh_wq[lane] = pq;
+      if (lane == 0) {
+        s_Smin = tm;
+        s_Z = tq;
+      }
     }
+    __syncthreads();
+    Smin = s_Smin;
+    Z = s_Z;
   }
 
-  // ------------------------------------------------------------------ phase D: residual / bonus sample
+  // ------------------------------------------------------------------ pass 4: residual / bonus sample
   if (need_acc || need_bonus) {
     const bool use_q = need_acc && Z > 0.0;
-    const double Wtot = use_q ? Z : St;
+    const double Wtot = use_q ? Z : s_St;
     const double t = (double)a.u_res[b] * Wtot;
     double P = 0.0;
-    for (int r = 0; r < rank; ++r) P += use_q ? Wq[r] : Wt[r];
-    const double Wr = use_q ? Wq[rank] : Wt[rank];
+    for (int r = 0; r < rank; ++r) P += use_q ? sh_wq[r] : sh_wt[r];
+    const double Wr = use_q ? sh_wq[rank] : sh_wt[rank];
     const double Pn = P + Wr;
     int last_nz = -1;
     for (int r = 0; r < CS; ++r)
-      if ((use_q ? Wq[r] : Wt[r]) > 0.0) last_nz = r;
+      if ((use_q ? sh_wq[r] : sh_wt[r]) > 0.0) last_nz = r;
     const bool cross = (Wr > 0.0) && (P <= t) && (t < Pn || rank == last_nz);
     if (cross) {  // uniform over the CTA
+      const double fbonus = s_ft;  // element weights of the bonus row in units of exp(z - M_t)
       const int seg = (n + nthr - 1) / nthr;
       const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
       double tsum = 0.0;
       for (int i = i0; i < i1; ++i)
-        tsum += use_q ? (double)fmaxf(__fmul_rn(st[i], iSt) - __fmul_rn(sd[i], iSd), 0.f) : (double)st[i];
+        tsum += use_q ? (double)fmaxf(__fmul_rn(st[i], ct) - __fmul_rn(sd[i], cd), 0.f) : (double)st[i] * fbonus;
       const double incl = warp_incl_scan_d(tsum);
       double excl = __shfl_up_sync(0xffffffffu, incl, 1);
       if (lane == 0) excl = 0.0;
@@ -426,7 +476,8 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
         int pick = -1, last = -1;
         double lo = 0.0, hi = 0.0;
         for (int i = i0; i < i1; ++i) {
-          const double w = use_q ? (double)fmaxf(__fmul_rn(st[i], iSt) - __fmul_rn(sd[i], iSd), 0.f) : (double)st[i];
+          const double w =
+              use_q ? (double)fmaxf(__fmul_rn(st[i], ct) - __fmul_rn(sd[i], cd), 0.f) : (double)st[i] * fbonus;
           if (w > 0.0) {
             last = i;
             Rlast = R;
@@ -457,7 +508,8 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
         double lo = s_lo, hi = s_hi;
         if (pick < 0) {  // rounding left the threshold past every positive weight of the slice
           for (int i = n - 1; i >= 0; --i) {
-            const double w = use_q ? (double)fmaxf(__fmul_rn(st[i], iSt) - __fmul_rn(sd[i], iSd), 0.f) : (double)st[i];
+            const double w =
+                use_q ? (double)fmaxf(__fmul_rn(st[i], ct) - __fmul_rn(sd[i], cd), 0.f) : (double)st[i] * fbonus;
             if (w > 0.0) {
               pick = i;
               lo = hi = t;
@@ -474,12 +526,12 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
       }
     }
   }
-  cluster.sync();
+  cluster.sync();  // (3) the candidate token is in rank 0's slot
 
   // ------------------------------------------------------------------ row results (rank 0)
+  // no distributed shared memory access past this point: peers may have exited
   if (rank == 0 && tid == 0) {
-    uint32_t dfl = 0;
-    for (int r = 0; r < CS; ++r) dfl |= cluster.map_shared_rank(&slot, r)->data_fl;
+    uint32_t dfl = s_dfl;
     if (timed_out) dfl |= DSPARK_FLAG_DEVICE_TIMEOUT;
     if (need_cstar) {
       const double cs = (Z <= 0.5) ? 1.0 - Z : Smin;
@@ -491,10 +543,10 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
       if (need_acc) {
         const int xk = a.x[(size_t)b * a.gamma + kk];
         int acc = 0;
-        if ((unsigned)xk >= (unsigned)a.V || !x_found) {
+        if ((unsigned)xk >= (unsigned)a.V || !s_xfound) {
           dfl |= DSPARK_FLAG_TOKEN_RANGE;
         } else {
-          const double pd = (double)ed_x / Sd, pt = (double)et_x / St;
+          const double pd = s_pdx, pt = s_ptx;
           const double u = (double)a.u_acc[(size_t)b * a.gamma + kk];
           acc = (u * pd < pt) ? 1 : 0;
           if (pd > 0.0 && fabs(u - pt / pd) < 1e-6) rfl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
@@ -522,10 +574,15 @@ size_t verify_workspace_bytes(int B, int gamma, int V) {
   return kWsHeader + 3 * align_up(rows * 4, 256) + align_up((size_t)B * 4, 256);
 }
 
+// Cluster size: the smallest power of two whose per-CTA slices (ℓ_d and ℓ_t, fp32) fit the
+// budget (80 KB by default, so two CTAs share an SM).  A requested size is raised if its
+// slices would not fit in shared memory at all.
+constexpr size_t kVerifySmemMax = 200 * 1024;
+
 static int pick_cluster(int V, int requested) {
-  if (requested == 1 || requested == 2 || requested == 4 || requested == 8 || requested == 16) return requested;
-  const size_t budget = 80 * 1024;
-  int cs = 1;
+  const bool req = requested == 1 || requested == 2 || requested == 4 || requested == 8 || requested == 16;
+  const size_t budget = req ? kVerifySmemMax : 80 * 1024;
+  int cs = req ? requested : 1;
   while (cs < 16) {
     const size_t vc = align_up((size_t)(V + cs - 1) / cs, 4);
     if (8 * vc <= budget) break;
@@ -572,6 +629,10 @@ dspark_status launch_verify(const VerifyCall& c) {
   }
   const int cs = pick_cluster(c.V, options().verify_cluster);
   a.Vc = (int)align_up((size_t)(c.V + cs - 1) / cs, 4);
+  if ((size_t)8 * a.Vc > kVerifySmemMax) {
+    set_error("dspark_verify: V too large for one 16-CTA cluster per row (V <= 409600)");
+    return DSPARK_ENOTIMPL;
+  }
   a.bulk = (c.V % 4 == 0) && ((uintptr_t)c.lt % 16 == 0) && ((uintptr_t)c.ld % 16 == 0);
   const int nthr = a.Vc >= 4096 ? 512 : (a.Vc >= 1024 ? 256 : 128);
   const size_t smem = (size_t)8 * a.Vc;
