@@ -158,6 +158,27 @@ int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int3
                   void* ws, size_t ws_bytes, void* stream);
 
 /* --------------------------------------------------------------------------
+ * dspark_verify_noalloc -- dspark_verify without a caller workspace.
+ *
+ * The pages have no counterpart to this entry point: it exists for callers that
+ * cannot provide device scratch when they verify -- a serving engine that has
+ * reserved nearly all of HBM for its KV cache and allows no further allocation
+ * while decoding, or plugin code that gets raw device pointers from a host
+ * framework but no access to its allocator.  Arguments, results and flags are
+ * those of dspark_verify; the scratch is a fixed array inside libdspark.so
+ * (213,248 bytes per GPU, held from load until the process exits), so the call
+ * allocates and frees nothing.
+ * Limits: B <= 4096 and B*(gamma+1) <= 16384, else DSPARK_EINVAL with a message.
+ * The first call on a device looks up the array's device address; make that first
+ * call before any stream capture.  All calls share the array and each clears the
+ * parts that must start at zero: calls whose kernels overlap on the GPU race.
+ * -------------------------------------------------------------------------- */
+int dspark_verify_noalloc(const float* ld, const float* lt, const int32_t* x, const int32_t* L,
+                          const float* u_acc, const float* u_res,
+                          int B, int gamma, int V, float T,
+                          int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags, void* stream);
+
+/* --------------------------------------------------------------------------
  * dspark_tv_labels -- confidence-head supervision labels.
  *
  * [P3 §Confidence-Scheduled Verification] c*_k = 1 - ½ ‖p_d,k - p_t,k‖₁;

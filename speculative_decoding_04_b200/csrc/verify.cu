@@ -21,6 +21,8 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <mutex>
+#include <string>
 
 #include "common.cuh"
 #include "internal.h"
@@ -676,3 +678,70 @@ dspark_status launch_verify(const VerifyCall& c) {
 }
 
 }  // namespace dspark
+
+// ============================================================================ verify without allocation
+//
+// Some callers cannot hand this library a workspace at the moment they verify: a serving
+// engine that has reserved almost all of HBM for its KV cache and permits no further
+// cudaMalloc while decoding, or plugin code that receives raw device pointers from a host
+// framework with no access to that framework's allocator.  dspark_verify_noalloc serves them
+// from a fixed array in the library's own device memory instead of a caller workspace.
+//
+// The array below is that scratch.  Every GPU that loads the library holds it until the
+// process exits.  In host code its name is only a host-side stand-in, so its device address
+// is looked up once per device with cudaGetSymbolAddress (the first call on a device does
+// this, which is why that first call should come before any stream capture).  All calls
+// share the array: the per-call counters are cleared by each call, and calls whose kernels
+// overlap on the GPU race on it.
+
+namespace dspark {
+
+constexpr int kNoAllocMaxRows = 16384;  // B * (gamma + 1)
+constexpr int kNoAllocMaxB = 4096;
+constexpr size_t kNoAllocScratchBytes = kWsHeader + 3 * (size_t)kNoAllocMaxRows * 4 + (size_t)kNoAllocMaxB * 4;
+
+static __device__ __align__(256) uint8_t g_verify_scratch[kNoAllocScratchBytes];
+
+static dspark_status verify_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t rc = cudaGetDevice(&dev);
+  if (rc != cudaSuccess || dev < 0 || dev >= 64) {
+    set_error(std::string("dspark_verify_noalloc: cudaGetDevice: ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    rc = cudaGetSymbolAddress(&p, g_verify_scratch);
+    if (rc != cudaSuccess || !p) {
+      set_error(std::string("dspark_verify_noalloc: cudaGetSymbolAddress: ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
+    }
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return DSPARK_OK;
+}
+
+}  // namespace dspark
+
+extern "C" int dspark_verify_noalloc(const float* ld, const float* lt, const int32_t* x, const int32_t* L,
+                                     const float* u_acc, const float* u_res, int B, int gamma, int V, float T,
+                                     int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags, void* stream) {
+  using namespace dspark;
+  if (B > kNoAllocMaxB || (long long)B * (gamma + 1) > kNoAllocMaxRows) {
+    set_error("dspark_verify_noalloc: needs B <= 4096 and B*(gamma+1) <= 16384 (fixed scratch); use dspark_verify");
+    return DSPARK_EINVAL;
+  }
+  if (!ld || !lt || !x || !n_acc || !y_out || !flags) {
+    set_error("dspark_verify_noalloc: null pointer");
+    return DSPARK_EINVAL;
+  }
+  void* ws = nullptr;
+  dspark_status st = verify_scratch(&ws);
+  if (st != DSPARK_OK) return st;
+  return dspark_verify(ld, lt, x, L, u_acc, u_res, B, gamma, V, T, n_acc, y_out, c_star, flags, ws,
+                       kNoAllocScratchBytes, stream);
+}

@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
     lib.dspark_markov_draft.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.dspark_verify.restype = _i
     lib.dspark_verify.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_verify_noalloc.restype = _i
+    lib.dspark_verify_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp]
     lib.dspark_tv_labels.restype = _i
     lib.dspark_tv_labels.argtypes = [_vp, _vp, _i, _i, _i, _i, _f, _vp, _vp]
     lib.dspark_prefix_schedule.restype = _i
@@ -191,6 +193,29 @@ def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torc
     st = lib.dspark_verify(_p(ld), _p(lt), _p(x), _p(L), _p(u_acc), _p(u_res), B, G, V, float(T), _p(n_acc),
                            _p(y_out), _p(c_star), _p(flags), _p(ws), ws.numel(), _s(stream))
     _check("dspark_verify", st)
+    return n_acc, y_out, c_star, flags
+
+
+def verify_noalloc(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torch.Tensor],
+                   u_acc: Optional[torch.Tensor], u_res: Optional[torch.Tensor], T: float, *,
+                   want_c_star: bool = False, n_acc=None, y_out=None, c_star=None, flags=None, stream=None):
+    """verify() for callers that cannot provide device scratch: the library uses a fixed array of
+    its own (B <= 4096, B*(gamma+1) <= 16384).  Outputs are allocated here only when not passed."""
+    B, G, V = ld.shape
+    _need(ld, "ld", torch.float32)
+    _need(lt, "lt", torch.float32, (B, G + 1, V))
+    _need(x, "x", torch.int32, (B, G))
+    if L is not None:
+        _need(L, "L", torch.int32, (B,))
+    dev = ld.device
+    n_acc = torch.empty(B, dtype=torch.int32, device=dev) if n_acc is None else n_acc
+    y_out = torch.empty((B, G + 1), dtype=torch.int32, device=dev) if y_out is None else y_out
+    if c_star is None and want_c_star:
+        c_star = torch.empty((B, G), dtype=torch.float32, device=dev)
+    flags = torch.zeros(B, dtype=torch.int32, device=dev) if flags is None else flags
+    st = lib.dspark_verify_noalloc(_p(ld), _p(lt), _p(x), _p(L), _p(u_acc), _p(u_res), B, G, V, float(T), _p(n_acc),
+                                   _p(y_out), _p(c_star), _p(flags), _s(stream))
+    _check("dspark_verify_noalloc", st)
     return n_acc, y_out, c_star, flags
 
 
