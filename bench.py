@@ -180,7 +180,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dspark", choices=["dspark", "reference"])
     ap.add_argument("--workload", default="high_concurrency", choices=["high_concurrency", "profile"],
-                    help="profile: B=32, gamma=8 (same kernels, ~0.6 GB on the device) for ncu captures")
+                    help="profile: B=64, gamma=4 (same kernels as the headline, ~0.6 GB on the device) for ncu captures")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle timing (after the GPU timing)")
     ap.add_argument("--cpu-requests", type=int, default=4)
     args = ap.parse_args()
@@ -191,7 +191,7 @@ def main():
 
     wl = inputs.HIGH_CONCURRENCY
     if args.workload == "profile":
-        wl = wl.with_(name="profile", B=32, gamma=8)
+        wl = wl.with_(name="profile", B=64, gamma=4)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":

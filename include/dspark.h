@@ -62,7 +62,7 @@ enum { DSPARK_WS_DRAFT = 0, DSPARK_WS_VERIFY = 1, DSPARK_WS_SCHEDULE = 2 };
 #define DSPARK_FLAG_ACCEPT_NEAR_TIE   (1u << 1) /* |u - p_t/p_d| < 1e-6 at a verified position */
 #define DSPARK_FLAG_SAMPLE_NEAR_TIE   (1u << 2) /* |u - F| < 1e-6 at the residual or bonus token */
 #define DSPARK_FLAG_SMALL_RESIDUAL    (1u << 3) /* residual mass < 1e-3 at the first rejection */
-#define DSPARK_FLAG_NONFINITE         (1u << 4) /* NaN or Inf among the logits */
+#define DSPARK_FLAG_NONFINITE         (1u << 4) /* NaN or +Inf among the logits (-Inf is a masked token) */
 #define DSPARK_FLAG_TOKEN_RANGE       (1u << 5) /* a token id outside [0, V) */
 #define DSPARK_FLAG_CONF_RANGE        (1u << 6) /* a confidence outside [0, 1] */
 #define DSPARK_FLAG_SCHED_NEAR_TIE    (1u << 7) /* the chosen D is within 1e-12 (relative) of another */
@@ -78,7 +78,10 @@ const char* dspark_last_error(void);
  *   "draft_tc_min_b"  bf16 drafts with B >= value use the tensor-core main pass (default 9)
  *   "draft_path"      0 automatic, 1 always the CUDA-core GEMV pass, 2 always tensor cores
  *   "draft_pdl"       1 (default) chain draft kernels with programmatic dependent launch
+ *   "draft_w2_hint"   1 (default) W2 tile loads ask L2 to keep W2 (it is re-read every step)
  *   "verify_cluster"  0 automatic, else the cluster size of the verify kernel (1..16, power of 2)
+ *   "verify_persistent" 1 (default) sampled verification and labels run on persistent clusters
+ *                     with double-buffered rows; 2 the same single-buffered; 0 one cluster per row
  *   "sm_count"        0 query the device, else the SM count used to size persistent grids
  * Returns DSPARK_EINVAL for an unknown key. */
 int dspark_set_option(const char* key, long value);

@@ -26,6 +26,7 @@ Options& options() {
     if (const char* e = std::getenv("DSPARK_DRAFT_PATH")) o.draft_force_path = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_DRAFT_PDL")) o.draft_pdl = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_CLUSTER")) o.verify_cluster = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_VERIFY_PERSISTENT")) o.verify_persistent = std::atoi(e);
   });
   return o;
 }
@@ -68,7 +69,9 @@ int dspark_set_option(const char* key, long value) {
   if (!std::strcmp(key, "draft_tc_min_b")) o.draft_tc_min_b = (int)value;
   else if (!std::strcmp(key, "draft_path")) o.draft_force_path = (int)value;
   else if (!std::strcmp(key, "draft_pdl")) o.draft_pdl = (int)value;
+  else if (!std::strcmp(key, "draft_w2_hint")) o.draft_w2_hint = (int)value;
   else if (!std::strcmp(key, "verify_cluster")) o.verify_cluster = (int)value;
+  else if (!std::strcmp(key, "verify_persistent")) o.verify_persistent = (int)value;
   else if (!std::strcmp(key, "sm_count")) o.sm_count = (int)value;
   else return einval(std::string("dspark_set_option: unknown key ") + key);
   return DSPARK_OK;

@@ -37,12 +37,36 @@ struct DraftArgs {
   float* ld;
   const float* u_draft;
   uint32_t* flags;
-  ChunkStat* part;
+  ChunkStat* part;     // [nchunk][B]: per (32-column chunk, request) statistics
+  ChunkStat* cpart;    // [np][B]: per (main-pass partition, request) statistics
   uint32_t* status;
   int B, gamma, V, r, nchunk;
   float inv_T;
   int greedy;
+  int np;              // partitions of the vocabulary: partition p covers tiles
+  int ntiles;          //   [p*ntiles/np, (p+1)*ntiles/np) of tile_chunks chunks each
+  int tile_chunks;
 };
+
+// Fold statistics of a disjoint column range into `acc`: (max, sum of exp) pairs, or greedy top-2.
+__device__ __forceinline__ void stat_fold(ChunkStat& acc, const ChunkStat& o, int greedy) {
+  if (greedy) {
+    const Top2 r = top2_merge(Top2{acc.m, acc.idx, acc.m2}, Top2{o.m, o.idx, o.m2});
+    acc.m = r.best;
+    acc.idx = r.idx;
+    acc.m2 = r.second;
+  } else {
+    const float M = fmaxf(acc.m, o.m);
+    if (M == -INFINITY) {
+      acc.s = 0.f;
+    } else {
+      acc.s = acc.s * exp2f(__fmul_rn(__fsub_rn(acc.m, M), kLog2e)) + o.s * exp2f(__fmul_rn(__fsub_rn(o.m, M), kLog2e));
+    }
+    acc.m = M;
+  }
+}
+
+__device__ __forceinline__ ChunkStat stat_empty() { return ChunkStat{-INFINITY, 0.f, -1, -INFINITY}; }
 
 // exp(z - m) as 2^((z - m) log2 e); z and m are already-rounded fp32 values
 __device__ __forceinline__ float ex_shift(float z, float m) { return exp2f(__fmul_rn(__fsub_rn(z, m), kLog2e)); }
@@ -126,12 +150,14 @@ __device__ __forceinline__ ChunkStat chunk_stat_pair(float l0, float l1, bool va
   return st;
 }
 
-// Grid: x = 256-column tile, y = group of BG requests.  128 threads: the r rank-dimension is
-// split over the 4 warps, each lane owns 8 consecutive columns; the partial sums meet in
-// shared memory, then every thread finishes 2 columns for each request of the group.
+// Grid: x = 256-column tile (one partition of the combine's first level), y = group of BG
+// requests.  128 threads: the rank dimension r is split over the 4 warps, each lane owns 8
+// consecutive columns; the partial sums meet in shared memory, then every thread finishes 2
+// columns for each request of the group.
 template <typename WT, int BG>
 __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int vec_ok) {
   extern __shared__ __align__(16) float fsm[];
+  __shared__ ChunkStat s_stat[8][BG];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int v0 = blockIdx.x * 256;
   const int b0 = blockIdx.y * BG;
@@ -192,7 +218,8 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
   const int c = 2 * tid;
   const int v = v0 + c;
   const bool val0 = v < V, val1 = v + 1 < V;
-  const int chunk = v0 / kChunk + (tid >> 4);
+  const int lchunk = tid >> 4;  // chunk of this CTA, 0..7
+  const int chunk = v0 / kChunk + lchunk;
   for (int bb = 0; bb < nb; ++bb) {
     const int b = b0 + bb;
     float bias0 = 0.f, bias1 = 0.f;
@@ -211,46 +238,61 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
       l1 = a.U[row + v + 1] + bias1;
       a.ld[row + v + 1] = l1;
     }
-    if ((val0 && !isfinite(l0)) || (val1 && !isfinite(l1))) atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
+    if ((val0 && (isnan(l0) || l0 == INFINITY)) || (val1 && (isnan(l1) || l1 == INFINITY)))
+      atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
     const ChunkStat st = chunk_stat_pair(l0, l1, val0, val1, v, a.inv_T, a.greedy);
-    if ((tid & 15) == 0 && chunk < a.nchunk) a.part[(size_t)b * a.nchunk + chunk] = st;
+    if ((tid & 15) == 0) {
+      const bool ok = chunk < a.nchunk;
+      if (ok) a.part[(size_t)chunk * a.B + b] = st;
+      s_stat[lchunk][bb] = ok ? st : stat_empty();
+    }
+  }
+  __syncthreads();
+  if (tid < nb) {  // fold the CTA's 8 chunks into its partition record
+    ChunkStat acc = s_stat[0][tid];
+    for (int q = 1; q < 8; ++q) stat_fold(acc, s_stat[q][tid], a.greedy);
+    a.cpart[(size_t)blockIdx.x * a.B + b0 + tid] = acc;
   }
 }
 
 // ============================================================================ tcgen05 main pass
 //
-// One CTA per SM: a group of up to 128 requests (MMA M = 128, row = request) times a
-// contiguous run of 64-column tiles (MMA N = 64, K = r).  Warp roles:
-//   warp 0      TMA producer: W2 tile [r x 64] bf16 (MN-major, 128B swizzle) and the two
-//               U boxes [rows x 32] fp32 of the tile, 3 / 2 stage rings.
-//   warp 1      MMA issuer: r/16 tcgen05.mma kind::f16 per tile into one of two TMEM
-//               accumulators (64 fp32 columns each).
+// One CTA per SM over a contiguous run of 128-column tiles of the vocabulary (one partition of
+// the combine's first level), for one group of NB requests (NB = 32 or 64; larger batches use
+// several groups).  The MMA computes the bias tile transposed, D[v][b] = sum_k W2[k][v] B[b][k]:
+// M = 128 vocabulary columns on the TMEM lanes and N = NB requests on the TMEM columns, so no
+// MMA row is padding.
+//   warp 0      TMA producer: the W2 tile [r x 128] bf16 as two 64-column boxes (MN-major A
+//               operand, 128-byte swizzle) in a 2-stage ring.
+//   warp 1      MMA issuer: r/16 tcgen05.mma kind::f16 (M = 128, N = NB, K = 16) per tile into
+//               one of two TMEM accumulators of NB fp32 columns.
 //   warp 2      TMEM allocation owner.
-//   warps 4-11  epilogue, two warpgroups (columns 0-31 / 32-63 of each tile): thread = request
-//               row; TMEM -> registers, + U from the swizzled smem box, l_d written back to the
-//               box and stored by TMA, chunk statistics from registers.
-// A (the gathered W1 rows, K-major, 128B swizzle) is built once per step by warps 1-11.
+//   warps 4..   epilogue, NB/8 warps: warp w owns TMEM lane quadrant w%4 (32 vocabulary columns)
+//               for the 32 requests of its column group.  Its [32 requests x 32 columns] block of
+//               U arrives by TMA two tiles ahead into a per-warp double buffer; l = U + bias is
+//               written back in place (lane = column), then each lane reads its own request's
+//               row (rotated 16-byte chunks, free of bank conflicts), streams l_d out with 16-byte
+//               stores and reduces the chunk statistics sequentially.  The statistics are also
+//               folded into one record per (CTA, request) for the combine's first level.
+// The B operand (the gathered W1 rows, K-major, 128-byte swizzle) is built once per step.
 
-constexpr int kTcN = 64;
-constexpr int kTcStagesW = 3;
-constexpr int kTcStagesU = 2;
+constexpr int kTcTile = 128;
 constexpr int kTcThreads = 384;
-constexpr uint32_t kTcTmemCols = 128;
+constexpr int kTcStages = 2;
 
 struct TcLayout {
   uint32_t g, w2, u, bars, misc, total;
-  uint32_t w2_stage_bytes, u_box_bytes;
+  uint32_t w2_stage_bytes;
 };
 
-__host__ __device__ inline TcLayout tc_layout(int r, int box_rows) {
+__host__ __device__ inline TcLayout tc_layout(int r, int nb) {
   TcLayout L;
   L.g = 0;
-  L.w2_stage_bytes = (uint32_t)r * 128u;
-  L.w2 = L.g + (uint32_t)(r / 64) * 16384u;
-  L.u_box_bytes = (uint32_t)box_rows * 128u;
-  L.u = L.w2 + kTcStagesW * L.w2_stage_bytes;
-  L.bars = L.u + kTcStagesU * 2 * L.u_box_bytes;
-  L.misc = L.bars + 8u * (2 * kTcStagesW + 2 * kTcStagesU + 2 + 2 + 1);
+  L.w2_stage_bytes = (uint32_t)r * 256u;  // two 64-column atoms of r rows x 128 B
+  L.w2 = ((uint32_t)nb * (uint32_t)r * 2u + 1023u) & ~1023u;
+  L.u = L.w2 + kTcStages * L.w2_stage_bytes;
+  L.bars = L.u + (uint32_t)(nb / 8) * 2u * 4096u;  // per epilogue warp: 2 x [32 x 32] fp32
+  L.misc = L.bars + 8u * (2 * kTcStages + 2 + 2 + 1 + 2 * (nb / 8));
   L.total = L.misc + 16u;
   return L;
 }
@@ -272,25 +314,25 @@ __device__ __forceinline__ bool tc_wait(const TcSync& s, uint64_t* bar, uint32_t
   return false;
 }
 
+template <int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    draft_main_tc(const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmU,
-                  const __grid_constant__ CUtensorMap tmLD, DraftArgs a, int k, int ntiles, int n_bgroups,
-                  int ctas_per_group, int box_rows) {
+    draft_main_tc(const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmU, DraftArgs a,
+                  int k, int n_bgroups, int ctas_per_group, int w2_hint) {
+  constexpr int EPI_WARPS = NB / 8;  // 4 per 32-request column group
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-  const TcLayout L = tc_layout(a.r, box_rows);
+  const TcLayout L = tc_layout(a.r, NB);
   uint8_t* sG = sm + L.g;
   uint8_t* sW = sm + L.w2;
-  uint8_t* sU = sm + L.u;
+  float* sU = reinterpret_cast<float*>(sm + L.u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* w_full = bars;
-  uint64_t* w_empty = w_full + kTcStagesW;
-  uint64_t* u_full = w_empty + kTcStagesW;
-  uint64_t* u_empty = u_full + kTcStagesU;
-  uint64_t* t_full = u_empty + kTcStagesU;
+  uint64_t* w_empty = w_full + kTcStages;
+  uint64_t* t_full = w_empty + kTcStages;
   uint64_t* t_empty = t_full + 2;
   uint64_t* mma_done = t_empty + 2;
+  uint64_t* u_full = mma_done + 1;  // [EPI_WARPS][2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L.misc + 4);
   const TcSync sy{s_abort, a.status};
@@ -298,34 +340,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % n_bgroups;
   const int jc = blockIdx.x / n_bgroups;
-  const int t_beg = (int)((long long)jc * ntiles / ctas_per_group);
-  const int t_end = (int)((long long)(jc + 1) * ntiles / ctas_per_group);
+  const int t_beg = (int)((long long)jc * a.ntiles / ctas_per_group);
+  const int t_end = (int)((long long)(jc + 1) * a.ntiles / ctas_per_group);
   const int nt = t_end - t_beg;
-  const int b0 = g * 128;
+  const int b0 = g * NB;
   const int ksteps = a.r / 16;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kTcStagesW; ++i) {
+    for (int i = 0; i < kTcStages; ++i) {
       mbar_init(&w_full[i], 1);
       mbar_init(&w_empty[i], 1);
     }
-    for (int i = 0; i < kTcStagesU; ++i) {
-      mbar_init(&u_full[i], 1);
-      mbar_init(&u_empty[i], 2);
-    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&t_full[i], 1);
-      mbar_init(&t_empty[i], 8);
+      mbar_init(&t_empty[i], EPI_WARPS);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 2 * EPI_WARPS; ++i) mbar_init(&u_full[i], 1);
     *s_abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tmW2);
     prefetch_tmap(&tmU);
-    prefetch_tmap(&tmLD);
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, kTcTmemCols);
+    tmem_alloc(tmem_slot, 2 * NB);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -334,47 +372,65 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   pdl_trigger();
 
+  // epilogue geometry (warps 4 .. 4+EPI_WARPS-1)
+  const bool epi = warp >= 4 && warp < 4 + EPI_WARPS;
+  const int q = warp & 3, h = (warp - 4) >> 2, ew = warp - 4;
+  const int bb = b0 + h * 32;
+  float* ubuf = sU + (size_t)ew * 2 * 1024;  // two [32 requests][32 columns] fp32 blocks
+  // U block of tile i into buffer j (lane 0 issues; U is an input of the call, so the first
+  // blocks are requested before waiting for the previous kernel)
+  auto load_u = [&](int i) {
+    const int j = i & 1;
+    mbar_arrive_expect_tx(&u_full[ew * 2 + j], 4096u);
+    tma_load_3d(ubuf + j * 1024, &tmU, (t_beg + i) * kTcTile + q * 32, k, bb, &u_full[ew * 2 + j]);
+  };
+  if (epi && lane == 0) {
+    if (nt > 0) load_u(0);
+    if (nt > 1) load_u(1);
+  }
+
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // W2 and U are inputs of the call, so the ring fills before the previous kernel finishes.
+    // W2 is an input of the call: the ring fills before the previous kernel has finished.
     if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();
       int issued = 0;
       for (int i = 0; i < nt; ++i) {
-        const int v0 = (t_beg + i) * kTcN;
-        const int s = i % kTcStagesW, su = i % kTcStagesU;
-        if (!tc_wait(sy, &w_empty[s], ((i / kTcStagesW) & 1) ^ 1)) break;
+        const int v0 = (t_beg + i) * kTcTile;
+        const int s = i % kTcStages;
+        if (!tc_wait(sy, &w_empty[s], ((i / kTcStages) & 1) ^ 1)) break;
+        uint8_t* st = sW + s * L.w2_stage_bytes;
         mbar_arrive_expect_tx(&w_full[s], L.w2_stage_bytes);
-        tma_load_2d(sW + s * L.w2_stage_bytes, &tmW2, v0, 0, &w_full[s]);
-        if (!tc_wait(sy, &u_empty[su], ((i / kTcStagesU) & 1) ^ 1)) {
-          issued = i + 1;
-          break;
+        if (w2_hint) {
+          tma_load_2d_hint(st, &tmW2, v0, 0, &w_full[s], pol);
+          tma_load_2d_hint(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s], pol);
+        } else {
+          tma_load_2d(st, &tmW2, v0, 0, &w_full[s]);
+          tma_load_2d(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s]);
         }
-        uint8_t* ub = sU + su * 2 * L.u_box_bytes;
-        mbar_arrive_expect_tx(&u_full[su], 2 * L.u_box_bytes);
-        tma_load_3d(ub, &tmU, v0, k, b0, &u_full[su]);
-        tma_load_3d(ub + L.u_box_bytes, &tmU, v0 + 32, k, b0, &u_full[su]);
         issued = i + 1;
       }
       if (*s_abort) {
         // give the copies already issued a bounded chance to land before the CTA exits
-        for (int i = max(0, issued - kTcStagesW); i < issued; ++i)
-          for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(&w_full[i % kTcStagesW], (i / kTcStagesW) & 1); ++t) {
+        for (int i = max(0, issued - kTcStages); i < issued; ++i)
+          for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(&w_full[i % kTcStages], (i / kTcStages) & 1); ++t) {
           }
       }
     }
   } else {
     pdl_wait();
-    // ---------------------------------------------------------------- gather A = W1[x_{k-1}] rows
+    // ---------------------------------------------------------------- gather B = W1[x_{k-1}] rows
     {
       const int cpr = a.r / 8;  // 16-byte chunks per row
       const __nv_bfloat16* W1 = static_cast<const __nv_bfloat16*>(a.W1);
-      for (int i = threadIdx.x - 32; i < 128 * cpr; i += kTcThreads - 32) {
+      for (int i = threadIdx.x - 32; i < NB * cpr; i += kTcThreads - 32) {
         const int row = i / cpr, c = i - row * cpr;
         const int b = b0 + row;
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (b < a.B) val = __ldg(reinterpret_cast<const uint4*>(W1 + (size_t)prev_token(a, b, k, c == 0) * a.r + c * 8));
+        if (b < a.B)
+          val = __ldg(reinterpret_cast<const uint4*>(W1 + (size_t)prev_token(a, b, k, c == 0) * a.r + c * 8));
         const int kb = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(sG + kb * 16384 + row * 128 + ((cc ^ (row & 7)) << 4)) = val;
+        *reinterpret_cast<uint4*>(sG + kb * (NB * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = val;
       }
       fence_proxy_async_smem();
       named_bar(1, kTcThreads - 32);
@@ -382,22 +438,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (warp == 1) {
       // ---------------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        const uint32_t idesc = (1u << 4)                        // D fp32
-                               | (1u << 7) | (1u << 10)         // A, B bf16
-                               | (1u << 16)                     // B MN-major (W2 is [r][V])
-                               | ((uint32_t)(kTcN >> 3) << 17)  // N
+        const uint32_t idesc = (1u << 4)                       // D fp32
+                               | (1u << 7) | (1u << 10)        // A, B bf16
+                               | (1u << 15)                    // A MN-major (W2 is [r][V])
+                               | ((uint32_t)(NB >> 3) << 17)   // N
                                | ((uint32_t)(128 >> 4) << 24);  // M
         const uint32_t g_addr = smem_u32(sG), w_addr = smem_u32(sW);
         for (int i = 0; i < nt; ++i) {
-          const int acc = i & 1, s = i % kTcStagesW;
+          const int acc = i & 1, s = i % kTcStages;
           if (!tc_wait(sy, &t_empty[acc], ((i >> 1) & 1) ^ 1)) break;
-          if (!tc_wait(sy, &w_full[s], (i / kTcStagesW) & 1)) break;
+          if (!tc_wait(sy, &w_full[s], (i / kTcStages) & 1)) break;
           tc_fence_after();
           const uint32_t wst = w_addr + s * L.w2_stage_bytes;
           for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t ad = smem_desc(g_addr + (kk >> 2) * 16384u + (kk & 3) * 32u, 16u, 1024u, 2u);
-            const uint64_t bd = smem_desc(wst + kk * 2048u, L.w2_stage_bytes, 1024u, 2u);
-            tc_mma_f16(tmem_base + acc * kTcN, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            const uint64_t ad = smem_desc(wst + kk * 2048u, L.w2_stage_bytes / 2, 1024u, 2u);
+            const uint64_t bd = smem_desc(g_addr + (kk >> 2) * (NB * 128u) + (kk & 3) * 32u, 16u, 1024u, 2u);
+            tc_mma_f16(tmem_base + acc * NB, ad, bd, idesc, kk > 0 ? 1u : 0u);
           }
           tc_commit(&w_empty[s]);
           tc_commit(&t_full[acc]);
@@ -405,108 +461,102 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_commit(mma_done);
       }
       __syncwarp();
-    } else if (warp >= 4) {
+    } else if (epi) {
       // ---------------------------------------------------------------- epilogue
-      const int ew = warp - 4, h = ew >> 2, q = ew & 3;
-      const int row = q * 32 + lane;
-      const int b = b0 + row;
-      const bool live = (b < a.B) && (row < box_rows);
+      const float inv_T = a.inv_T;
+      const int b = bb + lane;  // this lane's request in the row phase
+      const bool bok = b < a.B;
+      float* ldrow = a.ld + ((size_t)b * a.gamma + k) * a.V;
       bool bad = false;
+      ChunkStat run = stat_empty();
       for (int i = 0; i < nt; ++i) {
-        const int v0 = (t_beg + i) * kTcN;
-        const int acc = i & 1, su = i % kTcStagesU;
-        const int vb = v0 + h * 32;
-        float bias[32];
-        const bool ok_t = tc_wait(sy, &t_full[acc], (i >> 1) & 1);
-        const bool all_t = __all_sync(0xffffffffu, ok_t);
-        if (all_t) {
+        const int j = i & 1;
+        const int acc = i & 1;
+        const int v0w = (t_beg + i) * kTcTile + q * 32;  // this warp's 32 columns
+        const bool ok_u = tc_wait(sy, &u_full[ew * 2 + j], (i >> 1) & 1);
+        const bool ok_t = __all_sync(0xffffffffu, tc_wait(sy, &t_full[acc], (i >> 1) & 1) && ok_u);
+        float x[32];
+        if (ok_t) {
           tc_fence_after();
-          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * kTcN + h * 32, bias);
-          tc_fence_before();
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * NB + h * 32, x);
         }
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&t_empty[acc]);
-        const bool ok_u = tc_wait(sy, &u_full[su], (i / kTcStagesU) & 1);
-        uint8_t* ubox = sU + su * 2 * L.u_box_bytes + h * L.u_box_bytes;
-        if (live && all_t && ok_u) {
-          uint8_t* rp = ubox + row * 128;
-          float l[32];
+        float* ub = ubuf + j * 1024;
+        if (ok_t) {
+          // column phase: lane = column, row jj = request: l = U + bias in place
 #pragma unroll
-          for (int j8 = 0; j8 < 8; ++j8) {
-            float4* p = reinterpret_cast<float4*>(rp + ((j8 ^ (row & 7)) << 4));
-            float4 u4 = *p;
-            u4.x += bias[4 * j8 + 0];
-            u4.y += bias[4 * j8 + 1];
-            u4.z += bias[4 * j8 + 2];
-            u4.w += bias[4 * j8 + 3];
-            *p = u4;
-            l[4 * j8 + 0] = u4.x;
-            l[4 * j8 + 1] = u4.y;
-            l[4 * j8 + 2] = u4.z;
-            l[4 * j8 + 3] = u4.w;
+          for (int jj = 0; jj < 32; ++jj) ub[jj * 32 + lane] += x[jj];
+          __syncwarp();
+          // row phase: lane = request; rotated 16-byte chunks keep the eight lanes of each
+          // shared-memory phase on distinct banks
+          float lv[32];
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const int c = (lane + s4) & 7;
+            const float4 f = *reinterpret_cast<const float4*>(ub + lane * 32 + c * 4);
+            lv[4 * s4 + 0] = f.x;
+            lv[4 * s4 + 1] = f.y;
+            lv[4 * s4 + 2] = f.z;
+            lv[4 * s4 + 3] = f.w;
+            if (bok && v0w + c * 4 < a.V) __stcs(reinterpret_cast<float4*>(ldrow + v0w + c * 4), f);
           }
-          const int nvalid = min(32, a.V - vb);
+          const int nval = min(32, a.V - v0w);  // valid columns of this chunk (multiple of 8)
           ChunkStat st;
           if (a.greedy) {
-            Top2 t;
-            t.best = -INFINITY;
-            t.idx = -1;
-            t.second = -INFINITY;
+            Top2 t{-INFINITY, -1, -INFINITY};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < nvalid) {
-                bad |= !isfinite(l[j]);
-                const float x = l[j];
-                if (t.idx < 0 || x > t.best) {
-                  t.second = fmaxf(t.second, t.best);
-                  t.best = x;
-                  t.idx = vb + j;
-                } else {
-                  t.second = fmaxf(t.second, x);
+            for (int s4 = 0; s4 < 8; ++s4) {
+              const int c = (lane + s4) & 7;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int col = c * 4 + e;
+                const float l = lv[4 * s4 + e];
+                if (col < nval) {
+                  bad |= isnan(l) || l == INFINITY;
+                  const Top2 o{l, v0w + col, -INFINITY};
+                  t = top2_merge(t, o);
                 }
               }
             }
-            st.m = t.best;
-            st.s = 0.f;
-            st.idx = t.idx;
-            st.m2 = t.second;
+            st = ChunkStat{t.best, 0.f, t.idx, t.second};
           } else {
-            float z[32];
-            float m = -INFINITY;
+            float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              z[j] = __fmul_rn(l[j], a.inv_T);
-              if (j < nvalid) {
-                bad |= !isfinite(l[j]);
-                m = fmaxf(m, z[j]);
+            for (int s4 = 0; s4 < 8; ++s4) {
+              const int c = (lane + s4) & 7;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                lv[4 * s4 + e] = (c * 4 + e < nval) ? __fmul_rn(lv[4 * s4 + e], inv_T) : -INFINITY;  // z
+                mx = fmaxf(mx, lv[4 * s4 + e]);
               }
             }
+            float sm = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) z[j] = (j < nvalid) ? ex_shift(z[j], m) : 0.f;
-#pragma unroll
-            for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-              for (int j = 0; j < w; ++j) z[j] += z[j + w];
-            st.m = m;
-            st.s = z[0];
-            st.idx = 0;
-            st.m2 = 0.f;
+            for (int e = 0; e < 32; ++e) sm += (lv[e] == -INFINITY) ? 0.f : ex_shift(lv[e], mx);
+            bad |= isnan(sm) || mx == INFINITY;
+            st = ChunkStat{mx, sm, 0, 0.f};
           }
-          if (vb < a.V) a.part[(size_t)b * a.nchunk + vb / kChunk] = st;
-        }
-        fence_proxy_async_smem();
-        named_bar(2 + h, 128);
-        if (q == 0 && lane == 0) {
-          if (vb < a.V && ok_u && !*s_abort) {
-            tma_store_3d(&tmLD, ubox, vb, k, b0);
-            bulk_commit();
-            bulk_wait_read0();
+          if (v0w < a.V) {
+            if (bok) a.part[(size_t)(v0w >> 5) * a.B + b] = st;
+            stat_fold(run, st, a.greedy);
           }
-          mbar_arrive(&u_empty[su]);
         }
+        __syncwarp();  // every lane is done with this buffer: refill it with the tile after next
+        if (lane == 0 && i + 2 < nt) load_u(i + 2);
       }
-      if (q == 0 && lane == 0) bulk_wait0();
-      if (bad) atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
+      // partition record: fold the four lane quadrants (through shared memory: the G region,
+      // free once every MMA has completed, which the last accumulator wait guarantees)
+      ChunkStat* comb = reinterpret_cast<ChunkStat*>(sG);
+      comb[q * NB + h * 32 + lane] = run;
+      named_bar(2, EPI_WARPS * 32);
+      if (q == 0 && bok) {
+        ChunkStat r = comb[h * 32 + lane];
+        for (int qq = 1; qq < 4; ++qq) stat_fold(r, comb[qq * NB + h * 32 + lane], a.greedy);
+        a.cpart[(size_t)jc * a.B + b] = r;
+      }
+      if (bad && bok) atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
     }
   }
   __syncthreads();
@@ -515,165 +565,150 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(mma_done, 0); ++t) {
     }
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTcTmemCols);
+    tmem_dealloc(tmem_base, 2 * NB);
   }
   if (threadIdx.x == 0 && *s_abort && a.flags)
-    for (int i = 0; i < min(128, a.B - b0); ++i) atomicOr(a.flags + b0 + i, DSPARK_FLAG_DEVICE_TIMEOUT);
+    for (int i = 0; i < min(NB, a.B - b0); ++i) atomicOr(a.flags + b0 + i, DSPARK_FLAG_DEVICE_TIMEOUT);
 }
 
 // ============================================================================ combine + sample
+//
+// One warp per request, three short levels, all weights relative to the row maximum M:
+//   1  the np partition records -> M, S and the partition holding u*S (fp64 warp scan over
+//      contiguous ranges of records, exact partition of [0, S));
+//   2  that partition's chunk records -> the chunk holding u*S;
+//   3  that chunk's 32 stored logits, exp in fp64 -> the token (and the near-tie flag).
+// Greedy: the partition records already carry the argmax (lowest index) and the runner-up.
+constexpr int kCombWarps = 4;
 
-// One CTA per request.  Softmax: load the chunk (max, sum) pairs, global max M, per-thread
-// fp64 sums over contiguous chunk ranges, block scan, the crossing thread walks its chunks to
-// the chunk holding u*S, and one warp rescans that chunk's 32 stored logits in fp64.
-constexpr int kCombThreads = 256;
+// Warp-cooperative search of `t` in the running sum of w[0..n) (lane l owns the contiguous
+// range [l*per, min(n, (l+1)*per)), element weights from `wf`).  Returns the index (or -1),
+// writes its interval [lo, hi) in the running sum started at `base`.
+template <typename WF>
+__device__ __forceinline__ int warp_crossing(int n, double base, double t, WF wf, double& lo, double& hi) {
+  const int lane = threadIdx.x & 31;
+  const int per = (n + 31) / 32;
+  const int i0 = min(n, lane * per), i1 = min(n, i0 + per);
+  double ts = 0.0;
+  for (int i = i0; i < i1; ++i) ts += wf(i);
+  const double incl = warp_incl_scan_d(ts);
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  const double pre = base + excl, nxt = base + incl;
+  const bool last_nonempty = (i0 < i1) && (i1 == n);
+  const bool mine = (i0 < i1) && pre <= t && (t < nxt || last_nonempty);
+  int pick = -1;
+  double plo = 0.0, phi = 0.0;
+  if (mine) {
+    double R = pre, Rlast = pre, wlast = 0.0;
+    int last = -1;
+    for (int i = i0; i < i1; ++i) {
+      const double w = wf(i);
+      if (w > 0.0) {
+        last = i;
+        Rlast = R;
+        wlast = w;
+        if (t < R + w) {
+          pick = i;
+          plo = R;
+          phi = R + w;
+          break;
+        }
+      }
+      R += w;
+    }
+    if (pick < 0 && last >= 0) {
+      pick = last;
+      plo = Rlast;
+      phi = Rlast + wlast;
+    }
+  }
+  const unsigned who = __ballot_sync(0xffffffffu, mine && pick >= 0);
+  if (!who) return -1;
+  const int src = __ffs(who) - 1;
+  lo = __shfl_sync(0xffffffffu, plo, src);
+  hi = __shfl_sync(0xffffffffu, phi, src);
+  return __shfl_sync(0xffffffffu, pick, src);
+}
 
-__global__ void __launch_bounds__(kCombThreads) draft_combine(DraftArgs a, int k) {
-  extern __shared__ __align__(16) float csm[];
-  __shared__ double s_warp[kCombThreads / 32];
-  __shared__ float s_wmax[kCombThreads / 32];
-  __shared__ Top2 s_top[kCombThreads / 32];
-  __shared__ int s_chunk;
-  __shared__ double s_base, s_S, s_t;
-  __shared__ float s_M;
-  const int b = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nchunk = a.nchunk;
-  const ChunkStat* P = a.part + (size_t)b * nchunk;
+__global__ void __launch_bounds__(kCombWarps * 32) draft_combine(DraftArgs a, int k) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x * kCombWarps + warp;
   pdl_trigger();
   pdl_wait();
+  if (b >= a.B) return;
+  const size_t B = (size_t)a.B;
+  const int np = a.np;
 
   if (a.greedy) {
-    Top2 t;
-    t.best = -INFINITY;
-    t.idx = -1;
-    t.second = -INFINITY;
-    for (int c = tid; c < nchunk; c += kCombThreads) {
-      const ChunkStat s = P[c];
-      Top2 u;
-      u.best = s.m;
-      u.idx = s.idx;
-      u.second = s.m2;
-      t = top2_merge(t, u);
+    Top2 t{-INFINITY, -1, -INFINITY};
+    for (int p = lane; p < np; p += 32) {
+      const ChunkStat s = a.cpart[p * B + b];
+      t = top2_merge(t, Top2{s.m, s.idx, s.m2});
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t = top2_merge(t, top2_shfl_xor(t, o));
-    if (lane == 0) s_top[warp] = t;
-    __syncthreads();
-    if (tid == 0) {
-      Top2 r = s_top[0];
-      for (int w = 1; w < kCombThreads / 32; ++w) r = top2_merge(r, s_top[w]);
-      int x = r.idx;
+    if (lane == 0) {
+      int x = t.idx;
       if (x < 0 || x >= a.V) {
         atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
         x = min(max(x, 0), a.V - 1);
       }
-      if (r.best - r.second <= 1e-6f * fmaxf(1.f, fabsf(r.best))) atomicOr(a.flags + b, DSPARK_FLAG_DRAFT_NEAR_TIE);
+      if (t.best - t.second <= 1e-6f * fmaxf(1.f, fabsf(t.best))) atomicOr(a.flags + b, DSPARK_FLAG_DRAFT_NEAR_TIE);
       a.x_out[b * a.gamma + k] = x;
     }
     return;
   }
 
-  float* sm_m = csm;           // [nchunk]
-  float* sm_s = csm + nchunk;  // [nchunk]
+  // level 1: partitions
   float mloc = -INFINITY;
-  for (int c = tid; c < nchunk; c += kCombThreads) {
-    const float2 ms = *reinterpret_cast<const float2*>(P + c);
-    sm_m[c] = ms.x;
-    sm_s[c] = ms.y;
-    mloc = fmaxf(mloc, ms.x);
-  }
-  mloc = warp_max(mloc);
-  if (lane == 0) s_wmax[warp] = mloc;
-  __syncthreads();
-  if (tid == 0) {
-    float M = s_wmax[0];
-    for (int w = 1; w < kCombThreads / 32; ++w) M = fmaxf(M, s_wmax[w]);
-    s_M = M;
-  }
-  __syncthreads();
-  const float M = s_M;
+  for (int p = lane; p < np; p += 32) mloc = fmaxf(mloc, a.cpart[p * B + b].m);
+  const float M = warp_max(mloc);
   const double Md = (double)M;
-
-  // contiguous chunk range of this thread
-  const int per = (nchunk + kCombThreads - 1) / kCombThreads;
-  const int c0 = min(nchunk, tid * per), c1 = min(nchunk, c0 + per);
-  double tsum = 0.0;
-  for (int c = c0; c < c1; ++c) tsum += (double)sm_s[c] * exp((double)sm_m[c] - Md);
-  // block exclusive scan of tsum (fp64); [pre, nxt) of consecutive threads tile [0, S) exactly
-  const double incl = warp_incl_scan_d(tsum);
-  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
-  if (lane == 0) excl = 0.0;
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  double wpre = 0.0;
-  for (int w = 0; w < warp; ++w) wpre += s_warp[w];
+  auto w1 = [&](int p) -> double {
+    const ChunkStat s = a.cpart[p * B + b];
+    return s.m == -INFINITY ? 0.0 : (double)s.s * (double)ex_shift(s.m, M);
+  };
   double S = 0.0;
-  for (int w = 0; w < kCombThreads / 32; ++w) S += s_warp[w];
-  const double pre = wpre + excl;
-  const double nxt = wpre + incl;
-  const double u = (double)a.u_draft[b * a.gamma + k];
-  const double t = u * S;
-  if (tid == 0) {
-    s_chunk = -1;
-    s_S = S;
-    s_t = t;
+  {
+    const int per = (np + 31) / 32;
+    const int i0 = min(np, lane * per), i1 = min(np, i0 + per);
+    double ts = 0.0;
+    for (int i = i0; i < i1; ++i) ts += w1(i);
+    S = __shfl_sync(0xffffffffu, warp_incl_scan_d(ts), 31);
   }
-  __syncthreads();
-  const bool last_nonempty = (c0 < c1) && (c1 == nchunk);
-  if (c0 < c1 && pre <= t && (t < nxt || last_nonempty)) {
-    double R = pre;
-    int cf = -1, clast = -1;
-    double Rlast = pre;
-    for (int c = c0; c < c1; ++c) {
-      const double w = (double)sm_s[c] * exp((double)sm_m[c] - Md);
-      if (w > 0.0) {
-        clast = c;
-        Rlast = R;
-      }
-      if (t < R + w) {
-        cf = c;
-        break;
-      }
-      R += w;
+  const double t = (double)a.u_draft[b * a.gamma + k] * S;
+  double lo1 = 0.0, hi1 = 0.0;
+  const int p = warp_crossing(np, 0.0, t, w1, lo1, hi1);
+  int x = 0;
+  uint32_t fl = 0;
+  if (p < 0 || !(S > 0.0) || !isfinite(S)) {
+    fl |= DSPARK_FLAG_NONFINITE;
+  } else {
+    // level 2: chunks of partition p
+    const int t0 = (int)((long long)p * a.ntiles / np), t1 = (int)((long long)(p + 1) * a.ntiles / np);
+    const int c0 = t0 * a.tile_chunks, c1 = min(a.nchunk, t1 * a.tile_chunks);
+    auto w2 = [&](int i) -> double {
+      const ChunkStat s = a.part[(size_t)(c0 + i) * B + b];
+      return s.m == -INFINITY ? 0.0 : (double)s.s * (double)ex_shift(s.m, M);
+    };
+    double lo2 = 0.0, hi2 = 0.0;
+    int c = warp_crossing(c1 - c0, lo1, t, w2, lo2, hi2);
+    if (c < 0) {  // rounding: fall back to the partition's last chunk with weight
+      c = c1 - c0 - 1;
+      while (c > 0 && w2(c) <= 0.0) --c;
+      lo2 = hi2 = t;
     }
-    if (cf < 0) {
-      cf = clast;
-      R = Rlast;
-    }
-    if (cf >= 0) {
-      s_chunk = cf;
-      s_base = R;
-    }
-  }
-  __syncthreads();
-  if (s_chunk < 0) {
-    // every weight zero or non-finite: no valid distribution
-    if (tid == 0) {
-      int x = 0;
-      for (int c = 0; c < nchunk; ++c)
-        if (sm_m[c] == M) {
-          x = c * kChunk;
-          break;
-        }
-      atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
-      a.x_out[b * a.gamma + k] = min(x, a.V - 1);
-    }
-    return;
-  }
-  if (warp == 0) {
-    const int c = s_chunk;
+    c += c0;
+    // level 3: the chunk's 32 logits
     const int v = c * kChunk + lane;
     const bool valid = v < a.V;
-    double e = 0.0;
-    if (valid) {
-      const float l = a.ld[((size_t)b * a.gamma + k) * a.V + v];
-      const float z = __fmul_rn(l, a.inv_T);
-      e = exp((double)z - Md);
-    }
-    const double base = s_base, Stot = s_S, tt = s_t;
+    const float* row = a.ld + ((size_t)b * a.gamma + k) * a.V;
+    const float z = valid ? __fmul_rn(row[v], a.inv_T) : -INFINITY;
+    const double e = valid ? exp((double)z - Md) : 0.0;
     const double inc = warp_incl_scan_d(e);
-    const double upper = base + inc, lower = upper - e;
-    const unsigned cross = __ballot_sync(0xffffffffu, valid && e > 0.0 && tt < upper);
+    const double upper = lo2 + inc, lower = upper - e;
+    const unsigned cross = __ballot_sync(0xffffffffu, valid && e > 0.0 && t < upper);
     int pick;
     if (cross) {
       pick = __ffs(cross) - 1;
@@ -681,14 +716,13 @@ __global__ void __launch_bounds__(kCombThreads) draft_combine(DraftArgs a, int k
       const unsigned pos = __ballot_sync(0xffffffffu, valid && e > 0.0);
       pick = pos ? 31 - __clz(pos) : 0;
     }
-    const double lo = __shfl_sync(0xffffffffu, lower, pick);
-    const double hi = __shfl_sync(0xffffffffu, upper, pick);
-    if (lane == 0) {
-      const int x = min(c * kChunk + pick, a.V - 1);
-      if ((tt - lo) < 1e-6 * Stot || (hi - tt) < 1e-6 * Stot) atomicOr(a.flags + b, DSPARK_FLAG_DRAFT_NEAR_TIE);
-      if (!(Stot > 0.0) || !isfinite(Stot)) atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
-      a.x_out[b * a.gamma + k] = x;
-    }
+    const double plo = __shfl_sync(0xffffffffu, lower, pick), phi = __shfl_sync(0xffffffffu, upper, pick);
+    x = min(c * kChunk + pick, a.V - 1);
+    if ((t - plo) < 1e-6 * S || (phi - t) < 1e-6 * S) fl |= DSPARK_FLAG_DRAFT_NEAR_TIE;
+  }
+  if (lane == 0) {
+    if (fl) atomicOr(a.flags + b, fl);
+    a.x_out[b * a.gamma + k] = x;
   }
 }
 
@@ -698,7 +732,9 @@ size_t draft_workspace_bytes(int B, int gamma, int V, int r) {
   (void)gamma;
   (void)r;
   const size_t nchunk = (size_t)(V + kChunk - 1) / kChunk;
-  return kWsHeader + align_up((size_t)B * nchunk * sizeof(ChunkStat), 256);
+  const size_t np_max = std::max<size_t>((size_t)(V + 255) / 256, 1024);
+  return kWsHeader + align_up((size_t)B * nchunk * sizeof(ChunkStat), 256) +
+         align_up((size_t)B * np_max * sizeof(ChunkStat), 256);
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -715,12 +751,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, void* base, const uint64_t* dims,
-                     const uint64_t* strides_bytes, const uint32_t* box) {
+                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128 = true) {
   auto fn = encode_fn();
   if (!fn) return false;
   uint32_t es[3] = {1, 1, 1};
   CUresult rc = fn(m, dt, rank, base, dims, strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return rc == CUDA_SUCCESS;
 }
 
@@ -747,7 +784,7 @@ static cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaS
 template <typename WT, int BG>
 static cudaError_t launch_fma(const DraftArgs& a, int k, cudaStream_t st, bool pdl) {
   const int vec_ok = (a.V % (int)(16 / sizeof(WT)) == 0 && (uintptr_t)a.W2 % 16 == 0) ? 1 : 0;
-  const size_t smem = (align_up((size_t)BG * a.r, 4) + (size_t)4 * BG * 256) * sizeof(float);
+  const size_t smem = (size_t)(((BG * a.r + 3) & ~3) + 4 * BG * 256) * sizeof(float);
   auto kern = draft_main_fma<WT, BG>;
   static cudaError_t attr_rc = cudaSuccess;
   static size_t attr_smem = 0;
@@ -768,6 +805,17 @@ static cudaError_t launch_fma_bg(const DraftArgs& a, int k, cudaStream_t st, boo
   return launch_fma<WT, 8>(a, k, st, pdl);
 }
 
+static cudaError_t tc_set_smem(int nb, size_t smem) {
+  static size_t done[2] = {0, 0};
+  const int i = nb == 32 ? 0 : 1;
+  if (smem <= done[i]) return cudaSuccess;
+  const cudaError_t rc =
+      nb == 32 ? cudaFuncSetAttribute(draft_main_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+               : cudaFuncSetAttribute(draft_main_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (rc == cudaSuccess) done[i] = smem;
+  return rc;
+}
+
 dspark_status launch_draft(const DraftCall& c) {
   const Options& opt = options();
   DraftArgs a{};
@@ -780,18 +828,20 @@ dspark_status launch_draft(const DraftCall& c) {
   a.u_draft = c.u_draft;
   a.flags = c.flags;
   a.status = reinterpret_cast<uint32_t*>(c.ws);
-  a.part = reinterpret_cast<ChunkStat*>(static_cast<uint8_t*>(c.ws) + kWsHeader);
   a.B = c.B;
   a.gamma = c.gamma;
   a.V = c.V;
   a.r = c.r;
   a.nchunk = (c.V + kChunk - 1) / kChunk;
+  a.part = reinterpret_cast<ChunkStat*>(static_cast<uint8_t*>(c.ws) + kWsHeader);
+  a.cpart = reinterpret_cast<ChunkStat*>(static_cast<uint8_t*>(c.ws) + kWsHeader +
+                                         align_up((size_t)c.B * a.nchunk * sizeof(ChunkStat), 256));
   a.greedy = (c.T == 0.f) ? 1 : 0;
   a.inv_T = a.greedy ? 1.f : 1.f / c.T;
   const bool pdl = opt.draft_pdl != 0;
 
-  const bool aligned16 = ((uintptr_t)c.U % 16 == 0) && ((uintptr_t)c.W1 % 16 == 0) &&
-                         ((uintptr_t)c.W2 % 16 == 0) && ((uintptr_t)c.ld_out % 16 == 0);
+  const bool aligned16 = ((uintptr_t)c.W1 % 16 == 0) && ((uintptr_t)c.W2 % 16 == 0) && ((uintptr_t)c.U % 16 == 0) &&
+                         ((uintptr_t)c.ld_out % 16 == 0);
   const bool tc_ok = c.w_dtype == DSPARK_BF16 && c.r % 64 == 0 && c.r <= 256 && c.V % 8 == 0 && aligned16;
   bool use_tc = tc_ok && c.B >= opt.draft_tc_min_b;
   if (opt.draft_force_path == 1) use_tc = false;
@@ -809,67 +859,55 @@ dspark_status launch_draft(const DraftCall& c) {
     return DSPARK_ECUDA;
   }
 
-  CUtensorMap mW2, mU, mLD;
-  int n_bgroups = 1, cpg = 1, ntiles = 0, box_rows = 0;
+  CUtensorMap mW2, mU;
+  int n_bgroups = 1, cpg = 1, nb = 0;
   size_t tc_smem = 0;
   if (use_tc) {
-    ntiles = (c.V + kTcN - 1) / kTcN;
-    n_bgroups = (c.B + 127) / 128;
+    nb = c.B <= 32 ? 32 : 64;
+    a.ntiles = (c.V + kTcTile - 1) / kTcTile;
+    a.tile_chunks = kTcTile / kChunk;
+    n_bgroups = (c.B + nb - 1) / nb;
     const int sms = device_sm_count();
     cpg = std::max(1, sms / n_bgroups);
-    cpg = std::min(cpg, ntiles);
-    box_rows = std::min(128, (c.B + 7) / 8 * 8);
-    {
-      uint64_t dims[2] = {(uint64_t)c.V, (uint64_t)c.r};
-      uint64_t strides[1] = {(uint64_t)c.V * 2};
-      uint32_t box[2] = {64, (uint32_t)c.r};
-      if (!make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(c.W2), dims, strides, box)) {
-        set_error("cuTensorMapEncodeTiled failed for W2");
-        return DSPARK_ECUDA;
-      }
+    cpg = std::min(cpg, a.ntiles);
+    a.np = cpg;
+    uint64_t dims[2] = {(uint64_t)c.V, (uint64_t)c.r};
+    uint64_t strides[1] = {(uint64_t)c.V * 2};
+    uint32_t box[2] = {64, (uint32_t)c.r};
+    if (!make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(c.W2), dims, strides, box)) {
+      set_error("cuTensorMapEncodeTiled failed for W2");
+      return DSPARK_ECUDA;
     }
-    {
-      uint64_t dims[3] = {(uint64_t)c.V, (uint64_t)c.gamma, (uint64_t)c.B};
-      uint64_t strides[2] = {(uint64_t)c.V * 4, (uint64_t)c.gamma * c.V * 4};
-      uint32_t box[3] = {32, 1, (uint32_t)box_rows};
-      if (!make_map(&mU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(c.U), dims, strides, box) ||
-          !make_map(&mLD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, c.ld_out, dims, strides, box)) {
-        set_error("cuTensorMapEncodeTiled failed for U / l_d");
-        return DSPARK_ECUDA;
-      }
+    uint64_t udims[3] = {(uint64_t)c.V, (uint64_t)c.gamma, (uint64_t)c.B};
+    uint64_t ustrides[2] = {(uint64_t)c.V * 4, (uint64_t)c.gamma * c.V * 4};
+    uint32_t ubox[3] = {32, 1, 32};
+    if (!make_map(&mU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(c.U), udims, ustrides, ubox, false)) {
+      set_error("cuTensorMapEncodeTiled failed for U");
+      return DSPARK_ECUDA;
     }
-    tc_smem = tc_layout(c.r, box_rows).total + 1024;
-    static size_t attr_smem = 0;
-    if (tc_smem > attr_smem) {
-      rc = cudaFuncSetAttribute(draft_main_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem);
-      if (rc != cudaSuccess) {
-        set_error(std::string("cudaFuncSetAttribute(draft_main_tc): ") + cudaGetErrorString(rc));
-        return DSPARK_ECUDA;
-      }
-      attr_smem = tc_smem;
+    tc_smem = tc_layout(c.r, nb).total + 1024;
+    rc = tc_set_smem(nb, tc_smem);
+    if (rc != cudaSuccess) {
+      set_error(std::string("cudaFuncSetAttribute(draft_main_tc): ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
     }
-  }
-
-  const size_t comb_smem = a.greedy ? 0 : (size_t)2 * a.nchunk * sizeof(float);
-  {
-    static size_t attr_smem = 0;
-    if (comb_smem > 48 * 1024 && comb_smem > attr_smem) {
-      rc = cudaFuncSetAttribute(draft_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)comb_smem);
-      if (rc != cudaSuccess) {
-        set_error(std::string("cudaFuncSetAttribute(draft_combine): ") + cudaGetErrorString(rc));
-        return DSPARK_ECUDA;
-      }
-      attr_smem = comb_smem;
-    }
+  } else {
+    a.ntiles = (c.V + 255) / 256;
+    a.tile_chunks = 256 / kChunk;
+    a.np = a.ntiles;
   }
 
   for (int k = 0; k < c.gamma; ++k) {
-    // The first main pass waits for everything before the call in full: its TMA producer reads
-    // U and W2 without a grid-dependency wait, which is only safe behind this call's own kernels.
+    // The first main pass waits for everything before the call in full: its producers read U
+    // and W2 before the grid-dependency wait, which is only safe behind this call's own kernels.
     const bool pdl_k = pdl && k > 0;
     if (use_tc) {
-      rc = launch_ex(draft_main_tc, dim3(cpg * n_bgroups), dim3(kTcThreads), tc_smem, c.stream, pdl_k, mW2, mU, mLD,
-                     a, k, ntiles, n_bgroups, cpg, box_rows);
+      const dim3 grid(cpg * n_bgroups), block(kTcThreads);
+      const int hint = opt.draft_w2_hint;
+      if (nb == 32)
+        rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, a, k, n_bgroups, cpg, hint);
+      else
+        rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, a, k, n_bgroups, cpg, hint);
     } else if (c.w_dtype == DSPARK_BF16) {
       rc = launch_fma_bg<__nv_bfloat16>(a, k, c.stream, pdl_k);
     } else {
@@ -879,7 +917,8 @@ dspark_status launch_draft(const DraftCall& c) {
       set_error(std::string("draft main pass launch: ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;
     }
-    rc = launch_ex(draft_combine, dim3(c.B), dim3(kCombThreads), comb_smem, c.stream, pdl, a, k);
+    rc = launch_ex(draft_combine, dim3((c.B + kCombWarps - 1) / kCombWarps), dim3(kCombWarps * 32), 0, c.stream, pdl,
+                   a, k);
     if (rc != cudaSuccess) {
       set_error(std::string("draft combine launch: ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;

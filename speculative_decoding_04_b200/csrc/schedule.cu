@@ -61,20 +61,38 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
   const int B = s.B, G = s.gamma, N = B * G, P = s.P, Dm = s.D_max;
 
   // ---------------------------------------------------------------- survival and keys
+  // c is staged in shared memory (the key array's space) with coalesced loads; each request's
+  // running product is then taken in place, left to right, and the keys are built afterwards.
+  float* cs = reinterpret_cast<float*>(keys);  // N floats fit in the first N/2 keys
+  for (int i = tid; i < N; i += kSchedThreads) cs[i] = s.c[i];
+  __syncthreads();
   for (int b = tid; b < B; b += kSchedThreads) {
     float prod = 1.f;
     bool bad = false;
     for (int j = 0; j < G; ++j) {
-      const float cj = s.c[(size_t)b * G + j];
+      const float cj = cs[b * G + j];
       bad |= !(cj >= 0.f && cj <= 1.f);
       prod = (j == 0) ? cj : __fmul_rn(prod, cj);
-      if (s.a_out) s.a_out[(size_t)b * G + j] = prod;
-      keys[b * G + j] = ((uint64_t)desc_key(prod) << 32) | (uint32_t)(b * G + j);
+      cs[b * G + j] = prod;
     }
     if (bad && s.flags) atomicOr(s.flags + b, DSPARK_FLAG_CONF_RANGE);
     cnt[b] = 0;
   }
-  for (int i = N + tid; i < P; i += kSchedThreads) keys[i] = ~0ull;
+  __syncthreads();
+  constexpr int kMaxPer = kMaxScheduleItems / kSchedThreads;
+  float av[kMaxPer];
+#pragma unroll
+  for (int m = 0; m < kMaxPer; ++m) {
+    const int i = tid + m * kSchedThreads;
+    av[m] = i < N ? cs[i] : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < kMaxPer; ++m) {
+    const int i = tid + m * kSchedThreads;
+    if (i < P) keys[i] = i < N ? (((uint64_t)desc_key(av[m]) << 32) | (uint32_t)i) : ~0ull;
+    if (i < N && s.a_out) s.a_out[i] = av[m];
+  }
   __syncthreads();
 
   // ---------------------------------------------------------------- bitonic sort (ascending)

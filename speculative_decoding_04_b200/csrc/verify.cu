@@ -71,6 +71,9 @@ struct __align__(16) Slot {
 
 constexpr int kMaxWarps = 16;
 
+// A logit that breaks the softmax: NaN or +Inf (-Inf is a masked token with probability 0).
+__device__ __forceinline__ bool bad_logit(float x) { return isnan(x) || x == INFINITY; }
+
 // exp(z - m) as 2^((z - m) log2 e); z and m are already-rounded fp32 values
 __device__ __forceinline__ float vex(float z, float m) { return exp2f(__fmul_rn(__fsub_rn(z, m), kLog2e)); }
 
@@ -137,30 +140,25 @@ __device__ __forceinline__ void top2_push(Top2& t, float x, int idx) {
   }
 }
 
-// Assemble n_acc / y for request b once every one of its rows has reported.
-__device__ void finalize_request(const VerifyArgs& a, int b, int Lb) {
+// Assemble n_acc / y for every request from the per-row results (one thread per request),
+// after the row kernel has finished.
+__global__ void verify_finalize(VerifyArgs a) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= a.B) return;
+  const int Lb = a.L ? min(max(a.L[b], 0), a.gamma) : a.gamma;
   const int R = a.gamma + 1;
   const int32_t* acc = a.row_acc + (size_t)b * R;
-  const int32_t* cand = a.row_cand + (size_t)b * R;
   const uint32_t* rfl = a.row_fl + (size_t)b * R;
   int n = 0;
-  while (n < Lb && __ldcg(acc + n)) ++n;
+  while (n < Lb && acc[n]) ++n;
   uint32_t fl = 0;
-  for (int j = 0; j <= n && j < Lb; ++j) fl |= __ldcg(rfl + j) & DSPARK_FLAG_ACCEPT_NEAR_TIE;
-  fl |= __ldcg(rfl + n) & (DSPARK_FLAG_SAMPLE_NEAR_TIE | DSPARK_FLAG_SMALL_RESIDUAL);
+  for (int j = 0; j <= n && j < Lb; ++j) fl |= rfl[j] & DSPARK_FLAG_ACCEPT_NEAR_TIE;
+  fl |= rfl[n] & (DSPARK_FLAG_SAMPLE_NEAR_TIE | DSPARK_FLAG_SMALL_RESIDUAL);
   int32_t* y = a.y_out + (size_t)b * R;
-  for (int j = 0; j < R; ++j) y[j] = (j < n) ? a.x[(size_t)b * a.gamma + j] : (j == n ? __ldcg(cand + n) : -1);
+  const int cand = a.row_cand[(size_t)b * R + n];
+  for (int j = 0; j < R; ++j) y[j] = (j < n) ? a.x[(size_t)b * a.gamma + j] : (j == n ? cand : -1);
   a.n_acc[b] = n;
   if (fl && a.flags) atomicOr(a.flags + b, fl);
-}
-
-__device__ void row_done(const VerifyArgs& a, int b, int Lb) {
-  __threadfence();
-  const int old = atomicAdd(a.counter + b, 1);
-  if (old == a.rows_per_req - 1) {
-    __threadfence();
-    finalize_request(a, b, Lb);
-  }
 }
 
 __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
@@ -197,10 +195,7 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
   const bool need_d = need_cstar || need_acc;
   const bool need_t = need_d || need_bonus;
 
-  if (!need_t) {  // uniform over the cluster: nothing of this row is needed
-    if (a.do_verify && rank == 0 && tid == 0) row_done(a, b, Lb);
-    return;
-  }
+  if (!need_t) return;  // uniform over the cluster: nothing of this row is needed
 
   const int v_beg = rank * a.Vc;
   const int n = max(0, min(a.V, v_beg + a.Vc) - v_beg);
@@ -245,11 +240,11 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
     Top2 gd{-INFINITY, -1, -INFINITY}, gt{-INFINITY, -1, -INFINITY};
     for (int i = tid; i < n; i += nthr) {
       const float lt_ = st[i];
-      nonfin |= !isfinite(lt_);
+      nonfin |= isnan(lt_) || lt_ == INFINITY;
       top2_push(gt, lt_, v_beg + i);
       if (need_d) {
         const float ld_ = sd[i];
-        nonfin |= !isfinite(ld_);
+        nonfin |= isnan(ld_) || ld_ == INFINITY;
         top2_push(gd, ld_, v_beg + i);
       }
     }
@@ -287,7 +282,6 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
       if (dfl && a.flags) atomicOr(a.flags + b, dfl);
     }
     cluster.sync();
-    if (a.do_verify && rank == 0 && tid == 0) row_done(a, b, Lb);
     return;
   }
 
@@ -298,21 +292,21 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
     const float4* st4 = reinterpret_cast<const float4*>(st);
     for (int i = tid; i < n4; i += nthr) {
       const float4 t4 = st4[i];
-      nonfin |= !(isfinite(t4.x) && isfinite(t4.y) && isfinite(t4.z) && isfinite(t4.w));
+      nonfin |= bad_logit(t4.x) || bad_logit(t4.y) || bad_logit(t4.z) || bad_logit(t4.w);
       mt = fmaxf(mt, fmaxf(fmaxf(__fmul_rn(t4.x, inv_T), __fmul_rn(t4.y, inv_T)),
                            fmaxf(__fmul_rn(t4.z, inv_T), __fmul_rn(t4.w, inv_T))));
       if (need_d) {
         const float4 d4 = sd4[i];
-        nonfin |= !(isfinite(d4.x) && isfinite(d4.y) && isfinite(d4.z) && isfinite(d4.w));
+        nonfin |= bad_logit(d4.x) || bad_logit(d4.y) || bad_logit(d4.z) || bad_logit(d4.w);
         md = fmaxf(md, fmaxf(fmaxf(__fmul_rn(d4.x, inv_T), __fmul_rn(d4.y, inv_T)),
                              fmaxf(__fmul_rn(d4.z, inv_T), __fmul_rn(d4.w, inv_T))));
       }
     }
     for (int i = 4 * n4 + tid; i < n; i += nthr) {
-      nonfin |= !isfinite(st[i]);
+      nonfin |= bad_logit(st[i]);
       mt = fmaxf(mt, __fmul_rn(st[i], inv_T));
       if (need_d) {
-        nonfin |= !isfinite(sd[i]);
+        nonfin |= bad_logit(sd[i]);
         md = fmaxf(md, __fmul_rn(sd[i], inv_T));
       }
     }
@@ -564,8 +558,488 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
       a.row_fl[ri] = rfl;
     }
     if (dfl && a.flags) atomicOr(a.flags + b, dfl);
-    if (a.do_verify) row_done(a, b, Lb);
   }
+}
+
+// ============================================================================ persistent verify (T > 0)
+//
+// Each cluster walks the rows cid, cid + ncl, ... with the row slices double-buffered in
+// shared memory: the bulk copies of row i+1 are in flight while row i is computed.  Per row:
+//   pass 1  each thread takes its float4s of l_d and l_t into registers, z = l * (1/T), its own
+//           max m_th and e = exp(z - m_th), sum e  (one pass, no block barrier in between);
+//           a warp / block combine of (max, sum) pairs gives the CTA's pair;
+//   S1      cluster barrier; warp 0 folds the CS pairs into M, S (fp64, rank order);
+//   pass 2  p = e * exp(m_th - M) / S; sum min(p_d, p_t), sum max(0, p_t - p_d); the sample
+//           weights (residual q and target p_t) are written back to the row's buffer;
+//   S2      cluster barrier (only when TV labels or a residual are needed); fold the sums;
+//   pass 3  the CTA holding u_res * W scans its slice in fp64 and writes the token into rank 0's
+//           slot; rank 0 commits the row after the next barrier (S1 of the next row).
+
+struct __align__(16) PSlot {
+  double s_d, s_t;    // CTA sums of exp(z - m_cta)
+  double smin, sq;    // CTA sums of min(p_d, p_t) and max(0, p_t - p_d)
+  float m_d, m_t;     // CTA maxima of z
+  float ex_d, ex_t;   // drafted token: exp(z - m_th) of its owner thread ...
+  float mx_d, mx_t;   // ... and that thread's maxima
+  int has_x;
+  uint32_t data_fl;
+  int cand;           // sampled token, written into rank 0's slot by the CTA holding it
+  uint32_t cand_fl;
+};
+
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (max, sum-of-exp) pair combine; the sums are relative to their own maxima.
+__device__ __forceinline__ void ms_combine(float& m, float& s, float m2, float s2) {
+  const float M = fmaxf(m, m2);
+  if (M == -INFINITY) {
+    s = 0.f;
+  } else {
+    s = s * ex2a((m - M) * kLog2e) + s2 * ex2a((m2 - M) * kLog2e);
+  }
+  m = M;
+}
+
+struct RowNeed {
+  int b, kk, Lb;
+  bool cstar, acc, bonus, d, t;
+};
+
+__device__ __forceinline__ RowNeed row_need(const VerifyArgs& a, long long row) {
+  RowNeed r;
+  r.b = (int)(row / a.rows_per_req);
+  r.kk = (int)(row - (long long)r.b * a.rows_per_req);
+  r.Lb = a.gamma;
+  if (a.do_verify && a.L) r.Lb = min(max(a.L[r.b], 0), a.gamma);
+  r.cstar = (a.c_star != nullptr) && r.kk < a.gamma;
+  r.acc = a.do_verify && r.kk < r.Lb;
+  r.bonus = a.do_verify && r.kk == r.Lb;
+  r.d = r.cstar || r.acc;
+  r.t = r.d || r.bonus;
+  return r;
+}
+
+template <int NI, int NBUF>
+__global__ void __launch_bounds__(512, 1) verify_rows_pc(VerifyArgs a) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CS = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int cid = blockIdx.x / CS, ncl = gridDim.x / CS;
+  const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
+
+  extern __shared__ __align__(16) float psm[];  // [NBUF][2][Vc]: draft then target slice
+  __shared__ PSlot slot[2];
+  __shared__ __align__(8) uint64_t bar[2];
+  __shared__ float4 sh_ms[16];       // per warp: (m_d, s_d, m_t, s_t)
+  __shared__ double2 sh_d2[16];
+  __shared__ double sh_wq[16], sh_wt[16], sh_w[16];
+  __shared__ float s_Md, s_Mt;
+  __shared__ double s_iSd, s_iSt, s_pdx, s_ptx, s_Smin, s_Z, s_WtT;
+  __shared__ int s_xfound, s_pick;
+  __shared__ uint32_t s_dfl;
+  __shared__ double s_lo, s_hi;
+
+  const int v_beg = rank * a.Vc;
+  const int n = max(0, min(a.V, v_beg + a.Vc) - v_beg);
+  const int n4 = n >> 2;  // the bulk path needs V % 4 == 0, so n % 4 == 0
+  const long long nrows = (long long)a.B * a.rows_per_req;
+  const float inv_T = a.inv_T;
+
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+    for (int q = 0; q < 2; ++q) {
+      slot[q].cand = -1;
+      slot[q].cand_fl = 0;
+      slot[q].data_fl = 0;
+      slot[q].has_x = 0;
+    }
+  }
+  __syncthreads();
+
+  uint32_t uses[2] = {0u, 0u}, par[2] = {0u, 0u};
+  bool loaded[2] = {false, false};
+  // issue the slices of `row` into buffer j; identical bookkeeping in every thread
+  auto issue = [&](long long row, int j) {
+    const RowNeed rn = row_need(a, row);
+    loaded[j] = rn.t && n > 0;
+    if (!loaded[j]) return;
+    par[j] = uses[j] & 1u;
+    ++uses[j];
+    if (tid == 0) {
+      float* sd = psm + (size_t)j * 2 * a.Vc;
+      const uint32_t bytes = (uint32_t)n * 4u;
+      const size_t rowd = ((size_t)rn.b * a.gamma + rn.kk) * a.V + v_beg;
+      const size_t rowt = ((size_t)rn.b * a.lt_rows + rn.kk) * a.V + v_beg;
+      mbar_arrive_expect_tx(&bar[j], rn.d ? 2u * bytes : bytes);
+      if (rn.d) bulk_g2s(sd, a.ld + rowd, bytes, &bar[j]);
+      bulk_g2s(sd + a.Vc, a.lt + rowt, bytes, &bar[j]);
+    }
+  };
+
+  // rank 0 commits a row once its sampled token is visible (after the next cluster barrier)
+  bool pend = false;
+  int p_b = 0, p_kk = 0, p_Lb = 0, p_acc = 0, p_j = 0;
+  uint32_t p_fl = 0, p_dfl = 0;
+  bool p_sample = false;
+  auto commit = [&]() {
+    if (!pend) return;
+    pend = false;
+    uint32_t dfl = p_dfl;
+    if (p_sample) {
+      const size_t ri = (size_t)p_b * (a.gamma + 1) + p_kk;
+      int cand = slot[p_j].cand;
+      if (cand < 0 || cand >= a.V) {
+        dfl |= DSPARK_FLAG_NONFINITE;
+        cand = min(max(cand, 0), a.V - 1);
+      }
+      if (p_kk < p_Lb) a.row_acc[ri] = p_acc;
+      a.row_cand[ri] = cand;
+      a.row_fl[ri] = p_fl | slot[p_j].cand_fl;
+      slot[p_j].cand = -1;
+      slot[p_j].cand_fl = 0;
+    }
+    if (dfl && a.flags) atomicOr(a.flags + p_b, dfl);
+  };
+
+  bool timed_out = false;
+  int processed = 0;
+  long long row = cid;
+  if (row < nrows) issue(row, 0);
+  for (int it = 0; row < nrows; row += ncl, ++it) {
+    const int j = NBUF == 2 ? (it & 1) : 0;  // shared-memory buffer of this row
+    const RowNeed rn = row_need(a, row);
+    const long long nxt = row + ncl;
+    if (NBUF == 2 && nxt < nrows) issue(nxt, j ^ 1);  // its last reader passed the barrier that ended row it-1
+    if (!rn.t) {
+      if (NBUF == 1 && nxt < nrows) {
+        __syncthreads();
+        issue(nxt, 0);
+      }
+      continue;
+    }
+    // exchange slot: alternates over the rows this cluster processes (skipped rows have no
+    // cluster barrier, so the slot of the previous processed row is the one reset at S1)
+    const int sj = processed & 1;
+    ++processed;
+    if (loaded[j] && !mbar_wait(&bar[j], par[j])) timed_out = true;
+    float* sd = psm + (size_t)j * 2 * a.Vc;
+    float* st = sd + a.Vc;
+    float4* sd4 = reinterpret_cast<float4*>(sd);
+    float4* st4 = reinterpret_cast<float4*>(st);
+
+    // ---------------------------------------------------------------- pass 1 (registers)
+    float4 ev_d[NI], ev_t[NI];
+    float mthd = -INFINITY, mtht = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int f = tid + i * nthr;
+      float4 t4 = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY), d4 = t4;
+      if (f < n4) {
+        t4 = st4[f];
+        t4 = make_float4(__fmul_rn(t4.x, inv_T), __fmul_rn(t4.y, inv_T), __fmul_rn(t4.z, inv_T), __fmul_rn(t4.w, inv_T));
+        if (rn.d) {
+          d4 = sd4[f];
+          d4 = make_float4(__fmul_rn(d4.x, inv_T), __fmul_rn(d4.y, inv_T), __fmul_rn(d4.z, inv_T), __fmul_rn(d4.w, inv_T));
+        }
+      }
+      ev_t[i] = t4;
+      ev_d[i] = d4;
+      mtht = fmaxf(mtht, fmaxf(fmaxf(t4.x, t4.y), fmaxf(t4.z, t4.w)));
+      mthd = fmaxf(mthd, fmaxf(fmaxf(d4.x, d4.y), fmaxf(d4.z, d4.w)));
+    }
+    float sthd = 0.f, stht = 0.f;
+    {
+      // a thread with no finite maximum (no elements, or all -inf) contributes e = 0
+      const float cd = mthd == -INFINITY ? 0.f : mthd * kLog2e, ct = mtht == -INFINITY ? 0.f : mtht * kLog2e;
+#pragma unroll
+      for (int i = 0; i < NI; ++i) {
+        float4& t4 = ev_t[i];
+        t4.x = ex2a(fmaf(t4.x, kLog2e, -ct));
+        t4.y = ex2a(fmaf(t4.y, kLog2e, -ct));
+        t4.z = ex2a(fmaf(t4.z, kLog2e, -ct));
+        t4.w = ex2a(fmaf(t4.w, kLog2e, -ct));
+        stht += (t4.x + t4.y) + (t4.z + t4.w);
+        float4& d4 = ev_d[i];
+        d4.x = ex2a(fmaf(d4.x, kLog2e, -cd));
+        d4.y = ex2a(fmaf(d4.y, kLog2e, -cd));
+        d4.z = ex2a(fmaf(d4.z, kLog2e, -cd));
+        d4.w = ex2a(fmaf(d4.w, kLog2e, -cd));
+        sthd += (d4.x + d4.y) + (d4.z + d4.w);
+      }
+    }
+    const bool nonfin = (mtht == INFINITY) || (mthd == INFINITY) || isnan(stht) || isnan(sthd);
+    // drafted token: its owner thread reports e and its thread maxima
+    if (rn.acc) {
+      const int xk = a.x[(size_t)rn.b * a.gamma + rn.kk];
+      const int off = xk - v_beg;
+      if (off >= 0 && off < n && ((off >> 2) % nthr) == tid) {
+        const int i = (off >> 2) / nthr, c = off & 3;
+        float exd = 0.f, ext = 0.f;
+#pragma unroll
+        for (int ii = 0; ii < NI; ++ii)
+          if (ii == i) {
+            exd = c == 0 ? ev_d[ii].x : c == 1 ? ev_d[ii].y : c == 2 ? ev_d[ii].z : ev_d[ii].w;
+            ext = c == 0 ? ev_t[ii].x : c == 1 ? ev_t[ii].y : c == 2 ? ev_t[ii].z : ev_t[ii].w;
+          }
+        slot[sj].ex_d = exd;
+        slot[sj].ex_t = ext;
+        slot[sj].mx_d = mthd;
+        slot[sj].mx_t = mtht;
+        slot[sj].has_x = 1;
+      }
+    }
+    // CTA (max, sum) pairs
+    {
+      float md = mthd, sdd = sthd, mt = mtht, stt = stht;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ms_combine(md, sdd, __shfl_xor_sync(0xffffffffu, md, o), __shfl_xor_sync(0xffffffffu, sdd, o));
+        ms_combine(mt, stt, __shfl_xor_sync(0xffffffffu, mt, o), __shfl_xor_sync(0xffffffffu, stt, o));
+      }
+      const unsigned nf = __ballot_sync(0xffffffffu, nonfin);
+      if (lane == 0) sh_ms[warp] = make_float4(md, sdd, mt, stt);
+      if (lane == 0 && nf) atomicOr(&slot[sj].data_fl, DSPARK_FLAG_NONFINITE);
+      __syncthreads();
+      if (warp == 0) {
+        float4 v = lane < nw ? sh_ms[lane] : make_float4(-INFINITY, 0.f, -INFINITY, 0.f);
+        const float Md = warp_max(v.x), Mt = warp_max(v.z);
+        const double wd = (v.x == -INFINITY) ? 0.0 : (double)v.y * (double)ex2a((v.x - Md) * kLog2e);
+        const double wt = (v.z == -INFINITY) ? 0.0 : (double)v.w * (double)ex2a((v.z - Mt) * kLog2e);
+        const double Sd = __shfl_sync(0xffffffffu, warp_incl_scan_d(wd), 31);
+        const double St = __shfl_sync(0xffffffffu, warp_incl_scan_d(wt), 31);
+        if (lane == 0) {
+          slot[sj].m_d = Md;
+          slot[sj].m_t = Mt;
+          slot[sj].s_d = Sd;
+          slot[sj].s_t = St;
+        }
+      }
+    }
+    cluster.sync();  // S1: every CTA's (max, sum) pair, and the previous row's token, are visible
+    if (rank == 0 && tid == 0) commit();
+    if (warp == 0) {
+      const bool live = lane < CS;
+      const PSlot* p = cluster.map_shared_rank(&slot[sj], live ? lane : 0);
+      const float pmd = live ? p->m_d : -INFINITY, pmt = live ? p->m_t : -INFINITY;
+      const double psd = live ? p->s_d : 0.0, pst = live ? p->s_t : 0.0;
+      const uint32_t pfl = live ? p->data_fl : 0u;
+      const int phx = live ? p->has_x : 0;
+      const float pexd = live ? p->ex_d : 0.f, pext = live ? p->ex_t : 0.f;
+      const float pmxd = live ? p->mx_d : -INFINITY, pmxt = live ? p->mx_t : -INFINITY;
+      const float Md = warp_max(pmd), Mt = warp_max(pmt);
+      const double wd = (pmd == -INFINITY) ? 0.0 : psd * exp((double)pmd - (double)Md);
+      const double wt = (pmt == -INFINITY) ? 0.0 : pst * exp((double)pmt - (double)Mt);
+      const double Sd = __shfl_sync(0xffffffffu, warp_incl_scan_d(wd), 31);
+      const double St = __shfl_sync(0xffffffffu, warp_incl_scan_d(wt), 31);
+      const uint32_t fl = __reduce_or_sync(0xffffffffu, pfl);
+      const unsigned xm = __ballot_sync(0xffffffffu, phx != 0);
+      const int owner = xm ? __ffs(xm) - 1 : 0;
+      const double pdx = (double)pexd * exp((double)pmxd - (double)Md) / Sd;
+      const double ptx = (double)pext * exp((double)pmxt - (double)Mt) / St;
+      const double wt_norm = wt / St;  // this rank's target probability mass
+      const double WtT = __shfl_sync(0xffffffffu, warp_incl_scan_d(live ? wt_norm : 0.0), 31);
+      if (live) sh_wt[lane] = wt_norm;
+      if (lane == 0) {
+        s_Md = Md;
+        s_Mt = Mt;
+        s_iSd = 1.0 / Sd;
+        s_iSt = 1.0 / St;
+        s_WtT = WtT;
+        s_dfl = fl;
+        s_xfound = xm != 0;
+      }
+      const double pdx0 = __shfl_sync(0xffffffffu, pdx, owner), ptx0 = __shfl_sync(0xffffffffu, ptx, owner);
+      if (lane == 0) {
+        s_pdx = pdx0;
+        s_ptx = ptx0;
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {  // the other slot was last read before this S1: ready for the next row
+      slot[sj ^ 1].data_fl = 0;
+      slot[sj ^ 1].has_x = 0;
+    }
+
+    // ---------------------------------------------------------------- pass 2: probabilities
+    const bool sample = rn.acc || rn.bonus;
+    const bool phase_c = rn.cstar || rn.acc;
+    const float fd = (rn.d && mthd != -INFINITY) ? (float)((double)ex2a((mthd - s_Md) * kLog2e) * s_iSd) : 0.f;
+    const float ft = (mtht != -INFINITY) ? (float)((double)ex2a((mtht - s_Mt) * kLog2e) * s_iSt) : 0.f;
+    double Smin = 0.0, Z = 0.0;
+    if (phase_c || sample) {
+      float amin = 0.f, aq = 0.f;
+#pragma unroll
+      for (int i = 0; i < NI; ++i) {
+        const int f = tid + i * nthr;
+        if (f < n4) {
+          const float4 d4 = ev_d[i], t4 = ev_t[i];
+          const float4 pd = make_float4(__fmul_rn(d4.x, fd), __fmul_rn(d4.y, fd), __fmul_rn(d4.z, fd), __fmul_rn(d4.w, fd));
+          const float4 pt = make_float4(__fmul_rn(t4.x, ft), __fmul_rn(t4.y, ft), __fmul_rn(t4.z, ft), __fmul_rn(t4.w, ft));
+          const float4 q = make_float4(fmaxf(pt.x - pd.x, 0.f), fmaxf(pt.y - pd.y, 0.f), fmaxf(pt.z - pd.z, 0.f),
+                                       fmaxf(pt.w - pd.w, 0.f));
+          amin += (fminf(pd.x, pt.x) + fminf(pd.y, pt.y)) + (fminf(pd.z, pt.z) + fminf(pd.w, pt.w));
+          aq += (q.x + q.y) + (q.z + q.w);
+          if (sample) {
+            sd4[f] = q;
+            st4[f] = pt;
+          }
+        }
+      }
+      if (phase_c) {
+        double m2 = warp_sum_d((double)amin), q2 = warp_sum_d((double)aq);
+        if (lane == 0) sh_d2[warp] = make_double2(m2, q2);
+        __syncthreads();
+        if (tid == 0) {
+          double tm = 0.0, tq = 0.0;
+          for (int w = 0; w < nw; ++w) {
+            tm += sh_d2[w].x;
+            tq += sh_d2[w].y;
+          }
+          slot[sj].smin = tm;
+          slot[sj].sq = tq;
+        }
+        cluster.sync();  // S2
+        if (warp == 0) {
+          const bool live = lane < CS;
+          const PSlot* p = cluster.map_shared_rank(&slot[sj], live ? lane : 0);
+          const double pm = live ? p->smin : 0.0, pq = live ? p->sq : 0.0;
+          const double tm = __shfl_sync(0xffffffffu, warp_incl_scan_d(pm), 31);
+          const double tq = __shfl_sync(0xffffffffu, warp_incl_scan_d(pq), 31);
+          if (live) sh_wq[lane] = pq;
+          if (lane == 0) {
+            s_Smin = tm;
+            s_Z = tq;
+          }
+        }
+      }
+      __syncthreads();
+      if (phase_c) {
+        Smin = s_Smin;
+        Z = s_Z;
+      }
+    }
+
+    // ---------------------------------------------------------------- pass 3: residual / bonus sample
+    if (sample) {
+      const bool use_q = rn.acc && Z > 0.0;
+      const double* W = use_q ? sh_wq : sh_wt;
+      const float* wbuf = use_q ? sd : st;
+      double Wtot = 0.0;
+      for (int r = 0; r < CS; ++r) Wtot += W[r];
+      const double t = (double)a.u_res[rn.b] * Wtot;
+      double P = 0.0;
+      for (int r = 0; r < rank; ++r) P += W[r];
+      const double Wr = W[rank];
+      const double Pn = P + Wr;
+      int last_nz = -1;
+      for (int r = 0; r < CS; ++r)
+        if (W[r] > 0.0) last_nz = r;
+      const bool cross = (Wr > 0.0) && (P <= t) && (t < Pn || rank == last_nz);
+      if (cross) {  // uniform over the CTA
+        const int seg = (n + nthr - 1) / nthr;
+        const int i0 = min(n, tid * seg), i1 = min(n, i0 + seg);
+        double tsum = 0.0;
+        for (int i = i0; i < i1; ++i) tsum += (double)wbuf[i];
+        const double incl = warp_incl_scan_d(tsum);
+        double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+        if (lane == 0) excl = 0.0;
+        if (lane == 31) sh_w[warp] = incl;
+        if (tid == 0) s_pick = -1;
+        __syncthreads();
+        double wpre = P;
+        for (int w = 0; w < warp; ++w) wpre += sh_w[w];
+        const double pre = wpre + excl, nx = wpre + incl;
+        const bool last_nonempty = (i0 < i1) && (i1 == n);
+        if (i0 < i1 && pre <= t && (t < nx || last_nonempty)) {
+          double R = pre, Rlast = pre, wlast = 0.0, lo = 0.0, hi = 0.0;
+          int pick = -1, last = -1;
+          for (int i = i0; i < i1; ++i) {
+            const double w = (double)wbuf[i];
+            if (w > 0.0) {
+              last = i;
+              Rlast = R;
+              wlast = w;
+              if (t < R + w) {
+                pick = i;
+                lo = R;
+                hi = R + w;
+                break;
+              }
+            }
+            R += w;
+          }
+          if (pick < 0 && last >= 0) {
+            pick = last;
+            lo = Rlast;
+            hi = Rlast + wlast;
+          }
+          if (pick >= 0) {
+            s_pick = pick;
+            s_lo = lo;
+            s_hi = hi;
+          }
+        }
+        __syncthreads();
+        if (tid == 0) {
+          int pick = s_pick;
+          double lo = s_lo, hi = s_hi;
+          if (pick < 0) {  // rounding left the threshold past every positive weight of the slice
+            for (int i = n - 1; i >= 0; --i)
+              if (wbuf[i] > 0.f) {
+                pick = i;
+                lo = hi = t;
+                break;
+              }
+          }
+          uint32_t fl = 0;
+          if ((t - lo) < 1e-6 * Wtot || (hi - t) < 1e-6 * Wtot) fl |= DSPARK_FLAG_SAMPLE_NEAR_TIE;
+          if (rn.acc && Z < 1e-3) fl |= DSPARK_FLAG_SMALL_RESIDUAL;
+          PSlot* s0 = cluster.map_shared_rank(&slot[sj], 0);
+          s0->cand = pick >= 0 ? v_beg + pick : -1;
+          s0->cand_fl = fl;
+        }
+      }
+    }
+
+    // ---------------------------------------------------------------- row results (rank 0)
+    if (rank == 0 && tid == 0) {
+      uint32_t dfl = s_dfl | (timed_out ? DSPARK_FLAG_DEVICE_TIMEOUT : 0u);
+      if (rn.cstar) a.c_star[(size_t)rn.b * a.gamma + rn.kk] = (float)((Z <= 0.5) ? 1.0 - Z : Smin);
+      uint32_t rfl = 0;
+      int acc = 0;
+      if (rn.acc) {
+        const int xk = a.x[(size_t)rn.b * a.gamma + rn.kk];
+        if ((unsigned)xk >= (unsigned)a.V || !s_xfound) {
+          dfl |= DSPARK_FLAG_TOKEN_RANGE;
+        } else {
+          const double u = (double)a.u_acc[(size_t)rn.b * a.gamma + rn.kk];
+          acc = (u * s_pdx < s_ptx) ? 1 : 0;
+          if (s_pdx > 0.0 && fabs(u - s_ptx / s_pdx) < 1e-6) rfl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
+        }
+      }
+      pend = true;
+      p_b = rn.b;
+      p_kk = rn.kk;
+      p_Lb = rn.Lb;
+      p_acc = acc;
+      p_j = sj;
+      p_fl = rfl;
+      p_dfl = dfl;
+      p_sample = sample;
+      if (!sample) commit();  // nothing to wait for
+    }
+    __syncthreads();  // every reader of buffer j is done: it may be refilled
+    if (NBUF == 1 && nxt < nrows) issue(nxt, 0);
+  }
+  cluster.sync();  // the last row's token is visible; no shared-memory access across CTAs after this
+  if (rank == 0 && tid == 0) commit();
+  if (timed_out && a.status) atomicOr(a.status, (uint32_t)DSPARK_ETIMEOUT);
 }
 
 // ============================================================================ host side
@@ -591,6 +1065,82 @@ static int pick_cluster(int V, int requested) {
     cs *= 2;
   }
   return cs;
+}
+
+template <int NI, int NBUF>
+static dspark_status launch_pc(const VerifyArgs& a, int cs, cudaStream_t stream) {
+  auto kern = verify_rows_pc<NI, NBUF>;
+  const size_t smem = (size_t)NBUF * 8 * a.Vc;
+  static size_t attr_smem = 0;
+  static bool np_set = false;
+  cudaError_t rc = cudaSuccess;
+  if (smem > attr_smem) {
+    rc = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (rc != cudaSuccess) {
+      set_error(std::string("cudaFuncSetAttribute(verify_rows_pc, smem): ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
+    }
+    attr_smem = smem;
+  }
+  if (cs > 8 && !np_set) {
+    rc = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (rc != cudaSuccess) {
+      set_error(std::string("cudaFuncSetAttribute(verify_rows_pc, cluster 16): ") + cudaGetErrorString(rc));
+      return DSPARK_ECUDA;
+    }
+    np_set = true;
+  }
+  const long long nrows = (long long)a.B * a.rows_per_req;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(512);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)cs);
+  int ncl = 0;
+  rc = cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg);
+  if (rc != cudaSuccess || ncl <= 0) {
+    (void)cudaGetLastError();
+    return DSPARK_ENOTIMPL;
+  }
+  ncl = (int)std::min<long long>(ncl, nrows);
+  cfg.gridDim = dim3((unsigned)(ncl * cs));
+  rc = cudaLaunchKernelEx(&cfg, kern, a);
+  if (rc != cudaSuccess) {
+    set_error(std::string("verify launch (persistent, cluster ") + std::to_string(cs) + "): " + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
+  }
+  return DSPARK_OK;
+}
+
+static dspark_status launch_finalize(const VerifyArgs& a, cudaStream_t stream) {
+  if (!a.do_verify) return DSPARK_OK;
+  verify_finalize<<<(a.B + 127) / 128, 128, 0, stream>>>(a);
+  const cudaError_t rc = cudaGetLastError();
+  if (rc != cudaSuccess) {
+    set_error(std::string("verify finalize launch: ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
+  }
+  return DSPARK_OK;
+}
+
+// double_buffer: rows double-buffered in shared memory (else single-buffered; also used when two
+// buffers do not fit).  One CTA of 512 threads per SM either way.
+static dspark_status launch_verify_persistent(const VerifyArgs& a, int cs, cudaStream_t stream, bool double_buffer) {
+  const int per_thread = (a.Vc / 4 + 511) / 512;  // float4s per thread
+  const bool two = double_buffer && (size_t)16 * a.Vc <= kVerifySmemMax;
+  if (per_thread <= 1) return two ? launch_pc<1, 2>(a, cs, stream) : launch_pc<1, 1>(a, cs, stream);
+  if (per_thread <= 2) return two ? launch_pc<2, 2>(a, cs, stream) : launch_pc<2, 1>(a, cs, stream);
+  if (per_thread <= 4) return two ? launch_pc<4, 2>(a, cs, stream) : launch_pc<4, 1>(a, cs, stream);
+  if (per_thread <= 6) return two ? launch_pc<6, 2>(a, cs, stream) : launch_pc<6, 1>(a, cs, stream);
+  if (per_thread <= 8) return two ? launch_pc<8, 2>(a, cs, stream) : launch_pc<8, 1>(a, cs, stream);
+  return DSPARK_ENOTIMPL;
 }
 
 dspark_status launch_verify(const VerifyCall& c) {
@@ -623,7 +1173,6 @@ dspark_status launch_verify(const VerifyCall& c) {
     a.row_fl = reinterpret_cast<uint32_t*>(ws + kWsHeader + 2 * align_up(rows * 4, 256));
     a.counter = reinterpret_cast<int32_t*>(ws + kWsHeader + 3 * align_up(rows * 4, 256));
     rc = cudaMemsetAsync(ws, 0, kWsHeader, c.stream);
-    if (rc == cudaSuccess) rc = cudaMemsetAsync(a.counter, 0, (size_t)c.B * 4, c.stream);
     if (rc != cudaSuccess) {
       set_error(std::string("cudaMemsetAsync: ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;
@@ -636,6 +1185,11 @@ dspark_status launch_verify(const VerifyCall& c) {
     return DSPARK_ENOTIMPL;
   }
   a.bulk = (c.V % 4 == 0) && ((uintptr_t)c.lt % 16 == 0) && ((uintptr_t)c.ld % 16 == 0);
+  if (!a.greedy && a.bulk && options().verify_persistent) {
+    dspark_status st = launch_verify_persistent(a, cs, c.stream, options().verify_persistent != 2);
+    if (st == DSPARK_OK) st = launch_finalize(a, c.stream);
+    if (st != DSPARK_ENOTIMPL) return st;  // else: no resident cluster fits; use the one-row-per-cluster kernel
+  }
   const int nthr = a.Vc >= 4096 ? 512 : (a.Vc >= 1024 ? 256 : 128);
   const size_t smem = (size_t)8 * a.Vc;
   static size_t attr_smem = 0;
@@ -674,7 +1228,7 @@ dspark_status launch_verify(const VerifyCall& c) {
     set_error(std::string("verify launch (cluster ") + std::to_string(cs) + "): " + cudaGetErrorString(rc));
     return DSPARK_ECUDA;
   }
-  return DSPARK_OK;
+  return launch_finalize(a, c.stream);
 }
 
 }  // namespace dspark

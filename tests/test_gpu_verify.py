@@ -33,16 +33,19 @@ def run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=True):
 @pytest.mark.parametrize("T", [1.0, 0.7, 0.0])
 @pytest.mark.parametrize("scheduled", [False, True])
 @pytest.mark.parametrize("cluster", [0, 1, 4, 16])
-def test_verify_matches_oracle(V, T, scheduled, cluster):
+@pytest.mark.parametrize("labels", [True, False])
+def test_verify_matches_oracle(V, T, scheduled, cluster, labels):
     if cluster and V < 4096 and cluster > 4:
         pytest.skip("slice smaller than the block")
     D.set_option("verify_cluster", cluster)
     B, G = 6, 4
     ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=V + int(T * 10) + cluster)
+    # without labels, rows past L_b + 1 are skipped by the kernels
     L = np.array([0, 1, 2, 3, 4, 2], dtype=np.int32) if scheduled else None
-    n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, T)
+    n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=labels)
     check_verify(ld, lt, x, L, u_acc, u_res, T, n, y)
-    check_labels(ld, lt, T, c)
+    if labels:
+        check_labels(ld, lt, T, c)
     G_ = G if L is None else L
     assert np.all(n <= G_)
 
@@ -111,3 +114,14 @@ def test_acceptance_rate_matches_label_statistically():
     c1 = O.tv_labels(ld[:1], lt[:1, :1], 1.0)[0, 0]
     rate = n.mean()
     assert abs(rate - c1) < 4 * np.sqrt(c1 * (1 - c1) / B)
+
+
+@pytest.mark.parametrize("persistent", [1, 0])
+def test_scheduled_rows_skipped_many_requests(persistent):
+    D.set_option("verify_persistent", persistent)
+    B, G, V = 40, 6, 20000
+    ld, lt, x, u_acc, u_res = case(B, G, V, 1.0, seed=77)
+    L = (np.arange(B) * 7 % (G + 1)).astype(np.int32)
+    n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, 1.0, want_c=False)
+    check_verify(ld, lt, x, L, u_acc, u_res, 1.0, n, y)
+    assert np.all(n <= L)
