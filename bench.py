@@ -213,6 +213,7 @@ def main():
 
     # ---------------------------------------------------------------- inputs (each rank its own batch)
     d = inputs.full_inputs(rank_workload(wl, rank))
+    d["U"] = d["U"].transpose(1, 0, 2)      # the draft's base logits are position-major [gamma, B, V]
     pin = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
            for k, v in d.items() if k in ("U", "lt", "x0", "u_draft", "u_acc", "u_res", "c")}
     W1 = torch.from_numpy(d["W1"]).to(torch.bfloat16).to(dev)
@@ -221,7 +222,7 @@ def main():
     B, G, V, r = wl.B, wl.gamma, wl.V, wl.r
     sps = torch.ones(B * G + 1, dtype=torch.float64, device=dev)       # flat: every drafted token is worth verifying
     x = torch.empty((B, G), dtype=torch.int32, device=dev)
-    ld = torch.empty((B, G, V), dtype=torch.float32, device=dev)
+    ld = torch.empty((G, B, V), dtype=torch.float32, device=dev)
     fl = torch.zeros(B, dtype=torch.int32, device=dev)
     L = torch.empty(B, dtype=torch.int32, device=dev)
     theta = torch.empty(1, dtype=torch.float64, device=dev)

@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
       bias0 += red[(w * BG + bb) * 256 + c];
       bias1 += red[(w * BG + bb) * 256 + c + 1];
     }
-    const size_t row = ((size_t)b * a.gamma + k) * V;
+    const size_t row = ((size_t)k * a.B + b) * V;  // position-major [gamma][B][V]
     float l0 = 0.f, l1 = 0.f;
     if (val0) {
       l0 = a.U[row + v] + bias0;
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto load_u = [&](int i) {
     const int j = i & 1;
     mbar_arrive_expect_tx(&u_full[ew * 2 + j], 4096u);
-    tma_load_3d(ubuf + j * 1024, &tmU, (t_beg + i) * kTcTile + q * 32, k, bb, &u_full[ew * 2 + j]);
+    tma_load_3d(ubuf + j * 1024, &tmU, (t_beg + i) * kTcTile + q * 32, bb, k, &u_full[ew * 2 + j]);
   };
   if (epi && lane == 0) {
     if (nt > 0) load_u(0);
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float inv_T = a.inv_T;
       const int b = bb + lane;  // this lane's request in the row phase
       const bool bok = b < a.B;
-      float* ldrow = a.ld + ((size_t)b * a.gamma + k) * a.V;
+      float* ldrow = a.ld + ((size_t)k * a.B + b) * a.V;
       bool bad = false;
       ChunkStat run = stat_empty();
       for (int i = 0; i < nt; ++i) {
@@ -703,7 +703,7 @@ __global__ void __launch_bounds__(kCombWarps * 32) draft_combine(DraftArgs a, in
     // level 3: the chunk's 32 logits
     const int v = c * kChunk + lane;
     const bool valid = v < a.V;
-    const float* row = a.ld + ((size_t)b * a.gamma + k) * a.V;
+    const float* row = a.ld + ((size_t)k * a.B + b) * a.V;
     const float z = valid ? __fmul_rn(row[v], a.inv_T) : -INFINITY;
     const double e = valid ? exp((double)z - Md) : 0.0;
     const double inc = warp_incl_scan_d(e);
@@ -878,9 +878,10 @@ dspark_status launch_draft(const DraftCall& c) {
       set_error("cuTensorMapEncodeTiled failed for W2");
       return DSPARK_ECUDA;
     }
-    uint64_t udims[3] = {(uint64_t)c.V, (uint64_t)c.gamma, (uint64_t)c.B};
-    uint64_t ustrides[2] = {(uint64_t)c.V * 4, (uint64_t)c.gamma * c.V * 4};
-    uint32_t ubox[3] = {32, 1, 32};
+    // U is position-major [gamma][B][V]: a box is 32 columns of 32 requests at one position
+    uint64_t udims[3] = {(uint64_t)c.V, (uint64_t)c.B, (uint64_t)c.gamma};
+    uint64_t ustrides[2] = {(uint64_t)c.V * 4, (uint64_t)c.B * c.V * 4};
+    uint32_t ubox[3] = {32, 32, 1};
     if (!make_map(&mU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(c.U), udims, ustrides, ubox, false)) {
       set_error("cuTensorMapEncodeTiled failed for U");
       return DSPARK_ECUDA;

@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
 
   const int v_beg = rank * a.Vc;
   const int n = max(0, min(a.V, v_beg + a.Vc) - v_beg);
-  const size_t rowd = ((size_t)b * a.gamma + kk) * a.V + v_beg;
+  const size_t rowd = ((size_t)kk * a.B + b) * a.V + v_beg;  // l_d is [gamma][B][V]
   const size_t rowt = ((size_t)b * a.lt_rows + kk) * a.V + v_beg;
   bool timed_out = false;
 
@@ -674,7 +674,7 @@ __global__ void __launch_bounds__(512, 1) verify_rows_pc(VerifyArgs a) {
     if (tid == 0) {
       float* sd = psm + (size_t)j * 2 * a.Vc;
       const uint32_t bytes = (uint32_t)n * 4u;
-      const size_t rowd = ((size_t)rn.b * a.gamma + rn.kk) * a.V + v_beg;
+      const size_t rowd = ((size_t)rn.kk * a.B + rn.b) * a.V + v_beg;
       const size_t rowt = ((size_t)rn.b * a.lt_rows + rn.kk) * a.V + v_beg;
       mbar_arrive_expect_tx(&bar[j], rn.d ? 2u * bytes : bytes);
       if (rn.d) bulk_g2s(sd, a.ld + rowd, bytes, &bar[j]);

@@ -138,8 +138,10 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
 def markov_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, x0: torch.Tensor,
                  u_draft: Optional[torch.Tensor], T: float, *, x_out=None, ld_out=None, flags=None, ws=None,
                  stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Markov-head draft of gamma tokens per request; returns (x [B, gamma], l_d [B, gamma, V], flags [B])."""
-    B, G, V = U.shape
+    """Markov-head draft of gamma tokens per request.
+
+    U is position-major [gamma, B, V]; returns (x [B, gamma], l_d [gamma, B, V], flags [B])."""
+    G, B, V = U.shape
     r = W1.shape[1]
     _need(U, "U", torch.float32)
     if W1.dtype not in (torch.bfloat16, torch.float32) or W2.dtype != W1.dtype:
@@ -151,11 +153,11 @@ def markov_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, x0: torch.
         _need(u_draft, "u_draft", torch.float32, (B, G))
     dev = U.device
     x_out = torch.empty((B, G), dtype=torch.int32, device=dev) if x_out is None else x_out
-    ld_out = torch.empty((B, G, V), dtype=torch.float32, device=dev) if ld_out is None else ld_out
+    ld_out = torch.empty((G, B, V), dtype=torch.float32, device=dev) if ld_out is None else ld_out
     flags = torch.zeros(B, dtype=torch.int32, device=dev) if flags is None else flags
     ws = workspace(WS_DRAFT, B, G, V, r, dev) if ws is None else ws
     _need(x_out, "x_out", torch.int32, (B, G))
-    _need(ld_out, "ld_out", torch.float32, (B, G, V))
+    _need(ld_out, "ld_out", torch.float32, (G, B, V))
     _need(flags, "flags", torch.int32, (B,))
     st = lib.dspark_markov_draft(_p(U), _p(W1), _p(W2), BF16 if W1.dtype == torch.bfloat16 else F32, _p(x0),
                                  _p(u_draft), B, G, V, r, float(T), _p(x_out), _p(ld_out), _p(flags), _p(ws),
@@ -167,8 +169,9 @@ def markov_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, x0: torch.
 def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torch.Tensor],
            u_acc: Optional[torch.Tensor], u_res: Optional[torch.Tensor], T: float, *, want_c_star: bool = False,
            n_acc=None, y_out=None, c_star=None, flags=None, ws=None, stream=None):
-    """Rejection-sampling verification; returns (n_acc [B], y [B, gamma+1], c_star [B, gamma] or None, flags [B])."""
-    B, G, V = ld.shape
+    """Rejection-sampling verification of l_d [gamma, B, V] (position-major) against l_t [B, gamma+1, V];
+    returns (n_acc [B], y [B, gamma+1], c_star [B, gamma] or None, flags [B])."""
+    G, B, V = ld.shape
     _need(ld, "ld", torch.float32)
     _need(lt, "lt", torch.float32, (B, G + 1, V))
     _need(x, "x", torch.int32, (B, G))
@@ -201,7 +204,7 @@ def verify_noalloc(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optio
                    want_c_star: bool = False, n_acc=None, y_out=None, c_star=None, flags=None, stream=None):
     """verify() for callers that cannot provide device scratch: the library uses a fixed array of
     its own (B <= 4096, B*(gamma+1) <= 16384).  Outputs are allocated here only when not passed."""
-    B, G, V = ld.shape
+    G, B, V = ld.shape
     _need(ld, "ld", torch.float32)
     _need(lt, "lt", torch.float32, (B, G + 1, V))
     _need(x, "x", torch.int32, (B, G))
@@ -220,8 +223,9 @@ def verify_noalloc(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optio
 
 
 def tv_labels(ld: torch.Tensor, lt: torch.Tensor, T: float, *, c_star=None, stream=None) -> torch.Tensor:
-    """c*_k = 1 - ½‖p_d,k - p_t,k‖₁ for every drafted position; lt has gamma or gamma+1 rows."""
-    B, G, V = ld.shape
+    """c*_k = 1 - ½‖p_d,k - p_t,k‖₁ for every drafted position; l_d is [gamma, B, V] and l_t
+    [B, gamma or gamma+1, V]."""
+    G, B, V = ld.shape
     _need(ld, "ld", torch.float32)
     _need(lt, "lt", torch.float32)
     if lt.dim() != 3 or lt.shape[0] != B or lt.shape[2] != V or lt.shape[1] not in (G, G + 1):

@@ -211,7 +211,8 @@ def full_inputs(wl: Workload) -> dict:
 
 
 def device_logits(wl: Workload, device, requests=None):
-    """(U [n, gamma, V], lt [n, gamma+1, V]) fp32 drawn on `device` with a seeded torch generator.
+    """(U [gamma, n, V] position-major, lt [n, gamma+1, V]) fp32 drawn on `device` with a seeded
+    torch generator.
 
     Same shapes and value recipe as `logits`, for workloads too large to draw on
     the host (the vocabulary sweep); the values differ from `logits` but are
@@ -224,7 +225,7 @@ def device_logits(wl: Workload, device, requests=None):
     G, V = wl.gamma, wl.V
     prior = torch.from_numpy(logzipf_prior(wl)).to(device) if wl.logits == "logzipf" else None
     sig = torch.from_numpy(target_sigmas(wl)).to(device)[:, None]
-    U = torch.empty((len(reqs), G, V), dtype=torch.float32, device=device)
+    U = torch.empty((G, len(reqs), V), dtype=torch.float32, device=device)
     lt = torch.empty((len(reqs), G + 1, V), dtype=torch.float32, device=device)
     g = torch.Generator(device=device)
     for i, b in enumerate(reqs):
@@ -232,6 +233,6 @@ def device_logits(wl: Workload, device, requests=None):
         u_ext = torch.randn((G + 1, V), generator=g, device=device) * wl.u_sigma
         if prior is not None:
             u_ext += prior
-        U[i] = u_ext[:G]
+        U[:, i] = u_ext[:G]
         lt[i] = u_ext + torch.randn((G + 1, V), generator=g, device=device) * sig
     return U, lt

@@ -29,6 +29,16 @@ def dev(a, dtype=None):
     return t.cuda()
 
 
+def pm(a):
+    """Host [B, gamma, V] -> device position-major [gamma, B, V] (the layout of U and l_d)."""
+    return dev(np.ascontiguousarray(np.asarray(a).transpose(1, 0, 2)))
+
+
+def host_rm(t):
+    """Device position-major [gamma, B, V] -> host [B, gamma, V]."""
+    return host(t).transpose(1, 0, 2)
+
+
 def dev_weights(W1, W2, w_dtype):
     dt = torch.bfloat16 if w_dtype == "bf16" else torch.float32
     return dev(W1, dt), dev(W2, dt)

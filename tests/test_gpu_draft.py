@@ -6,7 +6,7 @@ import torch
 
 from speculative_decoding_04_b200 import dspark as D
 from speculative_decoding_04_b200 import inputs
-from tests.parity import check_draft, dev, dev_weights, host
+from tests.parity import check_draft, dev, dev_weights, host, host_rm, pm
 
 pytestmark = pytest.mark.gpu
 
@@ -14,9 +14,9 @@ pytestmark = pytest.mark.gpu
 def run_draft(d, wl, path=0):
     D.set_option("draft_path", path)
     W1, W2 = dev_weights(d["W1"], d["W2"], wl.w_dtype)
-    x, ld, fl = D.markov_draft(dev(d["U"]), W1, W2, dev(d["x0"]), dev(d["u_draft"]), wl.T)
+    x, ld, fl = D.markov_draft(pm(d["U"]), W1, W2, dev(d["x0"]), dev(d["u_draft"]), wl.T)
     torch.cuda.synchronize()
-    return host(x), host(ld), host(fl)
+    return host(x), host_rm(ld), host(fl)
 
 
 def small(B, gamma, V, r, T, w_dtype="bf16", seed=77, logits="logzipf"):
@@ -76,7 +76,7 @@ def test_forced_markov_chain():
     for path in (1, 2):
         D.set_option("draft_path", path)
         Wd1, Wd2 = dev_weights(W1, W2, "bf16")
-        x, ld, fl = D.markov_draft(dev(U), Wd1, Wd2, dev(x0), dev(u), 1.0)
+        x, ld, fl = D.markov_draft(pm(U), Wd1, Wd2, dev(x0), dev(u), 1.0)
         x = host(x)
         want = (x0[:, None] + 1 + np.arange(G)[None, :]) % r
         assert np.array_equal(x, want), path
@@ -101,9 +101,9 @@ def test_nonfinite_logits_are_flagged():
 def test_graph_capture_replays_the_same_draft():
     wl, d = small(16, 4, 4104, 256, 1.0, seed=6)
     W1, W2 = dev_weights(d["W1"], d["W2"], "bf16")
-    U, x0, u = dev(d["U"]), dev(d["x0"]), dev(d["u_draft"])
+    U, x0, u = pm(d["U"]), dev(d["x0"]), dev(d["u_draft"])
     x = torch.empty((16, 4), dtype=torch.int32, device="cuda")
-    ld = torch.empty((16, 4, wl.V), dtype=torch.float32, device="cuda")
+    ld = torch.empty((4, 16, wl.V), dtype=torch.float32, device="cuda")
     fl = torch.zeros(16, dtype=torch.int32, device="cuda")
     ws = D.workspace(D.WS_DRAFT, 16, 4, wl.V, 256)
     s = torch.cuda.Stream()

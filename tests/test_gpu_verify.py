@@ -7,7 +7,7 @@ import torch
 import oracle as O
 from speculative_decoding_04_b200 import dspark as D
 from speculative_decoding_04_b200 import inputs
-from tests.parity import check_labels, check_verify, dev, draw_tokens, host
+from tests.parity import check_labels, check_verify, dev, draw_tokens, host, pm
 
 pytestmark = pytest.mark.gpu
 
@@ -23,7 +23,7 @@ def case(B, G, V, T, seed, sigma_t=0.7, logits="logzipf"):
 
 
 def run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=True):
-    n, y, c, fl = D.verify(dev(ld), dev(lt), dev(x), None if L is None else dev(L), dev(u_acc), dev(u_res), T,
+    n, y, c, fl = D.verify(pm(ld), dev(lt), dev(x), None if L is None else dev(L), dev(u_acc), dev(u_res), T,
                            want_c_star=want_c)
     torch.cuda.synchronize()
     return host(n), host(y), (host(c) if c is not None else None), host(fl)
@@ -84,7 +84,7 @@ def test_tv_labels_entry_point(lt_rows, T):
     ld, lt, x, u_acc, u_res = case(4, 5, 50000, T, seed=11, sigma_t=1.5)
     if lt_rows == "gamma":
         lt = np.ascontiguousarray(lt[:, :5])
-    c = host(D.tv_labels(dev(ld), dev(lt), T))
+    c = host(D.tv_labels(pm(ld), dev(lt), T))
     check_labels(ld, lt, T, c)
     assert np.all((c >= 0) & (c <= 1))
 

@@ -12,7 +12,7 @@ import torch
 import oracle as O
 from speculative_decoding_04_b200 import dspark as D
 from speculative_decoding_04_b200 import inputs
-from tests.parity import check_draft, check_labels, check_verify, dev, dev_weights, host
+from tests.parity import check_draft, check_labels, check_verify, dev, dev_weights, host, host_rm, pm
 
 pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -20,11 +20,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 
 def gpu_round(d, wl, L=None, want_c=True):
     W1, W2 = dev_weights(d["W1"], d["W2"], wl.w_dtype)
-    x, ld, fl = D.markov_draft(dev(d["U"]), W1, W2, dev(d["x0"]), dev(d["u_draft"]), wl.T)
+    x, ld, fl = D.markov_draft(pm(d["U"]), W1, W2, dev(d["x0"]), dev(d["u_draft"]), wl.T)
     n, y, c, fl = D.verify(ld, dev(d["lt"]), x, None if L is None else dev(L), dev(d["u_acc"]), dev(d["u_res"]),
                            wl.T, want_c_star=want_c, flags=fl)
     torch.cuda.synchronize()
-    return host(x), host(ld), host(n), host(y), (host(c) if c is not None else None), host(fl)
+    return host(x), host_rm(ld), host(n), host(y), (host(c) if c is not None else None), host(fl)
 
 
 def test_tiny_round_matches_golden_fixture():
@@ -92,7 +92,7 @@ def test_vocabulary_sweep(B, gamma):
         assert np.array_equal(yh[b, :nh[b]], xh[b, :nh[b]]) and np.all(yh[b, nh[b] + 1:] == -1)
     # oracle on sampled requests (the requests are independent)
     reqs = sorted({0, B - 1, B // 2})
-    Uh, lth, ldh = host(U[reqs]), host(lt[reqs]), host(ld[reqs])
+    Uh, lth, ldh = host_rm(U[:, reqs]), host(lt[reqs]), host_rm(ld[:, reqs])
     sub = dict(U=Uh, x0=x0[reqs], u=u_draft[reqs])
     check_draft(sub["U"], W1h, W2h, sub["x0"], sub["u"], wl.T, xh[reqs], ldh)
     check_verify(ldh, lth, xh[reqs], None, u_acc[reqs], u_res[reqs], wl.T, nh[reqs], yh[reqs])

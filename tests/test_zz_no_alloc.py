@@ -10,7 +10,7 @@ import torch
 
 from speculative_decoding_04_b200 import dspark as D
 from speculative_decoding_04_b200 import inputs
-from tests.parity import P_ATOL, P_RTOL, dev, draw_tokens, host
+from tests.parity import P_ATOL, P_RTOL, dev, draw_tokens, host, pm
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +29,7 @@ def test_noalloc_matches_workspace_verify_twice_in_a_row(T):
     L = np.array([6, 0, 3, 5, 1, 6, 2, 4, 6, 6, 0, 1], dtype=np.int32)
     for call, seed in enumerate((21, 22)):   # two calls in a row on the shared scratch
         ld, lt, x, u_acc, u_res = _case(seed, B, G, V, T)
-        args = (dev(ld), dev(lt), dev(x), dev(L) if call else None, dev(u_acc), dev(u_res), T)
+        args = (pm(ld), dev(lt), dev(x), dev(L) if call else None, dev(u_acc), dev(u_res), T)
         n0, y0, c0, f0 = D.verify(*args, want_c_star=True)
         # outputs prepared by the caller: the no-allocation call itself allocates nothing
         n1 = torch.empty(B, dtype=torch.int32, device="cuda")
@@ -47,7 +47,7 @@ def test_noalloc_matches_workspace_verify_twice_in_a_row(T):
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     B, G, V = 4097, 1, 64
-    ld = torch.zeros((B, G, V), device="cuda")
+    ld = torch.zeros((G, B, V), device="cuda")
     lt = torch.zeros((B, G + 1, V), device="cuda")
     x = torch.zeros((B, G), dtype=torch.int32, device="cuda")
     u = torch.zeros((B, G), device="cuda")
