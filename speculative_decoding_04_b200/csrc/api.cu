@@ -27,6 +27,8 @@ Options& options() {
     if (const char* e = std::getenv("DSPARK_DRAFT_PDL")) o.draft_pdl = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_CLUSTER")) o.verify_cluster = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_PERSISTENT")) o.verify_persistent = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_VERIFY_STREAM")) o.verify_stream = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_VERIFY_STREAM_CLUSTER")) o.verify_stream_cluster = std::atoi(e);
   });
   return o;
 }
@@ -72,6 +74,8 @@ int dspark_set_option(const char* key, long value) {
   else if (!std::strcmp(key, "draft_w2_hint")) o.draft_w2_hint = (int)value;
   else if (!std::strcmp(key, "verify_cluster")) o.verify_cluster = (int)value;
   else if (!std::strcmp(key, "verify_persistent")) o.verify_persistent = (int)value;
+  else if (!std::strcmp(key, "verify_stream")) o.verify_stream = (int)value;
+  else if (!std::strcmp(key, "verify_stream_cluster")) o.verify_stream_cluster = (int)value;
   else if (!std::strcmp(key, "sm_count")) o.sm_count = (int)value;
   else return einval(std::string("dspark_set_option: unknown key ") + key);
   return DSPARK_OK;

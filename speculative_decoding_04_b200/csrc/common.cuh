@@ -279,6 +279,17 @@ __device__ __forceinline__ Top2 top2_merge(Top2 a, Top2 b) {
   return r;
 }
 
+// Add one value; indices must arrive in increasing order (the lowest index wins a tie).
+__device__ __forceinline__ void top2_push(Top2& t, float x, int idx) {
+  if (t.idx < 0 || x > t.best) {
+    t.second = fmaxf(t.second, t.best);
+    t.best = x;
+    t.idx = idx;
+  } else {
+    t.second = fmaxf(t.second, x);
+  }
+}
+
 __device__ __forceinline__ Top2 top2_shfl_xor(Top2 t, int o) {
   Top2 u;
   u.best = __shfl_xor_sync(0xffffffffu, t.best, o);

@@ -20,6 +20,8 @@ struct Options {
   int draft_w2_hint = 1;         // W2 tile loads carry an L2 evict-last hint
   int verify_cluster = 0;        // 0 auto, else the cluster size (1, 2, 4, 8, 16)
   int verify_persistent = 1;     // sampled verify / labels: persistent double-buffered clusters
+  int verify_stream = 1;         // verify with a workspace: streaming kernels (one HBM read + one L2 read)
+  int verify_stream_cluster = 8; // CTAs per cluster of the streaming verify (1, 2, 4, 8)
   int sm_count = 0;              // 0: query the device
 };
 Options& options();
@@ -78,6 +80,8 @@ size_t verify_workspace_bytes(int B, int gamma, int V);
 
 dspark_status launch_draft(const DraftCall& c);
 dspark_status launch_verify(const VerifyCall& c);
+dspark_status launch_verify_stream(const VerifyCall& c);
+size_t stream_verify_workspace_bytes(int B, int gamma, int V);
 dspark_status launch_schedule(const ScheduleCall& c);
 
 constexpr int kMaxGamma = 64;

@@ -130,16 +130,6 @@ __device__ Top2 block_top2(Top2 t, Top2* sh) {
   return r;
 }
 
-__device__ __forceinline__ void top2_push(Top2& t, float x, int idx) {
-  if (t.idx < 0 || x > t.best) {
-    t.second = fmaxf(t.second, t.best);
-    t.best = x;
-    t.idx = idx;
-  } else {
-    t.second = fmaxf(t.second, x);
-  }
-}
-
 // Assemble n_acc / y for every request from the per-row results (one thread per request),
 // after the row kernel has finished.
 __global__ void verify_finalize(VerifyArgs a) {
@@ -1044,10 +1034,12 @@ __global__ void __launch_bounds__(512, 1) verify_rows_pc(VerifyArgs a) {
 
 // ============================================================================ host side
 
+// Per-row kernels need the first part; the streaming kernels (the default with a workspace)
+// the second.
 size_t verify_workspace_bytes(int B, int gamma, int V) {
-  (void)V;
   const size_t rows = (size_t)B * (gamma + 1);
-  return kWsHeader + 3 * align_up(rows * 4, 256) + align_up((size_t)B * 4, 256);
+  const size_t per_row = kWsHeader + 3 * align_up(rows * 4, 256) + align_up((size_t)B * 4, 256);
+  return std::max(per_row, stream_verify_workspace_bytes(B, gamma, V));
 }
 
 // Cluster size: the smallest power of two whose per-CTA slices (ℓ_d and ℓ_t, fp32) fit the
@@ -1144,6 +1136,10 @@ static dspark_status launch_verify_persistent(const VerifyArgs& a, int cs, cudaS
 }
 
 dspark_status launch_verify(const VerifyCall& c) {
+  if (c.do_verify) {
+    const dspark_status st = launch_verify_stream(c);
+    if (st != DSPARK_ENOTIMPL) return st;  // else: the per-row kernels below
+  }
   VerifyArgs a{};
   a.ld = c.ld;
   a.lt = c.lt;

@@ -29,15 +29,33 @@ def run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=True):
     return host(n), host(y), (host(c) if c is not None else None), host(fl)
 
 
+# kernels: "stream-C" = streaming kernels with clusters of C CTAs (the default with a
+# workspace); "rows-C" = one cluster of C CTAs per row (0: chosen from V), which serves calls
+# without a workspace, V not a multiple of 4 and the labels entry point.
+IMPLS = ["stream-8", "stream-4", "stream-1", "rows-0", "rows-1", "rows-4", "rows-16"]
+
+
+def use_impl(impl):
+    kind, c = impl.split("-")
+    D.set_option("verify_stream", 1 if kind == "stream" else 0)
+    if kind == "stream":
+        D.set_option("verify_stream_cluster", int(c))
+    else:
+        D.set_option("verify_cluster", int(c))
+    return kind, int(c)
+
+
 @pytest.mark.parametrize("V", [1003, 4096, 30000])
 @pytest.mark.parametrize("T", [1.0, 0.7, 0.0])
 @pytest.mark.parametrize("scheduled", [False, True])
-@pytest.mark.parametrize("cluster", [0, 1, 4, 16])
+@pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("labels", [True, False])
-def test_verify_matches_oracle(V, T, scheduled, cluster, labels):
-    if cluster and V < 4096 and cluster > 4:
+def test_verify_matches_oracle(V, T, scheduled, impl, labels):
+    kind, cluster = use_impl(impl)
+    if kind == "rows" and cluster and V < 4096 and cluster > 4:
         pytest.skip("slice smaller than the block")
-    D.set_option("verify_cluster", cluster)
+    if kind == "stream" and V % 4:
+        pytest.skip("the streaming kernels need V % 4 == 0 (other V take the per-row kernels)")
     B, G = 6, 4
     ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=V + int(T * 10) + cluster)
     # without labels, rows past L_b + 1 are skipped by the kernels
@@ -116,12 +134,32 @@ def test_acceptance_rate_matches_label_statistically():
     assert abs(rate - c1) < 4 * np.sqrt(c1 * (1 - c1) / B)
 
 
-@pytest.mark.parametrize("persistent", [1, 0])
-def test_scheduled_rows_skipped_many_requests(persistent):
-    D.set_option("verify_persistent", persistent)
+@pytest.mark.parametrize("impl", ["stream-8", "stream-2", "persistent-1", "persistent-0"])
+def test_scheduled_rows_skipped_many_requests(impl):
+    kind, v = impl.split("-")
+    D.set_option("verify_stream", 1 if kind == "stream" else 0)
+    if kind == "stream":
+        D.set_option("verify_stream_cluster", int(v))
+    else:
+        D.set_option("verify_persistent", int(v))
     B, G, V = 40, 6, 20000
     ld, lt, x, u_acc, u_res = case(B, G, V, 1.0, seed=77)
     L = (np.arange(B) * 7 % (G + 1)).astype(np.int32)
     n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, 1.0, want_c=False)
     check_verify(ld, lt, x, L, u_acc, u_res, 1.0, n, y)
     assert np.all(n <= L)
+
+
+@pytest.mark.parametrize("T", [1.0, 0.0])
+def test_stream_vocabulary_beyond_per_row_kernels(T):
+    # V = 500,000: more than one 16-CTA cluster can hold per row; only the streaming kernels
+    # take it (rows of 489 tiles, the last one 288 columns wide)
+    B, G, V = 3, 3, 500_000
+    ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=91)
+    n, y, c, fl = run_verify(ld, lt, x, None, u_acc, u_res, T)
+    check_verify(ld, lt, x, None, u_acc, u_res, T, n, y)
+    check_labels(ld, lt, T, c)
+    D.set_option("verify_stream", 0)
+    with pytest.raises(D.DsparkError) as e:
+        run_verify(ld, lt, x, None, u_acc, u_res, T)
+    assert e.value.status == D.ENOTIMPL
