@@ -21,9 +21,13 @@
 // stalls the tile pipeline, and a row's two reads are at most two rows of the whole grid
 // apart (a few tens of MB against a 126 MB L2).
 //
-// Roles in a CTA of 320 threads: warps 0-7 consume tiles (tile g goes to warp g mod 8 and ring
-// stage g mod 16), warp 8 issues the bulk copies, warp 9 combines partial results, exchanges
-// them with the cluster, decides acceptance and writes the per-row records.  A small second
+// Roles in a CTA of 320 threads: warp 8 streams the rows through a 3-stage ring, one 32 KB bulk
+// copy per row and stage (copies of 4 KB were measured to cap the stream at under half the HBM
+// bandwidth, whatever the number of issuing threads); warps 0-7 each take one 1024-column piece
+// of a stage (the assignment rotates from stage to stage, so uneven segments even out); warp 9
+// combines partial results, exchanges them with the cluster, decides acceptance and writes the
+// per-row records.
+// A small second
 // kernel (one warp per request) finds n, samples the residual / bonus token by an inverse CDF
 // over the per-tile weights and one rescanned tile, and writes y, n and c*.
 // Every wait is bounded; after a timeout all roles stop and the status word is set.
@@ -45,7 +49,8 @@ namespace {
 
 constexpr int kSvTile = 1024;  // columns per tile
 constexpr int kSvWarps = 8;    // consumer warps
-constexpr int kSvStages = 16;  // ring stages of (l_d tile, l_t tile)
+constexpr int kSvBig = kSvWarps * kSvTile;  // columns per ring stage: one 32 KB copy per row
+constexpr int kSvStages = 3;                 // ring stages of (l_d 8192 columns, l_t 8192 columns)
 constexpr int kSvThreads = (kSvWarps + 2) * 32;
 constexpr int kSvProducer = kSvWarps;
 constexpr int kSvController = kSvWarps + 1;
@@ -54,7 +59,7 @@ constexpr int kSvJobSlots = 4;
 constexpr int kSvMaxCluster = 8;
 constexpr int kRNone = -(1 << 28);  // reference of an empty sum
 constexpr int kRMax = 1 << 24;
-constexpr size_t kSvRingBytes = (size_t)kSvStages * 2 * kSvTile * sizeof(float);
+constexpr size_t kSvRingBytes = (size_t)kSvStages * 2 * kSvBig * sizeof(float);
 
 // A partial result: of a warp for one phase, or of a CTA for one row.
 // P1: sd / st are sums of 2^(z log2e - rd / rt); P2: sd = sum min(p_d, p_t), st = sum q.
@@ -132,6 +137,61 @@ __device__ __forceinline__ int sv_next(const SvArgs& a, int j, int ncl, SvJob& J
 }
 
 __device__ __forceinline__ bool sv_p2(const SvArgs& a, const SvJob& J) { return !a.greedy && J.d; }
+
+// One phase of the tile stream: the first pass of a row, or its second pass.
+struct SvPhase {
+  SvJob J;
+  bool second;
+  int i;  // index of the row among this cluster's rows (exchange / decision slots)
+};
+
+// The phase sequence of a cluster: P1(row 0), then P1(row i), P2(row i-1) for i = 1, 2, ...,
+// then P2(last row).  Every role walks the same sequence.
+struct SvGen {
+  int j, ncl, i, step;
+  SvJob cur, prev;
+  bool have_prev, done;
+  __device__ void init(const SvArgs& a, int cid, int ncl_) {
+    ncl = ncl_;
+    j = sv_next(a, cid, ncl, cur);
+    i = 0;
+    step = 0;
+    have_prev = false;
+    done = false;
+  }
+  __device__ bool next(const SvArgs& a, SvPhase& ph) {
+    while (!done) {
+      if (step == 0) {
+        step = 1;
+        if (j >= 0) {
+          ph.J = cur;
+          ph.second = false;
+          ph.i = i;
+          return true;
+        }
+      }
+      if (step == 1) {
+        step = 2;
+        if (have_prev && sv_p2(a, prev)) {
+          ph.J = prev;
+          ph.second = true;
+          ph.i = i - 1;
+          return true;
+        }
+      }
+      if (j < 0) {
+        done = true;
+        return false;
+      }
+      prev = cur;
+      have_prev = true;
+      ++i;
+      j = sv_next(a, j + ncl, ncl, cur);
+      step = 0;
+    }
+    return false;
+  }
+};
 
 __device__ __forceinline__ float sv_ex2(float x) {
   float y;
@@ -280,6 +340,62 @@ __device__ __forceinline__ bool sv_wait(const SvSync& s, uint64_t* bar, uint32_t
 
 __device__ __forceinline__ float f4c(const float4& v, int c) { return c == 0 ? v.x : (c == 1 ? v.y : (c == 2 ? v.z : v.w)); }
 
+// Packed fp32 pairs (sm_100): per element the same correctly rounded results as the scalar
+// instructions, at half the instruction count.
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+// max of three (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
+
+// First pass over one lane's 32 values of a tile: z = l * (1/T) in place, the integer
+// reference R of their maximum and the fp32 sum of 2^(z log2e - R).
+__device__ __forceinline__ float sv_lane_sum(float4 (&v)[8], float2 invT2, int& R) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const float2 a = f2mul(lo2(v[jj]), invT2), b = f2mul(hi2(v[jj]), invT2);
+    v[jj] = make_float4(a.x, a.y, b.x, b.y);
+    m = fmax3(m, a.x, a.y);
+    m = fmax3(m, b.x, b.y);
+  }
+  R = sv_ref(m);
+  const float2 l2e2 = make_float2(kLog2e, kLog2e), nr2 = make_float2(-(float)R, -(float)R);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const float2 a = f2fma(lo2(v[jj]), l2e2, nr2), b = f2fma(hi2(v[jj]), l2e2, nr2);
+    acc0 = f2add(acc0, make_float2(sv_ex2(a.x), sv_ex2(a.y)));
+    acc1 = f2add(acc1, make_float2(sv_ex2(b.x), sv_ex2(b.y)));
+  }
+  const float2 acc = f2add(acc0, acc1);
+  return acc.x + acc.y;
+}
+
 template <bool GREEDY>
 __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
@@ -288,7 +404,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   const int cid = blockIdx.x / C, ncl = gridDim.x / C;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  extern __shared__ __align__(128) float ring[];  // [kSvStages][2][kSvTile]: l_d tile, l_t tile
+  extern __shared__ __align__(128) float ring[];  // [kSvStages][2][kSvBig]: l_d columns, l_t columns
   __shared__ __align__(8) uint64_t full[kSvStages], empty[kSvStages];
   __shared__ __align__(8) uint64_t phbar[kSvPhaseSlots];
   __shared__ __align__(8) uint64_t xbar[kSvJobSlots], dbar[kSvJobSlots];
@@ -301,7 +417,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSvStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], kSvWarps);
     }
     for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
     for (int i = 0; i < kSvJobSlots; ++i) {
@@ -318,47 +434,49 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   const int nt = (int)((long long)(rank + 1) * a.ntile / C) - tb;  // tiles of this CTA per row (may be 0)
   const float inv_T = a.inv_T;
 
+  const int nbig = (nt + kSvWarps - 1) / kSvWarps;  // ring stages per row and pass
+  const int c_end = min((tb + nt) * kSvTile, a.V);     // end column of this CTA's segment
+
   if (warp == kSvProducer) {
     // ------------------------------------------------------------------ bulk copies
-    if (lane == 0) {
-      uint32_t G = 0;
+    // Stage gb of the stream holds up to 8192 columns of both rows: one copy per row.  A bulk
+    // copy costs the copy engine about the same time whatever its size (measured on this part:
+    // 4 KB copies stream at under half the HBM bandwidth, 32 KB ones at full bandwidth).
+    if (lane < 2) {
+      SvGen gen;
+      gen.init(a, cid, ncl);
+      SvPhase ph;
+      uint32_t Gb = 0;
       bool ok = true;
-      auto issue = [&](const SvJob& J, bool with_d) {
-        const float* rd = a.ld + ((size_t)J.k * a.B + J.b) * a.V;
-        const float* rt = a.lt + ((size_t)J.b * a.lt_rows + J.k) * a.V;
-        for (int t = 0; t < nt && ok; ++t) {
-          const uint32_t g = G + t;
-          const int s = (int)(g % kSvStages);
-          if (!sv_wait(sy, &empty[s], ((g / kSvStages) & 1) ^ 1)) {
+      while (ok && gen.next(a, ph)) {
+        const bool with_d = ph.second || ph.J.d;
+        const float* rd = a.ld + ((size_t)ph.J.k * a.B + ph.J.b) * a.V;
+        const float* rt = a.lt + ((size_t)ph.J.b * a.lt_rows + ph.J.k) * a.V;
+        for (int bt = 0; bt < nbig; ++bt) {
+          const uint32_t gb = Gb + bt;
+          const int s = (int)(gb % kSvStages);
+          // lane 0 arms the stage and copies l_d, lane 1 copies l_t
+          if (!sv_wait(sy, &empty[s], ((gb / kSvStages) & 1) ^ 1)) {
             ok = false;
             break;
           }
-          const int v0 = (tb + t) * kSvTile;
-          const uint32_t bytes = (uint32_t)min(kSvTile, a.V - v0) * 4u;
-          float* st = ring + (size_t)s * 2 * kSvTile;
-          mbar_arrive_expect_tx(&full[s], with_d ? 2 * bytes : bytes);
-          if (with_d) bulk_g2s(st, rd + v0, bytes, &full[s]);
-          bulk_g2s(st + kSvTile, rt + v0, bytes, &full[s]);
+          const int v0 = (tb + bt * kSvWarps) * kSvTile;
+          const uint32_t bytes = (uint32_t)min(kSvBig, c_end - v0) * 4u;
+          float* st = ring + (size_t)s * 2 * kSvBig;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[s], with_d ? 2 * bytes : bytes);
+            if (with_d) bulk_g2s(st, rd + v0, bytes, &full[s]);
+          } else {
+            bulk_g2s(st + kSvBig, rt + v0, bytes, &full[s]);
+          }
         }
-        G += nt;
-      };
-      SvJob cur, prev;
-      int j = sv_next(a, cid, ncl, cur);
-      bool have_prev = false;
-      while (ok) {
-        const bool have_cur = j >= 0;
-        if (have_cur) issue(cur, cur.d);
-        if (have_prev && sv_p2(a, prev)) issue(prev, true);
-        if (!have_cur) break;
-        prev = cur;
-        have_prev = true;
-        j = sv_next(a, j + ncl, ncl, cur);
+        Gb += (uint32_t)nbig;
       }
       if (!ok) {
-        // let the copies already issued land before the CTA can exit
-        const uint32_t lo = G > (uint32_t)kSvStages ? G - kSvStages : 0u;
-        for (uint32_t g = lo; g < G; ++g)
-          for (uint32_t i = 0; i < kSpinLimit && !mbar_try_wait(&full[g % kSvStages], (g / kSvStages) & 1); ++i) {
+        // let the copies still in flight land before the CTA can exit
+        const uint32_t lo = Gb > (uint32_t)kSvStages ? Gb - kSvStages : 0u;
+        for (uint32_t gb = lo; gb < Gb; ++gb)
+          for (uint32_t i = 0; i < kSpinLimit && !mbar_try_wait(&full[gb % kSvStages], (gb / kSvStages) & 1); ++i) {
           }
       }
     }
@@ -472,7 +590,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   } else {
     // ------------------------------------------------------------------ tile consumers
     const int w = warp;
-    uint32_t G = 0;
+    uint32_t Gb = 0;
     int p = 0;
     bool ok = true;
     auto run_phase = [&](const SvJob& J, bool second, int i) {
@@ -492,18 +610,21 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
         if (ok) nm = dec[js];
       }
       const bool with_d = second || J.d;
-      const uint32_t g0 = G + (uint32_t)((w - (int)(G % kSvWarps) + kSvWarps) % kSvWarps);
-      for (uint32_t g = g0; ok && g < G + (uint32_t)nt; g += kSvWarps) {
-        const int t = (int)(g - G);
-        const int s = (int)(g % kSvStages);
-        if (!sv_wait(sy, &full[s], (g / kSvStages) & 1)) {
+      for (int bt = 0; ok && bt < nbig; ++bt) {
+        const uint32_t gb = Gb + bt;
+        const int s = (int)(gb % kSvStages);
+        if (!sv_wait(sy, &full[s], (gb / kSvStages) & 1)) {
           ok = false;
           break;
         }
+        // this warp's 1024-column piece of the stage; the assignment rotates from stage to stage
+        const int q = (w + (int)(gb % kSvWarps)) % kSvWarps;
+        const int t = bt * kSvWarps + q;  // tile of this CTA's segment
+        const bool mine = t < nt;
         const int v0 = (tb + t) * kSvTile;
-        const int cnt = min(kSvTile, a.V - v0);
-        const float* sd = ring + (size_t)s * 2 * kSvTile;
-        const float* st = sd + kSvTile;
+        const int cnt = mine ? min(kSvTile, a.V - v0) : 0;
+        const float* sd = ring + (size_t)s * 2 * kSvBig + q * kSvTile;
+        const float* st = sd + kSvBig;
         float4 fd[8], ft[8];
         const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
 #pragma unroll
@@ -515,6 +636,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);  // the values are in registers
+        if (!mine) continue;
         if (!second) {
           // drafted token in this tile: keep its raw logits
           const int xi = xk - v0;
@@ -541,25 +663,9 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
               }
             }
           } else {
-            float mt = -INFINITY, md = -INFINITY;
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              ft[jj] = make_float4(__fmul_rn(ft[jj].x, inv_T), __fmul_rn(ft[jj].y, inv_T), __fmul_rn(ft[jj].z, inv_T),
-                                   __fmul_rn(ft[jj].w, inv_T));
-              mt = fmaxf(mt, fmaxf(fmaxf(ft[jj].x, ft[jj].y), fmaxf(ft[jj].z, ft[jj].w)));
-              if (with_d) {
-                fd[jj] = make_float4(__fmul_rn(fd[jj].x, inv_T), __fmul_rn(fd[jj].y, inv_T),
-                                     __fmul_rn(fd[jj].z, inv_T), __fmul_rn(fd[jj].w, inv_T));
-                md = fmaxf(md, fmaxf(fmaxf(fd[jj].x, fd[jj].y), fmaxf(fd[jj].z, fd[jj].w)));
-              }
-            }
-            const int rt = sv_ref(mt);
-            const float rtf = (float)rt;
-            float stl = 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-              stl += (sv_ex2(fmaf(ft[jj].x, kLog2e, -rtf)) + sv_ex2(fmaf(ft[jj].y, kLog2e, -rtf))) +
-                     (sv_ex2(fmaf(ft[jj].z, kLog2e, -rtf)) + sv_ex2(fmaf(ft[jj].w, kLog2e, -rtf)));
+            const float2 invT2 = make_float2(inv_T, inv_T);
+            int rt;
+            const float stl = sv_lane_sum(ft, invT2, rt);
             bad |= (stl <= FLT_MAX) ? 0u : 1u;
             sv_merge(Rt, St, rt, (double)stl);
             if (a.do_verify) {
@@ -569,39 +675,41 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
               if (lane == 0) a.trec[(size_t)J.rec * a.ntile + tb + t] = make_float2((float)R, sw);
             }
             if (with_d) {
-              const int rd = sv_ref(md);
-              const float rdf = (float)rd;
-              float sdl = 0.f;
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj)
-                sdl += (sv_ex2(fmaf(fd[jj].x, kLog2e, -rdf)) + sv_ex2(fmaf(fd[jj].y, kLog2e, -rdf))) +
-                       (sv_ex2(fmaf(fd[jj].z, kLog2e, -rdf)) + sv_ex2(fmaf(fd[jj].w, kLog2e, -rdf)));
+              int rd;
+              const float sdl = sv_lane_sum(fd, invT2, rd);
               bad |= (sdl <= FLT_MAX) ? 0u : 1u;
               sv_merge(Rd, Sd, rd, (double)sdl);
             }
           }
         } else {
-          float sml = 0.f, ql = 0.f;
+          // p = 2^(z log2e - K - lam) for both rows; sum min(p_d, p_t) and q = p_t - min
+          const float2 invT2 = make_float2(inv_T, inv_T), l2e2 = make_float2(kLog2e, kLog2e);
+          const float2 nkd = make_float2(-nm.Kd, -nm.Kd), nkt = make_float2(-nm.Kt, -nm.Kt);
+          const float2 nld = make_float2(-nm.lamd, -nm.lamd), nlt = make_float2(-nm.lamt, -nm.lamt);
+          float2 sm2 = make_float2(0.f, 0.f), q2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float pd, pt;
-              sv_probs(f4c(fd[jj], c), f4c(ft[jj], c), inv_T, nm, pd, pt);
-              const float mn = fminf(pd, pt);
-              sml += mn;
-              ql += pt - mn;
+            for (int h = 0; h < 2; ++h) {
+              const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
+              const float2 ad = f2add(f2fma(f2mul(ld2, invT2), l2e2, nkd), nld);
+              const float2 at = f2add(f2fma(f2mul(lt2, invT2), l2e2, nkt), nlt);
+              const float2 pt = make_float2(sv_ex2(at.x), sv_ex2(at.y));
+              const float2 mn = make_float2(fminf(sv_ex2(ad.x), pt.x), fminf(sv_ex2(ad.y), pt.y));
+              sm2 = f2add(sm2, mn);
+              q2 = f2add(q2, make_float2(pt.x - mn.x, pt.y - mn.y));
             }
           }
+          const float sml = sm2.x + sm2.y, ql = q2.x + q2.y;
           smin += (double)sml;
           sq += (double)ql;
           if (J.verify) {
-            const double qw = warp_sum_d((double)ql);
-            if (lane == 0) a.qrec[(size_t)J.rec * a.ntile + tb + t] = (float)qw;
+            const float qw = warp_sum_f(ql);
+            if (lane == 0) a.qrec[(size_t)J.rec * a.ntile + tb + t] = qw;
           }
         }
       }
-      G += (uint32_t)nt;
+      Gb += (uint32_t)nbig;
       if (!ok) return;
       // ---- phase result of this warp
       if (!second) {
@@ -640,18 +748,10 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       }
       ++p;
     };
-    SvJob cur, prev;
-    int j = sv_next(a, cid, ncl, cur);
-    bool have_prev = false;
-    for (int i = 0; ok; ++i) {
-      const bool have_cur = j >= 0;
-      if (have_cur) run_phase(cur, false, i);
-      if (ok && have_prev && sv_p2(a, prev)) run_phase(prev, true, i - 1);
-      if (!have_cur) break;
-      prev = cur;
-      have_prev = true;
-      j = sv_next(a, j + ncl, ncl, cur);
-    }
+    SvGen cgen;
+    cgen.init(a, cid, ncl);
+    SvPhase ph;
+    while (ok && cgen.next(a, ph)) run_phase(ph.J, ph.second, ph.i);
   }
 
   __syncwarp();
@@ -860,7 +960,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   const SvLayout Ly = sv_layout(c.B, c.gamma, c.V);
   if (c.ws_bytes < Ly.total) return DSPARK_ENOTIMPL;
   int C = options().verify_stream_cluster;
-  if (C != 1 && C != 2 && C != 4 && C != 8) C = 8;
+  if (C != 1 && C != 2 && C != 4 && C != 8) C = 2;
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   SvArgs a{};
   a.ld = c.ld;

@@ -29,4 +29,4 @@ def _default_options():
         D.set_option("draft_w2_hint", 1)
         D.set_option("verify_persistent", 1)
         D.set_option("verify_stream", 1)
-        D.set_option("verify_stream_cluster", 8)
+        D.set_option("verify_stream_cluster", 2)
