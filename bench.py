@@ -25,6 +25,7 @@ cpu_baseline= the CPU oracle on a bounded sample of requests of the same workloa
 """
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -50,6 +51,22 @@ def peaks():
             j = json.load(f)
         return float(j["hbm_gbs"]), float(j.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), "measured"
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def measured_traffic(key, units):
+    """DRAM bytes (read + write) of one launch of kernel `key` from the ncu capture summarised in
+    profiles/traffic.json, scaled to `units` of work; None when that kernel's source file has
+    changed since the counters were taken (its SHA-1 is stored beside them)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)[key]
+        with open(os.path.join(ROOT, "speculative_decoding_04_b200", "csrc", t["source"]), "rb") as f:
+            sha = hashlib.sha1(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    if sha != t.get("source_sha1"):
+        return None
+    return t["dram_bytes_per_launch"] * units / t["units_per_launch"]
 
 
 def workload_bytes(wl):
@@ -233,7 +250,7 @@ def main():
     ws_v = D.workspace(D.WS_VERIFY, B, G, V, 0, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    n_launch = 2 * G + 1 + 1
+    n_launch = 2 * G + 1 + 2  # draft: main pass + combine per position; schedule; verify: stream + finalize
 
     def round_(src):
         D.markov_draft(src["U"], W1, W2, src["x0"], src["u_draft"], wl.T, x_out=x, ld_out=ld, flags=fl, ws=ws_d,
@@ -334,14 +351,17 @@ def main():
             "verified_tokens_per_s": accepted_all / (args.steps * t_step),
             "draft_ms": t_draft * 1e3, "verify_ms": t_verify * 1e3,
             "hbm_gbs_round": (draft_b + verify_b) / t_step / 1e9,
-            "roofline": {"kernel": "markov_draft stage (16 x tcgen05 main pass + combine, PDL-chained)",
+            "roofline": {"kernel": f"markov_draft ({G} draft_main_tc + {G} draft_combine launches, timed "
+                                   "together with CUDA events around the call)",
                          "bound": "hbm", "achieved": draft_b / t_draft / 1e9, "peak": hbm, "unit": "GB/s",
-                         "frac": draft_b / t_draft / 1e9 / hbm, "traffic": None, "peak_source": src,
-                         "algorithmic_bytes": draft_b, "bias_tflops": flops / t_draft / 1e12,
+                         "frac": draft_b / t_draft / 1e9 / hbm,
+                         "traffic": measured_traffic("draft_main_tc", B * G),
+                         "peak_source": src, "algorithmic_bytes": draft_b, "bias_tflops": flops / t_draft / 1e12,
                          "frac_of_nominal_8TBs": draft_b / t_draft / 8e12},
-            "roofline_verify": {"kernel": "verify_rows (one launch)", "bound": "hbm",
-                                "achieved": verify_b / t_verify / 1e9, "peak": hbm, "unit": "GB/s",
-                                "frac": verify_b / t_verify / 1e9 / hbm, "traffic": None,
+            "roofline_verify": {"kernel": "verify (verify_stream + verify_stream_finalize, timed together)",
+                                "bound": "hbm", "achieved": verify_b / t_verify / 1e9, "peak": hbm, "unit": "GB/s",
+                                "frac": verify_b / t_verify / 1e9 / hbm,
+                                "traffic": measured_traffic("verify_stream", verify_b),
                                 "algorithmic_bytes": verify_b},
             "e2e": {"value": world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": n_launch * args.steps,

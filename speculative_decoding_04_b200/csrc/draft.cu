@@ -267,13 +267,17 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
 //   warp 1      MMA issuer: r/16 tcgen05.mma kind::f16 (M = 128, N = NB, K = 16) per tile into
 //               one of two TMEM accumulators of NB fp32 columns.
 //   warp 2      TMEM allocation owner.
+//   warp 3      U and l_d: one TMA box per tile brings U [NB requests x 128 columns] (32 KB at
+//               NB = 64) into a 2-stage buffer; when the epilogue has written l = U + bias in
+//               place, one TMA store writes the tile of l_d and the stage is refilled two tiles
+//               ahead (copies this size keep the copy engine near full HBM bandwidth; 4 KB ones
+//               were measured to stream at under half).
 //   warps 4..   epilogue, NB/8 warps: warp w owns TMEM lane quadrant w%4 (32 vocabulary columns)
-//               for the 32 requests of its column group.  Its [32 requests x 32 columns] block of
-//               U arrives by TMA two tiles ahead into a per-warp double buffer; l = U + bias is
-//               written back in place (lane = column), then each lane reads its own request's
-//               row (rotated 16-byte chunks, free of bank conflicts), streams l_d out with 16-byte
-//               stores and reduces the chunk statistics sequentially.  The statistics are also
-//               folded into one record per (CTA, request) for the combine's first level.
+//               for the 32 requests of its column group: it adds the bias to its [32 x 32] block
+//               of the U stage (lane = column), then each lane reads its own request's row
+//               (rotated 16-byte chunks, free of bank conflicts) and reduces the chunk statistics
+//               sequentially.  The statistics are also folded into one record per (CTA, request)
+//               for the combine's first level.
 // The B operand (the gathered W1 rows, K-major, 128-byte swizzle) is built once per step.
 
 constexpr int kTcTile = 128;
@@ -291,8 +295,8 @@ __host__ __device__ inline TcLayout tc_layout(int r, int nb) {
   L.w2_stage_bytes = (uint32_t)r * 256u;  // two 64-column atoms of r rows x 128 B
   L.w2 = ((uint32_t)nb * (uint32_t)r * 2u + 1023u) & ~1023u;
   L.u = L.w2 + kTcStages * L.w2_stage_bytes;
-  L.bars = L.u + (uint32_t)(nb / 8) * 2u * 4096u;  // per epilogue warp: 2 x [32 x 32] fp32
-  L.misc = L.bars + 8u * (2 * kTcStages + 2 + 2 + 1 + 2 * (nb / 8));
+  L.bars = L.u + 2u * (uint32_t)nb * kTcTile * 4u;  // two [nb requests x 128 columns] fp32 stages
+  L.misc = L.bars + 8u * (2 * kTcStages + 2 + 2 + 1 + 2 + 2 + 2);
   L.total = L.misc + 16u;
   return L;
 }
@@ -316,8 +320,9 @@ __device__ __forceinline__ bool tc_wait(const TcSync& s, uint64_t* bar, uint32_t
 
 template <int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    draft_main_tc(const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmU, DraftArgs a,
-                  int k, int n_bgroups, int ctas_per_group, int w2_hint) {
+    draft_main_tc(const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmU,
+                  const __grid_constant__ CUtensorMap tmLd, DraftArgs a, int k, int n_bgroups, int ctas_per_group,
+                  int w2_hint) {
   constexpr int EPI_WARPS = NB / 8;  // 4 per 32-request column group
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -332,7 +337,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* t_full = w_empty + kTcStages;
   uint64_t* t_empty = t_full + 2;
   uint64_t* mma_done = t_empty + 2;
-  uint64_t* u_full = mma_done + 1;  // [EPI_WARPS][2]
+  uint64_t* u_full = mma_done + 1;  // [2] U stage landed
+  uint64_t* u_empty = u_full + 2;   // [2] every epilogue warp is done reading the stage
+  uint64_t* c_done = u_empty + 2;   // [2] every epilogue warp has written l = U + bias in place
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L.misc + 4);
   const TcSync sy{s_abort, a.status};
@@ -356,11 +363,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&t_empty[i], EPI_WARPS);
     }
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 2 * EPI_WARPS; ++i) mbar_init(&u_full[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&u_full[i], 1);
+      mbar_init(&u_empty[i], EPI_WARPS);
+      mbar_init(&c_done[i], EPI_WARPS);
+    }
     *s_abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tmW2);
     prefetch_tmap(&tmU);
+    prefetch_tmap(&tmLd);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, 2 * NB);
@@ -374,19 +386,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // epilogue geometry (warps 4 .. 4+EPI_WARPS-1)
   const bool epi = warp >= 4 && warp < 4 + EPI_WARPS;
-  const int q = warp & 3, h = (warp - 4) >> 2, ew = warp - 4;
+  const int q = warp & 3, h = (warp - 4) >> 2;
   const int bb = b0 + h * 32;
-  float* ubuf = sU + (size_t)ew * 2 * 1024;  // two [32 requests][32 columns] fp32 blocks
-  // U block of tile i into buffer j (lane 0 issues; U is an input of the call, so the first
-  // blocks are requested before waiting for the previous kernel)
-  auto load_u = [&](int i) {
-    const int j = i & 1;
-    mbar_arrive_expect_tx(&u_full[ew * 2 + j], 4096u);
-    tma_load_3d(ubuf + j * 1024, &tmU, (t_beg + i) * kTcTile + q * 32, bb, k, &u_full[ew * 2 + j]);
-  };
-  if (epi && lane == 0) {
-    if (nt > 0) load_u(0);
-    if (nt > 1) load_u(1);
+  constexpr uint32_t kUStage = (uint32_t)NB * kTcTile;  // floats of one U stage: [NB requests][128 columns]
+  // U (an input of the call) for the first two tiles is requested before waiting for the previous
+  // kernel: one 128-column x NB-request box per tile
+  if (warp == 3 && lane == 0) {
+    for (int i = 0; i < 2 && i < nt; ++i) {
+      mbar_arrive_expect_tx(&u_full[i], kUStage * 4u);
+      tma_load_3d(sU + i * kUStage, &tmU, (t_beg + i) * kTcTile, b0, k, &u_full[i]);
+    }
   }
 
   if (warp == 0) {
@@ -435,7 +444,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       fence_proxy_async_smem();
       named_bar(1, kTcThreads - 32);
     }
-    if (warp == 1) {
+    if (warp == 3) {
+      // ---------------------------------------------------------------- U refills and l_d stores
+      // l_d = U + bias is written in place in the U stage by the epilogue; one TMA store per tile
+      // writes it out, and the stage is refilled with the U tile two ahead once the store has
+      // read it and every epilogue warp is done with it.
+      if (lane == 0) {
+        int last_load[2] = {nt > 0 ? 0 : -1, nt > 1 ? 1 : -1};  // last tile loaded into each stage
+        for (int i = 0; i < nt; ++i) {
+          const int j = i & 1;
+          if (!tc_wait(sy, &c_done[j], (i >> 1) & 1)) break;
+          tma_store_3d(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k);
+          bulk_commit();
+          if (i + 2 < nt) {
+            if (!tc_wait(sy, &u_empty[j], (i >> 1) & 1)) break;
+            bulk_wait_read0();
+            mbar_arrive_expect_tx(&u_full[j], kUStage * 4u);
+            tma_load_3d(sU + j * kUStage, &tmU, (t_beg + i + 2) * kTcTile, b0, k, &u_full[j]);
+            last_load[j] = i + 2;
+          }
+        }
+        bulk_wait0();  // the stores are complete before the CTA exits
+        if (*s_abort) {
+          // let U copies still in flight land before the CTA exits
+          for (int j = 0; j < 2; ++j)
+            if (last_load[j] >= 0)
+              for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(&u_full[j], (last_load[j] >> 1) & 1); ++t) {
+              }
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1) {
       // ---------------------------------------------------------------- MMA issuer
       if (lane == 0) {
         const uint32_t idesc = (1u << 4)                       // D fp32
@@ -466,14 +505,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float inv_T = a.inv_T;
       const int b = bb + lane;  // this lane's request in the row phase
       const bool bok = b < a.B;
-      float* ldrow = a.ld + ((size_t)k * a.B + b) * a.V;
       bool bad = false;
       ChunkStat run = stat_empty();
       for (int i = 0; i < nt; ++i) {
         const int j = i & 1;
         const int acc = i & 1;
         const int v0w = (t_beg + i) * kTcTile + q * 32;  // this warp's 32 columns
-        const bool ok_u = tc_wait(sy, &u_full[ew * 2 + j], (i >> 1) & 1);
+        const bool ok_u = tc_wait(sy, &u_full[j], (i >> 1) & 1);
         const bool ok_t = __all_sync(0xffffffffu, tc_wait(sy, &t_full[acc], (i >> 1) & 1) && ok_u);
         float x[32];
         if (ok_t) {
@@ -483,24 +521,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&t_empty[acc]);
-        float* ub = ubuf + j * 1024;
+        // this warp's [32 requests x 32 columns] block of the stage (row stride 128 columns)
+        float* ub = sU + j * kUStage + (h * 32) * kTcTile + q * 32;
         if (ok_t) {
           // column phase: lane = column, row jj = request: l = U + bias in place
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) ub[jj * 32 + lane] += x[jj];
+          for (int jj = 0; jj < 32; ++jj) ub[jj * kTcTile + lane] += x[jj];
+          fence_proxy_async_smem();  // the TMA store reads these values
           __syncwarp();
+          if (lane == 0) mbar_arrive(&c_done[j]);
           // row phase: lane = request; rotated 16-byte chunks keep the eight lanes of each
           // shared-memory phase on distinct banks
           float lv[32];
 #pragma unroll
           for (int s4 = 0; s4 < 8; ++s4) {
             const int c = (lane + s4) & 7;
-            const float4 f = *reinterpret_cast<const float4*>(ub + lane * 32 + c * 4);
+            const float4 f = *reinterpret_cast<const float4*>(ub + lane * kTcTile + c * 4);
             lv[4 * s4 + 0] = f.x;
             lv[4 * s4 + 1] = f.y;
             lv[4 * s4 + 2] = f.z;
             lv[4 * s4 + 3] = f.w;
-            if (bok && v0w + c * 4 < a.V) __stcs(reinterpret_cast<float4*>(ldrow + v0w + c * 4), f);
           }
           const int nval = min(32, a.V - v0w);  // valid columns of this chunk (multiple of 8)
           ChunkStat st;
@@ -543,8 +583,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             stat_fold(run, st, a.greedy);
           }
         }
-        __syncwarp();  // every lane is done with this buffer: refill it with the tile after next
-        if (lane == 0 && i + 2 < nt) load_u(i + 2);
+        __syncwarp();  // every lane is done with this stage
+        if (lane == 0) mbar_arrive(&u_empty[j]);
       }
       // partition record: fold the four lane quadrants (through shared memory: the G region,
       // free once every MMA has completed, which the last accumulator wait guarantees)
@@ -859,7 +899,7 @@ dspark_status launch_draft(const DraftCall& c) {
     return DSPARK_ECUDA;
   }
 
-  CUtensorMap mW2, mU;
+  CUtensorMap mW2, mU, mLd;
   int n_bgroups = 1, cpg = 1, nb = 0;
   size_t tc_smem = 0;
   if (use_tc) {
@@ -878,12 +918,18 @@ dspark_status launch_draft(const DraftCall& c) {
       set_error("cuTensorMapEncodeTiled failed for W2");
       return DSPARK_ECUDA;
     }
-    // U is position-major [gamma][B][V]: a box is 32 columns of 32 requests at one position
+    // U and l_d are position-major [gamma][B][V]: a box is one 128-column tile of the nb
+    // requests of a group at one position (32 KB at nb = 64: large copies keep the copy
+    // engine near full bandwidth, where 4 KB copies were measured to stream at under half)
     uint64_t udims[3] = {(uint64_t)c.V, (uint64_t)c.B, (uint64_t)c.gamma};
     uint64_t ustrides[2] = {(uint64_t)c.V * 4, (uint64_t)c.B * c.V * 4};
-    uint32_t ubox[3] = {32, 32, 1};
+    uint32_t ubox[3] = {(uint32_t)kTcTile, (uint32_t)nb, 1};
     if (!make_map(&mU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(c.U), udims, ustrides, ubox, false)) {
       set_error("cuTensorMapEncodeTiled failed for U");
+      return DSPARK_ECUDA;
+    }
+    if (!make_map(&mLd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, c.ld_out, udims, ustrides, ubox, false)) {
+      set_error("cuTensorMapEncodeTiled failed for l_d");
       return DSPARK_ECUDA;
     }
     tc_smem = tc_layout(c.r, nb).total + 1024;
@@ -906,9 +952,11 @@ dspark_status launch_draft(const DraftCall& c) {
       const dim3 grid(cpg * n_bgroups), block(kTcThreads);
       const int hint = opt.draft_w2_hint;
       if (nb == 32)
-        rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, a, k, n_bgroups, cpg, hint);
+        rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, mLd, a, k, n_bgroups, cpg,
+                       hint);
       else
-        rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, a, k, n_bgroups, cpg, hint);
+        rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, mLd, a, k, n_bgroups, cpg,
+                       hint);
     } else if (c.w_dtype == DSPARK_BF16) {
       rc = launch_fma_bg<__nv_bfloat16>(a, k, c.stream, pdl_k);
     } else {
