@@ -25,6 +25,7 @@ Options& options() {
     if (const char* e = std::getenv("DSPARK_DRAFT_TC_MIN_B")) o.draft_tc_min_b = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_DRAFT_PATH")) o.draft_force_path = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_DRAFT_PDL")) o.draft_pdl = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_DRAFT_FUSED")) o.draft_fused = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_CLUSTER")) o.verify_cluster = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_PERSISTENT")) o.verify_persistent = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_STREAM")) o.verify_stream = std::atoi(e);
@@ -72,6 +73,7 @@ int dspark_set_option(const char* key, long value) {
   else if (!std::strcmp(key, "draft_path")) o.draft_force_path = (int)value;
   else if (!std::strcmp(key, "draft_pdl")) o.draft_pdl = (int)value;
   else if (!std::strcmp(key, "draft_w2_hint")) o.draft_w2_hint = (int)value;
+  else if (!std::strcmp(key, "draft_fused")) o.draft_fused = (int)value;
   else if (!std::strcmp(key, "verify_cluster")) o.verify_cluster = (int)value;
   else if (!std::strcmp(key, "verify_persistent")) o.verify_persistent = (int)value;
   else if (!std::strcmp(key, "verify_stream")) o.verify_stream = (int)value;

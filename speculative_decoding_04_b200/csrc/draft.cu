@@ -10,15 +10,16 @@
 //                 32-column chunk) softmax statistics (max, sum of exp) or greedy top-2.
 //                 Two variants: a CUDA-core GEMV for few requests (or fp32 weights) and a
 //                 tcgen05 tensor-core GEMM with TMA-staged W2 / U / l_d tiles.
-//   combine    -- per request: global max and normaliser from the chunk statistics (fp64),
-//                 exclusive scan to the chunk that crosses u * S, exact rescan of that one
-//                 chunk, x_k and the near-tie flag.
+//   combine    -- per request: global max and normaliser from the per-partition statistics
+//                 (fp64 sums), the partition that crosses u * S, a rescan of that partition's
+//                 stored logits for x_k and the near-tie flag.
 // The main pass of step k+1 prefetches its W2 / U tiles before waiting on step k's combine.
 
 #include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -37,8 +38,8 @@ struct DraftArgs {
   float* ld;
   const float* u_draft;
   uint32_t* flags;
-  ChunkStat* part;     // [nchunk][B]: per (32-column chunk, request) statistics
   ChunkStat* cpart;    // [np][B]: per (main-pass partition, request) statistics
+  __nv_bfloat16* gbuf; // [B][r]: W1 rows of the tokens just drafted (next step's B operand), or null
   uint32_t* status;
   int B, gamma, V, r, nchunk;
   float inv_T;
@@ -72,7 +73,7 @@ __device__ __forceinline__ ChunkStat stat_empty() { return ChunkStat{-INFINITY, 
 __device__ __forceinline__ float ex_shift(float z, float m) { return exp2f(__fmul_rn(__fsub_rn(z, m), kLog2e)); }
 
 __device__ __forceinline__ int prev_token(const DraftArgs& a, int b, int k, bool report) {
-  int prev = (k == 0) ? a.x0[b] : a.x_out[b * a.gamma + k - 1];
+  int prev = (k == 0) ? a.x0[b] : __ldcg(a.x_out + b * a.gamma + k - 1);  // may be this launch's
   if ((unsigned)prev >= (unsigned)a.V) {
     if (report) atomicOr(a.flags + b, DSPARK_FLAG_TOKEN_RANGE);
     prev = prev < 0 ? 0 : a.V - 1;
@@ -241,11 +242,7 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
     if ((val0 && (isnan(l0) || l0 == INFINITY)) || (val1 && (isnan(l1) || l1 == INFINITY)))
       atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
     const ChunkStat st = chunk_stat_pair(l0, l1, val0, val1, v, a.inv_T, a.greedy);
-    if ((tid & 15) == 0) {
-      const bool ok = chunk < a.nchunk;
-      if (ok) a.part[(size_t)chunk * a.B + b] = st;
-      s_stat[lchunk][bb] = ok ? st : stat_empty();
-    }
+    if ((tid & 15) == 0) s_stat[lchunk][bb] = chunk < a.nchunk ? st : stat_empty();
   }
   __syncthreads();
   if (tid < nb) {  // fold the CTA's 8 chunks into its partition record
@@ -296,7 +293,7 @@ __host__ __device__ inline TcLayout tc_layout(int r, int nb) {
   L.w2 = ((uint32_t)nb * (uint32_t)r * 2u + 1023u) & ~1023u;
   L.u = L.w2 + kTcStages * L.w2_stage_bytes;
   L.bars = L.u + 2u * (uint32_t)nb * kTcTile * 4u;  // two [nb requests x 128 columns] fp32 stages
-  L.misc = L.bars + 8u * (2 * kTcStages + 2 + 2 + 1 + 2 + 2 + 2);
+  L.misc = L.bars + 8u * (2 * kTcStages + 2 + 2 + 1 + 2 + 2 + 2 + 1);
   L.total = L.misc + 16u;
   return L;
 }
@@ -318,11 +315,83 @@ __device__ __forceinline__ bool tc_wait(const TcSync& s, uint64_t* bar, uint32_t
   return false;
 }
 
+// A group of nth threads (a multiple of 32, ranks tid = 0..nth-1) that synchronises with
+// __syncthreads (bar < 0) or with named barrier `bar`.
+struct Grp {
+  int tid, nth, bar;
+  __device__ __forceinline__ void sync() const {
+    if (bar < 0) __syncthreads();
+    else named_bar(bar, nth);
+  }
+};
+
+// Inclusive fp64 scan over the group in rank order; `total` gets the group's sum.  sh: >= 33 doubles.
+__device__ __forceinline__ double grp_incl_scan_d(double v, double* sh, const Grp& g, double& total) {
+  const int lane = g.tid & 31, w = g.tid >> 5, nw = g.nth >> 5;
+  v = warp_incl_scan_d(v);
+  if (lane == 31) sh[w] = v;
+  g.sync();
+  if (w == 0) {
+    double x = lane < nw ? sh[lane] : 0.0;
+    x = warp_incl_scan_d(x);
+    if (lane < nw) sh[lane] = x;
+  }
+  g.sync();
+  const double pre = w > 0 ? sh[w - 1] : 0.0;
+  total = sh[nw - 1];
+  g.sync();
+  return v + pre;
+}
+
+__device__ __forceinline__ float grp_max_f(float v, float* sh, const Grp& g) {
+  const int lane = g.tid & 31, w = g.tid >> 5, nw = g.nth >> 5;
+  v = warp_max(v);
+  if (lane == 0) sh[w] = v;
+  g.sync();
+  float r = sh[0];
+  for (int i = 1; i < nw; ++i) r = fmaxf(r, sh[i]);
+  g.sync();
+  return r;
+}
+
+// Grid-wide barrier of the multi-step launch (cooperative, so every CTA is resident): one thread
+// per CTA after a CTA-level barrier.  Bounded: gives up with the timeout status and the abort flag.
+__device__ __forceinline__ bool grid_sync(uint32_t* count, uint32_t* gen, uint32_t nblocks, uint32_t& epoch,
+                                          const TcSync& sy) {
+  if (*sy.abort) return false;
+  __threadfence();
+  const uint32_t target = ++epoch;
+  if (atomicAdd(count, 1u) == nblocks - 1) {
+    atomicExch(count, 0u);
+    __threadfence();
+    atomicExch(gen, target);
+    return true;
+  }
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (*reinterpret_cast<volatile uint32_t*>(gen) == target) {
+      __threadfence();
+      return true;
+    }
+    if ((i & 1023u) == 1023u && *sy.abort) return false;
+  }
+  *sy.abort = 1;
+  atomicOr(sy.status, (uint32_t)DSPARK_ETIMEOUT);
+  return false;
+}
+
+__device__ void combine_group(const DraftArgs& a, int k, int b, const Grp& g, double* sh);
+
+// Steps k0 .. k1-1 of the draft.  With fused = 0 the launch is one step and a separate combine
+// kernel samples its tokens; with fused = 1 (a cooperative launch, all CTAs resident) every step
+// ends with a grid barrier, the combine of that step inside the kernel (the epilogue warps take one
+// request each) and a second grid barrier, after which the next step gathers its W1 rows.  The
+// W2 and U streams run on across steps (tile counter gi = step * nt + tile), so the next step's
+// first tiles are already loaded when its gather finishes.
 template <int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
     draft_main_tc(const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmU,
-                  const __grid_constant__ CUtensorMap tmLd, DraftArgs a, int k, int n_bgroups, int ctas_per_group,
-                  int w2_hint) {
+                  const __grid_constant__ CUtensorMap tmLd, const __grid_constant__ CUtensorMap tmG, DraftArgs a,
+                  int k0, int k1, int n_bgroups, int ctas_per_group, int w2_hint, int fused) {
   constexpr int EPI_WARPS = NB / 8;  // 4 per 32-request column group
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -340,9 +409,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* u_full = mma_done + 1;  // [2] U stage landed
   uint64_t* u_empty = u_full + 2;   // [2] every epilogue warp is done reading the stage
   uint64_t* c_done = u_empty + 2;   // [2] every epilogue warp has written l = U + bias in place
+  uint64_t* g_full = c_done + 2;    // the B operand arrived by TMA from gbuf
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L.misc + 4);
   const TcSync sy{s_abort, a.status};
+  __shared__ double s_comb[72];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % n_bgroups;
@@ -352,6 +423,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int nt = t_end - t_beg;
   const int b0 = g * NB;
   const int ksteps = a.r / 16;
+  const int total = (k1 - k0) * nt;  // tiles of this CTA over the launch
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kTcStages; ++i) {
@@ -368,11 +440,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&u_empty[i], EPI_WARPS);
       mbar_init(&c_done[i], EPI_WARPS);
     }
+    mbar_init(g_full, 1);
     *s_abort = 0;
     fence_mbar_init();
     prefetch_tmap(&tmW2);
     prefetch_tmap(&tmU);
     prefetch_tmap(&tmLd);
+    if (a.gbuf) prefetch_tmap(&tmG);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, 2 * NB);
@@ -390,24 +464,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int bb = b0 + h * 32;
   constexpr uint32_t kUStage = (uint32_t)NB * kTcTile;  // floats of one U stage: [NB requests][128 columns]
   // U (an input of the call) for the first two tiles is requested before waiting for the previous
-  // kernel: one 128-column x NB-request box per tile
+  // kernel: one 128-column x NB-request box per tile.  With the L2 hint on, U and l_d (streamed
+  // once per step) are evict-first, so that W2 (read by every step) can stay in L2.
+  auto load_u = [&](int gi, uint64_t pol) {
+    const int j = gi & 1, ku = k0 + gi / nt, iu = gi % nt;
+    mbar_arrive_expect_tx(&u_full[j], kUStage * 4u);
+    if (w2_hint) tma_load_3d_hint(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j], pol);
+    else tma_load_3d(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j]);
+  };
   if (warp == 3 && lane == 0) {
-    for (int i = 0; i < 2 && i < nt; ++i) {
-      mbar_arrive_expect_tx(&u_full[i], kUStage * 4u);
-      tma_load_3d(sU + i * kUStage, &tmU, (t_beg + i) * kTcTile, b0, k, &u_full[i]);
-    }
+    const uint64_t pol = l2_policy_evict_first();
+    for (int gi = 0; gi < 2 && gi < total; ++gi) load_u(gi, pol);
   }
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // W2 is an input of the call: the ring fills before the previous kernel has finished.
+    // W2 is an input of the call: the ring fills before the previous kernel has finished, and
+    // across steps (the same tiles every step).
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_last();
       int issued = 0;
-      for (int i = 0; i < nt; ++i) {
-        const int v0 = (t_beg + i) * kTcTile;
-        const int s = i % kTcStages;
-        if (!tc_wait(sy, &w_empty[s], ((i / kTcStages) & 1) ^ 1)) break;
+      for (int gi = 0; gi < total; ++gi) {
+        const int v0 = (t_beg + gi % nt) * kTcTile;
+        const int s = gi % kTcStages;
+        if (!tc_wait(sy, &w_empty[s], ((gi / kTcStages) & 1) ^ 1)) break;
         uint8_t* st = sW + s * L.w2_stage_bytes;
         mbar_arrive_expect_tx(&w_full[s], L.w2_stage_bytes);
         if (w2_hint) {
@@ -417,7 +497,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tma_load_2d(st, &tmW2, v0, 0, &w_full[s]);
           tma_load_2d(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s]);
         }
-        issued = i + 1;
+        issued = gi + 1;
       }
       if (*s_abort) {
         // give the copies already issued a bounded chance to land before the CTA exits
@@ -427,177 +507,212 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   } else {
+    // All other warps walk the steps together: every named barrier below is reached by all of
+    // them on every step, also after a timeout (the waits then return at once).
     pdl_wait();
-    // ---------------------------------------------------------------- gather B = W1[x_{k-1}] rows
-    {
-      const int cpr = a.r / 8;  // 16-byte chunks per row
-      const __nv_bfloat16* W1 = static_cast<const __nv_bfloat16*>(a.W1);
-      for (int i = threadIdx.x - 32; i < NB * cpr; i += kTcThreads - 32) {
-        const int row = i / cpr, c = i - row * cpr;
-        const int b = b0 + row;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (b < a.B)
-          val = __ldg(reinterpret_cast<const uint4*>(W1 + (size_t)prev_token(a, b, k, c == 0) * a.r + c * 8));
-        const int kb = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(sG + kb * (NB * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = val;
+    uint32_t epoch = 0;
+    uint32_t* gcount = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.status) + 64);
+    uint32_t* ggen = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.status) + 128);
+    bool bad = false;
+    int last_load[2] = {total > 0 ? 0 : -1, total > 1 ? 1 : -1};  // (warp 3) last tile loaded into each U stage
+    for (int k = k0; k < k1; ++k) {
+      const int gbase = (k - k0) * nt;
+      // ---------------------------------------------------------------- B operand = W1[x_{k-1}] rows
+      // Step 0 gathers the rows of x0; later steps load the rows the previous combine copied to
+      // gbuf, with r/64 TMA boxes of [NB rows x 64 columns] (the same 128-byte swizzled K-major
+      // layout as the gather writes).
+      const bool tma_g = a.gbuf != nullptr && k > 0;
+      if (!tma_g) {
+        const int cpr = a.r / 8;  // 16-byte chunks per row
+        const __nv_bfloat16* W1 = static_cast<const __nv_bfloat16*>(a.W1);
+        for (int i = threadIdx.x - 32; i < NB * cpr; i += kTcThreads - 32) {
+          const int row = i / cpr, c = i - row * cpr;
+          const int b = b0 + row;
+          uint4 val = make_uint4(0u, 0u, 0u, 0u);
+          if (b < a.B)
+            val = __ldg(reinterpret_cast<const uint4*>(W1 + (size_t)prev_token(a, b, k, c == 0) * a.r + c * 8));
+          const int kb = c >> 3, cc = c & 7;
+          *reinterpret_cast<uint4*>(sG + kb * (NB * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = val;
+        }
+        fence_proxy_async_smem();
+      } else if (warp == 1 && lane == 0) {
+        fence_proxy_async_smem();  // earlier generic accesses to the G region come first
+        mbar_arrive_expect_tx(g_full, (uint32_t)NB * a.r * 2u);
+        for (int kb = 0; kb < a.r / 64; ++kb) tma_load_2d(sG + kb * (NB * 128), &tmG, kb * 64, b0, g_full);
       }
-      fence_proxy_async_smem();
       named_bar(1, kTcThreads - 32);
-    }
-    if (warp == 3) {
-      // ---------------------------------------------------------------- U refills and l_d stores
-      // l_d = U + bias is written in place in the U stage by the epilogue; one TMA store per tile
-      // writes it out, and the stage is refilled with the U tile two ahead once the store has
-      // read it and every epilogue warp is done with it.
-      if (lane == 0) {
-        int last_load[2] = {nt > 0 ? 0 : -1, nt > 1 ? 1 : -1};  // last tile loaded into each stage
-        for (int i = 0; i < nt; ++i) {
-          const int j = i & 1;
-          if (!tc_wait(sy, &c_done[j], (i >> 1) & 1)) break;
-          tma_store_3d(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k);
-          bulk_commit();
-          if (i + 2 < nt) {
-            if (!tc_wait(sy, &u_empty[j], (i >> 1) & 1)) break;
-            bulk_wait_read0();
-            mbar_arrive_expect_tx(&u_full[j], kUStage * 4u);
-            tma_load_3d(sU + j * kUStage, &tmU, (t_beg + i + 2) * kTcTile, b0, k, &u_full[j]);
-            last_load[j] = i + 2;
+      if (warp == 3) {
+        // ---------------------------------------------------------------- U refills and l_d stores
+        // l_d = U + bias is written in place in the U stage by the epilogue; one TMA store per tile
+        // writes it out, and the stage is refilled with the U tile two ahead (possibly of the next
+        // step) once the store has read it and every epilogue warp is done with it.
+        if (lane == 0) {
+          const uint64_t pol = l2_policy_evict_first();
+          for (int i = 0; i < nt; ++i) {
+            const int gi = gbase + i, j = gi & 1;
+            if (!tc_wait(sy, &c_done[j], (gi >> 1) & 1)) break;
+            if (w2_hint) tma_store_3d_hint(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k, pol);
+            else tma_store_3d(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k);
+            bulk_commit();
+            if (gi + 2 < total) {
+              if (!tc_wait(sy, &u_empty[j], (gi >> 1) & 1)) break;
+              bulk_wait_read0();
+              load_u(gi + 2, pol);
+              last_load[j] = gi + 2;
+            }
           }
+          bulk_wait0();     // this step's l_d is written before anyone samples from it
+          __threadfence();
         }
-        bulk_wait0();  // the stores are complete before the CTA exits
-        if (*s_abort) {
-          // let U copies still in flight land before the CTA exits
-          for (int j = 0; j < 2; ++j)
-            if (last_load[j] >= 0)
-              for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(&u_full[j], (last_load[j] >> 1) & 1); ++t) {
-              }
-        }
-      }
-      __syncwarp();
-    } else if (warp == 1) {
-      // ---------------------------------------------------------------- MMA issuer
-      if (lane == 0) {
-        const uint32_t idesc = (1u << 4)                       // D fp32
-                               | (1u << 7) | (1u << 10)        // A, B bf16
-                               | (1u << 15)                    // A MN-major (W2 is [r][V])
-                               | ((uint32_t)(NB >> 3) << 17)   // N
-                               | ((uint32_t)(128 >> 4) << 24);  // M
-        const uint32_t g_addr = smem_u32(sG), w_addr = smem_u32(sW);
-        for (int i = 0; i < nt; ++i) {
-          const int acc = i & 1, s = i % kTcStages;
-          if (!tc_wait(sy, &t_empty[acc], ((i >> 1) & 1) ^ 1)) break;
-          if (!tc_wait(sy, &w_full[s], (i / kTcStages) & 1)) break;
-          tc_fence_after();
-          const uint32_t wst = w_addr + s * L.w2_stage_bytes;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t ad = smem_desc(wst + kk * 2048u, L.w2_stage_bytes / 2, 1024u, 2u);
-            const uint64_t bd = smem_desc(g_addr + (kk >> 2) * (NB * 128u) + (kk & 3) * 32u, 16u, 1024u, 2u);
-            tc_mma_f16(tmem_base + acc * NB, ad, bd, idesc, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&w_empty[s]);
-          tc_commit(&t_full[acc]);
-        }
-        tc_commit(mma_done);
-      }
-      __syncwarp();
-    } else if (epi) {
-      // ---------------------------------------------------------------- epilogue
-      const float inv_T = a.inv_T;
-      const int b = bb + lane;  // this lane's request in the row phase
-      const bool bok = b < a.B;
-      bool bad = false;
-      ChunkStat run = stat_empty();
-      for (int i = 0; i < nt; ++i) {
-        const int j = i & 1;
-        const int acc = i & 1;
-        const int v0w = (t_beg + i) * kTcTile + q * 32;  // this warp's 32 columns
-        const bool ok_u = tc_wait(sy, &u_full[j], (i >> 1) & 1);
-        const bool ok_t = __all_sync(0xffffffffu, tc_wait(sy, &t_full[acc], (i >> 1) & 1) && ok_u);
-        float x[32];
-        if (ok_t) {
-          tc_fence_after();
-          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * NB + h * 32, x);
-        }
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&t_empty[acc]);
-        // this warp's [32 requests x 32 columns] block of the stage (row stride 128 columns)
-        float* ub = sU + j * kUStage + (h * 32) * kTcTile + q * 32;
-        if (ok_t) {
-          // column phase: lane = column, row jj = request: l = U + bias in place
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) ub[jj * kTcTile + lane] += x[jj];
-          fence_proxy_async_smem();  // the TMA store reads these values
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&c_done[j]);
-          // row phase: lane = request; rotated 16-byte chunks keep the eight lanes of each
-          // shared-memory phase on distinct banks
-          float lv[32];
-#pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4) {
-            const int c = (lane + s4) & 7;
-            const float4 f = *reinterpret_cast<const float4*>(ub + lane * kTcTile + c * 4);
-            lv[4 * s4 + 0] = f.x;
-            lv[4 * s4 + 1] = f.y;
-            lv[4 * s4 + 2] = f.z;
-            lv[4 * s4 + 3] = f.w;
+      } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+          const uint32_t idesc = (1u << 4)                       // D fp32
+                                 | (1u << 7) | (1u << 10)        // A, B bf16
+                                 | (1u << 15)                    // A MN-major (W2 is [r][V])
+                                 | ((uint32_t)(NB >> 3) << 17)   // N
+                                 | ((uint32_t)(128 >> 4) << 24);  // M
+          const uint32_t g_addr = smem_u32(sG), w_addr = smem_u32(sW);
+          // the n-th TMA load of the B operand in this launch completes phase n of g_full
+          const bool g_ok = !tma_g || tc_wait(sy, g_full, (uint32_t)(k - max(k0, 1)) & 1u);
+          for (int i = 0; g_ok && i < nt; ++i) {
+            const int gi = gbase + i, acc = gi & 1, s = gi % kTcStages;
+            if (!tc_wait(sy, &t_empty[acc], ((gi >> 1) & 1) ^ 1)) break;
+            if (!tc_wait(sy, &w_full[s], (gi / kTcStages) & 1)) break;
+            tc_fence_after();
+            const uint32_t wst = w_addr + s * L.w2_stage_bytes;
+            for (int kk = 0; kk < ksteps; ++kk) {
+              const uint64_t ad = smem_desc(wst + kk * 2048u, L.w2_stage_bytes / 2, 1024u, 2u);
+              const uint64_t bd = smem_desc(g_addr + (kk >> 2) * (NB * 128u) + (kk & 3) * 32u, 16u, 1024u, 2u);
+              tc_mma_f16(tmem_base + acc * NB, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&w_empty[s]);
+            tc_commit(&t_full[acc]);
           }
-          const int nval = min(32, a.V - v0w);  // valid columns of this chunk (multiple of 8)
-          ChunkStat st;
-          if (a.greedy) {
-            Top2 t{-INFINITY, -1, -INFINITY};
+        }
+        __syncwarp();
+      } else if (epi) {
+        // ---------------------------------------------------------------- epilogue
+        const float inv_T = a.inv_T;
+        const int b = bb + lane;  // this lane's request in the row phase
+        const bool bok = b < a.B;
+        ChunkStat run = stat_empty();
+        for (int i = 0; i < nt; ++i) {
+          const int gi = gbase + i, j = gi & 1, acc = gi & 1;
+          const int v0w = (t_beg + i) * kTcTile + q * 32;  // this warp's 32 columns
+          const bool ok_u = tc_wait(sy, &u_full[j], (gi >> 1) & 1);
+          const bool ok_t = __all_sync(0xffffffffu, tc_wait(sy, &t_full[acc], (gi >> 1) & 1) && ok_u);
+          float x[32];
+          if (ok_t) {
+            tc_fence_after();
+            tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * NB + h * 32, x);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&t_empty[acc]);
+          // this warp's [32 requests x 32 columns] block of the stage (row stride 128 columns)
+          float* ub = sU + j * kUStage + (h * 32) * kTcTile + q * 32;
+          if (ok_t) {
+            // column phase: lane = column, row jj = request: l = U + bias in place
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) ub[jj * kTcTile + lane] += x[jj];
+            fence_proxy_async_smem();  // the TMA store reads these values
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&c_done[j]);
+            // row phase: lane = request; rotated 16-byte chunks keep the eight lanes of each
+            // shared-memory phase on distinct banks
+            float lv[32];
 #pragma unroll
             for (int s4 = 0; s4 < 8; ++s4) {
               const int c = (lane + s4) & 7;
+              const float4 f = *reinterpret_cast<const float4*>(ub + lane * kTcTile + c * 4);
+              lv[4 * s4 + 0] = f.x;
+              lv[4 * s4 + 1] = f.y;
+              lv[4 * s4 + 2] = f.z;
+              lv[4 * s4 + 3] = f.w;
+            }
+            const int nval = min(32, a.V - v0w);  // valid columns of this chunk (multiple of 8)
+            ChunkStat st;
+            if (a.greedy) {
+              Top2 t{-INFINITY, -1, -INFINITY};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int col = c * 4 + e;
-                const float l = lv[4 * s4 + e];
-                if (col < nval) {
-                  bad |= isnan(l) || l == INFINITY;
-                  const Top2 o{l, v0w + col, -INFINITY};
-                  t = top2_merge(t, o);
+              for (int s4 = 0; s4 < 8; ++s4) {
+                const int c = (lane + s4) & 7;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int col = c * 4 + e;
+                  const float l = lv[4 * s4 + e];
+                  if (col < nval) {
+                    bad |= isnan(l) || l == INFINITY;
+                    const Top2 o{l, v0w + col, -INFINITY};
+                    t = top2_merge(t, o);
+                  }
                 }
               }
-            }
-            st = ChunkStat{t.best, 0.f, t.idx, t.second};
-          } else {
-            float mx = -INFINITY;
+              st = ChunkStat{t.best, 0.f, t.idx, t.second};
+            } else {
+              float mx = -INFINITY;
 #pragma unroll
-            for (int s4 = 0; s4 < 8; ++s4) {
-              const int c = (lane + s4) & 7;
+              for (int s4 = 0; s4 < 8; ++s4) {
+                const int c = (lane + s4) & 7;
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                lv[4 * s4 + e] = (c * 4 + e < nval) ? __fmul_rn(lv[4 * s4 + e], inv_T) : -INFINITY;  // z
-                mx = fmaxf(mx, lv[4 * s4 + e]);
+                for (int e = 0; e < 4; ++e) {
+                  lv[4 * s4 + e] = (c * 4 + e < nval) ? __fmul_rn(lv[4 * s4 + e], inv_T) : -INFINITY;  // z
+                  mx = fmaxf(mx, lv[4 * s4 + e]);
+                }
               }
-            }
-            float sm = 0.f;
+              float sm = 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) sm += (lv[e] == -INFINITY) ? 0.f : ex_shift(lv[e], mx);
-            bad |= isnan(sm) || mx == INFINITY;
-            st = ChunkStat{mx, sm, 0, 0.f};
+              for (int e = 0; e < 32; ++e) sm += (lv[e] == -INFINITY) ? 0.f : ex_shift(lv[e], mx);
+              bad |= isnan(sm) || mx == INFINITY;
+              st = ChunkStat{mx, sm, 0, 0.f};
+            }
+            if (v0w < a.V) stat_fold(run, st, a.greedy);
           }
-          if (v0w < a.V) {
-            if (bok) a.part[(size_t)(v0w >> 5) * a.B + b] = st;
-            stat_fold(run, st, a.greedy);
-          }
+          __syncwarp();  // every lane is done with this stage
+          if (lane == 0) mbar_arrive(&u_empty[j]);
         }
-        __syncwarp();  // every lane is done with this stage
-        if (lane == 0) mbar_arrive(&u_empty[j]);
+        // partition record: fold the four lane quadrants (through shared memory: the G region,
+        // free once every MMA of the step has completed, which the last accumulator wait
+        // guarantees)
+        ChunkStat* comb = reinterpret_cast<ChunkStat*>(sG);
+        comb[q * NB + h * 32 + lane] = run;
+        named_bar(2, EPI_WARPS * 32);
+        if (q == 0 && bok) {
+          ChunkStat r = comb[h * 32 + lane];
+          for (int qq = 1; qq < 4; ++qq) stat_fold(r, comb[qq * NB + h * 32 + lane], a.greedy);
+          a.cpart[(size_t)jc * a.B + b] = r;
+        }
+        fence_proxy_async_smem();      // the next B operand arrives in the G region by TMA
+        named_bar(2, EPI_WARPS * 32);  // the G region is read before anyone reuses it
       }
-      // partition record: fold the four lane quadrants (through shared memory: the G region,
-      // free once every MMA has completed, which the last accumulator wait guarantees)
-      ChunkStat* comb = reinterpret_cast<ChunkStat*>(sG);
-      comb[q * NB + h * 32 + lane] = run;
-      named_bar(2, EPI_WARPS * 32);
-      if (q == 0 && bok) {
-        ChunkStat r = comb[h * 32 + lane];
-        for (int qq = 1; qq < 4; ++qq) stat_fold(r, comb[qq * NB + h * 32 + lane], a.greedy);
-        a.cpart[(size_t)jc * a.B + b] = r;
+      if (fused) {
+        // ---------------------------------------------------------------- sample this step
+        named_bar(3, kTcThreads - 32);
+        if (warp == 1 && lane == 0) grid_sync(gcount, ggen, gridDim.x, epoch, sy);
+        named_bar(3, kTcThreads - 32);
+        // one request per CTA at a time, all non-producer warps together
+        // (no test of the abort flag here: every thread of the group must take the same path)
+        for (int rq = blockIdx.x; rq < a.B; rq += gridDim.x)
+          combine_group(a, k, rq, Grp{(int)threadIdx.x - 32, kTcThreads - 32, 4}, s_comb);
+        named_bar(3, kTcThreads - 32);
+        if (warp == 1 && lane == 0) grid_sync(gcount, ggen, gridDim.x, epoch, sy);
+        named_bar(3, kTcThreads - 32);
       }
-      if (bad && bok) atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
     }
+    if (epi) {
+      const int b = bb + lane;
+      if (bad && b < a.B) atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
+    }
+    if (warp == 3 && lane == 0 && *s_abort) {
+      // let U copies still in flight land before the CTA exits
+      for (int j = 0; j < 2; ++j)
+        if (last_load[j] >= 0)
+          for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(&u_full[j], (last_load[j] >> 1) & 1); ++t) {
+          }
+    }
+    if (warp == 1 && lane == 0) tc_commit(mma_done);
   }
   __syncthreads();
   if (warp == 2) {
@@ -613,168 +728,202 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // ============================================================================ combine + sample
 //
-// One warp per request, three short levels, all weights relative to the row maximum M:
+// One warp per request, two short levels, all weights exp(z - M) relative to the row maximum M:
 //   1  the np partition records -> M, S and the partition holding u*S (fp64 warp scan over
 //      contiguous ranges of records, exact partition of [0, S));
-//   2  that partition's chunk records -> the chunk holding u*S;
-//   3  that chunk's 32 stored logits, exp in fp64 -> the token (and the near-tie flag).
+//   2  that partition's stored logits (about 1000 columns, each lane a contiguous run) -> the
+//      token (and the near-tie flag).  The main passes keep no finer records: one more
+//      dependent level cost more than the rescan.
 // Greedy: the partition records already carry the argmax (lowest index) and the runner-up.
-constexpr int kCombWarps = 4;
 
-// Warp-cooperative search of `t` in the running sum of w[0..n) (lane l owns the contiguous
-// range [l*per, min(n, (l+1)*per)), element weights from `wf`).  Returns the index (or -1),
-// writes its interval [lo, hi) in the running sum started at `base`.
-template <typename WF>
-__device__ __forceinline__ int warp_crossing(int n, double base, double t, WF wf, double& lo, double& hi) {
-  const int lane = threadIdx.x & 31;
-  const int per = (n + 31) / 32;
-  const int i0 = min(n, lane * per), i1 = min(n, i0 + per);
-  double ts = 0.0;
-  for (int i = i0; i < i1; ++i) ts += wf(i);
-  const double incl = warp_incl_scan_d(ts);
-  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
-  if (lane == 0) excl = 0.0;
-  const double pre = base + excl, nxt = base + incl;
-  const bool last_nonempty = (i0 < i1) && (i1 == n);
-  const bool mine = (i0 < i1) && pre <= t && (t < nxt || last_nonempty);
-  int pick = -1;
-  double plo = 0.0, phi = 0.0;
-  if (mine) {
-    double R = pre, Rlast = pre, wlast = 0.0;
-    int last = -1;
-    for (int i = i0; i < i1; ++i) {
-      const double w = wf(i);
-      if (w > 0.0) {
-        last = i;
-        Rlast = R;
-        wlast = w;
-        if (t < R + w) {
-          pick = i;
-          plo = R;
-          phi = R + w;
-          break;
-        }
-      }
-      R += w;
-    }
-    if (pick < 0 && last >= 0) {
-      pick = last;
-      plo = Rlast;
-      phi = Rlast + wlast;
-    }
-  }
-  const unsigned who = __ballot_sync(0xffffffffu, mine && pick >= 0);
-  if (!who) return -1;
-  const int src = __ffs(who) - 1;
-  lo = __shfl_sync(0xffffffffu, plo, src);
-  hi = __shfl_sync(0xffffffffu, phi, src);
-  return __shfl_sync(0xffffffffu, pick, src);
+__device__ __forceinline__ ChunkStat ld_stat_cg(const ChunkStat* p) {
+  const float4 v = __ldcg(reinterpret_cast<const float4*>(p));
+  return ChunkStat{v.x, v.y, __float_as_int(v.z), v.w};
 }
 
-__global__ void __launch_bounds__(kCombWarps * 32) draft_combine(DraftArgs a, int k) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.x * kCombWarps + warp;
-  pdl_trigger();
-  pdl_wait();
-  if (b >= a.B) return;
+// Combine of one request by a whole group of threads (one element per thread per level, scans
+// in fp64): partitions -> M, S and the partition holding u*S; that partition's stored logits ->
+// the token x_k (and the near-tie flag).  Weights are exp(z - M) through exp2, as in the main
+// passes.  Records and logits are read through L2 (ld.global.cg): in the multi-step launch other
+// CTAs wrote them during this kernel.  The group then copies W1[x_k] into row b of `gbuf`
+// (the next step's B operand) when gbuf is given.  sh: >= 72 doubles of shared memory.
+__device__ void combine_group(const DraftArgs& a, int k, int b, const Grp& g, double* sh) {
   const size_t B = (size_t)a.B;
-  const int np = a.np;
+  const int np = a.np, nth = g.nth, tid = g.tid;
+  double* shs = sh;                                   // scan scratch (33)
+  float* shf = reinterpret_cast<float*>(sh + 34);     // max scratch (32 floats = 16 doubles)
+  int* shi = reinterpret_cast<int*>(sh + 52);         // [0] pick, [1] token, [2] flags
+  double* shd = sh + 56;                              // [0] lo of the pick, [1] hi
+  const float u = __ldg(a.u_draft + b * a.gamma + k);  // requested before the first dependent load
+  if (tid == 0) shi[0] = -1;
 
   if (a.greedy) {
     Top2 t{-INFINITY, -1, -INFINITY};
-    for (int p = lane; p < np; p += 32) {
-      const ChunkStat s = a.cpart[p * B + b];
+    for (int p = tid; p < np; p += nth) {
+      const ChunkStat s = ld_stat_cg(a.cpart + p * B + b);
       t = top2_merge(t, Top2{s.m, s.idx, s.m2});
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t = top2_merge(t, top2_shfl_xor(t, o));
-    if (lane == 0) {
-      int x = t.idx;
+    Top2* sht = reinterpret_cast<Top2*>(sh);
+    if ((tid & 31) == 0) sht[tid >> 5] = t;
+    g.sync();
+    if (tid == 0) {
+      Top2 r = sht[0];
+      for (int i = 1; i < nth / 32; ++i) r = top2_merge(r, sht[i]);
+      int x = r.idx;
+      uint32_t fl = 0;
       if (x < 0 || x >= a.V) {
-        atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
+        fl |= DSPARK_FLAG_NONFINITE;
         x = min(max(x, 0), a.V - 1);
       }
-      if (t.best - t.second <= 1e-6f * fmaxf(1.f, fabsf(t.best))) atomicOr(a.flags + b, DSPARK_FLAG_DRAFT_NEAR_TIE);
+      if (r.best - r.second <= 1e-6f * fmaxf(1.f, fabsf(r.best))) fl |= DSPARK_FLAG_DRAFT_NEAR_TIE;
+      if (fl) atomicOr(a.flags + b, fl);
       a.x_out[b * a.gamma + k] = x;
+      shi[1] = x;
     }
-    return;
-  }
-
-  // level 1: partitions
-  float mloc = -INFINITY;
-  for (int p = lane; p < np; p += 32) mloc = fmaxf(mloc, a.cpart[p * B + b].m);
-  const float M = warp_max(mloc);
-  const double Md = (double)M;
-  auto w1 = [&](int p) -> double {
-    const ChunkStat s = a.cpart[p * B + b];
-    return s.m == -INFINITY ? 0.0 : (double)s.s * (double)ex_shift(s.m, M);
-  };
-  double S = 0.0;
-  {
-    const int per = (np + 31) / 32;
-    const int i0 = min(np, lane * per), i1 = min(np, i0 + per);
-    double ts = 0.0;
-    for (int i = i0; i < i1; ++i) ts += w1(i);
-    S = __shfl_sync(0xffffffffu, warp_incl_scan_d(ts), 31);
-  }
-  const double t = (double)a.u_draft[b * a.gamma + k] * S;
-  double lo1 = 0.0, hi1 = 0.0;
-  const int p = warp_crossing(np, 0.0, t, w1, lo1, hi1);
-  int x = 0;
-  uint32_t fl = 0;
-  if (p < 0 || !(S > 0.0) || !isfinite(S)) {
-    fl |= DSPARK_FLAG_NONFINITE;
+    g.sync();
   } else {
-    // level 2: chunks of partition p
-    const int t0 = (int)((long long)p * a.ntiles / np), t1 = (int)((long long)(p + 1) * a.ntiles / np);
-    const int c0 = t0 * a.tile_chunks, c1 = min(a.nchunk, t1 * a.tile_chunks);
-    auto w2 = [&](int i) -> double {
-      const ChunkStat s = a.part[(size_t)(c0 + i) * B + b];
+    // ---- level 1: each thread a contiguous run of partition records
+    const int e1 = (np + nth - 1) / nth;
+    const int i0 = min(np, tid * e1), i1 = min(np, i0 + e1);
+    float ml = -INFINITY;
+    for (int i = i0; i < i1; ++i) ml = fmaxf(ml, ld_stat_cg(a.cpart + (size_t)i * B + b).m);
+    const float M = grp_max_f(ml, shf, g);
+    auto w1 = [&](int i) -> double {
+      const ChunkStat s = ld_stat_cg(a.cpart + (size_t)i * B + b);
       return s.m == -INFINITY ? 0.0 : (double)s.s * (double)ex_shift(s.m, M);
     };
-    double lo2 = 0.0, hi2 = 0.0;
-    int c = warp_crossing(c1 - c0, lo1, t, w2, lo2, hi2);
-    if (c < 0) {  // rounding: fall back to the partition's last chunk with weight
-      c = c1 - c0 - 1;
-      while (c > 0 && w2(c) <= 0.0) --c;
-      lo2 = hi2 = t;
+    double own = 0.0;
+    for (int i = i0; i < i1; ++i) own += w1(i);
+    double S = 0.0;
+    const double incl = grp_incl_scan_d(own, shs, g, S);
+    const double t = (double)u * S;
+    {
+      const double excl = incl - own;
+      if (i0 < i1 && excl <= t && (t < incl || i1 == np)) {
+        double R = excl;
+        int pick = -1, last = -1;
+        double plo = 0.0, lastlo = 0.0;
+        for (int i = i0; i < i1; ++i) {
+          const double w = w1(i);
+          if (w > 0.0) {
+            last = i;
+            lastlo = R;
+            if (t < R + w) {
+              pick = i;
+              plo = R;
+              break;
+            }
+          }
+          R += w;
+        }
+        if (pick < 0) {
+          pick = last;
+          plo = lastlo;
+        }
+        if (pick >= 0) {
+          shi[0] = pick;
+          shd[0] = plo;
+        }
+      }
     }
-    c += c0;
-    // level 3: the chunk's 32 logits
-    const int v = c * kChunk + lane;
-    const bool valid = v < a.V;
-    const float* row = a.ld + ((size_t)k * a.B + b) * a.V;
-    const float z = valid ? __fmul_rn(row[v], a.inv_T) : -INFINITY;
-    const double e = valid ? exp((double)z - Md) : 0.0;
-    const double inc = warp_incl_scan_d(e);
-    const double upper = lo2 + inc, lower = upper - e;
-    const unsigned cross = __ballot_sync(0xffffffffu, valid && e > 0.0 && t < upper);
-    int pick;
-    if (cross) {
-      pick = __ffs(cross) - 1;
+    g.sync();
+    const int p = shi[0];
+    const double lo1 = shd[0];
+    g.sync();
+    if (p < 0 || !(S > 0.0) || !isfinite(S)) {
+      if (tid == 0) {
+        atomicOr(a.flags + b, DSPARK_FLAG_NONFINITE);
+        a.x_out[b * a.gamma + k] = 0;
+        shi[1] = 0;
+      }
     } else {
-      const unsigned pos = __ballot_sync(0xffffffffu, valid && e > 0.0);
-      pick = pos ? 31 - __clz(pos) : 0;
+      // ---- level 2: the partition's stored logits, each thread a contiguous run of columns
+      const int t0 = (int)((long long)p * a.ntiles / np), t1 = (int)((long long)(p + 1) * a.ntiles / np);
+      const int tw = a.tile_chunks * kChunk;
+      const int v0 = t0 * tw, n = min(t1 * tw, a.V) - v0;
+      const float* row = a.ld + ((size_t)k * a.B + b) * a.V + v0;
+      const float inv_T = a.inv_T;
+      auto w2 = [&](int j) -> double {
+        const float z = __fmul_rn(__ldcg(row + j), inv_T);
+        return z == -INFINITY ? 0.0 : (double)ex_shift(z, M);
+      };
+      const int e2 = (n + nth - 1) / nth;
+      const int j0 = min(n, tid * e2), j1 = min(n, j0 + e2);
+      double own2 = 0.0;
+      for (int j = j0; j < j1; ++j) own2 += w2(j);
+      double tot2 = 0.0;
+      const double incl2 = lo1 + grp_incl_scan_d(own2, shs, g, tot2);
+      const double excl2 = incl2 - own2;
+      if (tid == 0) shi[1] = -1;
+      g.sync();
+      if (j0 < j1 && excl2 <= t && (t < incl2 || j1 == n)) {
+        double R = excl2;
+        int pick = -1, last = -1;
+        double plo = 0.0, phi = 0.0;
+        for (int j = j0; j < j1; ++j) {
+          const double w = w2(j);
+          if (w > 0.0) {
+            last = j;
+            if (t < R + w) {
+              pick = j;
+              plo = R;
+              phi = R + w;
+              break;
+            }
+          }
+          R += w;
+        }
+        if (pick < 0 && last >= 0) {
+          pick = last;
+          plo = phi = t;  // rounding left u*S past the partition: a boundary, flagged
+        }
+        if (pick >= 0) {
+          shi[1] = v0 + pick;
+          uint32_t fl = 0;
+          if ((t - plo) < 1e-6 * S || (phi - t) < 1e-6 * S) fl |= DSPARK_FLAG_DRAFT_NEAR_TIE;
+          shi[2] = (int)fl;
+        }
+      }
+      g.sync();
+      if (tid == 0) {
+        int x = shi[1];
+        uint32_t fl = x >= 0 ? (uint32_t)shi[2] : (uint32_t)DSPARK_FLAG_NONFINITE;
+        x = min(max(x, 0), a.V - 1);
+        if (fl) atomicOr(a.flags + b, fl);
+        a.x_out[b * a.gamma + k] = x;
+        shi[1] = x;
+      }
     }
-    const double plo = __shfl_sync(0xffffffffu, lower, pick), phi = __shfl_sync(0xffffffffu, upper, pick);
-    x = min(c * kChunk + pick, a.V - 1);
-    if ((t - plo) < 1e-6 * S || (phi - t) < 1e-6 * S) fl |= DSPARK_FLAG_DRAFT_NEAR_TIE;
+    g.sync();
   }
-  if (lane == 0) {
-    if (fl) atomicOr(a.flags + b, fl);
-    a.x_out[b * a.gamma + k] = x;
+  // the next step's B operand row: W1[x_k] (bf16 weights only)
+  if (a.gbuf && k + 1 < a.gamma) {
+    const int x = shi[1];
+    const int cpr = a.r / 8;  // 16-byte chunks per row
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.W1) + (size_t)x * a.r);
+    uint4* dst = reinterpret_cast<uint4*>(a.gbuf + (size_t)b * a.r);
+    for (int c = tid; c < cpr; c += nth) dst[c] = __ldg(src + c);
   }
+  g.sync();
+}
+
+// Combine kernel of the per-step launches: one CTA of kCombThreads per request.
+constexpr int kCombThreads = 512;
+__global__ void __launch_bounds__(kCombThreads) draft_combine(DraftArgs a, int k) {
+  __shared__ double sh[72];
+  pdl_trigger();
+  pdl_wait();
+  combine_group(a, k, blockIdx.x, Grp{(int)threadIdx.x, kCombThreads, -1}, sh);
 }
 
 // ============================================================================ host side
 
 size_t draft_workspace_bytes(int B, int gamma, int V, int r) {
   (void)gamma;
-  (void)r;
-  const size_t nchunk = (size_t)(V + kChunk - 1) / kChunk;
-  const size_t np_max = std::max<size_t>((size_t)(V + 255) / 256, 1024);
-  return kWsHeader + align_up((size_t)B * nchunk * sizeof(ChunkStat), 256) +
-         align_up((size_t)B * np_max * sizeof(ChunkStat), 256);
+  const size_t np_max = std::max<size_t>((size_t)(V + 255) / 256, 1024);  // partitions (either main pass)
+  return kWsHeader + align_up((size_t)B * np_max * sizeof(ChunkStat), 256) + align_up((size_t)B * r * 2, 256);
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -802,18 +951,23 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, void* bas
 }
 
 template <typename K, typename... Args>
-static cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+static cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl, bool coop,
                              Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   int na = 0;
   if (pdl) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (coop) {  // all CTAs resident at once (the launch fails otherwise)
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
     ++na;
   }
   cfg.attrs = attr;
@@ -834,7 +988,7 @@ static cudaError_t launch_fma(const DraftArgs& a, int k, cudaStream_t st, bool p
   }
   if (attr_rc != cudaSuccess) return attr_rc;
   dim3 grid((a.V + 255) / 256, (a.B + BG - 1) / BG);
-  return launch_ex(kern, grid, dim3(128), smem, st, pdl, a, k, vec_ok);
+  return launch_ex(kern, grid, dim3(128), smem, st, pdl, false, a, k, vec_ok);
 }
 
 template <typename WT>
@@ -873,9 +1027,12 @@ dspark_status launch_draft(const DraftCall& c) {
   a.V = c.V;
   a.r = c.r;
   a.nchunk = (c.V + kChunk - 1) / kChunk;
-  a.part = reinterpret_cast<ChunkStat*>(static_cast<uint8_t*>(c.ws) + kWsHeader);
-  a.cpart = reinterpret_cast<ChunkStat*>(static_cast<uint8_t*>(c.ws) + kWsHeader +
-                                         align_up((size_t)c.B * a.nchunk * sizeof(ChunkStat), 256));
+  a.cpart = reinterpret_cast<ChunkStat*>(static_cast<uint8_t*>(c.ws) + kWsHeader);
+  {
+    const size_t np_max = std::max<size_t>((size_t)(c.V + 255) / 256, 1024);
+    uint8_t* gb = static_cast<uint8_t*>(c.ws) + kWsHeader + align_up((size_t)c.B * np_max * sizeof(ChunkStat), 256);
+    a.gbuf = (c.w_dtype == DSPARK_BF16 && c.r % 64 == 0) ? reinterpret_cast<__nv_bfloat16*>(gb) : nullptr;
+  }
   a.greedy = (c.T == 0.f) ? 1 : 0;
   a.inv_T = a.greedy ? 1.f : 1.f / c.T;
   const bool pdl = opt.draft_pdl != 0;
@@ -899,7 +1056,8 @@ dspark_status launch_draft(const DraftCall& c) {
     return DSPARK_ECUDA;
   }
 
-  CUtensorMap mW2, mU, mLd;
+  CUtensorMap mW2, mU, mLd, mG;
+  memset(&mG, 0, sizeof(mG));
   int n_bgroups = 1, cpg = 1, nb = 0;
   size_t tc_smem = 0;
   if (use_tc) {
@@ -932,6 +1090,15 @@ dspark_status launch_draft(const DraftCall& c) {
       set_error("cuTensorMapEncodeTiled failed for l_d");
       return DSPARK_ECUDA;
     }
+    if (a.gbuf) {  // the B operand rows copied by the combine: [B][r] bf16, boxes of 64 x nb, 128-byte swizzle
+      uint64_t gdims[2] = {(uint64_t)c.r, (uint64_t)c.B};
+      uint64_t gstrides[1] = {(uint64_t)c.r * 2};
+      uint32_t gbox[2] = {64, (uint32_t)nb};
+      if (!make_map(&mG, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.gbuf, gdims, gstrides, gbox)) {
+        set_error("cuTensorMapEncodeTiled failed for the B-operand rows");
+        return DSPARK_ECUDA;
+      }
+    }
     tc_smem = tc_layout(c.r, nb).total + 1024;
     rc = tc_set_smem(nb, tc_smem);
     if (rc != cudaSuccess) {
@@ -944,6 +1111,19 @@ dspark_status launch_draft(const DraftCall& c) {
     a.np = a.ntiles;
   }
 
+  if (use_tc && opt.draft_fused) {
+    // all gamma steps in one cooperative launch (every CTA resident; grid barriers between steps)
+    const dim3 grid(cpg * n_bgroups), block(kTcThreads);
+    const int hint = opt.draft_w2_hint;
+    if (nb == 32)
+      rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, false, true, mW2, mU, mLd, mG, a, 0, c.gamma,
+                     n_bgroups, cpg, hint, 1);
+    else
+      rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, false, true, mW2, mU, mLd, mG, a, 0, c.gamma,
+                     n_bgroups, cpg, hint, 1);
+    if (rc == cudaSuccess) return DSPARK_OK;
+    (void)cudaGetLastError();  // e.g. not all CTAs can be resident: one launch pair per step below
+  }
   for (int k = 0; k < c.gamma; ++k) {
     // The first main pass waits for everything before the call in full: its producers read U
     // and W2 before the grid-dependency wait, which is only safe behind this call's own kernels.
@@ -952,11 +1132,11 @@ dspark_status launch_draft(const DraftCall& c) {
       const dim3 grid(cpg * n_bgroups), block(kTcThreads);
       const int hint = opt.draft_w2_hint;
       if (nb == 32)
-        rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, mLd, a, k, n_bgroups, cpg,
-                       hint);
+        rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, pdl_k, false, mW2, mU, mLd, mG, a, k, k + 1,
+                       n_bgroups, cpg, hint, 0);
       else
-        rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, pdl_k, mW2, mU, mLd, a, k, n_bgroups, cpg,
-                       hint);
+        rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, pdl_k, false, mW2, mU, mLd, mG, a, k, k + 1,
+                       n_bgroups, cpg, hint, 0);
     } else if (c.w_dtype == DSPARK_BF16) {
       rc = launch_fma_bg<__nv_bfloat16>(a, k, c.stream, pdl_k);
     } else {
@@ -966,8 +1146,7 @@ dspark_status launch_draft(const DraftCall& c) {
       set_error(std::string("draft main pass launch: ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;
     }
-    rc = launch_ex(draft_combine, dim3((c.B + kCombWarps - 1) / kCombWarps), dim3(kCombWarps * 32), 0, c.stream, pdl,
-                   a, k);
+    rc = launch_ex(draft_combine, dim3(c.B), dim3(kCombThreads), 0, c.stream, pdl, false, a, k);
     if (rc != cudaSuccess) {
       set_error(std::string("draft combine launch: ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;

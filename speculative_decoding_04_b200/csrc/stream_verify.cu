@@ -21,12 +21,13 @@
 // stalls the tile pipeline, and a row's two reads are at most two rows of the whole grid
 // apart (a few tens of MB against a 126 MB L2).
 //
-// Roles in a CTA of 320 threads: warp 8 streams the rows through a 3-stage ring, one 32 KB bulk
+// Roles in a CTA of 352 threads: warp 8 streams the rows through a 3-stage ring, one 32 KB bulk
 // copy per row and stage (copies of 4 KB were measured to cap the stream at under half the HBM
 // bandwidth, whatever the number of issuing threads); warps 0-7 each take one 1024-column piece
 // of a stage (the assignment rotates from stage to stage, so uneven segments even out); warp 9
-// combines partial results, exchanges them with the cluster, decides acceptance and writes the
-// per-row records.
+// folds the warps' partials and exchanges them with the cluster; warp 10 folds the cluster's
+// partials, decides acceptance and writes the per-row records (two warps, so that a row's
+// decision never waits behind the next row's exchange).
 // A small second
 // kernel (one warp per request) finds n, samples the residual / bonus token by an inverse CDF
 // over the per-tile weights and one rescanned tile, and writes y, n and c*.
@@ -51,9 +52,10 @@ constexpr int kSvTile = 1024;  // columns per tile
 constexpr int kSvWarps = 8;    // consumer warps
 constexpr int kSvBig = kSvWarps * kSvTile;  // columns per ring stage: one 32 KB copy per row
 constexpr int kSvStages = 3;                 // ring stages of (l_d 8192 columns, l_t 8192 columns)
-constexpr int kSvThreads = (kSvWarps + 2) * 32;
+constexpr int kSvThreads = (kSvWarps + 3) * 32;
 constexpr int kSvProducer = kSvWarps;
-constexpr int kSvController = kSvWarps + 1;
+constexpr int kSvCombiner = kSvWarps + 1;
+constexpr int kSvDecider = kSvWarps + 2;
 constexpr int kSvPhaseSlots = 8;
 constexpr int kSvJobSlots = 4;
 constexpr int kSvMaxCluster = 8;
@@ -268,19 +270,18 @@ __device__ __forceinline__ SvPart sv_empty_part() {
 // Fold the partials held by lanes 0..n-1 of a warp (the other lanes hold empty partials);
 // every lane returns the same result (each step is commutative, so the butterfly gives
 // identical bits in all lanes and in every CTA that folds the same inputs).
-__device__ __forceinline__ SvPart sv_fold(SvPart p, bool sums_are_plain) {
+template <bool GREEDY>
+__device__ __forceinline__ SvPart sv_fold(SvPart p) {
   SvPart r = p;
-  if (sums_are_plain) {
-    r.sd = warp_sum_d(p.sd);
-    r.st = warp_sum_d(p.st);
+  if (GREEDY) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      r.gd = top2_merge(r.gd, top2_shfl_xor(r.gd, o));
+      r.gt = top2_merge(r.gt, top2_shfl_xor(r.gt, o));
+    }
   } else {
     sv_warp_ref_sum(r.rd, r.sd);
     sv_warp_ref_sum(r.rt, r.st);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    r.gd = top2_merge(r.gd, top2_shfl_xor(r.gd, o));
-    r.gt = top2_merge(r.gt, top2_shfl_xor(r.gt, o));
   }
   const unsigned hx = __ballot_sync(0xffffffffu, p.has_x != 0);
   if (hx) {
@@ -412,6 +413,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   __shared__ SvPart xs[kSvJobSlots][kSvMaxCluster];
   __shared__ SvNorm dec[kSvJobSlots];
   __shared__ int s_abort;
+  __shared__ volatile int s_decided;  // rows of this cluster's sequence decided by this CTA
 
   const SvSync sy{&s_abort, a.status};
   if (threadIdx.x == 0) {
@@ -425,6 +427,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       mbar_init(&dbar[i], 1);
     }
     s_abort = 0;
+    s_decided = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -480,112 +483,113 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           }
       }
     }
-  } else if (warp == kSvController) {
-    // ------------------------------------------------------------------ combine, exchange, decide
+  } else if (warp == kSvCombiner) {
+    // ------------------------------------------------------------------ combine and exchange
+    // Per first pass: fold the eight warps' partials and push the CTA's into slot [i % 4][rank]
+    // of every CTA of the cluster.  Per second pass: the CTA's label partials to global memory.
+    // A push for row i waits until this CTA has decided row i-2: a peer that has decided row
+    // i-2 has then seen this CTA's push of row i-2, so every peer has decided row i-4, the
+    // previous user of the slot (the second passes give the same order when T > 0; greedy
+    // verification has none).
+    SvGen gen;
+    gen.init(a, cid, ncl);
+    SvPhase ph;
     int p = 0;
     bool ok = true;
-    int xk_prev = -1, xk_cur = -1;
-    float u_prev = 0.f, u_cur = 0.f;
-    auto p1_end = [&](const SvJob& J, int i) {
+    while (ok && gen.next(a, ph)) {
       const int ps = p % kSvPhaseSlots;
       ok = sv_wait(sy, &phbar[ps], (p / kSvPhaseSlots) & 1);
       ++p;
-      if (!ok) return;
+      if (!ok) break;
       SvPart w = lane < kSvWarps ? wpart[ps][lane] : sv_empty_part();
-      w = sv_fold(w, false);
-      // push this CTA's partial into slot [i % 4][rank] of every CTA of the cluster
-      if (lane < C) {
-        SvPart* dst = cluster.map_shared_rank(&xs[i % kSvJobSlots][rank], lane);
-        *dst = w;
-        sv_remote_arrive(&xbar[i % kSvJobSlots], lane);
-      }
-      (void)J;
-    };
-    auto p2_end = [&](const SvJob& J) {
-      const int ps = p % kSvPhaseSlots;
-      ok = sv_wait(sy, &phbar[ps], (p / kSvPhaseSlots) & 1);
-      ++p;
-      if (!ok) return;
-      SvPart w = lane < kSvWarps ? wpart[ps][lane] : sv_empty_part();
-      const double sm = warp_sum_d(w.sd), sq = warp_sum_d(w.st);
-      if (lane == 0 && J.k < a.gamma) a.part[((size_t)J.b * a.gamma + J.k) * C + rank] = make_double2(sm, sq);
-    };
-    SvJob cur, prev;
-    int j = sv_next(a, cid, ncl, cur);
-    bool have_prev = false;
-    for (int i = 0; ok; ++i) {
-      const bool have_cur = j >= 0;
-      if (have_cur) {
-        xk_cur = cur.verify ? __ldg(a.x + (size_t)cur.b * a.gamma + cur.k) : -1;
-        u_cur = (cur.verify && !GREEDY) ? __ldg(a.u_acc + (size_t)cur.b * a.gamma + cur.k) : 0.f;
-      }
-      if (have_prev) {
-        // ---- decide the previous row: fold the cluster's partials in rank order
-        const int js = (i - 1) % kSvJobSlots;
-        ok = sv_wait(sy, &xbar[js], ((i - 1) / kSvJobSlots) & 1, true);
-        if (!ok) break;
-        SvPart x = lane < C ? xs[js][lane] : sv_empty_part();
-        x = sv_fold(x, false);
-        SvRow row;
-        row.acc = 0;
-        row.fl = 0;
-        row.cand = 0;
-        row.cstar = 0.f;
-        uint32_t dfl = x.fl;
-        if (GREEDY) {
-          row.nm = SvNorm{0.f, 0.f, 0.f, 0.f};
-          const bool ttie = x.gt.best - x.gt.second <= 1e-6f * fmaxf(1.f, fabsf(x.gt.best));
-          row.cand = min(max(x.gt.idx, 0), a.V - 1);
-          if (x.gt.idx < 0) dfl |= DSPARK_FLAG_NONFINITE;
-          row.cstar = (x.gd.idx == x.gt.idx) ? 1.f : 0.f;
-          row.fl = ttie ? (DSPARK_FLAG_ACCEPT_NEAR_TIE | DSPARK_FLAG_SAMPLE_NEAR_TIE) : 0u;
-          if (prev.verify) {
-            if ((unsigned)xk_prev >= (unsigned)a.V) dfl |= DSPARK_FLAG_TOKEN_RANGE;
-            row.acc = (xk_prev == x.gt.idx) ? 1 : 0;
-          }
-        } else {
-          SvNorm nm;
-          bool good = sv_norm(x.rt, x.st, nm.Kt, nm.lamt);
-          if (prev.d) good &= sv_norm(x.rd, x.sd, nm.Kd, nm.lamd);
-          else nm.Kd = nm.lamd = 0.f;
-          if (!good) dfl |= DSPARK_FLAG_NONFINITE;
-          row.nm = nm;
-          if (lane == 0) dec[js] = nm;
-          if (prev.verify) {
-            if ((unsigned)xk_prev >= (unsigned)a.V || !x.has_x) {
-              dfl |= DSPARK_FLAG_TOKEN_RANGE;
-            } else {
-              const double l2e = (double)kLog2e;
-              const double zd = (double)__fmul_rn(x.ldx, inv_T), zt = (double)__fmul_rn(x.ltx, inv_T);
-              const double pd = exp2(zd * l2e - (double)x.rd) / x.sd;
-              const double pt = exp2(zt * l2e - (double)x.rt) / x.st;
-              const double u = (double)u_prev;
-              row.acc = (u * pd < pt) ? 1 : 0;
-              if (pd > 0.0 && fabs(u - pt / pd) < 1e-6) row.fl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
+      if (!ph.second) {
+        w = sv_fold<GREEDY>(w);
+        const int i = ph.i;
+        for (uint32_t t = 0; s_decided < i - 1; ++t)  // s_decided counts rows, so row i-2 is decided
+          if (t >= kSpinLimit || *sy.abort) {
+            if (!*sy.abort) {
+              *sy.abort = 1;
+              atomicOr(sy.status, (uint32_t)DSPARK_ETIMEOUT);
             }
+            ok = false;
+            break;
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&dbar[js]);  // the second pass of this row may start
-        }
-        if (rank == 0 && lane == 0) {
-          a.rows[prev.rec] = row;
-          if (dfl && a.flags) atomicOr(a.flags + prev.b, dfl);
-        }
-      }
-      if (have_cur) {
-        p1_end(cur, i);
         if (!ok) break;
+        if (lane < C) {
+          SvPart* dst = cluster.map_shared_rank(&xs[i % kSvJobSlots][rank], lane);
+          *dst = w;
+          sv_remote_arrive(&xbar[i % kSvJobSlots], lane);
+        }
+      } else {
+        const double sm = warp_sum_d(w.sd), sq = warp_sum_d(w.st);
+        if (lane == 0 && ph.J.k < a.gamma)
+          a.part[((size_t)ph.J.b * a.gamma + ph.J.k) * C + rank] = make_double2(sm, sq);
       }
-      if (have_prev && sv_p2(a, prev)) {
-        p2_end(prev);
-        if (!ok) break;
+    }
+  } else if (warp == kSvDecider) {
+    // ------------------------------------------------------------------ decide, row by row
+    SvJob J;
+    int j = sv_next(a, cid, ncl, J);
+    bool ok = true;
+    for (int i = 0; ok && j >= 0; ++i) {
+      const int js = i % kSvJobSlots;
+      // the drafted token and its uniform are requested before the wait for the peers
+      const int xk = J.verify ? __ldg(a.x + (size_t)J.b * a.gamma + J.k) : -1;
+      const float u_acc = (J.verify && !GREEDY) ? __ldg(a.u_acc + (size_t)J.b * a.gamma + J.k) : 0.f;
+      ok = sv_wait(sy, &xbar[js], (i / kSvJobSlots) & 1, true);
+      if (!ok) break;
+      SvPart x = lane < C ? xs[js][lane] : sv_empty_part();
+      x = sv_fold<GREEDY>(x);
+      SvRow row;
+      row.acc = 0;
+      row.fl = 0;
+      row.cand = 0;
+      row.cstar = 0.f;
+      uint32_t dfl = x.fl;
+      if (GREEDY) {
+        row.nm = SvNorm{0.f, 0.f, 0.f, 0.f};
+        const bool ttie = x.gt.best - x.gt.second <= 1e-6f * fmaxf(1.f, fabsf(x.gt.best));
+        row.cand = min(max(x.gt.idx, 0), a.V - 1);
+        if (x.gt.idx < 0) dfl |= DSPARK_FLAG_NONFINITE;
+        row.cstar = (x.gd.idx == x.gt.idx) ? 1.f : 0.f;
+        row.fl = ttie ? (DSPARK_FLAG_ACCEPT_NEAR_TIE | DSPARK_FLAG_SAMPLE_NEAR_TIE) : 0u;
+        if (J.verify) {
+          if ((unsigned)xk >= (unsigned)a.V) dfl |= DSPARK_FLAG_TOKEN_RANGE;
+          row.acc = (xk == x.gt.idx) ? 1 : 0;
+        }
+      } else {
+        SvNorm nm;
+        bool good = sv_norm(x.rt, x.st, nm.Kt, nm.lamt);
+        if (J.d) good &= sv_norm(x.rd, x.sd, nm.Kd, nm.lamd);
+        else nm.Kd = nm.lamd = 0.f;
+        if (!good) dfl |= DSPARK_FLAG_NONFINITE;
+        row.nm = nm;
+        if (lane == 0) dec[js] = nm;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dbar[js]);  // the second pass of this row may start
+        if (J.verify) {
+          if ((unsigned)xk >= (unsigned)a.V || !x.has_x) {
+            dfl |= DSPARK_FLAG_TOKEN_RANGE;
+          } else {
+            // u p_d(x) < p_t(x) with p = 2^(z log2e - R) / S, in fp64
+            const double l2e = (double)kLog2e;
+            const double zd = (double)__fmul_rn(x.ldx, inv_T), zt = (double)__fmul_rn(x.ltx, inv_T);
+            const double pd = exp2(zd * l2e - (double)x.rd) / x.sd;
+            const double pt = exp2(zt * l2e - (double)x.rt) / x.st;
+            const double u = (double)u_acc;
+            row.acc = (u * pd < pt) ? 1 : 0;
+            if (pd > 0.0 && fabs(u - pt / pd) < 1e-6) row.fl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
+          }
+        }
       }
-      if (!have_cur) break;
-      prev = cur;
-      xk_prev = xk_cur;
-      u_prev = u_cur;
-      have_prev = true;
-      j = sv_next(a, j + ncl, ncl, cur);
+      if (rank == 0 && lane == 0) {
+        a.rows[J.rec] = row;
+        if (dfl && a.flags) atomicOr(a.flags + J.b, dfl);
+      }
+      __syncwarp();
+      __threadfence_block();  // this row's slot reads come before the count that frees the slot
+      if (lane == 0) s_decided = i + 1;
+      j = sv_next(a, j + ncl, ncl, J);
     }
   } else {
     // ------------------------------------------------------------------ tile consumers

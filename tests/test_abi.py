@@ -38,9 +38,9 @@ def test_workspace_sizes():
     w1 = D.workspace_size(D.WS_DRAFT, 64, 16, 151936, 256)
     w2 = D.workspace_size(D.WS_DRAFT, 128, 16, 151936, 256)
     assert 256 < w1 < w2
-    assert w1 >= 64 * (151936 // 32) * 16
+    assert w1 >= 256 + 64 * 148 * 16            # one 16-byte record per (partition, request)
     v = D.workspace_size(D.WS_VERIFY, 64, 16, 151936, 0)
-    assert v >= 256 + 3 * 64 * 17 * 4 + 64 * 4
+    assert v >= 256 + 64 * 17 * 32 + 64 * 17 * 149 * 12   # row records + per-1024-column tile records
     assert D.workspace_size(D.WS_SCHEDULE, 64, 16, 151936, 0) == 0
     assert D.workspace_size(7, 64, 16, 151936, 0) == 0
     assert D.workspace_size(D.WS_DRAFT, 0, 16, 151936, 256) == 0

@@ -46,6 +46,19 @@ def test_bf16_paths_ragged_tail(path, B, T, r):
     assert x.min() >= 0 and x.max() < wl.V
 
 
+@pytest.mark.parametrize("fused", [1, 0])
+@pytest.mark.parametrize("B", [16, 64, 100])
+@pytest.mark.parametrize("T", [1.0, 0.0])
+def test_tensor_core_steps_fused_and_per_step(fused, B, T):
+    # fused: all positions in one cooperative launch with grid barriers; else one launch pair
+    # (main pass + combine) per position.  V = 30000: partitions of about 200 columns, a ragged
+    # last tile; B = 100 takes two request groups.
+    D.set_option("draft_fused", fused)
+    wl, d = small(B, 6, 30000, 256, T, seed=2000 + B + fused)
+    x, ld, fl = run_draft(d, wl, 2)
+    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld, fl)
+
+
 def test_tensor_core_and_gemv_passes_agree():
     wl, d = small(24, 6, 8192, 256, 1.0, seed=5)
     x1, ld1, _ = run_draft(d, wl, 1)
