@@ -250,7 +250,8 @@ def main():
     ws_v = D.workspace(D.WS_VERIFY, B, G, V, 0, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    n_launch = 2 * G + 1 + 2  # draft: main pass + combine per position; schedule; verify: stream + finalize
+    D.set_option("draft_fused", 1)  # the draft's gamma positions in one cooperative launch
+    n_launch = 1 + 1 + 2  # draft; schedule; verify: stream + finalize
 
     def round_(src):
         D.markov_draft(src["U"], W1, W2, src["x0"], src["u_draft"], wl.T, x_out=x, ld_out=ld, flags=fl, ws=ws_d,
@@ -351,8 +352,8 @@ def main():
             "verified_tokens_per_s": accepted_all / (args.steps * t_step),
             "draft_ms": t_draft * 1e3, "verify_ms": t_verify * 1e3,
             "hbm_gbs_round": (draft_b + verify_b) / t_step / 1e9,
-            "roofline": {"kernel": f"markov_draft ({G} draft_main_tc + {G} draft_combine launches, timed "
-                                   "together with CUDA events around the call)",
+            "roofline": {"kernel": f"markov_draft (draft_main_tc<64>: {G} positions in one cooperative launch, "
+                                   "timed with CUDA events around the call)",
                          "bound": "hbm", "achieved": draft_b / t_draft / 1e9, "peak": hbm, "unit": "GB/s",
                          "frac": draft_b / t_draft / 1e9 / hbm,
                          "traffic": measured_traffic("draft_main_tc", B * G),
