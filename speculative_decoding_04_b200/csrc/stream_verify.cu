@@ -8,10 +8,10 @@
 //  §Confidence-Scheduled Verification: label c*_k = 1 - ½‖p_d - p_t‖₁]
 //
 // Layout of the work.  A cluster of C CTAs takes rows (position k, request b) in turn; CTA r
-// owns the r-th contiguous run of 1024-column tiles of every row.  Per row each CTA runs
+// owns the r-th contiguous run of 512-column tiles of every row.  Per row each CTA runs
 //   P1  (tiles from HBM)  per-lane maxima and sums of 2^(z log2e - R) against an integer
 //       reference R, so that every later rescaling is an exact power of two; the sums of l_t
-//       per tile are kept for the bonus sample; the raw logits at the drafted token are kept;
+//       per tile are kept for the bonus sample;
 //   --  the CTA's (R, S) pairs go to every CTA of the cluster (distributed shared memory and a
 //       remote mbarrier arrive); each CTA folds them in rank order into the row's normalisers
 //       log2 p = z log2e - K - lam (K an integer, lam in [0, 1)) and decides the acceptance;
@@ -21,11 +21,12 @@
 // stalls the tile pipeline, and a row's two reads are at most two rows of the whole grid
 // apart (a few tens of MB against a 126 MB L2).
 //
-// Roles in a CTA of 352 threads: warp 8 streams the rows through a 3-stage ring, one 32 KB bulk
+// Roles in a CTA of 608 threads: warp 16 streams the rows through a 3-stage ring, one 32 KB bulk
 // copy per row and stage (copies of 4 KB were measured to cap the stream at under half the HBM
-// bandwidth, whatever the number of issuing threads); warps 0-7 each take one 1024-column piece
-// of a stage (the assignment rotates from stage to stage, so uneven segments even out); warp 9
-// folds the warps' partials and exchanges them with the cluster; warp 10 folds the cluster's
+// bandwidth, whatever the number of issuing threads); warps 0-15 each take one 512-column piece
+// of a stage (the assignment rotates from stage to stage, so uneven segments even out; the
+// passes are latency-bound, and 16 warps with 512 columns each measured faster than 8 with
+// 1024); warp 17 folds the warps' partials and exchanges them with the cluster; warp 18 folds the cluster's
 // partials, decides acceptance and writes the per-row records (two warps, so that a row's
 // decision never waits behind the next row's exchange).
 // A small second
@@ -48,15 +49,18 @@ namespace dspark {
 
 namespace {
 
-constexpr int kSvTile = 1024;  // columns per tile
-constexpr int kSvWarps = 8;    // consumer warps
-constexpr int kSvBig = kSvWarps * kSvTile;  // columns per ring stage: one 32 KB copy per row
-constexpr int kSvStages = 3;                 // ring stages of (l_d 8192 columns, l_t 8192 columns)
+constexpr int kSvTile = 512;    // columns per tile (one consumer warp's piece of a stage)
+constexpr int kSvWarps = 16;    // consumer warps (four per scheduler: the passes are latency-bound)
+constexpr int kSvVec = kSvTile / 128;  // float4s per lane and row in a piece
+constexpr int kSvGroups = 1;                       // consumer groups; stage g goes to group g mod kSvGroups
+constexpr int kSvGroupWarps = kSvWarps / kSvGroups;  // warps per group, one piece each
+constexpr int kSvBig = kSvGroupWarps * kSvTile;      // columns per ring stage: one 32 KB copy per row
+constexpr int kSvStages = 3;                         // ring stages of (l_d 8192 columns, l_t 8192 columns)
 constexpr int kSvThreads = (kSvWarps + 3) * 32;
 constexpr int kSvProducer = kSvWarps;
 constexpr int kSvCombiner = kSvWarps + 1;
 constexpr int kSvDecider = kSvWarps + 2;
-constexpr int kSvPhaseSlots = 8;
+constexpr int kSvPhaseSlots = 16;
 constexpr int kSvJobSlots = 4;
 constexpr int kSvMaxCluster = 8;
 constexpr int kRNone = -(1 << 28);  // reference of an empty sum
@@ -69,8 +73,8 @@ struct __align__(16) SvPart {
   double sd, st;
   int rd, rt;
   Top2 gd, gt;
-  float ldx, ltx;  // raw logits at the drafted token (has_x)
-  int has_x;
+  float pad0, pad1;
+  int pad2;
   uint32_t fl;
 };
 
@@ -95,7 +99,7 @@ struct SvArgs {
   const int32_t* L;
   const float* u_acc;
   const float* u_res;
-  int B, gamma, V, lt_rows, njobs, ntile, C;
+  int B, gamma, V, lt_rows, njobs, ntile, C, lag;
   float inv_T;
   int greedy, do_verify;
   float* c_star;
@@ -147,26 +151,29 @@ struct SvPhase {
   int i;  // index of the row among this cluster's rows (exchange / decision slots)
 };
 
-// The phase sequence of a cluster: P1(row 0), then P1(row i), P2(row i-1) for i = 1, 2, ...,
-// then P2(last row).  Every role walks the same sequence.
+// The phase sequence of a cluster with a lag of L rows (a.lag, 1 to 3): P1(row i) then
+// P2(row i-L), for i = 0, 1, ..., until both have run out.  Every role walks the same sequence.
 struct SvGen {
-  int j, ncl, i, step;
-  SvJob cur, prev;
-  bool have_prev, done;
+  int j, ncl, i, step, nrows, lag;
+  bool exhausted;
+  SvJob ring[4];  // rows i-L .. i
   __device__ void init(const SvArgs& a, int cid, int ncl_) {
     ncl = ncl_;
-    j = sv_next(a, cid, ncl, cur);
+    lag = a.lag;
     i = 0;
     step = 0;
-    have_prev = false;
-    done = false;
+    nrows = 0;
+    exhausted = false;
+    j = sv_next(a, cid, ncl, ring[0]);
+    if (j >= 0) nrows = 1;
+    else exhausted = true;
   }
   __device__ bool next(const SvArgs& a, SvPhase& ph) {
-    while (!done) {
+    while (true) {
       if (step == 0) {
         step = 1;
-        if (j >= 0) {
-          ph.J = cur;
+        if (i < nrows) {
+          ph.J = ring[i & 3];
           ph.second = false;
           ph.i = i;
           return true;
@@ -174,24 +181,23 @@ struct SvGen {
       }
       if (step == 1) {
         step = 2;
-        if (have_prev && sv_p2(a, prev)) {
-          ph.J = prev;
+        const int q = i - lag;
+        if (q >= 0 && q < nrows && sv_p2(a, ring[q & 3])) {
+          ph.J = ring[q & 3];
           ph.second = true;
-          ph.i = i - 1;
+          ph.i = q;
           return true;
         }
       }
-      if (j < 0) {
-        done = true;
-        return false;
-      }
-      prev = cur;
-      have_prev = true;
       ++i;
-      j = sv_next(a, j + ncl, ncl, cur);
       step = 0;
+      if (!exhausted) {
+        j = sv_next(a, j + ncl, ncl, ring[i & 3]);
+        if (j >= 0) nrows = i + 1;
+        else exhausted = true;
+      }
+      if (exhausted && i - lag >= nrows) return false;
     }
-    return false;
   }
 };
 
@@ -230,6 +236,14 @@ __device__ __forceinline__ void sv_warp_ref_sum(int& R, double& S) {
   R = M;
 }
 
+// Same across the lanes of a warp with the lane sums rounded to fp32 first (32 terms, one
+// rounding each; the per-lane sums themselves are accumulated in fp64).
+__device__ __forceinline__ void sv_warp_ref_sum_f(int& R, double& S) {
+  const int M = __reduce_max_sync(0xffffffffu, R);
+  S = (double)warp_sum_f((float)(S * sv_pow2d(R - M)));
+  R = M;
+}
+
 // p_d and p_t of one column from its raw logits (shared by the second pass and the rescan
 // in the finalize kernel, so that both see the same weights).
 __device__ __forceinline__ void sv_probs(float ld, float lt, float inv_T, const SvNorm& n, float& pd, float& pt) {
@@ -261,8 +275,8 @@ __device__ __forceinline__ SvPart sv_empty_part() {
   p.rd = p.rt = kRNone;
   p.gd = Top2{-INFINITY, -1, -INFINITY};
   p.gt = Top2{-INFINITY, -1, -INFINITY};
-  p.ldx = p.ltx = 0.f;
-  p.has_x = 0;
+  p.pad0 = p.pad1 = 0.f;
+  p.pad2 = 0;
   p.fl = 0;
   return p;
 }
@@ -282,15 +296,6 @@ __device__ __forceinline__ SvPart sv_fold(SvPart p) {
   } else {
     sv_warp_ref_sum(r.rd, r.sd);
     sv_warp_ref_sum(r.rt, r.st);
-  }
-  const unsigned hx = __ballot_sync(0xffffffffu, p.has_x != 0);
-  if (hx) {
-    const int src = __ffs(hx) - 1;
-    r.ldx = __shfl_sync(0xffffffffu, p.ldx, src);
-    r.ltx = __shfl_sync(0xffffffffu, p.ltx, src);
-    r.has_x = 1;
-  } else {
-    r.has_x = 0;
   }
   r.fl = __reduce_or_sync(0xffffffffu, p.fl);
   return r;
@@ -375,10 +380,10 @@ __device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z,
 
 // First pass over one lane's 32 values of a tile: z = l * (1/T) in place, the integer
 // reference R of their maximum and the fp32 sum of 2^(z log2e - R).
-__device__ __forceinline__ float sv_lane_sum(float4 (&v)[8], float2 invT2, int& R) {
+__device__ __forceinline__ float sv_lane_sum(float4 (&v)[kSvVec], float2 invT2, int& R) {
   float m = -INFINITY;
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
+  for (int jj = 0; jj < kSvVec; ++jj) {
     const float2 a = f2mul(lo2(v[jj]), invT2), b = f2mul(hi2(v[jj]), invT2);
     v[jj] = make_float4(a.x, a.y, b.x, b.y);
     m = fmax3(m, a.x, a.y);
@@ -388,7 +393,7 @@ __device__ __forceinline__ float sv_lane_sum(float4 (&v)[8], float2 invT2, int& 
   const float2 l2e2 = make_float2(kLog2e, kLog2e), nr2 = make_float2(-(float)R, -(float)R);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
+  for (int jj = 0; jj < kSvVec; ++jj) {
     const float2 a = f2fma(lo2(v[jj]), l2e2, nr2), b = f2fma(hi2(v[jj]), l2e2, nr2);
     acc0 = f2add(acc0, make_float2(sv_ex2(a.x), sv_ex2(a.y)));
     acc1 = f2add(acc1, make_float2(sv_ex2(b.x), sv_ex2(b.y)));
@@ -419,7 +424,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSvStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kSvWarps);
+      mbar_init(&empty[i], kSvGroupWarps);
     }
     for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
     for (int i = 0; i < kSvJobSlots; ++i) {
@@ -437,7 +442,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   const int nt = (int)((long long)(rank + 1) * a.ntile / C) - tb;  // tiles of this CTA per row (may be 0)
   const float inv_T = a.inv_T;
 
-  const int nbig = (nt + kSvWarps - 1) / kSvWarps;  // ring stages per row and pass
+  const int nbig = (nt + kSvGroupWarps - 1) / kSvGroupWarps;  // ring stages per row and pass
   const int c_end = min((tb + nt) * kSvTile, a.V);     // end column of this CTA's segment
 
   if (warp == kSvProducer) {
@@ -463,7 +468,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
             ok = false;
             break;
           }
-          const int v0 = (tb + bt * kSvWarps) * kSvTile;
+          const int v0 = (tb + bt * kSvGroupWarps) * kSvTile;
           const uint32_t bytes = (uint32_t)min(kSvBig, c_end - v0) * 4u;
           float* st = ring + (size_t)s * 2 * kSvBig;
           if (lane == 0) {
@@ -534,8 +539,14 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     for (int i = 0; ok && j >= 0; ++i) {
       const int js = i % kSvJobSlots;
       // the drafted token and its uniform are requested before the wait for the peers
+      // (and, for T > 0, the two logits at the drafted token)
       const int xk = J.verify ? __ldg(a.x + (size_t)J.b * a.gamma + J.k) : -1;
       const float u_acc = (J.verify && !GREEDY) ? __ldg(a.u_acc + (size_t)J.b * a.gamma + J.k) : 0.f;
+      float ldx = 0.f, ltx = 0.f;
+      if (!GREEDY && J.verify && (unsigned)xk < (unsigned)a.V) {
+        ldx = __ldg(a.ld + ((size_t)J.k * a.B + J.b) * a.V + xk);
+        ltx = __ldg(a.lt + ((size_t)J.b * a.lt_rows + J.k) * a.V + xk);
+      }
       ok = sv_wait(sy, &xbar[js], (i / kSvJobSlots) & 1, true);
       if (!ok) break;
       SvPart x = lane < C ? xs[js][lane] : sv_empty_part();
@@ -568,12 +579,12 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&dbar[js]);  // the second pass of this row may start
         if (J.verify) {
-          if ((unsigned)xk >= (unsigned)a.V || !x.has_x) {
+          if ((unsigned)xk >= (unsigned)a.V) {
             dfl |= DSPARK_FLAG_TOKEN_RANGE;
           } else {
             // u p_d(x) < p_t(x) with p = 2^(z log2e - R) / S, in fp64
             const double l2e = (double)kLog2e;
-            const double zd = (double)__fmul_rn(x.ldx, inv_T), zt = (double)__fmul_rn(x.ltx, inv_T);
+            const double zd = (double)__fmul_rn(ldx, inv_T), zt = (double)__fmul_rn(ltx, inv_T);
             const double pd = exp2(zd * l2e - (double)x.rd) / x.sd;
             const double pt = exp2(zt * l2e - (double)x.rt) / x.st;
             const double u = (double)u_acc;
@@ -607,7 +618,6 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       // second pass state
       double smin = 0.0, sq = 0.0;
       SvNorm nm{0.f, 0.f, 0.f, 0.f};
-      const int xk = (!second && J.verify) ? __ldg(a.x + (size_t)J.b * a.gamma + J.k) : -1;
       if (second) {
         const int js = i % kSvJobSlots;
         ok = sv_wait(sy, &dbar[js], (i / kSvJobSlots) & 1);
@@ -616,23 +626,24 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       const bool with_d = second || J.d;
       for (int bt = 0; ok && bt < nbig; ++bt) {
         const uint32_t gb = Gb + bt;
+        if ((int)(gb % kSvGroups) != w / kSvGroupWarps) continue;  // the other group's stage
         const int s = (int)(gb % kSvStages);
         if (!sv_wait(sy, &full[s], (gb / kSvStages) & 1)) {
           ok = false;
           break;
         }
         // this warp's 1024-column piece of the stage; the assignment rotates from stage to stage
-        const int q = (w + (int)(gb % kSvWarps)) % kSvWarps;
-        const int t = bt * kSvWarps + q;  // tile of this CTA's segment
+        const int q = ((w % kSvGroupWarps) + (int)(gb / kSvGroups)) % kSvGroupWarps;
+        const int t = bt * kSvGroupWarps + q;  // tile of this CTA's segment
         const bool mine = t < nt;
         const int v0 = (tb + t) * kSvTile;
         const int cnt = mine ? min(kSvTile, a.V - v0) : 0;
         const float* sd = ring + (size_t)s * 2 * kSvBig + q * kSvTile;
         const float* st = sd + kSvBig;
-        float4 fd[8], ft[8];
+        float4 fd[kSvVec], ft[kSvVec];
         const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
+        for (int jj = 0; jj < kSvVec; ++jj) {
           const int idx = (jj * 32 + lane) * 4;
           const bool v = idx < cnt;
           ft[jj] = v ? *reinterpret_cast<const float4*>(st + idx) : ninf;
@@ -642,21 +653,9 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
         if (lane == 0) mbar_arrive(&empty[s]);  // the values are in registers
         if (!mine) continue;
         if (!second) {
-          // drafted token in this tile: keep its raw logits
-          const int xi = xk - v0;
-          if (xi >= 0 && xi < cnt && ((xi >> 2) & 31) == lane) {
-            const int jj = xi >> 7, c = xi & 3;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              if (q == jj) {
-                out.ldx = f4c(fd[q], c);
-                out.ltx = f4c(ft[q], c);
-              }
-            out.has_x = 1;
-          }
           if (GREEDY) {
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
+            for (int jj = 0; jj < kSvVec; ++jj) {
               const int base = v0 + (jj * 32 + lane) * 4;
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
@@ -692,7 +691,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           const float2 nld = make_float2(-nm.lamd, -nm.lamd), nlt = make_float2(-nm.lamt, -nm.lamt);
           float2 sm2 = make_float2(0.f, 0.f), q2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
+          for (int jj = 0; jj < kSvVec; ++jj) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
@@ -726,24 +725,17 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           out.gd = gd;
           out.gt = gt;
         } else {
-          sv_warp_ref_sum(Rd, Sd);
-          sv_warp_ref_sum(Rt, St);
+          sv_warp_ref_sum_f(Rd, Sd);
+          sv_warp_ref_sum_f(Rt, St);
           out.rd = Rd;
           out.sd = Sd;
           out.rt = Rt;
           out.st = St;
         }
-        const unsigned hx = __ballot_sync(0xffffffffu, out.has_x != 0);
-        if (hx) {
-          const int src = __ffs(hx) - 1;
-          out.ldx = __shfl_sync(0xffffffffu, out.ldx, src);
-          out.ltx = __shfl_sync(0xffffffffu, out.ltx, src);
-          out.has_x = 1;
-        }
         out.fl = __any_sync(0xffffffffu, bad != 0) ? (uint32_t)DSPARK_FLAG_NONFINITE : 0u;
       } else {
-        out.sd = warp_sum_d(smin);
-        out.st = warp_sum_d(sq);
+        out.sd = (double)warp_sum_f((float)smin);
+        out.st = (double)warp_sum_f((float)sq);
       }
       const int ps = p % kSvPhaseSlots;
       if (lane == 0) {
@@ -979,6 +971,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.lt_rows = c.lt_rows;
   a.njobs = c.B * (c.gamma + 1);
   a.ntile = (c.V + kSvTile - 1) / kSvTile;
+  a.lag = std::min(std::max(options().verify_stream_lag, 1), 3);
   a.greedy = c.T == 0.f ? 1 : 0;
   a.inv_T = a.greedy ? 1.f : 1.f / c.T;
   a.do_verify = 1;

@@ -31,3 +31,4 @@ def _default_options():
         D.set_option("verify_persistent", 1)
         D.set_option("verify_stream", 1)
         D.set_option("verify_stream_cluster", 2)
+        D.set_option("verify_stream_lag", 1)

@@ -163,3 +163,20 @@ def test_stream_vocabulary_beyond_per_row_kernels(T):
     with pytest.raises(D.DsparkError) as e:
         run_verify(ld, lt, x, None, u_acc, u_res, T)
     assert e.value.status == D.ENOTIMPL
+
+
+@pytest.mark.parametrize("lag", [1, 2, 3])
+@pytest.mark.parametrize("cluster", [2, 8])
+@pytest.mark.parametrize("T", [1.0, 0.0])
+def test_stream_lag_between_passes(lag, cluster, T):
+    # the second pass of a row runs `lag` rows after its first pass; scheduled rows are skipped
+    D.set_option("verify_stream_cluster", cluster)
+    D.set_option("verify_stream_lag", lag)
+    B, G, V = 24, 5, 20000
+    ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=300 + lag + cluster)
+    L = (np.arange(B) * 5 % (G + 1)).astype(np.int32)
+    for want_c in (True, False):
+        n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=want_c)
+        check_verify(ld, lt, x, L, u_acc, u_res, T, n, y)
+        if want_c:
+            check_labels(ld, lt, T, c)
