@@ -355,23 +355,18 @@ __device__ __forceinline__ float grp_max_f(float v, float* sh, const Grp& g) {
 }
 
 // Grid-wide barrier of the multi-step launch (cooperative, so every CTA is resident): one thread
-// per CTA after a CTA-level barrier.  Bounded: gives up with the timeout status and the abort flag.
-__device__ __forceinline__ bool grid_sync(uint32_t* count, uint32_t* gen, uint32_t nblocks, uint32_t& epoch,
-                                          const TcSync& sy) {
+// per CTA after a CTA-level barrier adds 1 to a monotonic counter with a release reduction (no
+// returned value, so the arrivals do not queue on each other) and waits, with acquire loads, for
+// it to reach nblocks times the barrier's number.  Bounded: gives up with the timeout status and
+// the abort flag.
+__device__ __forceinline__ bool grid_sync(uint32_t* count, uint32_t nblocks, uint32_t& epoch, const TcSync& sy) {
   if (*sy.abort) return false;
-  __threadfence();
-  const uint32_t target = ++epoch;
-  if (atomicAdd(count, 1u) == nblocks - 1) {
-    atomicExch(count, 0u);
-    __threadfence();
-    atomicExch(gen, target);
-    return true;
-  }
+  const uint32_t target = ++epoch * nblocks;
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (*reinterpret_cast<volatile uint32_t*>(gen) == target) {
-      __threadfence();
-      return true;
-    }
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
+    if ((int32_t)(v - target) >= 0) return true;
     if ((i & 1023u) == 1023u && *sy.abort) return false;
   }
   *sy.abort = 1;
@@ -469,7 +464,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto load_u = [&](int gi, uint64_t pol) {
     const int j = gi & 1, ku = k0 + gi / nt, iu = gi % nt;
     mbar_arrive_expect_tx(&u_full[j], kUStage * 4u);
-    if (w2_hint) tma_load_3d_hint(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j], pol);
+    if (w2_hint == 1 || w2_hint == 2)
+      tma_load_3d_hint(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j], pol);
     else tma_load_3d(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j]);
   };
   if (warp == 3 && lane == 0) {
@@ -512,7 +508,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     pdl_wait();
     uint32_t epoch = 0;
     uint32_t* gcount = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.status) + 64);
-    uint32_t* ggen = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.status) + 128);
     bool bad = false;
     int last_load[2] = {total > 0 ? 0 : -1, total > 1 ? 1 : -1};  // (warp 3) last tile loaded into each U stage
     for (int k = k0; k < k1; ++k) {
@@ -551,7 +546,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < nt; ++i) {
             const int gi = gbase + i, j = gi & 1;
             if (!tc_wait(sy, &c_done[j], (gi >> 1) & 1)) break;
-            if (w2_hint) tma_store_3d_hint(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k, pol);
+            if (w2_hint == 1) tma_store_3d_hint(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k, pol);
             else tma_store_3d(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k);
             bulk_commit();
             if (gi + 2 < total) {
@@ -690,14 +685,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (fused) {
         // ---------------------------------------------------------------- sample this step
         named_bar(3, kTcThreads - 32);
-        if (warp == 1 && lane == 0) grid_sync(gcount, ggen, gridDim.x, epoch, sy);
+        if (warp == 1 && lane == 0) grid_sync(gcount, gridDim.x, epoch, sy);
         named_bar(3, kTcThreads - 32);
         // one request per CTA at a time, all non-producer warps together
         // (no test of the abort flag here: every thread of the group must take the same path)
         for (int rq = blockIdx.x; rq < a.B; rq += gridDim.x)
           combine_group(a, k, rq, Grp{(int)threadIdx.x - 32, kTcThreads - 32, 4}, s_comb);
         named_bar(3, kTcThreads - 32);
-        if (warp == 1 && lane == 0) grid_sync(gcount, ggen, gridDim.x, epoch, sy);
+        if (warp == 1 && lane == 0) grid_sync(gcount, gridDim.x, epoch, sy);
         named_bar(3, kTcThreads - 32);
       }
     }

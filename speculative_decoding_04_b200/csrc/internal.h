@@ -17,7 +17,7 @@ struct Options {
   int draft_tc_min_b = 9;        // bf16 drafts with at least this many requests use the tensor-core path
   int draft_force_path = 0;      // 0 auto, 1 CUDA-core GEMV, 2 tensor cores
   int draft_pdl = 1;             // chain the draft kernels with programmatic dependent launch
-  int draft_w2_hint = 0;         // L2 hints: W2 tiles evict-last, U tiles and l_d stores evict-first (measured slower)
+  int draft_w2_hint = 0;         // L2 hints: 1 W2 evict-last, U and l_d evict-first; 2 W2 and U only; 3 W2 only
   int draft_fused = 1;           // tensor-core draft: all steps in one cooperative launch
   int verify_cluster = 0;        // 0 auto, else the cluster size (1, 2, 4, 8, 16)
   int verify_persistent = 1;     // sampled verify / labels: persistent double-buffered clusters
