@@ -8,30 +8,34 @@
 //  §Confidence-Scheduled Verification: label c*_k = 1 - ½‖p_d - p_t‖₁]
 //
 // Layout of the work.  A cluster of C CTAs takes rows (position k, request b) in turn; CTA r
-// owns the r-th contiguous run of 512-column tiles of every row.  Per row each CTA runs
-//   P1  (tiles from HBM)  per-lane maxima and sums of 2^(z log2e - R) against an integer
-//       reference R, so that every later rescaling is an exact power of two; the sums of l_t
-//       per tile are kept for the bonus sample;
+// owns the r-th contiguous run of 512-column tiles of every row.  With c = log2(e) / T every
+// exponent is a = fma(l, c, -ref) in fp32 (l·c exact inside the fma).  Per row each CTA runs
+//   P1  (tiles from HBM)  per-lane maxima and sums of 2^a against an integer reference, so that
+//       every later rescaling is an exact power of two;
 //   --  the CTA's (R, S) pairs go to every CTA of the cluster (distributed shared memory and a
 //       remote mbarrier arrive); each CTA folds them in rank order into the row's normalisers
-//       log2 p = z log2e - K - lam (K an integer, lam in [0, 1)) and decides the acceptance;
-//   P2  (the same tiles again, now from L2)  p_d, p_t, sum min(p_d, p_t) and
-//       q = max(0, p_t - p_d) per tile (the residual sample's weights).
-// The tiles of P1 of the next row sit between P1 and P2 of a row, so the exchange never
-// stalls the tile pipeline, and a row's two reads are at most two rows of the whole grid
-// apart (a few tens of MB against a 126 MB L2).
+//       log2 p = l c - K - lam (K an integer, lam in [0, 1)) and decides the acceptance;
+//   P2  (the same tiles again, now from L2)  sum min(p_d, p_t), taken as one 2^x per column
+//       with x = min(a_d - (lam_d - lam_t), a_t) and the factor 2^-lam_t applied per tile, and
+//       whether any column has p_t > p_d (without one, q = 0 everywhere and the label is exactly
+//       1); a rejection that may be its request's first also keeps sum q per tile,
+//       q = p_t - min(p_d, p_t) (the residual sample's weights).
+// The passes of a CTA form one stream of tiles (P1 of row i, then P2 of row i - lag, and so
+// on) cut into ring stages of 16 tiles without regard to row boundaries, so a row's last
+// stage is shared with the next pass and no consumer idles at the end of a row; the exchange
+// sits between P1 and P2 of a row and never stalls the stream.  A row's two reads are at most
+// a few rows of the whole grid apart (tens of MB against a 126 MB L2).
 //
-// Roles in a CTA of 608 threads: warp 16 streams the rows through a 3-stage ring, one 32 KB bulk
-// copy per row and stage (copies of 4 KB were measured to cap the stream at under half the HBM
-// bandwidth, whatever the number of issuing threads); warps 0-15 each take one 512-column piece
-// of a stage (the assignment rotates from stage to stage, so uneven segments even out; the
-// passes are latency-bound, and 16 warps with 512 columns each measured faster than 8 with
-// 1024); warp 17 folds the warps' partials and exchanges them with the cluster; warp 18 folds the cluster's
-// partials, decides acceptance and writes the per-row records (two warps, so that a row's
-// decision never waits behind the next row's exchange).
-// A small second
-// kernel (one warp per request) finds n, samples the residual / bonus token by an inverse CDF
-// over the per-tile weights and one rescanned tile, and writes y, n and c*.
+// Roles in a CTA of 608 threads: warp 16 streams the tiles through a 3-stage ring (per stage
+// and pass one bulk copy of each row: copies of 4 KB were measured to cap the stream at under
+// half the HBM bandwidth, 32 KB ones reach it); warps 0-15 each take one 512-column tile of a
+// stage (the assignment rotates from stage to stage; the passes are latency-bound, and 16
+// warps with 512 columns each measured faster than 8 with 1024); warp 17 folds the warps'
+// partials and exchanges them with the cluster; warp 18 folds the cluster's partials, decides
+// acceptance and writes the per-row records (two warps, so that a row's decision never waits
+// behind the next row's exchange).
+// A small second kernel (one warp per request) finds n, samples the residual / bonus token by
+// an inverse CDF over the per-tile weights and one rescanned tile, and writes y, n and c*.
 // Every wait is bounded; after a timeout all roles stop and the status word is set.
 
 #include <cooperative_groups.h>
@@ -63,6 +67,8 @@ constexpr int kSvDecider = kSvWarps + 2;
 constexpr int kSvPhaseSlots = 16;
 constexpr int kSvJobSlots = 4;
 constexpr int kSvMaxCluster = 8;
+constexpr uint32_t kSvSuspendNs = 100000;            // longest single suspension of a waiting warp
+constexpr uint64_t kSvTimeoutNs = 2000000000ull;     // a wait gives up after 2 s
 constexpr int kRNone = -(1 << 28);  // reference of an empty sum
 constexpr int kRMax = 1 << 24;
 constexpr size_t kSvRingBytes = (size_t)kSvStages * 2 * kSvBig * sizeof(float);
@@ -99,23 +105,24 @@ struct SvArgs {
   const int32_t* L;
   const float* u_acc;
   const float* u_res;
-  int B, gamma, V, lt_rows, njobs, ntile, C, lag;
-  float inv_T;
+  int B, gamma, V, lt_rows, njobs, ntile, C, lag, l2hint;
+  float zscale;  // log2(e) / T (T > 0)
   int greedy, do_verify;
   float* c_star;
   int32_t* n_acc;
   int32_t* y_out;
   uint32_t* flags;
   uint32_t* status;
+  int* rej;         // [B]: gamma + 1 - k of the earliest rejection seen so far (0: none)
   SvRow* rows;      // [B][gamma+1]
-  double2* part;    // [B][gamma][C]: (sum min, sum q) of each CTA
-  float2* trec;     // [B][gamma+1][ntile]: (R, s) of l_t per tile
-  float* qrec;      // [B][gamma+1][ntile]: sum q per tile
+  double2* part;    // [B][gamma][C]: (sum min(p_d, p_t), warps that saw p_t > p_d) of each CTA
+  float2* trec;     // [B][gamma+1][ntile]: (R, s) of l_t per tile (bonus rows)
+  float* qrec;      // [B][gamma+1][ntile]: sum q per tile (rejected rows)
 };
 
 struct SvJob {
   int b, k, rec;
-  bool t, d, verify;
+  bool t, d, verify, bonus;
 };
 
 __device__ __forceinline__ SvJob sv_job(const SvArgs& a, int j) {
@@ -130,6 +137,7 @@ __device__ __forceinline__ SvJob sv_job(const SvArgs& a, int j) {
   const bool bonus = a.do_verify && J.k == Lb;
   J.d = cstar || (J.verify && !a.greedy);  // greedy acceptance needs only argmax l_t
   J.t = cstar || J.verify || bonus;
+  J.bonus = bonus;
   return J;
 }
 
@@ -156,7 +164,7 @@ struct SvPhase {
 struct SvGen {
   int j, ncl, i, step, nrows, lag;
   bool exhausted;
-  SvJob ring[4];  // rows i-L .. i
+  int r0, r1, r2, r3;  // job indices of rows i, i-1, i-2, i-3 (registers, not an indexed array)
   __device__ void init(const SvArgs& a, int cid, int ncl_) {
     ncl = ncl_;
     lag = a.lag;
@@ -164,7 +172,10 @@ struct SvGen {
     step = 0;
     nrows = 0;
     exhausted = false;
-    j = sv_next(a, cid, ncl, ring[0]);
+    SvJob J;
+    j = sv_next(a, cid, ncl, J);
+    r0 = j;
+    r1 = r2 = r3 = -1;
     if (j >= 0) nrows = 1;
     else exhausted = true;
   }
@@ -173,7 +184,7 @@ struct SvGen {
       if (step == 0) {
         step = 1;
         if (i < nrows) {
-          ph.J = ring[i & 3];
+          ph.J = sv_job(a, r0);
           ph.second = false;
           ph.i = i;
           return true;
@@ -182,19 +193,31 @@ struct SvGen {
       if (step == 1) {
         step = 2;
         const int q = i - lag;
-        if (q >= 0 && q < nrows && sv_p2(a, ring[q & 3])) {
-          ph.J = ring[q & 3];
-          ph.second = true;
-          ph.i = q;
-          return true;
+        if (q >= 0 && q < nrows) {
+          const SvJob J = sv_job(a, lag == 1 ? r1 : (lag == 2 ? r2 : r3));
+          if (sv_p2(a, J)) {
+            ph.J = J;
+            ph.second = true;
+            ph.i = q;
+            return true;
+          }
         }
       }
       ++i;
       step = 0;
+      r3 = r2;
+      r2 = r1;
+      r1 = r0;
+      r0 = -1;
       if (!exhausted) {
-        j = sv_next(a, j + ncl, ncl, ring[i & 3]);
-        if (j >= 0) nrows = i + 1;
-        else exhausted = true;
+        SvJob J;
+        j = sv_next(a, j + ncl, ncl, J);
+        if (j >= 0) {
+          nrows = i + 1;
+          r0 = j;
+        } else {
+          exhausted = true;
+        }
       }
       if (exhausted && i - lag >= nrows) return false;
     }
@@ -213,21 +236,19 @@ __device__ __forceinline__ double sv_pow2d(int d) {
 }
 __device__ __forceinline__ float sv_pow2f(int d) { return d < -126 ? 0.f : __int_as_float((127 + d) << 23); }
 
-// Integer reference for a maximum m of z: R = ceil(m log2e), clamped; kRNone for an empty max.
-__device__ __forceinline__ int sv_ref(float m) {
+// Integer reference for a maximum m of the raw logits: R = ceil(m c), clamped; kRNone for an
+// empty max.  With it every 2^fma(l, c, -R) of those logits is at most about 1.
+__device__ __forceinline__ int sv_ref(float m, float c) {
   if (!(m > -INFINITY)) return kRNone;
-  const int R = __float2int_ru(m * kLog2e);
+  const int R = __float2int_ru(m * c);
   return min(max(R, -kRMax), kRMax);
 }
 
-// (R, S) += (r, s) with exact power-of-two rescaling
-__device__ __forceinline__ void sv_merge(int& R, double& S, int r, double s) {
-  if (r > R) {
-    S = S * sv_pow2d(R - r) + s;
-    R = r;
-  } else {
-    S += s * sv_pow2d(r - R);
-  }
+// (R, S) += (r, s) in fp32 with exact power-of-two rescaling (lane sums across the tiles of a pass)
+__device__ __forceinline__ void sv_merge_f(int& R, float& S, int r, float s) {
+  const int M = max(R, r);
+  S = fmaf(S, sv_pow2f(R - M), s * sv_pow2f(r - M));
+  R = M;
 }
 
 __device__ __forceinline__ void sv_warp_ref_sum(int& R, double& S) {
@@ -236,24 +257,35 @@ __device__ __forceinline__ void sv_warp_ref_sum(int& R, double& S) {
   R = M;
 }
 
-// Same across the lanes of a warp with the lane sums rounded to fp32 first (32 terms, one
-// rounding each; the per-lane sums themselves are accumulated in fp64).
-__device__ __forceinline__ void sv_warp_ref_sum_f(int& R, double& S) {
+// Same across the lanes of a warp for fp32 lane sums (32 terms, fp32 adds).
+__device__ __forceinline__ void sv_warp_ref_sum_f(int& R, float& S) {
   const int M = __reduce_max_sync(0xffffffffu, R);
-  S = (double)warp_sum_f((float)(S * sv_pow2d(R - M)));
+  S = warp_sum_f(S * sv_pow2f(R - M));
   R = M;
 }
 
-// p_d and p_t of one column from its raw logits (shared by the second pass and the rescan
-// in the finalize kernel, so that both see the same weights).
-__device__ __forceinline__ void sv_probs(float ld, float lt, float inv_T, const SvNorm& n, float& pd, float& pt) {
-  const float zd = __fmul_rn(ld, inv_T), zt = __fmul_rn(lt, inv_T);
-  pd = sv_ex2(__fsub_rn(fmaf(zd, kLog2e, -n.Kd), n.lamd));
-  pt = sv_ex2(__fsub_rn(fmaf(zt, kLog2e, -n.Kt), n.lamt));
+// Constants of the second pass of a row: x_d = fma(l_d, c, -K_d) - (lam_d - lam_t),
+// x_t = fma(l_t, c, -K_t); then p_t = 2^x_t * 2^-lam_t and min(p_d, p_t) = 2^min(x_d, x_t) * 2^-lam_t.
+struct SvP2 {
+  float nkd, nkt, ndl;  // -K_d, -K_t, -(lam_d - lam_t)
+  float scale;          // 2^-lam_t
+};
+__device__ __forceinline__ SvP2 sv_p2_consts(const SvNorm& n) {
+  SvP2 k;
+  k.nkd = -n.Kd;
+  k.nkt = -n.Kt;
+  k.ndl = -__fsub_rn(n.lamd, n.lamt);
+  k.scale = (float)exp2(-(double)n.lamt);
+  return k;
 }
-__device__ __forceinline__ float sv_pt(float lt, float inv_T, const SvNorm& n) {
-  return sv_ex2(__fsub_rn(fmaf(__fmul_rn(lt, inv_T), kLog2e, -n.Kt), n.lamt));
+// Unscaled terms of one column (the second pass computes the same values two columns at a time
+// with packed instructions, which round each element exactly like these).
+__device__ __forceinline__ void sv_p2_terms(float ld, float lt, float c, const SvP2& k, float& pt, float& mn) {
+  const float xd = __fadd_rn(fmaf(ld, c, k.nkd), k.ndl), xt = fmaf(lt, c, k.nkt);
+  pt = sv_ex2(xt);
+  mn = sv_ex2(fminf(xd, xt));
 }
+__device__ __forceinline__ float sv_pt_term(float lt, float c, const SvP2& k) { return sv_ex2(fmaf(lt, c, k.nkt)); }
 
 // Normalisers (K, lam) from (R, S): S = f 2^e with f in [0.5, 1), K = R + e - 1, lam = log2(2f).
 __device__ __forceinline__ bool sv_norm(int R, double S, float& K, float& lam) {
@@ -301,16 +333,33 @@ __device__ __forceinline__ SvPart sv_fold(SvPart p) {
   return r;
 }
 
-__device__ __forceinline__ bool sv_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+// One wait on the phase with the given parity that suspends the warp until the phase completes
+// or kSvSuspendNs pass (the hardware wakes it on completion), instead of polling in a loop.
+__device__ __forceinline__ bool sv_try_wait_suspend(uint64_t* bar, uint32_t parity, bool cluster_scope) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
+  if (cluster_scope)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSvSuspendNs)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSvSuspendNs)
+        : "memory");
   return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t sv_now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
 }
 
 // Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster; the
@@ -333,15 +382,37 @@ struct SvSync {
   uint32_t* status;
 };
 
+// Bounded wait: gives up (setting the abort flag and the status word) after kSvTimeoutNs, or
+// returns false at once when another role has given up.
 __device__ __forceinline__ bool sv_wait(const SvSync& s, uint64_t* bar, uint32_t parity, bool cluster_scope = false) {
   if (*s.abort) return false;
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (cluster_scope ? sv_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 1023u && *s.abort) return false;
+  if (sv_try_wait_suspend(bar, parity, cluster_scope)) return true;
+  const uint64_t t0 = sv_now_ns();
+  while (true) {
+    if (sv_try_wait_suspend(bar, parity, cluster_scope)) return true;
+    if (*s.abort) return false;
+    if (sv_now_ns() - t0 > kSvTimeoutNs) break;
   }
   *s.abort = 1;
   atomicOr(s.status, (uint32_t)DSPARK_ETIMEOUT);
   return false;
+}
+
+// Bounded wait until a shared counter reaches `target` (counters written by another warp of
+// the CTA), with a short sleep between polls.
+__device__ __forceinline__ bool sv_wait_count(const SvSync& s, volatile int* cnt, int target) {
+  if (*cnt >= target) return true;
+  const uint64_t t0 = sv_now_ns();
+  while (*cnt < target) {
+    if (*s.abort) return false;
+    if (sv_now_ns() - t0 > kSvTimeoutNs) {
+      *s.abort = 1;
+      atomicOr(s.status, (uint32_t)DSPARK_ETIMEOUT);
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
 }
 
 __device__ __forceinline__ float f4c(const float4& v, int c) { return c == 0 ? v.x : (c == 1 ? v.y : (c == 2 ? v.z : v.w)); }
@@ -378,29 +449,34 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
 
-// First pass over one lane's 32 values of a tile: z = l * (1/T) in place, the integer
-// reference R of their maximum and the fp32 sum of 2^(z log2e - R).
-__device__ __forceinline__ float sv_lane_sum(float4 (&v)[kSvVec], float2 invT2, int& R) {
+// First pass over one lane's 16 values of a tile row: the integer reference R of their maximum
+// and the fp32 sum of 2^fma(l, c, -R).
+__device__ __forceinline__ float sv_lane_sum(const float4 (&v)[kSvVec], float c, int& R) {
   float m = -INFINITY;
 #pragma unroll
   for (int jj = 0; jj < kSvVec; ++jj) {
-    const float2 a = f2mul(lo2(v[jj]), invT2), b = f2mul(hi2(v[jj]), invT2);
-    v[jj] = make_float4(a.x, a.y, b.x, b.y);
-    m = fmax3(m, a.x, a.y);
-    m = fmax3(m, b.x, b.y);
+    m = fmax3(m, v[jj].x, v[jj].y);
+    m = fmax3(m, v[jj].z, v[jj].w);
   }
-  R = sv_ref(m);
-  const float2 l2e2 = make_float2(kLog2e, kLog2e), nr2 = make_float2(-(float)R, -(float)R);
+  R = sv_ref(m, c);
+  const float2 c2 = make_float2(c, c), nr2 = make_float2(-(float)R, -(float)R);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int jj = 0; jj < kSvVec; ++jj) {
-    const float2 a = f2fma(lo2(v[jj]), l2e2, nr2), b = f2fma(hi2(v[jj]), l2e2, nr2);
-    acc0 = f2add(acc0, make_float2(sv_ex2(a.x), sv_ex2(a.y)));
-    acc1 = f2add(acc1, make_float2(sv_ex2(b.x), sv_ex2(b.y)));
+    const float2 x = f2fma(lo2(v[jj]), c2, nr2), y = f2fma(hi2(v[jj]), c2, nr2);
+    acc0 = f2add(acc0, make_float2(sv_ex2(x.x), sv_ex2(x.y)));
+    acc1 = f2add(acc1, make_float2(sv_ex2(y.x), sv_ex2(y.y)));
   }
   const float2 acc = f2add(acc0, acc1);
   return acc.x + acc.y;
 }
+
+// Decision of a row for its second pass.
+struct __align__(16) SvDec {
+  SvNorm nm;
+  int needq;  // rejected: the second pass also sums the residual weights q
+  int pad0, pad1, pad2;
+};
 
 template <bool GREEDY>
 __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
@@ -416,9 +492,10 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   __shared__ __align__(8) uint64_t xbar[kSvJobSlots], dbar[kSvJobSlots];
   __shared__ SvPart wpart[kSvPhaseSlots][kSvWarps];
   __shared__ SvPart xs[kSvJobSlots][kSvMaxCluster];
-  __shared__ SvNorm dec[kSvJobSlots];
+  __shared__ SvDec dec[kSvJobSlots];
   __shared__ int s_abort;
   __shared__ volatile int s_decided;  // rows of this cluster's sequence decided by this CTA
+  __shared__ volatile int s_combined;  // passes whose warp partials the combiner has read
 
   const SvSync sy{&s_abort, a.status};
   if (threadIdx.x == 0) {
@@ -433,65 +510,74 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     }
     s_abort = 0;
     s_decided = 0;
+    s_combined = 0;
     fence_mbar_init();
   }
   __syncthreads();
   sv_cluster_sync_all();  // peers' barriers are initialised before any remote arrive
 
+  // This CTA's segment of every row: tiles tb .. tb + nt - 1.  Pass number p of the CTA's
+  // sequence covers tiles p*nt .. p*nt + nt - 1 of the CTA's tile stream; stage g of the ring
+  // holds stream tiles 16g .. 16g + 15.
   const int tb = (int)((long long)rank * a.ntile / C);
-  const int nt = (int)((long long)(rank + 1) * a.ntile / C) - tb;  // tiles of this CTA per row (may be 0)
-  const float inv_T = a.inv_T;
-
-  const int nbig = (nt + kSvGroupWarps - 1) / kSvGroupWarps;  // ring stages per row and pass
-  const int c_end = min((tb + nt) * kSvTile, a.V);     // end column of this CTA's segment
+  const int nt = (int)((long long)(rank + 1) * a.ntile / C) - tb;  // may be 0
+  const float zc = a.zscale;
 
   if (warp == kSvProducer) {
     // ------------------------------------------------------------------ bulk copies
-    // Stage gb of the stream holds up to 8192 columns of both rows: one copy per row.  A bulk
-    // copy costs the copy engine about the same time whatever its size (measured on this part:
-    // 4 KB copies stream at under half the HBM bandwidth, 32 KB ones at full bandwidth).
-    if (lane < 2) {
+    if (lane == 0) {
+      const uint64_t pol_last = l2_policy_evict_last(), pol_first = l2_policy_evict_first();
       SvGen gen;
       gen.init(a, cid, ncl);
       SvPhase ph;
-      uint32_t Gb = 0;
+      bool have = nt > 0 && gen.next(a, ph);
+      int pbase = 0;  // first stream tile of the pass ph
+      uint32_t g = 0;
       bool ok = true;
-      while (ok && gen.next(a, ph)) {
-        const bool with_d = ph.second || ph.J.d;
-        const float* rd = a.ld + ((size_t)ph.J.k * a.B + ph.J.b) * a.V;
-        const float* rt = a.lt + ((size_t)ph.J.b * a.lt_rows + ph.J.k) * a.V;
-        for (int bt = 0; bt < nbig; ++bt) {
-          const uint32_t gb = Gb + bt;
-          const int s = (int)(gb % kSvStages);
-          // lane 0 arms the stage and copies l_d, lane 1 copies l_t
-          if (!sv_wait(sy, &empty[s], ((gb / kSvStages) & 1) ^ 1)) {
-            ok = false;
-            break;
-          }
-          const int v0 = (tb + bt * kSvGroupWarps) * kSvTile;
-          const uint32_t bytes = (uint32_t)min(kSvBig, c_end - v0) * 4u;
-          float* st = ring + (size_t)s * 2 * kSvBig;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[s], with_d ? 2 * bytes : bytes);
-            if (with_d) bulk_g2s(st, rd + v0, bytes, &full[s]);
-          } else {
-            bulk_g2s(st + kSvBig, rt + v0, bytes, &full[s]);
-          }
+      for (; have; ++g) {
+        const int s = (int)(g % kSvStages);
+        if (!sv_wait(sy, &empty[s], ((g / kSvStages) & 1) ^ 1)) {
+          ok = false;
+          break;
         }
-        Gb += (uint32_t)nbig;
+        const int T0 = (int)g * kSvGroupWarps, T1 = T0 + kSvGroupWarps;
+        float* stg = ring + (size_t)s * 2 * kSvBig;
+        // one copy per row for each pass that has tiles in this stage
+        while (have && pbase < T1) {
+          const int lo = max(T0, pbase), hi = min(T1, pbase + nt);
+          const int c0 = (tb + lo - pbase) * kSvTile, c1 = min((tb + hi - pbase) * kSvTile, a.V);
+          const uint32_t bytes = (uint32_t)(c1 - c0) * 4u;
+          const bool with_d = ph.second || ph.J.d;
+          const float* rd = a.ld + ((size_t)ph.J.k * a.B + ph.J.b) * a.V;
+          const float* rt = a.lt + ((size_t)ph.J.b * a.lt_rows + ph.J.k) * a.V;
+          mbar_expect_tx(&full[s], with_d ? 2 * bytes : bytes);
+          if (a.l2hint) {
+            // first pass: keep the lines for the second; second pass: they are done with
+            const uint64_t pol = (ph.second || !sv_p2(a, ph.J)) ? pol_first : pol_last;
+            if (with_d) bulk_g2s_hint(stg + (lo - T0) * kSvTile, rd + c0, bytes, &full[s], pol);
+            bulk_g2s_hint(stg + kSvBig + (lo - T0) * kSvTile, rt + c0, bytes, &full[s], pol);
+          } else {
+            if (with_d) bulk_g2s(stg + (lo - T0) * kSvTile, rd + c0, bytes, &full[s]);
+            bulk_g2s(stg + kSvBig + (lo - T0) * kSvTile, rt + c0, bytes, &full[s]);
+          }
+          if (hi < pbase + nt) break;  // the pass goes on in the next stage
+          have = gen.next(a, ph);
+          pbase += nt;
+        }
+        mbar_arrive(&full[s]);
       }
       if (!ok) {
         // let the copies still in flight land before the CTA can exit
-        const uint32_t lo = Gb > (uint32_t)kSvStages ? Gb - kSvStages : 0u;
-        for (uint32_t gb = lo; gb < Gb; ++gb)
+        const uint32_t lo = g > (uint32_t)kSvStages ? g - kSvStages : 0u;
+        for (uint32_t gb = lo; gb < g; ++gb)
           for (uint32_t i = 0; i < kSpinLimit && !mbar_try_wait(&full[gb % kSvStages], (gb / kSvStages) & 1); ++i) {
           }
       }
     }
   } else if (warp == kSvCombiner) {
     // ------------------------------------------------------------------ combine and exchange
-    // Per first pass: fold the eight warps' partials and push the CTA's into slot [i % 4][rank]
-    // of every CTA of the cluster.  Per second pass: the CTA's label partials to global memory.
+    // Per first pass: fold the warps' partials and push the CTA's into slot [i % 4][rank] of
+    // every CTA of the cluster.  Per second pass: the CTA's label partials to global memory.
     // A push for row i waits until this CTA has decided row i-2: a peer that has decided row
     // i-2 has then seen this CTA's push of row i-2, so every peer has decided row i-4, the
     // previous user of the slot (the second passes give the same order when T > 0; greedy
@@ -507,18 +593,13 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       ++p;
       if (!ok) break;
       SvPart w = lane < kSvWarps ? wpart[ps][lane] : sv_empty_part();
+      __syncwarp();
+      __threadfence_block();  // the slot's reads come before the count that frees it
+      if (lane == 0) s_combined = p;
       if (!ph.second) {
         w = sv_fold<GREEDY>(w);
         const int i = ph.i;
-        for (uint32_t t = 0; s_decided < i - 1; ++t)  // s_decided counts rows, so row i-2 is decided
-          if (t >= kSpinLimit || *sy.abort) {
-            if (!*sy.abort) {
-              *sy.abort = 1;
-              atomicOr(sy.status, (uint32_t)DSPARK_ETIMEOUT);
-            }
-            ok = false;
-            break;
-          }
+        ok = sv_wait_count(sy, &s_decided, i - 1);  // s_decided counts rows, so row i-2 is decided
         if (!ok) break;
         if (lane < C) {
           SvPart* dst = cluster.map_shared_rank(&xs[i % kSvJobSlots][rank], lane);
@@ -526,9 +607,9 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           sv_remote_arrive(&xbar[i % kSvJobSlots], lane);
         }
       } else {
-        const double sm = warp_sum_d(w.sd), sq = warp_sum_d(w.st);
+        const double sm = warp_sum_d(w.sd), nq = warp_sum_d(w.st);
         if (lane == 0 && ph.J.k < a.gamma)
-          a.part[((size_t)ph.J.b * a.gamma + ph.J.k) * C + rank] = make_double2(sm, sq);
+          a.part[((size_t)ph.J.b * a.gamma + ph.J.k) * C + rank] = make_double2(sm, nq);
       }
     }
   } else if (warp == kSvDecider) {
@@ -575,23 +656,27 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
         else nm.Kd = nm.lamd = 0.f;
         if (!good) dfl |= DSPARK_FLAG_NONFINITE;
         row.nm = nm;
-        if (lane == 0) dec[js] = nm;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dbar[js]);  // the second pass of this row may start
         if (J.verify) {
           if ((unsigned)xk >= (unsigned)a.V) {
             dfl |= DSPARK_FLAG_TOKEN_RANGE;
           } else {
-            // u p_d(x) < p_t(x) with p = 2^(z log2e - R) / S, in fp64
-            const double l2e = (double)kLog2e;
-            const double zd = (double)__fmul_rn(ldx, inv_T), zt = (double)__fmul_rn(ltx, inv_T);
-            const double pd = exp2(zd * l2e - (double)x.rd) / x.sd;
-            const double pt = exp2(zt * l2e - (double)x.rt) / x.st;
+            // u p_d(x) < p_t(x) with p = 2^(l c - R) / S, in fp64 (l c is exact there)
+            const double pd = exp2((double)ldx * (double)zc - (double)x.rd) / x.sd;
+            const double pt = exp2((double)ltx * (double)zc - (double)x.rt) / x.st;
             const double u = (double)u_acc;
             row.acc = (u * pd < pt) ? 1 : 0;
             if (pd > 0.0 && fabs(u - pt / pd) < 1e-6) row.fl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
           }
         }
+        // residual weights only for a rejection that may be the request's first (the others are
+        // never sampled); a rejection is published for the deciders of later rows
+        const int enc = a.gamma + 1 - J.k;
+        const bool rej = J.verify && !row.acc;
+        const bool needq = rej && __ldcg(a.rej + J.b) <= enc;
+        if (lane == 0) dec[js] = SvDec{nm, needq ? 1 : 0, 0, 0, 0};
+        if (rej && rank == 0 && lane == 0) atomicMax(a.rej + J.b, enc);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dbar[js]);  // the second pass of this row may start
       }
       if (rank == 0 && lane == 0) {
         a.rows[J.rec] = row;
@@ -605,117 +690,45 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   } else {
     // ------------------------------------------------------------------ tile consumers
     const int w = warp;
-    uint32_t Gb = 0;
-    int p = 0;
+    const int last_tile = a.ntile - 1 - tb;  // the segment's ragged tile, if it has it
+    const int last_cnt = a.V - (a.ntile - 1) * kSvTile;
+    const float2 c2 = make_float2(zc, zc);
     bool ok = true;
-    auto run_phase = [&](const SvJob& J, bool second, int i) {
+    int p = 0;  // passes finished by this warp (slot of the partials)
+    // state of the current pass
+    int Rd = kRNone, Rt = kRNone;
+    float Sd = 0.f, St = 0.f;
+    Top2 gd{-INFINITY, -1, -INFINITY}, gt{-INFINITY, -1, -INFINITY};
+    uint32_t bad = 0;
+    float smin = 0.f;       // second pass: unscaled sum of 2^min(x_d, x_t)
+    float dqmax = -INFINITY;  // second pass: max of x_t - x_d (> 0: some column has p_t > p_d)
+    SvP2 k2{0.f, 0.f, 0.f, 1.f};
+    bool needq = false;
+
+    SvGen cgen;
+    cgen.init(a, cid, ncl);
+    SvPhase ph;
+    auto start = [&]() {
+      Rd = Rt = kRNone;
+      Sd = St = 0.f;
+      gd = Top2{-INFINITY, -1, -INFINITY};
+      gt = Top2{-INFINITY, -1, -INFINITY};
+      bad = 0;
+      smin = 0.f;
+      dqmax = -INFINITY;
+      if (ph.second) {
+        const int js = ph.i % kSvJobSlots;
+        ok = __all_sync(0xffffffffu, sv_wait(sy, &dbar[js], (ph.i / kSvJobSlots) & 1));
+        if (ok) {
+          const SvDec dd = dec[js];
+          k2 = sv_p2_consts(dd.nm);
+          needq = dd.needq != 0;
+        }
+      }
+    };
+    auto finish = [&]() {
       SvPart out = sv_empty_part();
-      // first pass state (per lane)
-      int Rd = kRNone, Rt = kRNone;
-      double Sd = 0.0, St = 0.0;
-      Top2 gd{-INFINITY, -1, -INFINITY}, gt{-INFINITY, -1, -INFINITY};
-      uint32_t bad = 0;
-      // second pass state
-      double smin = 0.0, sq = 0.0;
-      SvNorm nm{0.f, 0.f, 0.f, 0.f};
-      if (second) {
-        const int js = i % kSvJobSlots;
-        ok = sv_wait(sy, &dbar[js], (i / kSvJobSlots) & 1);
-        if (ok) nm = dec[js];
-      }
-      const bool with_d = second || J.d;
-      for (int bt = 0; ok && bt < nbig; ++bt) {
-        const uint32_t gb = Gb + bt;
-        if ((int)(gb % kSvGroups) != w / kSvGroupWarps) continue;  // the other group's stage
-        const int s = (int)(gb % kSvStages);
-        if (!sv_wait(sy, &full[s], (gb / kSvStages) & 1)) {
-          ok = false;
-          break;
-        }
-        // this warp's 1024-column piece of the stage; the assignment rotates from stage to stage
-        const int q = ((w % kSvGroupWarps) + (int)(gb / kSvGroups)) % kSvGroupWarps;
-        const int t = bt * kSvGroupWarps + q;  // tile of this CTA's segment
-        const bool mine = t < nt;
-        const int v0 = (tb + t) * kSvTile;
-        const int cnt = mine ? min(kSvTile, a.V - v0) : 0;
-        const float* sd = ring + (size_t)s * 2 * kSvBig + q * kSvTile;
-        const float* st = sd + kSvBig;
-        float4 fd[kSvVec], ft[kSvVec];
-        const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-#pragma unroll
-        for (int jj = 0; jj < kSvVec; ++jj) {
-          const int idx = (jj * 32 + lane) * 4;
-          const bool v = idx < cnt;
-          ft[jj] = v ? *reinterpret_cast<const float4*>(st + idx) : ninf;
-          fd[jj] = (v && with_d) ? *reinterpret_cast<const float4*>(sd + idx) : ninf;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // the values are in registers
-        if (!mine) continue;
-        if (!second) {
-          if (GREEDY) {
-#pragma unroll
-            for (int jj = 0; jj < kSvVec; ++jj) {
-              const int base = v0 + (jj * 32 + lane) * 4;
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const float vt = f4c(ft[jj], c), vd = f4c(fd[jj], c);
-                bad |= (isnan(vt) || vt == INFINITY || isnan(vd) || vd == INFINITY) ? 1u : 0u;
-                if (vt > -INFINITY) top2_push(gt, vt, base + c);
-                if (with_d && vd > -INFINITY) top2_push(gd, vd, base + c);
-              }
-            }
-          } else {
-            const float2 invT2 = make_float2(inv_T, inv_T);
-            int rt;
-            const float stl = sv_lane_sum(ft, invT2, rt);
-            bad |= (stl <= FLT_MAX) ? 0u : 1u;
-            sv_merge(Rt, St, rt, (double)stl);
-            if (a.do_verify) {
-              // l_t weight of the tile for the bonus / fallback sample
-              const int R = __reduce_max_sync(0xffffffffu, rt);
-              const float sw = warp_sum_f(stl * sv_pow2f(rt - R));
-              if (lane == 0) a.trec[(size_t)J.rec * a.ntile + tb + t] = make_float2((float)R, sw);
-            }
-            if (with_d) {
-              int rd;
-              const float sdl = sv_lane_sum(fd, invT2, rd);
-              bad |= (sdl <= FLT_MAX) ? 0u : 1u;
-              sv_merge(Rd, Sd, rd, (double)sdl);
-            }
-          }
-        } else {
-          // p = 2^(z log2e - K - lam) for both rows; sum min(p_d, p_t) and q = p_t - min
-          const float2 invT2 = make_float2(inv_T, inv_T), l2e2 = make_float2(kLog2e, kLog2e);
-          const float2 nkd = make_float2(-nm.Kd, -nm.Kd), nkt = make_float2(-nm.Kt, -nm.Kt);
-          const float2 nld = make_float2(-nm.lamd, -nm.lamd), nlt = make_float2(-nm.lamt, -nm.lamt);
-          float2 sm2 = make_float2(0.f, 0.f), q2 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int jj = 0; jj < kSvVec; ++jj) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
-              const float2 ad = f2add(f2fma(f2mul(ld2, invT2), l2e2, nkd), nld);
-              const float2 at = f2add(f2fma(f2mul(lt2, invT2), l2e2, nkt), nlt);
-              const float2 pt = make_float2(sv_ex2(at.x), sv_ex2(at.y));
-              const float2 mn = make_float2(fminf(sv_ex2(ad.x), pt.x), fminf(sv_ex2(ad.y), pt.y));
-              sm2 = f2add(sm2, mn);
-              q2 = f2add(q2, make_float2(pt.x - mn.x, pt.y - mn.y));
-            }
-          }
-          const float sml = sm2.x + sm2.y, ql = q2.x + q2.y;
-          smin += (double)sml;
-          sq += (double)ql;
-          if (J.verify) {
-            const float qw = warp_sum_f(ql);
-            if (lane == 0) a.qrec[(size_t)J.rec * a.ntile + tb + t] = qw;
-          }
-        }
-      }
-      Gb += (uint32_t)nbig;
-      if (!ok) return;
-      // ---- phase result of this warp
-      if (!second) {
+      if (!ph.second) {
         if (GREEDY) {
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
@@ -728,26 +741,147 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           sv_warp_ref_sum_f(Rd, Sd);
           sv_warp_ref_sum_f(Rt, St);
           out.rd = Rd;
-          out.sd = Sd;
+          out.sd = (double)Sd;
           out.rt = Rt;
-          out.st = St;
+          out.st = (double)St;
         }
         out.fl = __any_sync(0xffffffffu, bad != 0) ? (uint32_t)DSPARK_FLAG_NONFINITE : 0u;
       } else {
-        out.sd = (double)warp_sum_f((float)smin);
-        out.st = (double)warp_sum_f((float)sq);
+        out.sd = (double)warp_sum_f(smin) * (double)k2.scale;
+        out.st = __any_sync(0xffffffffu, dqmax > 0.f) ? 1.0 : 0.0;
       }
       const int ps = p % kSvPhaseSlots;
+      // the slot's previous pass (p - 16) must have been read: without a pass that waits for a
+      // decision (greedy verification, or a CTA whose segment is empty) nothing else bounds
+      // how far the warps run ahead of the combiner
+      ok = __all_sync(0xffffffffu, sv_wait_count(sy, &s_combined, p - kSvPhaseSlots + 1));
+      if (!ok) return;
       if (lane == 0) {
         wpart[ps][w] = out;
         mbar_arrive(&phbar[ps]);
       }
       ++p;
     };
-    SvGen cgen;
-    cgen.init(a, cid, ncl);
-    SvPhase ph;
-    while (ok && cgen.next(a, ph)) run_phase(ph.J, ph.second, ph.i);
+
+    bool have = cgen.next(a, ph);
+    if (have) start();
+    int pbase = 0;
+    for (uint32_t g = 0; ok && have; ++g) {
+      const int q = (w + (int)g) & (kSvGroupWarps - 1);  // slot of this warp in stage g
+      const int T = (int)g * kSvGroupWarps + q;
+      while (T >= pbase + nt) {  // passes that end before this tile
+        finish();
+        if (!ok) break;
+        have = cgen.next(a, ph);
+        pbase += nt;
+        if (!have) break;
+        start();
+        if (!ok) break;
+      }
+      if (!have || !ok) break;
+      const int s = (int)(g % kSvStages);
+      if (!__all_sync(0xffffffffu, sv_wait(sy, &full[s], (g / kSvStages) & 1))) {
+        ok = false;
+        break;
+      }
+      const int t = T - pbase;  // tile of this CTA's segment
+      const int v0 = (tb + t) * kSvTile;
+      const float* sd = ring + (size_t)s * 2 * kSvBig + q * kSvTile;
+      const float* st = sd + kSvBig;
+      const bool with_d = ph.second || ph.J.d;
+      float4 fd[kSvVec], ft[kSvVec];
+      if (t != last_tile) {
+#pragma unroll
+        for (int jj = 0; jj < kSvVec; ++jj) {
+          const int idx = (jj * 32 + lane) * 4;
+          ft[jj] = *reinterpret_cast<const float4*>(st + idx);
+          fd[jj] = with_d ? *reinterpret_cast<const float4*>(sd + idx) : ft[jj];
+        }
+      } else {
+        const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+#pragma unroll
+        for (int jj = 0; jj < kSvVec; ++jj) {
+          const int idx = (jj * 32 + lane) * 4;
+          const bool v = idx < last_cnt;
+          ft[jj] = v ? *reinterpret_cast<const float4*>(st + idx) : ninf;
+          fd[jj] = (v && with_d) ? *reinterpret_cast<const float4*>(sd + idx) : ninf;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // the values are in registers
+      if (!ph.second) {
+        if (GREEDY) {
+#pragma unroll
+          for (int jj = 0; jj < kSvVec; ++jj) {
+            const int base = v0 + (jj * 32 + lane) * 4;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float vt = f4c(ft[jj], c), vd = f4c(fd[jj], c);
+              bad |= (isnan(vt) || vt == INFINITY || isnan(vd) || vd == INFINITY) ? 1u : 0u;
+              if (vt > -INFINITY) top2_push(gt, vt, base + c);
+              if (with_d && vd > -INFINITY) top2_push(gd, vd, base + c);
+            }
+          }
+        } else {
+          int rt;
+          const float stl = sv_lane_sum(ft, zc, rt);
+          bad |= (stl <= FLT_MAX) ? 0u : 1u;
+          sv_merge_f(Rt, St, rt, stl);
+          if (ph.J.bonus) {
+            // l_t weight of the tile for the bonus sample
+            const int R = __reduce_max_sync(0xffffffffu, rt);
+            const float sw = warp_sum_f(stl * sv_pow2f(rt - R));
+            if (lane == 0) a.trec[(size_t)ph.J.rec * a.ntile + tb + t] = make_float2((float)R, sw);
+          }
+          if (with_d) {
+            int rd;
+            const float sdl = sv_lane_sum(fd, zc, rd);
+            bad |= (sdl <= FLT_MAX) ? 0u : 1u;
+            sv_merge_f(Rd, Sd, rd, sdl);
+          }
+        }
+      } else {
+        // 2^min(x_d, x_t) per column, unscaled, and the max of x_t - x_d; a rejected row also
+        // keeps its tile's sum of q = 2^x_t - 2^min(x_d, x_t)
+        const float2 nkd = make_float2(k2.nkd, k2.nkd), nkt = make_float2(k2.nkt, k2.nkt);
+        const float2 ndl = make_float2(k2.ndl, k2.ndl), mone = make_float2(-1.f, -1.f);
+        float2 sm2 = make_float2(0.f, 0.f);
+        if (!needq) {
+          if (a.c_star) {
+#pragma unroll
+            for (int jj = 0; jj < kSvVec; ++jj) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
+                const float2 xd = f2add(f2fma(ld2, c2, nkd), ndl), xt = f2fma(lt2, c2, nkt);
+                sm2 = f2add(sm2, make_float2(sv_ex2(fminf(xd.x, xt.x)), sv_ex2(fminf(xd.y, xt.y))));
+                const float2 df = f2fma(xd, mone, xt);
+                dqmax = fmax3(dqmax, df.x, df.y);
+              }
+            }
+          }
+        } else {
+          float2 q2 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int jj = 0; jj < kSvVec; ++jj) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
+              const float2 xd = f2add(f2fma(ld2, c2, nkd), ndl), xt = f2fma(lt2, c2, nkt);
+              const float2 mn = make_float2(sv_ex2(fminf(xd.x, xt.x)), sv_ex2(fminf(xd.y, xt.y)));
+              const float2 pt = make_float2(sv_ex2(xt.x), sv_ex2(xt.y));
+              sm2 = f2add(sm2, mn);
+              q2 = f2add(q2, f2fma(mn, mone, pt));
+              const float2 df = f2fma(xd, mone, xt);
+              dqmax = fmax3(dqmax, df.x, df.y);
+            }
+          }
+          const float qw = warp_sum_f(q2.x + q2.y);
+          if (lane == 0) a.qrec[(size_t)ph.J.rec * a.ntile + tb + t] = qw * k2.scale;
+        }
+        smin += sm2.x + sm2.y;
+      }
+    }
   }
 
   __syncwarp();
@@ -756,18 +890,30 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
 
 // Inverse-CDF sample of row `rec` (one warp): weights q = max(0, p_t - p_d) when `resid`
 // (falling back to p_t when their sum is 0), else p_t.  Tile weights come from the records of
-// the main kernel; the tile holding u * W is rescanned element by element.
+// the main kernel (q of a rejected row, p_t of the bonus row); the p_t fallback of a rejected
+// row, which only an empty residual reaches, sums its tiles here.  The tile holding u * W is
+// rescanned element by element with the second pass's arithmetic.
 __device__ int sv_sample(const SvArgs& a, int b, int k, bool resid, const SvNorm& nm, uint32_t& fl) {
   const int lane = threadIdx.x & 31;
   const size_t rec = (size_t)b * (a.gamma + 1) + k;
   const float2* tr = a.trec + rec * a.ntile;
   const float* qr = a.qrec + rec * a.ntile;
+  const bool has_trec = !resid;  // the bonus row
+  const SvP2 k2 = sv_p2_consts(nm);
+  const float zc = a.zscale;
+  const float* rowd = a.ld + ((size_t)k * a.B + b) * a.V;
+  const float* rowt = a.lt + ((size_t)b * a.lt_rows + k) * a.V;
   const int per = (a.ntile + 31) / 32;
   const int t_lo = min(lane * per, a.ntile), t_hi = min(t_lo + per, a.ntile);
   auto tile_w = [&](int t, bool use_q) -> double {
     if (use_q) return (double)qr[t];
-    const float2 v = tr[t];  // (R, s): mass s * 2^(R - K_t - lam_t)
-    return (double)v.y * exp2((double)v.x - (double)nm.Kt - (double)nm.lamt);
+    if (has_trec) {
+      const float2 v = tr[t];  // (R, s): mass s * 2^(R - K_t - lam_t)
+      return (double)v.y * exp2((double)v.x - (double)nm.Kt - (double)nm.lamt);
+    }
+    double sum = 0.0;
+    for (int v = t * kSvTile, e = min(v + kSvTile, a.V); v < e; ++v) sum += (double)(sv_pt_term(rowt[v], zc, k2) * k2.scale);
+    return sum;
   };
   double own = 0.0;
   for (int t = t_lo; t < t_hi; ++t) own += tile_w(t, resid);
@@ -821,8 +967,6 @@ __device__ int sv_sample(const SvArgs& a, int b, int k, bool resid, const SvNorm
   // ---- rescan the tile: lane l takes columns v0 + 32 l .. v0 + 32 l + 31
   const int v0 = c * kSvTile;
   const int cnt = min(kSvTile, a.V - v0);
-  const float* rowd = a.ld + ((size_t)k * a.B + b) * a.V + v0;
-  const float* rowt = a.lt + ((size_t)b * a.lt_rows + k) * a.V + v0;
   float val[32];
   double lsum = 0.0;
 #pragma unroll
@@ -831,11 +975,11 @@ __device__ int sv_sample(const SvArgs& a, int b, int k, bool resid, const SvNorm
     float w = 0.f;
     if (i < cnt) {
       if (resid) {
-        float pd, pt;
-        sv_probs(rowd[i], rowt[i], a.inv_T, nm, pd, pt);
-        w = pt - fminf(pd, pt);
+        float pt, mn;
+        sv_p2_terms(rowd[v0 + i], rowt[v0 + i], zc, k2, pt, mn);
+        w = __fmul_rn(__fsub_rn(pt, mn), k2.scale);
       } else {
-        w = sv_pt(rowt[i], a.inv_T, nm);
+        w = __fmul_rn(sv_pt_term(rowt[v0 + i], zc, k2), k2.scale);
       }
     }
     val[e] = w;
@@ -890,13 +1034,14 @@ __global__ void __launch_bounds__(128) verify_stream_finalize(SvArgs a) {
       if (a.greedy) {
         cs = rr[k].cstar;
       } else {
-        double sm = 0.0, sq = 0.0;
+        // sum min(p_d, p_t); exactly 1 when no column has p_t > p_d (then q = 0 everywhere)
+        double sm = 0.0, nq = 0.0;
         for (int r = 0; r < a.C; ++r) {
           const double2 v = a.part[((size_t)b * G + k) * a.C + r];
           sm += v.x;
-          sq += v.y;
+          nq += v.y;
         }
-        cs = (float)(sq <= 0.5 ? 1.0 - sq : sm);
+        cs = nq > 0.0 ? (float)fmin(sm, 1.0) : 1.f;
       }
       a.c_star[(size_t)b * G + k] = cs;
     }
@@ -929,14 +1074,15 @@ __global__ void __launch_bounds__(128) verify_stream_finalize(SvArgs a) {
 }
 
 struct SvLayout {
-  size_t rows, part, trec, qrec, total;
+  size_t rej, rows, part, trec, qrec, total;
 };
 
 SvLayout sv_layout(int B, int gamma, int V) {
   const size_t R = (size_t)B * (gamma + 1);
   const size_t nt = (size_t)(V + kSvTile - 1) / kSvTile;
   SvLayout L;
-  L.rows = kWsHeader;
+  L.rej = kWsHeader;
+  L.rows = L.rej + align_up((size_t)B * sizeof(int), 256);
   L.part = L.rows + align_up(R * sizeof(SvRow), 256);
   L.trec = L.part + align_up((size_t)B * gamma * kSvMaxCluster * sizeof(double2), 256);
   L.qrec = L.trec + align_up(R * nt * sizeof(float2), 256);
@@ -972,14 +1118,16 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.njobs = c.B * (c.gamma + 1);
   a.ntile = (c.V + kSvTile - 1) / kSvTile;
   a.lag = std::min(std::max(options().verify_stream_lag, 1), 3);
+  a.l2hint = options().verify_stream_l2hint;
   a.greedy = c.T == 0.f ? 1 : 0;
-  a.inv_T = a.greedy ? 1.f : 1.f / c.T;
+  a.zscale = a.greedy ? 0.f : (float)(1.4426950408889634 / (double)c.T);
   a.do_verify = 1;
   a.c_star = c.c_star;
   a.n_acc = c.n_acc;
   a.y_out = c.y_out;
   a.flags = c.flags;
   a.status = reinterpret_cast<uint32_t*>(ws);
+  a.rej = reinterpret_cast<int*>(ws + Ly.rej);
   a.rows = reinterpret_cast<SvRow*>(ws + Ly.rows);
   a.part = reinterpret_cast<double2*>(ws + Ly.part);
   a.trec = reinterpret_cast<float2*>(ws + Ly.trec);
@@ -995,7 +1143,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
     }
     attr_set[a.greedy] = true;
   }
-  rc = cudaMemsetAsync(ws, 0, kWsHeader, c.stream);
+  rc = cudaMemsetAsync(ws, 0, Ly.rows, c.stream);  // status word and the rejection records
   if (rc != cudaSuccess) {
     set_error(std::string("cudaMemsetAsync: ") + cudaGetErrorString(rc));
     return DSPARK_ECUDA;
