@@ -22,7 +22,7 @@ struct Options {
   int verify_cluster = 0;        // 0 auto, else the cluster size (1, 2, 4, 8, 16)
   int verify_persistent = 1;     // sampled verify / labels: persistent double-buffered clusters
   int verify_stream = 1;         // verify with a workspace: streaming kernels (one HBM read + one L2 read)
-  int verify_stream_cluster = 4; // CTAs per cluster of the streaming verify (1, 2, 4, 8)
+  int verify_stream_cluster = 3; // CTAs per cluster of the streaming verify (1 to 8)
   int verify_stream_lag = 1;     // rows between a row's first and second pass (1 to 3)
   int verify_stream_l2hint = 1;  // streaming verify: first-pass copies evict-last, second-pass evict-first
   int sm_count = 0;              // 0: query the device

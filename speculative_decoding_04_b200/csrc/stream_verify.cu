@@ -1102,7 +1102,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   const SvLayout Ly = sv_layout(c.B, c.gamma, c.V);
   if (c.ws_bytes < Ly.total) return DSPARK_ENOTIMPL;
   int C = options().verify_stream_cluster;
-  if (C != 1 && C != 2 && C != 4 && C != 8) C = 2;
+  if (C < 1 || C > kSvMaxCluster) C = 3;
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   SvArgs a{};
   a.ld = c.ld;
@@ -1160,7 +1160,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int ncl = 0;
-  for (; C >= 1; C >>= 1) {
+  for (; C >= 1; --C) {
     attr[0].val.clusterDim.x = C;
     cfg.gridDim = dim3((unsigned)C);
     if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) == cudaSuccess && ncl > 0) break;

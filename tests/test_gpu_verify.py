@@ -32,7 +32,7 @@ def run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=True):
 # kernels: "stream-C" = streaming kernels with clusters of C CTAs (the default with a
 # workspace); "rows-C" = one cluster of C CTAs per row (0: chosen from V), which serves calls
 # without a workspace, V not a multiple of 4 and the labels entry point.
-IMPLS = ["stream-8", "stream-4", "stream-1", "rows-0", "rows-1", "rows-4", "rows-16"]
+IMPLS = ["stream-8", "stream-6", "stream-4", "stream-3", "stream-1", "rows-0", "rows-1", "rows-4", "rows-16"]
 
 
 def use_impl(impl):
