@@ -74,15 +74,30 @@ const char* dspark_status_string(int status);
 /* Text of the last host-side error of this thread ("" if none). */
 const char* dspark_last_error(void);
 
-/* Tuning knobs (process-wide, host side; no effect on results beyond the choice of kernel):
+/* Tuning knobs (process-wide, host side; no effect on results beyond the choice of kernel and,
+ * within the stated tolerances, the order of floating-point sums):
  *   "draft_tc_min_b"  bf16 drafts with B >= value use the tensor-core main pass (default 9)
  *   "draft_path"      0 automatic, 1 always the CUDA-core GEMV pass, 2 always tensor cores
  *   "draft_pdl"       1 (default) chain draft kernels with programmatic dependent launch
- *   "draft_w2_hint"   1 (default) W2 tile loads ask L2 to keep W2 (it is re-read every step)
- *   "verify_cluster"  0 automatic, else the cluster size of the verify kernel (1..16, power of 2)
- *   "verify_persistent" 1 (default) sampled verification and labels run on persistent clusters
- *                     with double-buffered rows; 2 the same single-buffered; 0 one cluster per row
+ *   "draft_fused"     1 (default) tensor-core draft: all gamma positions in one cooperative
+ *                     launch with grid barriers (falls back to one launch pair per position
+ *                     when the grid cannot be co-resident); 0 always one pair per position
+ *   "draft_w2_hint"   L2 policies of the tensor-core draft: 0 (default) none; 1 W2 evict-last,
+ *                     U loads and l_d stores evict-first; 2 W2 and U only; 3 W2 only
+ *   "verify_stream"   1 (default) verification with a workspace and V % 4 == 0 runs the
+ *                     streaming kernels; 0 the per-row cluster kernels
+ *   "verify_stream_cluster"  CTAs per cluster of the streaming verify, 1..8 (default 3)
+ *   "verify_stream_lag"      rows between a row's first and second pass, 1..3 (default 1)
+ *   "verify_stream_l2hint"   1 (default) first-pass copies evict-last, second-pass evict-first
+ *   "verify_cluster"  0 automatic, else the cluster size of the per-row verify kernels (1..16,
+ *                     power of 2)
+ *   "verify_persistent" 1 (default) per-row sampled verification and labels run on persistent
+ *                     clusters with double-buffered rows; 2 the same single-buffered; 0 one
+ *                     cluster per row
  *   "sm_count"        0 query the device, else the SM count used to size persistent grids
+ * The environment variables DSPARK_DRAFT_TC_MIN_B, DSPARK_DRAFT_PATH, DSPARK_DRAFT_PDL,
+ * DSPARK_DRAFT_FUSED, DSPARK_VERIFY_CLUSTER, DSPARK_VERIFY_PERSISTENT, DSPARK_VERIFY_STREAM and
+ * DSPARK_VERIFY_STREAM_CLUSTER set the initial values of the keys of the same names.
  * Returns DSPARK_EINVAL for an unknown key. */
 int dspark_set_option(const char* key, long value);
 
