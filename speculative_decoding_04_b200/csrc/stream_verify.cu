@@ -449,6 +449,20 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
 
+// fp32 sum of 2^fma(l, c, nR) over one lane's 16 values of a tile row (nR = minus a reference).
+__device__ __forceinline__ float sv_lane_sum_at(const float4 (&v)[kSvVec], float c, float nR) {
+  const float2 c2 = make_float2(c, c), nr2 = make_float2(nR, nR);
+  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int jj = 0; jj < kSvVec; ++jj) {
+    const float2 x = f2fma(lo2(v[jj]), c2, nr2), y = f2fma(hi2(v[jj]), c2, nr2);
+    acc0 = f2add(acc0, make_float2(sv_ex2(x.x), sv_ex2(x.y)));
+    acc1 = f2add(acc1, make_float2(sv_ex2(y.x), sv_ex2(y.y)));
+  }
+  const float2 acc = f2add(acc0, acc1);
+  return acc.x + acc.y;
+}
+
 // First pass over one lane's 16 values of a tile row: the integer reference R of their maximum
 // and the fp32 sum of 2^fma(l, c, -R).
 __device__ __forceinline__ float sv_lane_sum(const float4 (&v)[kSvVec], float c, int& R) {
@@ -459,16 +473,28 @@ __device__ __forceinline__ float sv_lane_sum(const float4 (&v)[kSvVec], float c,
     m = fmax3(m, v[jj].z, v[jj].w);
   }
   R = sv_ref(m, c);
-  const float2 c2 = make_float2(c, c), nr2 = make_float2(-(float)R, -(float)R);
-  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int jj = 0; jj < kSvVec; ++jj) {
-    const float2 x = f2fma(lo2(v[jj]), c2, nr2), y = f2fma(hi2(v[jj]), c2, nr2);
-    acc0 = f2add(acc0, make_float2(sv_ex2(x.x), sv_ex2(x.y)));
-    acc1 = f2add(acc1, make_float2(sv_ex2(y.x), sv_ex2(y.y)));
+  return sv_lane_sum_at(v, c, -(float)R);
+}
+
+// Adds one lane's tile row to the pass's running (R, S), nR = -R: against the reference that the
+// lane's first tile of the pass set, or, when that sum reaches 2^100 or is not finite (a maximum
+// far above the reference, or a non-finite logit), against the tile's own maximum with an exact
+// power-of-two rescale.  Terms far below the reference flush to zero, 2^-125 or less of the sum.
+// Returns the tile's sum; r is the reference it is taken against.
+__device__ __forceinline__ float sv_lane_acc(const float4 (&v)[kSvVec], float c, int& R, float& nR, float& S,
+                                             int& r) {
+  if (R != kRNone) {
+    const float s = sv_lane_sum_at(v, c, nR);
+    if (s < 0x1p100f) {
+      S += s;
+      r = R;
+      return s;
+    }
   }
-  const float2 acc = f2add(acc0, acc1);
-  return acc.x + acc.y;
+  const float s = sv_lane_sum(v, c, r);
+  sv_merge_f(R, S, r, s);
+  nR = -(float)R;
+  return s;
 }
 
 // Decision of a row for its second pass.
@@ -697,7 +723,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     int p = 0;  // passes finished by this warp (slot of the partials)
     // state of the current pass
     int Rd = kRNone, Rt = kRNone;
-    float Sd = 0.f, St = 0.f;
+    float Sd = 0.f, St = 0.f, nRd = 0.f, nRt = 0.f;
     Top2 gd{-INFINITY, -1, -INFINITY}, gt{-INFINITY, -1, -INFINITY};
     uint32_t bad = 0;
     float smin = 0.f;       // second pass: unscaled sum of 2^min(x_d, x_t)
@@ -738,6 +764,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           out.gd = gd;
           out.gt = gt;
         } else {
+          bad |= (St <= FLT_MAX && Sd <= FLT_MAX) ? 0u : 1u;  // a non-finite logit of the pass
           sv_warp_ref_sum_f(Rd, Sd);
           sv_warp_ref_sum_f(Rt, St);
           out.rd = Rd;
@@ -824,9 +851,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           }
         } else {
           int rt;
-          const float stl = sv_lane_sum(ft, zc, rt);
-          bad |= (stl <= FLT_MAX) ? 0u : 1u;
-          sv_merge_f(Rt, St, rt, stl);
+          const float stl = sv_lane_acc(ft, zc, Rt, nRt, St, rt);
           if (ph.J.bonus) {
             // l_t weight of the tile for the bonus sample
             const int R = __reduce_max_sync(0xffffffffu, rt);
@@ -835,9 +860,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           }
           if (with_d) {
             int rd;
-            const float sdl = sv_lane_sum(fd, zc, rd);
-            bad |= (sdl <= FLT_MAX) ? 0u : 1u;
-            sv_merge_f(Rd, Sd, rd, sdl);
+            sv_lane_acc(fd, zc, Rd, nRd, Sd, rd);
           }
         }
       } else {
