@@ -31,6 +31,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -87,10 +88,11 @@ def config_of(wl, n):
 
 
 class Clocks:
-    """nvidia-smi sampled during the timed region."""
+    """nvidia-smi sampled during the timed region; the raw samples go to clocks_<gpu>.csv in the
+    directory named by DSPARK_CLOCKS_DIR (default: the system temporary directory)."""
 
     def __init__(self, index):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{index}.csv")
+        self.path = os.path.join(os.environ.get("DSPARK_CLOCKS_DIR", tempfile.gettempdir()), f"clocks_{index}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
