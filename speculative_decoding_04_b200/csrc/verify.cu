@@ -164,13 +164,12 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
   float* st = vsm + a.Vc;
   __shared__ Slot slot;
   __shared__ __align__(8) uint64_t bar;
-  __shared__ float sh_f[kMaxWarps];
   __shared__ double2 sh_d[kMaxWarps];
   __shared__ Top2 sh_t[kMaxWarps];
   __shared__ double sh_w[kMaxWarps];
   __shared__ float2 sh_f2[kMaxWarps];
   __shared__ double sh_wt[16], sh_wq[16];
-  __shared__ double s_Sd, s_St, s_ft, s_pdx, s_ptx, s_Smin, s_Z;
+  __shared__ double s_St, s_ft, s_pdx, s_ptx, s_Smin, s_Z;
   __shared__ float s_cd, s_ct;
   __shared__ int s_xfound;
   __shared__ uint32_t s_dfl;
@@ -380,7 +379,6 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
     const double own_fd = __shfl_sync(0xffffffffu, fd, rank), own_ft = __shfl_sync(0xffffffffu, ft, rank);
     if (live) sh_wt[lane] = wt;
     if (lane == 0) {
-      s_Sd = Sd;
       s_St = St;
       s_ft = own_ft;
       s_cd = (float)(own_fd / Sd);
