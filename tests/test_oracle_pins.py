@@ -108,6 +108,23 @@ def test_temperature_sampling_breakpoint():
     assert m[1] == pytest.approx(expit(d / T), abs=1e-11)
 
 
+@pytest.mark.parametrize("T", [1.0, 0.7])
+def test_draft_sampler_distribution_is_the_softmax(T):
+    # the draft token, as a function of its uniform, takes each v on a set of measure p_d(v):
+    # p_d = softmax((U + W1[prev] W2) / T), here recomputed independently in fp64
+    rng = np.random.default_rng(21)
+    V, r = 8, 3
+    U = rng.normal(scale=1.5, size=V).astype(np.float32)
+    W1 = rng.normal(scale=0.7, size=(V, r)).astype(np.float32)
+    W2 = rng.normal(scale=0.7, size=(r, V)).astype(np.float32)
+    prev = 5
+    m = measure(lambda u: O.draft_step(U, W1, W2, prev, u, T)[0])
+    ld = U.astype(np.float64) + W1[prev].astype(np.float64) @ W2.astype(np.float64)
+    want = scipy_softmax(ld / T)
+    got = np.array([m.get(v, 0.0) for v in range(V)])
+    np.testing.assert_allclose(got, want, rtol=1e-5, atol=1e-9)
+
+
 def test_greedy_lowest_index_on_ties():
     x, alts = O.greedy_choice(np.array([1.0, 3.0, 3.0, -1.0], dtype=np.float32))
     assert x == 1 and alts == [1, 2]
