@@ -82,8 +82,6 @@ const char* dspark_last_error(void);
  *   "draft_fused"     1 (default) tensor-core draft: all gamma positions in one cooperative
  *                     launch with grid barriers (falls back to one launch pair per position
  *                     when the grid cannot be co-resident); 0 always one pair per position
- *   "draft_w2_hint"   L2 policies of the tensor-core draft: 0 (default) none; 1 W2 evict-last,
- *                     U loads and l_d stores evict-first; 2 W2 and U only; 3 W2 only
  *   "verify_stream"   1 (default) verification with a workspace and V % 4 == 0 runs the
  *                     streaming kernels; 0 the per-row cluster kernels
  *   "verify_stream_cluster"  CTAs per cluster of the streaming verify, 1..8 (default 3)
@@ -188,11 +186,15 @@ int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int3
  * framework but no access to its allocator.  Arguments, results and flags are
  * those of dspark_verify; the scratch is a fixed array inside libdspark.so
  * (213,248 bytes per GPU, held from load until the process exits), so the call
- * allocates and frees nothing.
- * Limits: B <= 4096 and B*(gamma+1) <= 16384, else DSPARK_EINVAL with a message.
- * The first call on a device looks up the array's device address; make that first
- * call before any stream capture.  All calls share the array and each clears the
- * parts that must start at zero: calls whose kernels overlap on the GPU race.
+ * allocates and frees nothing.  It always runs the per-row cluster kernels, whose
+ * scratch does not grow with V (results equal dspark_verify's within the stated
+ * tolerances; tokens and lengths agree except at flagged near-ties).
+ * Limits: B <= 4096 and B*(gamma+1) <= 16384, else DSPARK_EINVAL with a message;
+ * V <= 409600 (one 16-CTA cluster per row), else DSPARK_ENOTIMPL.
+ * The first call on a device (and the first after its context was destroyed and
+ * recreated) looks up the array's device address; make that first call before any
+ * stream capture.  All calls share the array and each clears the parts that must
+ * start at zero: calls whose kernels overlap on the GPU race.
  * -------------------------------------------------------------------------- */
 int dspark_verify_noalloc(const float* ld, const float* lt, const int32_t* x, const int32_t* L,
                           const float* u_acc, const float* u_res,

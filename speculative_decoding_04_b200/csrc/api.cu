@@ -7,8 +7,11 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <set>
 #include <string>
+#include <utility>
 
 #include "internal.h"
 
@@ -18,7 +21,9 @@ static thread_local std::string g_last_error;
 
 void set_error(const std::string& msg) { g_last_error = msg; }
 
-Options& options() {
+static std::mutex g_opt_mu;
+
+static Options& options_ref() {
   static Options o;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -34,8 +39,43 @@ Options& options() {
   return o;
 }
 
+Options options() {
+  std::lock_guard<std::mutex> lock(g_opt_mu);
+  return options_ref();
+}
+
+// (device, function) -> the largest dynamic shared-memory size set so far; a second map for the
+// non-portable cluster attribute.
+static std::mutex g_attr_mu;
+static std::map<std::pair<int, const void*>, size_t> g_smem_attr;
+static std::set<std::pair<int, const void*>> g_np_attr;
+
+cudaError_t ensure_smem_attr(const void* func, size_t bytes) {
+  int dev = 0;
+  cudaError_t rc = cudaGetDevice(&dev);
+  if (rc != cudaSuccess) return rc;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  size_t& done = g_smem_attr[{dev, func}];
+  if (bytes <= done) return cudaSuccess;
+  rc = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (rc == cudaSuccess) done = bytes;
+  return rc;
+}
+
+cudaError_t ensure_nonportable_cluster(const void* func) {
+  int dev = 0;
+  cudaError_t rc = cudaGetDevice(&dev);
+  if (rc != cudaSuccess) return rc;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  if (g_np_attr.count({dev, func})) return cudaSuccess;
+  rc = cudaFuncSetAttribute(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (rc == cudaSuccess) g_np_attr.insert({dev, func});
+  return rc;
+}
+
 int device_sm_count() {
-  if (options().sm_count > 0) return options().sm_count;
+  const int forced = options().sm_count;
+  if (forced > 0) return forced;
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
@@ -68,11 +108,11 @@ const char* dspark_last_error(void) { return g_last_error.c_str(); }
 
 int dspark_set_option(const char* key, long value) {
   if (!key) return einval("dspark_set_option: null key");
-  Options& o = options();
+  std::lock_guard<std::mutex> lock(g_opt_mu);
+  Options& o = options_ref();
   if (!std::strcmp(key, "draft_tc_min_b")) o.draft_tc_min_b = (int)value;
   else if (!std::strcmp(key, "draft_path")) o.draft_force_path = (int)value;
   else if (!std::strcmp(key, "draft_pdl")) o.draft_pdl = (int)value;
-  else if (!std::strcmp(key, "draft_w2_hint")) o.draft_w2_hint = (int)value;
   else if (!std::strcmp(key, "draft_fused")) o.draft_fused = (int)value;
   else if (!std::strcmp(key, "verify_cluster")) o.verify_cluster = (int)value;
   else if (!std::strcmp(key, "verify_persistent")) o.verify_persistent = (int)value;
@@ -134,7 +174,7 @@ int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int3
   if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_verify: T must be finite and >= 0");
   if (ws_bytes < verify_workspace_bytes(B, gamma, V)) return einval("dspark_verify: workspace too small");
   if ((uintptr_t)ws % 256) return einval("dspark_verify: workspace must be 256-byte aligned");
-  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, 1, n_acc, y_out, c_star, flags, ws, ws_bytes,
+  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, 1, 0, n_acc, y_out, c_star, flags, ws, ws_bytes,
                (cudaStream_t)stream};
   return launch_verify(c);
 }
@@ -146,7 +186,7 @@ int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, 
   if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_tv_labels: gamma must be in [1, 64]");
   if (lt_rows != gamma && lt_rows != gamma + 1) return einval("dspark_tv_labels: lt_rows must be gamma or gamma+1");
   if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_tv_labels: T must be finite and >= 0");
-  VerifyCall c{ld, lt, nullptr, nullptr, nullptr, nullptr, B, gamma, V, lt_rows, T, 0, nullptr, nullptr, c_star,
+  VerifyCall c{ld, lt, nullptr, nullptr, nullptr, nullptr, B, gamma, V, lt_rows, T, 0, 0, nullptr, nullptr, c_star,
                nullptr, nullptr, 0, (cudaStream_t)stream};
   return launch_verify(c);
 }

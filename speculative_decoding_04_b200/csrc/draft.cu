@@ -386,7 +386,7 @@ template <int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
     draft_main_tc(const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmU,
                   const __grid_constant__ CUtensorMap tmLd, const __grid_constant__ CUtensorMap tmG, DraftArgs a,
-                  int k0, int k1, int n_bgroups, int ctas_per_group, int w2_hint, int fused) {
+                  int k0, int k1, int n_bgroups, int ctas_per_group, int fused) {
   constexpr int EPI_WARPS = NB / 8;  // 4 per 32-request column group
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -459,26 +459,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int bb = b0 + h * 32;
   constexpr uint32_t kUStage = (uint32_t)NB * kTcTile;  // floats of one U stage: [NB requests][128 columns]
   // U (an input of the call) for the first two tiles is requested before waiting for the previous
-  // kernel: one 128-column x NB-request box per tile.  With the L2 hint on, U and l_d (streamed
-  // once per step) are evict-first, so that W2 (read by every step) can stay in L2.
-  auto load_u = [&](int gi, uint64_t pol) {
+  // kernel: one 128-column x NB-request box per tile.
+  auto load_u = [&](int gi) {
     const int j = gi & 1, ku = k0 + gi / nt, iu = gi % nt;
     mbar_arrive_expect_tx(&u_full[j], kUStage * 4u);
-    if (w2_hint == 1 || w2_hint == 2)
-      tma_load_3d_hint(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j], pol);
-    else tma_load_3d(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j]);
+    tma_load_3d(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j]);
   };
-  if (warp == 3 && lane == 0) {
-    const uint64_t pol = l2_policy_evict_first();
-    for (int gi = 0; gi < 2 && gi < total; ++gi) load_u(gi, pol);
-  }
+  if (warp == 3 && lane == 0)
+    for (int gi = 0; gi < 2 && gi < total; ++gi) load_u(gi);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     // W2 is an input of the call: the ring fills before the previous kernel has finished, and
     // across steps (the same tiles every step).
     if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_last();
       int issued = 0;
       for (int gi = 0; gi < total; ++gi) {
         const int v0 = (t_beg + gi % nt) * kTcTile;
@@ -486,13 +480,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!tc_wait(sy, &w_empty[s], ((gi / kTcStages) & 1) ^ 1)) break;
         uint8_t* st = sW + s * L.w2_stage_bytes;
         mbar_arrive_expect_tx(&w_full[s], L.w2_stage_bytes);
-        if (w2_hint) {
-          tma_load_2d_hint(st, &tmW2, v0, 0, &w_full[s], pol);
-          tma_load_2d_hint(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s], pol);
-        } else {
-          tma_load_2d(st, &tmW2, v0, 0, &w_full[s]);
-          tma_load_2d(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s]);
-        }
+        tma_load_2d(st, &tmW2, v0, 0, &w_full[s]);
+        tma_load_2d(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s]);
         issued = gi + 1;
       }
       if (*s_abort) {
@@ -542,17 +531,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // writes it out, and the stage is refilled with the U tile two ahead (possibly of the next
         // step) once the store has read it and every epilogue warp is done with it.
         if (lane == 0) {
-          const uint64_t pol = l2_policy_evict_first();
           for (int i = 0; i < nt; ++i) {
             const int gi = gbase + i, j = gi & 1;
             if (!tc_wait(sy, &c_done[j], (gi >> 1) & 1)) break;
-            if (w2_hint == 1) tma_store_3d_hint(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k, pol);
-            else tma_store_3d(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k);
+            tma_store_3d(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k);
             bulk_commit();
             if (gi + 2 < total) {
               if (!tc_wait(sy, &u_empty[j], (gi >> 1) & 1)) break;
               bulk_wait_read0();
-              load_u(gi + 2, pol);
+              load_u(gi + 2);
               last_load[j] = gi + 2;
             }
           }
@@ -975,12 +962,7 @@ static cudaError_t launch_fma(const DraftArgs& a, int k, cudaStream_t st, bool p
   const int vec_ok = (a.V % (int)(16 / sizeof(WT)) == 0 && (uintptr_t)a.W2 % 16 == 0) ? 1 : 0;
   const size_t smem = (size_t)(((BG * a.r + 3) & ~3) + 4 * BG * 256) * sizeof(float);
   auto kern = draft_main_fma<WT, BG>;
-  static cudaError_t attr_rc = cudaSuccess;
-  static size_t attr_smem = 0;
-  if (smem > attr_smem) {
-    attr_rc = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr_smem = smem;
-  }
+  const cudaError_t attr_rc = ensure_smem_attr((const void*)kern, smem);
   if (attr_rc != cudaSuccess) return attr_rc;
   dim3 grid((a.V + 255) / 256, (a.B + BG - 1) / BG);
   return launch_ex(kern, grid, dim3(128), smem, st, pdl, false, a, k, vec_ok);
@@ -995,18 +977,12 @@ static cudaError_t launch_fma_bg(const DraftArgs& a, int k, cudaStream_t st, boo
 }
 
 static cudaError_t tc_set_smem(int nb, size_t smem) {
-  static size_t done[2] = {0, 0};
-  const int i = nb == 32 ? 0 : 1;
-  if (smem <= done[i]) return cudaSuccess;
-  const cudaError_t rc =
-      nb == 32 ? cudaFuncSetAttribute(draft_main_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-               : cudaFuncSetAttribute(draft_main_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (rc == cudaSuccess) done[i] = smem;
-  return rc;
+  return nb == 32 ? ensure_smem_attr((const void*)draft_main_tc<32>, smem)
+                  : ensure_smem_attr((const void*)draft_main_tc<64>, smem);
 }
 
 dspark_status launch_draft(const DraftCall& c) {
-  const Options& opt = options();
+  const Options opt = options();
   DraftArgs a{};
   a.U = c.U;
   a.W1 = c.W1;
@@ -1109,13 +1085,12 @@ dspark_status launch_draft(const DraftCall& c) {
   if (use_tc && opt.draft_fused) {
     // all gamma steps in one cooperative launch (every CTA resident; grid barriers between steps)
     const dim3 grid(cpg * n_bgroups), block(kTcThreads);
-    const int hint = opt.draft_w2_hint;
     if (nb == 32)
       rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, false, true, mW2, mU, mLd, mG, a, 0, c.gamma,
-                     n_bgroups, cpg, hint, 1);
+                     n_bgroups, cpg, 1);
     else
       rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, false, true, mW2, mU, mLd, mG, a, 0, c.gamma,
-                     n_bgroups, cpg, hint, 1);
+                     n_bgroups, cpg, 1);
     if (rc == cudaSuccess) return DSPARK_OK;
     (void)cudaGetLastError();  // e.g. not all CTAs can be resident: one launch pair per step below
   }
@@ -1125,13 +1100,12 @@ dspark_status launch_draft(const DraftCall& c) {
     const bool pdl_k = pdl && k > 0;
     if (use_tc) {
       const dim3 grid(cpg * n_bgroups), block(kTcThreads);
-      const int hint = opt.draft_w2_hint;
       if (nb == 32)
         rc = launch_ex(draft_main_tc<32>, grid, block, tc_smem, c.stream, pdl_k, false, mW2, mU, mLd, mG, a, k, k + 1,
-                       n_bgroups, cpg, hint, 0);
+                       n_bgroups, cpg, 0);
       else
         rc = launch_ex(draft_main_tc<64>, grid, block, tc_smem, c.stream, pdl_k, false, mW2, mU, mLd, mG, a, k, k + 1,
-                       n_bgroups, cpg, hint, 0);
+                       n_bgroups, cpg, 0);
     } else if (c.w_dtype == DSPARK_BF16) {
       rc = launch_fma_bg<__nv_bfloat16>(a, k, c.stream, pdl_k);
     } else {

@@ -17,7 +17,6 @@ struct Options {
   int draft_tc_min_b = 9;        // bf16 drafts with at least this many requests use the tensor-core path
   int draft_force_path = 0;      // 0 auto, 1 CUDA-core GEMV, 2 tensor cores
   int draft_pdl = 1;             // chain the draft kernels with programmatic dependent launch
-  int draft_w2_hint = 0;         // L2 hints: 1 W2 evict-last, U and l_d evict-first; 2 W2 and U only; 3 W2 only
   int draft_fused = 1;           // tensor-core draft: all steps in one cooperative launch
   int verify_cluster = 0;        // 0 auto, else the cluster size (1, 2, 4, 8, 16)
   int verify_persistent = 1;     // sampled verify / labels: persistent double-buffered clusters
@@ -27,7 +26,15 @@ struct Options {
   int verify_stream_l2hint = 1;  // streaming verify: first-pass copies evict-last, second-pass evict-first
   int sm_count = 0;              // 0: query the device
 };
-Options& options();
+// A copy of the process-wide options, taken under their lock (dspark_set_option may run on
+// another thread).
+Options options();
+
+// cudaFuncSetAttribute for the dynamic shared-memory size of `func`, raised as needed and
+// remembered per device (a process may drive several GPUs; each needs the attribute once).
+cudaError_t ensure_smem_attr(const void* func, size_t bytes);
+// Allow cluster sizes above 8 for `func` on the current device (remembered per device).
+cudaError_t ensure_nonportable_cluster(const void* func);
 
 int device_sm_count();
 
@@ -58,6 +65,7 @@ struct VerifyCall {
   int B, gamma, V, lt_rows;
   float T;
   int do_verify;
+  int per_row_only;  // 1: the per-row cluster kernels only (their workspace layout), never the streaming ones
   int32_t* n_acc;
   int32_t* y_out;
   float* c_star;
@@ -80,6 +88,7 @@ struct ScheduleCall {
 
 size_t draft_workspace_bytes(int B, int gamma, int V, int r);
 size_t verify_workspace_bytes(int B, int gamma, int V);
+size_t verify_rows_workspace_bytes(int B, int gamma);
 
 dspark_status launch_draft(const DraftCall& c);
 dspark_status launch_verify(const VerifyCall& c);

@@ -274,15 +274,13 @@ dspark_status launch_schedule(const ScheduleCall& c) {
   s.theta_out = c.theta_out;
   s.flags = c.flags;
   const size_t smem = (size_t)P * 8 + align_up((size_t)c.B * 4, 16);
-  static size_t attr_smem = 0;
   cudaError_t rc;
-  if (smem > 48 * 1024 && smem > attr_smem) {
-    rc = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (smem > 48 * 1024) {
+    rc = ensure_smem_attr((const void*)schedule_kernel, smem);
     if (rc != cudaSuccess) {
       set_error(std::string("cudaFuncSetAttribute(schedule_kernel): ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;
     }
-    attr_smem = smem;
   }
   schedule_kernel<<<1, kSchedThreads, smem, c.stream>>>(s);
   rc = cudaGetLastError();

@@ -1120,11 +1120,12 @@ size_t stream_verify_workspace_bytes(int B, int gamma, int V) { return sv_layout
 // DSPARK_ENOTIMPL: this call is not for the streaming kernels (labels only, V not a multiple of
 // 4, unaligned rows, a workspace sized for the per-row kernels, or no cluster fits).
 dspark_status launch_verify_stream(const VerifyCall& c) {
-  if (!c.do_verify || !options().verify_stream) return DSPARK_ENOTIMPL;
+  const Options opt = options();
+  if (!c.do_verify || !opt.verify_stream) return DSPARK_ENOTIMPL;
   if (c.V % 4 || (uintptr_t)c.ld % 16 || (uintptr_t)c.lt % 16) return DSPARK_ENOTIMPL;
   const SvLayout Ly = sv_layout(c.B, c.gamma, c.V);
   if (c.ws_bytes < Ly.total) return DSPARK_ENOTIMPL;
-  int C = options().verify_stream_cluster;
+  int C = opt.verify_stream_cluster;
   if (C < 1 || C > kSvMaxCluster) C = 3;
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   SvArgs a{};
@@ -1140,8 +1141,8 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.lt_rows = c.lt_rows;
   a.njobs = c.B * (c.gamma + 1);
   a.ntile = (c.V + kSvTile - 1) / kSvTile;
-  a.lag = std::min(std::max(options().verify_stream_lag, 1), 3);
-  a.l2hint = options().verify_stream_l2hint;
+  a.lag = std::min(std::max(opt.verify_stream_lag, 1), 3);
+  a.l2hint = opt.verify_stream_l2hint;
   a.greedy = c.T == 0.f ? 1 : 0;
   a.zscale = a.greedy ? 0.f : (float)(1.4426950408889634 / (double)c.T);
   a.do_verify = 1;
@@ -1157,14 +1158,10 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.qrec = reinterpret_cast<float*>(ws + Ly.qrec);
   auto kern = a.greedy ? verify_stream<true> : verify_stream<false>;
   cudaError_t rc;
-  static bool attr_set[2] = {false, false};
-  if (!attr_set[a.greedy]) {
-    rc = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSvRingBytes);
-    if (rc != cudaSuccess) {
-      set_error(std::string("cudaFuncSetAttribute(verify_stream): ") + cudaGetErrorString(rc));
-      return DSPARK_ECUDA;
-    }
-    attr_set[a.greedy] = true;
+  rc = ensure_smem_attr((const void*)kern, kSvRingBytes);
+  if (rc != cudaSuccess) {
+    set_error(std::string("cudaFuncSetAttribute(verify_stream): ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
   }
   rc = cudaMemsetAsync(ws, 0, Ly.rows, c.stream);  // status word and the rejection records
   if (rc != cudaSuccess) {

@@ -21,6 +21,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <string>
 
@@ -1034,10 +1035,13 @@ __global__ void __launch_bounds__(512, 1) verify_rows_pc(VerifyArgs a) {
 
 // Per-row kernels need the first part; the streaming kernels (the default with a workspace)
 // the second.
-size_t verify_workspace_bytes(int B, int gamma, int V) {
+size_t verify_rows_workspace_bytes(int B, int gamma) {
   const size_t rows = (size_t)B * (gamma + 1);
-  const size_t per_row = kWsHeader + 3 * align_up(rows * 4, 256) + align_up((size_t)B * 4, 256);
-  return std::max(per_row, stream_verify_workspace_bytes(B, gamma, V));
+  return kWsHeader + 3 * align_up(rows * 4, 256) + align_up((size_t)B * 4, 256);
+}
+
+size_t verify_workspace_bytes(int B, int gamma, int V) {
+  return std::max(verify_rows_workspace_bytes(B, gamma), stream_verify_workspace_bytes(B, gamma, V));
 }
 
 // Cluster size: the smallest power of two whose per-CTA slices (ℓ_d and ℓ_t, fp32) fit the
@@ -1061,24 +1065,17 @@ template <int NI, int NBUF>
 static dspark_status launch_pc(const VerifyArgs& a, int cs, cudaStream_t stream) {
   auto kern = verify_rows_pc<NI, NBUF>;
   const size_t smem = (size_t)NBUF * 8 * a.Vc;
-  static size_t attr_smem = 0;
-  static bool np_set = false;
-  cudaError_t rc = cudaSuccess;
-  if (smem > attr_smem) {
-    rc = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (rc != cudaSuccess) {
-      set_error(std::string("cudaFuncSetAttribute(verify_rows_pc, smem): ") + cudaGetErrorString(rc));
-      return DSPARK_ECUDA;
-    }
-    attr_smem = smem;
+  cudaError_t rc = ensure_smem_attr((const void*)kern, smem);
+  if (rc != cudaSuccess) {
+    set_error(std::string("cudaFuncSetAttribute(verify_rows_pc, smem): ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
   }
-  if (cs > 8 && !np_set) {
-    rc = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (cs > 8) {
+    rc = ensure_nonportable_cluster((const void*)kern);
     if (rc != cudaSuccess) {
       set_error(std::string("cudaFuncSetAttribute(verify_rows_pc, cluster 16): ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;
     }
-    np_set = true;
   }
   const long long nrows = (long long)a.B * a.rows_per_req;
   cudaLaunchConfig_t cfg = {};
@@ -1134,7 +1131,7 @@ static dspark_status launch_verify_persistent(const VerifyArgs& a, int cs, cudaS
 }
 
 dspark_status launch_verify(const VerifyCall& c) {
-  if (c.do_verify) {
+  if (c.do_verify && !c.per_row_only) {
     const dspark_status st = launch_verify_stream(c);
     if (st != DSPARK_ENOTIMPL) return st;  // else: the per-row kernels below
   }
@@ -1172,37 +1169,32 @@ dspark_status launch_verify(const VerifyCall& c) {
       return DSPARK_ECUDA;
     }
   }
-  const int cs = pick_cluster(c.V, options().verify_cluster);
+  const Options opt = options();
+  const int cs = pick_cluster(c.V, opt.verify_cluster);
   a.Vc = (int)align_up((size_t)(c.V + cs - 1) / cs, 4);
   if ((size_t)8 * a.Vc > kVerifySmemMax) {
     set_error("dspark_verify: V too large for one 16-CTA cluster per row (V <= 409600)");
     return DSPARK_ENOTIMPL;
   }
   a.bulk = (c.V % 4 == 0) && ((uintptr_t)c.lt % 16 == 0) && ((uintptr_t)c.ld % 16 == 0);
-  if (!a.greedy && a.bulk && options().verify_persistent) {
-    dspark_status st = launch_verify_persistent(a, cs, c.stream, options().verify_persistent != 2);
+  if (!a.greedy && a.bulk && opt.verify_persistent) {
+    dspark_status st = launch_verify_persistent(a, cs, c.stream, opt.verify_persistent != 2);
     if (st == DSPARK_OK) st = launch_finalize(a, c.stream);
     if (st != DSPARK_ENOTIMPL) return st;  // else: no resident cluster fits; use the one-row-per-cluster kernel
   }
   const int nthr = a.Vc >= 4096 ? 512 : (a.Vc >= 1024 ? 256 : 128);
   const size_t smem = (size_t)8 * a.Vc;
-  static size_t attr_smem = 0;
-  static bool np_set = false;
-  if (smem > attr_smem) {
-    rc = cudaFuncSetAttribute(verify_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (rc != cudaSuccess) {
-      set_error(std::string("cudaFuncSetAttribute(verify_rows, smem): ") + cudaGetErrorString(rc));
-      return DSPARK_ECUDA;
-    }
-    attr_smem = smem;
+  rc = ensure_smem_attr((const void*)verify_rows, smem);
+  if (rc != cudaSuccess) {
+    set_error(std::string("cudaFuncSetAttribute(verify_rows, smem): ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
   }
-  if (cs > 8 && !np_set) {
-    rc = cudaFuncSetAttribute(verify_rows, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (cs > 8) {
+    rc = ensure_nonportable_cluster((const void*)verify_rows);
     if (rc != cudaSuccess) {
       set_error(std::string("cudaFuncSetAttribute(verify_rows, cluster 16): ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;
     }
-    np_set = true;
   }
   const long long nrows = (long long)c.B * a.rows_per_req;
   cudaLaunchConfig_t cfg = {};
@@ -1235,12 +1227,18 @@ dspark_status launch_verify(const VerifyCall& c) {
 // framework with no access to that framework's allocator.  dspark_verify_noalloc serves them
 // from a fixed array in the library's own device memory instead of a caller workspace.
 //
+// It always runs the per-row cluster kernels (verify_rows_pc / verify_rows + verify_finalize):
+// their scratch is a few words per row and request, so a fixed array covers every size up to
+// the limits below, whatever V is.  The streaming kernels keep per-tile records that grow with
+// V and are never used here.
+//
 // The array below is that scratch.  Every GPU that loads the library holds it until the
 // process exits.  In host code its name is only a host-side stand-in, so its device address
-// is looked up once per device with cudaGetSymbolAddress (the first call on a device does
-// this, which is why that first call should come before any stream capture).  All calls
-// share the array: the per-call counters are cleared by each call, and calls whose kernels
-// overlap on the GPU race on it.
+// is looked up with cudaGetSymbolAddress once per device and CUDA context, with that device
+// current (the first call on a device does this, which is why that first call should come
+// before any stream capture; a call after the context was destroyed and recreated looks it up
+// again).  All calls share the array: each call clears the words that must start at zero, and
+// calls whose kernels overlap on the GPU race on it.
 
 namespace dspark {
 
@@ -1250,24 +1248,45 @@ constexpr size_t kNoAllocScratchBytes = kWsHeader + 3 * (size_t)kNoAllocMaxRows 
 
 static __device__ __align__(256) uint8_t g_verify_scratch[kNoAllocScratchBytes];
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+static CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 static dspark_status verify_scratch(void** ptr) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
+  static CUcontext ctx_of[64] = {nullptr};
   int dev = 0;
   cudaError_t rc = cudaGetDevice(&dev);
   if (rc != cudaSuccess || dev < 0 || dev >= 64) {
     set_error(std::string("dspark_verify_noalloc: cudaGetDevice: ") + cudaGetErrorString(rc));
     return DSPARK_ECUDA;
   }
+  CUcontext ctx = nullptr;
+  const CtxGetCurrentFn cur = ctx_get_current_fn();
+  if (cur) (void)cur(&ctx);
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || !ctx || ctx_of[dev] != ctx) {
     void* p = nullptr;
-    rc = cudaGetSymbolAddress(&p, g_verify_scratch);
+    rc = cudaGetSymbolAddress(&p, g_verify_scratch);  // also makes the device's primary context current
     if (rc != cudaSuccess || !p) {
       set_error(std::string("dspark_verify_noalloc: cudaGetSymbolAddress: ") + cudaGetErrorString(rc));
       return DSPARK_ECUDA;
     }
+    if (!ctx && cur) (void)cur(&ctx);
     addr[dev] = p;
+    ctx_of[dev] = ctx;
   }
   *ptr = addr[dev];
   return DSPARK_OK;
@@ -1279,17 +1298,23 @@ extern "C" int dspark_verify_noalloc(const float* ld, const float* lt, const int
                                      const float* u_acc, const float* u_res, int B, int gamma, int V, float T,
                                      int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags, void* stream) {
   using namespace dspark;
-  if (B > kNoAllocMaxB || (long long)B * (gamma + 1) > kNoAllocMaxRows) {
-    set_error("dspark_verify_noalloc: needs B <= 4096 and B*(gamma+1) <= 16384 (fixed scratch); use dspark_verify");
-    return DSPARK_EINVAL;
-  }
-  if (!ld || !lt || !x || !n_acc || !y_out || !flags) {
-    set_error("dspark_verify_noalloc: null pointer");
-    return DSPARK_EINVAL;
-  }
+  auto einval = [](const char* msg) {
+    set_error(msg);
+    return (int)DSPARK_EINVAL;
+  };
+  if (!ld || !lt || !x || !n_acc || !y_out || !flags) return einval("dspark_verify_noalloc: null pointer");
+  if (T != 0.f && (!u_acc || !u_res)) return einval("dspark_verify_noalloc: u_acc and u_res are required when T > 0");
+  if (B <= 0 || V < 2) return einval("dspark_verify_noalloc: B must be >= 1 and V >= 2");
+  if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_verify_noalloc: gamma must be in [1, 64]");
+  if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_verify_noalloc: T must be finite and >= 0");
+  if (B > kNoAllocMaxB || (long long)B * (gamma + 1) > kNoAllocMaxRows)
+    return einval("dspark_verify_noalloc: needs B <= 4096 and B*(gamma+1) <= 16384 (fixed scratch); use dspark_verify");
+  if (verify_rows_workspace_bytes(B, gamma) > kNoAllocScratchBytes)  // holds within the limits above
+    return einval("dspark_verify_noalloc: fixed scratch too small for these sizes");
   void* ws = nullptr;
-  dspark_status st = verify_scratch(&ws);
+  const dspark_status st = verify_scratch(&ws);
   if (st != DSPARK_OK) return st;
-  return dspark_verify(ld, lt, x, L, u_acc, u_res, B, gamma, V, T, n_acc, y_out, c_star, flags, ws,
-                       kNoAllocScratchBytes, stream);
+  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, 1, 1, n_acc, y_out, c_star, flags, ws,
+               kNoAllocScratchBytes, (cudaStream_t)stream};
+  return launch_verify(c);
 }

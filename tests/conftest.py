@@ -26,7 +26,6 @@ def _default_options():
         D.set_option("draft_tc_min_b", 9)
         D.set_option("verify_cluster", 0)
         D.set_option("draft_pdl", 1)
-        D.set_option("draft_w2_hint", 0)
         D.set_option("draft_fused", 1)
         D.set_option("verify_persistent", 1)
         D.set_option("verify_stream", 1)
