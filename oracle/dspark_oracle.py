@@ -29,7 +29,7 @@ What each function follows:
                   candidate tokens by survival, add them one at a time, evaluate
                   expected throughput, stop when it falls; global search on the GPU).
 
-Readings where the pages leave a step open (each is listed in the design doc):
+Readings where the pages leave a step open:
   * temperature: p ∝ exp(ℓ/T) on both draft and target; the scaling is an fp32
     multiply of the fp32 logits by fl32(1/T), so that both sides take every
     sampling and acceptance decision from the same fp32 scaled logits; all
@@ -85,19 +85,20 @@ def softmax(logits, T: float) -> np.ndarray:
     return e / np.sum(e, axis=-1, keepdims=True)
 
 
-def greedy_choice(logits) -> Tuple[int, List[int]]:
-    """argmax with the lowest index on ties, plus every index within the near-tie gap."""
+def greedy_choice(logits, near: float = NEAR_TIE) -> Tuple[int, List[int]]:
+    """argmax with the lowest index on ties, plus every index within the near-tie gap
+    near·max(1, |max|) of the maximum."""
     z = np.asarray(logits, dtype=np.float32).astype(np.float64)
     x = int(np.argmax(z))
-    gap = NEAR_TIE * max(1.0, abs(z[x]))
+    gap = near * max(1.0, abs(z[x]))
     alts = [int(v) for v in np.nonzero(z >= z[x] - gap)[0]]
     return x, alts
 
 
-def inverse_cdf(p: np.ndarray, u: float) -> Tuple[int, List[int]]:
+def inverse_cdf(p: np.ndarray, u: float, near: float = NEAR_TIE) -> Tuple[int, List[int]]:
     """Sample index v = min{v : F_v > u}, F the running sum of p in vocabulary order.
 
-    Returns the index and every index whose CDF interval lies within NEAR_TIE of u.
+    Returns the index and every index whose CDF interval lies within `near` of u.
     """
     p = np.asarray(p, dtype=np.float64)
     F = np.cumsum(p)
@@ -106,8 +107,8 @@ def inverse_cdf(p: np.ndarray, u: float) -> Tuple[int, List[int]]:
     if v >= p.shape[0]:
         v = int(np.nonzero(p > 0)[0][-1])
     lo = np.concatenate([[0.0], F[:-1]])
-    near = (p > 0) & (lo - NEAR_TIE <= u) & (u < F + NEAR_TIE)
-    alts = sorted(set(int(i) for i in np.nonzero(near)[0]) | {v})
+    close = (p > 0) & (lo - near <= u) & (u < F + near)
+    alts = sorted(set(int(i) for i in np.nonzero(close)[0]) | {v})
     return v, alts
 
 
@@ -136,7 +137,7 @@ def draft_step(U_k, W1, W2, prev, u, T: float, W2_64: Optional[np.ndarray] = Non
     return x, ld32, alts
 
 
-def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None):
+def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None, near: float = NEAR_TIE):
     """The γ sequential Markov-head steps for every request.
 
     U [B, γ, V] fp32, x0 [B], u_draft [B, γ].  Step k uses the token chosen at
@@ -144,7 +145,7 @@ def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None
     ld [B, γ, V] fp32, alts) where alts[(b, k)] lists the valid tokens at a
     near-tie.  `follow` maps (b, k) to a token that must be one of the valid
     alternatives at that step; the chain then continues from it (used to
-    follow one branch of a near-tie).
+    follow one branch of a near-tie).  `near` is the near-tie window.
     """
     U = np.asarray(U, dtype=np.float32)
     B, G, V = U.shape
@@ -159,9 +160,9 @@ def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None
         ld[:, k] = (U[:, k].astype(np.float64) + bias).astype(np.float32)
         for b in range(B):
             if T == 0.0:
-                xk, a = greedy_choice(ld[b, k])
+                xk, a = greedy_choice(ld[b, k], near)
             else:
-                xk, a = inverse_cdf(softmax(ld[b, k], T), u_draft[b, k])
+                xk, a = inverse_cdf(softmax(ld[b, k], T), u_draft[b, k], near)
             if len(a) > 1:
                 alts[(b, k)] = a
             if follow is not None and (b, k) in follow:
@@ -177,7 +178,8 @@ def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None
 # --------------------------------------------------------------------------- verification
 
 def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
-                   force_accept: Optional[Dict[int, bool]] = None, force_token: Optional[int] = None):
+                   force_accept: Optional[Dict[int, bool]] = None, force_token: Optional[int] = None,
+                   near: float = NEAR_TIE):
     """Rejection-sampling verification of one request's block.
 
     ld_b [γ, V] draft logits, lt_b [≥L+1, V] target logits, x_b [γ] drafted
@@ -190,7 +192,8 @@ def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
     resampled/bonus token, then -1), accept_ties (positions whose decision is
     a near-tie), sample_alts (valid tokens for the last emitted one),
     residual_mass (Z when a residual was drawn) and kind ('residual'/'bonus').
-    `force_accept`/`force_token` pin a near-tie outcome to one of its valid values.
+    `force_accept`/`force_token` pin a near-tie outcome to one of its valid values
+    (an outcome outside the near-tie window raises ValueError); `near` is the window.
     """
     G = len(x_b)
     V = np.asarray(lt_b).shape[-1]
@@ -200,7 +203,7 @@ def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
     for k in range(L):
         xk = int(x_b[k])
         if T == 0.0:
-            tk, talts = greedy_choice(lt_b[k])
+            tk, talts = greedy_choice(lt_b[k], near)
             acc = (0 <= xk < V) and xk == tk
             if len(talts) > 1 and (xk in talts):
                 accept_ties.append(k)
@@ -212,7 +215,7 @@ def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
                 pt = softmax(lt_b[k], T)[xk]
                 u = float(u_acc_b[k])
                 acc = u * pd < pt
-                if pd > 0 and abs(u - pt / pd) < NEAR_TIE:
+                if pd > 0 and abs(u - pt / pd) < near:
                     accept_ties.append(k)
         if force_accept is not None and k in force_accept:
             if k not in accept_ties and force_accept[k] != acc:
@@ -224,7 +227,7 @@ def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
         n += 1
     residual_mass = None
     if T == 0.0:
-        tok, alts = greedy_choice(lt_b[n])
+        tok, alts = greedy_choice(lt_b[n], near)
         kind = "residual" if n < L else "bonus"
     elif n < L:
         q = np.maximum(0.0, softmax(lt_b[n], T) - softmax(ld_b[n], T))
@@ -232,12 +235,12 @@ def verify_request(ld_b, lt_b, x_b, L: int, u_acc_b, u_res: float, T: float,
         residual_mass = Z
         kind = "residual"
         if Z > 0.0:
-            tok, alts = inverse_cdf(q / Z, u_res)
+            tok, alts = inverse_cdf(q / Z, u_res, near)
         else:
-            tok, alts = inverse_cdf(softmax(lt_b[n], T), u_res)
+            tok, alts = inverse_cdf(softmax(lt_b[n], T), u_res, near)
     else:
         kind = "bonus"
-        tok, alts = inverse_cdf(softmax(lt_b[L], T), u_res)
+        tok, alts = inverse_cdf(softmax(lt_b[L], T), u_res, near)
     if force_token is not None:
         if force_token not in alts:
             raise ValueError(f"token {force_token} is not a valid outcome: {alts}")
@@ -299,7 +302,7 @@ def schedule_order(a) -> np.ndarray:
     return np.argsort(key, kind="stable")
 
 
-def prefix_schedule(c, sps, D_max: int, mode: int = SCHED_ARGMAX):
+def prefix_schedule(c, sps, D_max: int, mode: int = SCHED_ARGMAX, near: float = THETA_NEAR_TIE):
     """Greedy hardware-aware prefix scheduler.
 
     All B·γ candidate tokens are ranked by prefix survival; adding them one at a
@@ -308,7 +311,8 @@ def prefix_schedule(c, sps, D_max: int, mode: int = SCHED_ARGMAX):
     ARGMAX keeps the best D over 0..D_max; EARLY_STOP keeps the first D after
     which Θ no longer rises.  L_b is the number of request b's tokens kept.
 
-    Returns dict(L [B] int32, a [B, γ] fp32, theta (Θ at D*), D, thetas, near_tie).
+    Returns dict(L [B] int32, a [B, γ] fp32, theta (Θ at D*), D, thetas, near_tie); near_tie
+    says whether another D is within `near` (relative) of the decision.
     """
     a = prefix_survival(c)
     B, G = a.shape
@@ -321,20 +325,20 @@ def prefix_schedule(c, sps, D_max: int, mode: int = SCHED_ARGMAX):
     if mode == SCHED_ARGMAX:
         D = int(np.argmax(theta))
         others = np.delete(theta, D)
-        near = bool(others.size and np.any(np.abs(others - theta[D]) <= THETA_NEAR_TIE * abs(theta[D])))
+        tie = bool(others.size and np.any(np.abs(others - theta[D]) <= near * abs(theta[D])))
     elif mode == SCHED_EARLY_STOP:
         D = D_max
-        near = False
+        tie = False
         for d in range(D_max):
-            if abs(theta[d + 1] - theta[d]) <= THETA_NEAR_TIE * abs(theta[d]):
-                near = True
+            if abs(theta[d + 1] - theta[d]) <= near * abs(theta[d]):
+                tie = True
             if theta[d + 1] <= theta[d]:
                 D = d
                 break
     else:
         raise ValueError(mode)
     L = np.bincount(order[:D] // G, minlength=B).astype(np.int32)
-    return dict(L=L, a=a, theta=float(theta[D]), D=D, thetas=theta, near_tie=near)
+    return dict(L=L, a=a, theta=float(theta[D]), D=D, thetas=theta, near_tie=tie)
 
 
 def exhaustive_schedule(c, sps, D_max: int):

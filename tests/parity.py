@@ -8,6 +8,11 @@ Tolerances (stated once, used by every GPU parity test):
     near-tie (|u - F| < 1e-6, |u - p_t/p_d| < 1e-6, greedy top-2 gap <= 1e-6*max(1,|z|), or
     scheduler Θ within 1e-12 relative); there the GPU's choice must be one of the outcomes
     the oracle reports as valid, and the oracle then follows that branch.
+  * flag bits (near-ties, small residual): the device computes its decisions in its own
+    arithmetic, so the comparison has a margin of 4x on each side of the window: where the
+    oracle's distance to a decision threshold is below a quarter of the window the bit must be
+    set, and a set bit needs an oracle distance below four windows (residual mass: 0.9e-3 and
+    1.1e-3 around the 1e-3 threshold).
 """
 
 import numpy as np
@@ -20,6 +25,13 @@ P_RTOL = 1e-5
 P_ATOL = 1e-9
 
 FLAG_DRAFT_NEAR_TIE = 1 << 0
+FLAG_ACCEPT_NEAR_TIE = 1 << 1
+FLAG_SAMPLE_NEAR_TIE = 1 << 2
+FLAG_SMALL_RESIDUAL = 1 << 3
+
+STRICT = 0.25 * O.NEAR_TIE   # oracle distance below this: the device must flag
+LOOSE = 4.0 * O.NEAR_TIE     # a device flag needs an oracle distance below this
+SMALL_RES_STRICT, SMALL_RES_LOOSE = 0.9e-3, 1.1e-3
 
 
 def dev(a, dtype=None):
@@ -48,9 +60,43 @@ def host(t):
     return t.detach().cpu().numpy()
 
 
+def cdf_distance(p, u, x):
+    """Distance of u to the two ends of token x's interval of the running sum of p."""
+    F = np.cumsum(np.asarray(p, dtype=np.float64))
+    hi = F[x]
+    lo = hi - p[x]
+    return min(abs(float(u) - lo), abs(hi - float(u)))
+
+
+def greedy_gap(row):
+    """Top-2 gap of a logit row relative to max(1, |max|) (the greedy near-tie measure)."""
+    z = np.sort(np.asarray(row, dtype=np.float32).astype(np.float64))
+    return (z[-1] - z[-2]) / max(1.0, abs(z[-1]))
+
+
+def _flag_agrees(bit_set, dist, what, b, strict=STRICT, loose=LOOSE):
+    if dist < strict:
+        assert bit_set, f"request {b}: oracle {what} distance {dist:.3e} but the device did not flag it"
+    if bit_set:
+        assert dist < loose, f"request {b}: device flagged {what} but the oracle distance is {dist:.3e}"
+
+
+def check_draft_flags(ld_o, x_o, u_draft, T, flags_gpu, reqs):
+    """DRAFT_NEAR_TIE against the oracle's distances at every drafted position."""
+    for i, b in enumerate(reqs):
+        d = np.inf
+        for k in range(x_o.shape[1]):
+            if T == 0.0:
+                d = min(d, greedy_gap(ld_o[i, k]))
+            else:
+                d = min(d, cdf_distance(O.softmax(ld_o[i, k], T), u_draft[b, k], int(x_o[i, k])))
+        _flag_agrees(bool(int(flags_gpu[b]) & FLAG_DRAFT_NEAR_TIE), d, "draft sample", b)
+
+
 def check_draft(U, W1, W2, x0, u_draft, T, x_gpu, ld_gpu, flags_gpu=None, requests=None):
     """Run the oracle on the given requests, following the GPU's token wherever the oracle
-    reports it as a valid outcome, and check every token and the stored draft logits.
+    reports it as a valid outcome, and check every token and the stored draft logits (and,
+    given the device flags, the draft near-tie bit).
 
     Returns the number of near-tie positions met.
     """
@@ -62,6 +108,8 @@ def check_draft(U, W1, W2, x0, u_draft, T, x_gpu, ld_gpu, flags_gpu=None, reques
     ref = ld_o.astype(np.float64)
     err = np.abs(ld_g - ref) / np.maximum(1.0, np.abs(ref))
     assert err.max() <= LD_TOL, f"l_d max scaled error {err.max():.3e}"
+    if flags_gpu is not None:
+        check_draft_flags(ld_o, x_o, u_draft, T, flags_gpu, reqs)
     return len(alts)
 
 
@@ -87,13 +135,50 @@ def verify_outcome(ld_b, lt_b, x_b, Lb, u_acc_b, u_res_b, T, n_gpu, y_gpu):
     raise AssertionError("could not align the oracle with the GPU outcome")
 
 
-def check_verify(ld, lt, x, L, u_acc, u_res, T, n_gpu, y_gpu, requests=None):
+def check_verify_flags(ld_b, lt_b, x_b, Lb, u_acc_b, u_res_b, T, r, flags_b, b):
+    """ACCEPT_NEAR_TIE, SAMPLE_NEAR_TIE and SMALL_RESIDUAL of one request against the oracle's
+    outcome r (already aligned with the device's n and y)."""
+    n = r["n"]
+    fl = int(flags_b)
+    # acceptance decisions taken: positions 0..n (the first rejection included), below L
+    d_acc = np.inf
+    for k in range(min(n + 1, Lb)):
+        if T == 0.0:
+            d_acc = min(d_acc, greedy_gap(lt_b[k]))
+        elif 0 <= int(x_b[k]) < ld_b.shape[-1]:
+            pd = O.softmax(ld_b[k], T)[int(x_b[k])]
+            pt = O.softmax(lt_b[k], T)[int(x_b[k])]
+            if pd > 0:
+                d_acc = min(d_acc, abs(float(u_acc_b[k]) - pt / pd))
+    _flag_agrees(bool(fl & FLAG_ACCEPT_NEAR_TIE), d_acc, "acceptance", b)
+    # the residual or bonus sample
+    tok = int(r["y"][n])
+    if T == 0.0:
+        d_smp = greedy_gap(lt_b[n])
+    else:
+        pt = O.softmax(lt_b[n], T)
+        p = pt
+        if n < Lb:
+            q = np.maximum(0.0, pt - O.softmax(ld_b[n], T))
+            if q.sum() > 0:
+                p = q / q.sum()
+        d_smp = cdf_distance(p, u_res_b, tok)
+    _flag_agrees(bool(fl & FLAG_SAMPLE_NEAR_TIE), d_smp, "residual/bonus sample", b)
+    z = r["residual_mass"] if (T > 0 and n < Lb) else np.inf
+    _flag_agrees(bool(fl & FLAG_SMALL_RESIDUAL), z, "residual mass", b, SMALL_RES_STRICT, SMALL_RES_LOOSE)
+
+
+def check_verify(ld, lt, x, L, u_acc, u_res, T, n_gpu, y_gpu, requests=None, flags_gpu=None):
+    """Check n and y of every given request against the oracle (and, given the device flags,
+    the verification's flag bits).  Returns the number of requests with a near-tie."""
     reqs = list(range(ld.shape[0])) if requests is None else list(requests)
     G = ld.shape[1]
     ties = 0
     for b in reqs:
         Lb = G if L is None else int(L[b])
         r = verify_outcome(ld[b], lt[b], x[b], Lb, u_acc[b], u_res[b], T, int(n_gpu[b]), y_gpu[b])
+        if flags_gpu is not None:
+            check_verify_flags(ld[b], lt[b], x[b], Lb, u_acc[b], u_res[b], T, r, flags_gpu[b], b)
         ties += bool(r["accept_ties"]) or len(r["sample_alts"]) > 1
     return ties
 

@@ -59,12 +59,13 @@ def test_tensor_core_steps_fused_and_per_step(fused, B, T):
     check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld, fl)
 
 
-def test_tensor_core_and_gemv_passes_agree():
-    wl, d = small(24, 6, 8192, 256, 1.0, seed=5)
-    x1, ld1, _ = run_draft(d, wl, 1)
-    x2, ld2, _ = run_draft(d, wl, 2)
-    np.testing.assert_allclose(ld1, ld2, rtol=0, atol=2e-5 * max(1.0, float(np.abs(ld1).max())))
-    assert (x1 == x2).mean() > 0.99
+@pytest.mark.parametrize("T", [1.0, 0.0])
+def test_tensor_core_and_gemv_passes_both_match_the_oracle(T):
+    # the same 24 requests through both main passes, each checked against the oracle
+    wl, d = small(24, 6, 8192, 256, T, seed=5)
+    for path in (1, 2):
+        x, ld, fl = run_draft(d, wl, path)
+        check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld, fl)
 
 
 @pytest.mark.parametrize("w_dtype", ["f32", "bf16"])

@@ -61,7 +61,7 @@ def test_verify_matches_oracle(V, T, scheduled, impl, labels):
     # without labels, rows past L_b + 1 are skipped by the kernels
     L = np.array([0, 1, 2, 3, 4, 2], dtype=np.int32) if scheduled else None
     n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=labels)
-    check_verify(ld, lt, x, L, u_acc, u_res, T, n, y)
+    check_verify(ld, lt, x, L, u_acc, u_res, T, n, y, flags_gpu=fl)
     if labels:
         check_labels(ld, lt, T, c)
     G_ = G if L is None else L
@@ -78,7 +78,7 @@ def test_identical_logits_accept_all_and_label_one(T):
         want_n = np.full(5, 6) if L is None else L
         assert np.array_equal(n, want_n)
         assert np.all(c == 1.0)
-        check_verify(ld, lt, x, L, u_acc, u_res, T, n, y)
+        check_verify(ld, lt, x, L, u_acc, u_res, T, n, y, flags_gpu=fl)
 
 
 def test_disjoint_support_is_certain_rejection():
@@ -93,7 +93,7 @@ def test_disjoint_support_is_certain_rejection():
     n, y, c, fl = run_verify(ld, lt, x, None, u_acc, u_res, 1.0)
     assert np.all(n == 0) and np.all(c == 0.0)
     assert y[0, 0] == 0 and y[1, 0] == V - 1
-    check_verify(ld, lt, x, None, u_acc, u_res, 1.0, n, y)
+    check_verify(ld, lt, x, None, u_acc, u_res, 1.0, n, y, flags_gpu=fl)
 
 
 @pytest.mark.parametrize("lt_rows", ["gamma", "gamma+1"])
@@ -146,7 +146,7 @@ def test_scheduled_rows_skipped_many_requests(impl):
     ld, lt, x, u_acc, u_res = case(B, G, V, 1.0, seed=77)
     L = (np.arange(B) * 7 % (G + 1)).astype(np.int32)
     n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, 1.0, want_c=False)
-    check_verify(ld, lt, x, L, u_acc, u_res, 1.0, n, y)
+    check_verify(ld, lt, x, L, u_acc, u_res, 1.0, n, y, flags_gpu=fl)
     assert np.all(n <= L)
 
 
@@ -157,7 +157,7 @@ def test_stream_vocabulary_beyond_per_row_kernels(T):
     B, G, V = 3, 3, 500_000
     ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=91)
     n, y, c, fl = run_verify(ld, lt, x, None, u_acc, u_res, T)
-    check_verify(ld, lt, x, None, u_acc, u_res, T, n, y)
+    check_verify(ld, lt, x, None, u_acc, u_res, T, n, y, flags_gpu=fl)
     check_labels(ld, lt, T, c)
     D.set_option("verify_stream", 0)
     with pytest.raises(D.DsparkError) as e:
@@ -177,6 +177,6 @@ def test_stream_lag_between_passes(lag, cluster, T):
     L = (np.arange(B) * 5 % (G + 1)).astype(np.int32)
     for want_c in (True, False):
         n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=want_c)
-        check_verify(ld, lt, x, L, u_acc, u_res, T, n, y)
+        check_verify(ld, lt, x, L, u_acc, u_res, T, n, y, flags_gpu=fl)
         if want_c:
             check_labels(ld, lt, T, c)

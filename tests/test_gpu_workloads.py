@@ -36,15 +36,16 @@ def test_tiny_round_matches_golden_fixture():
     if not fl.any():
         assert x.tolist() == g["x"] and n.tolist() == g["n_acc"] and y.tolist() == g["y"]
     np.testing.assert_allclose(c, g["c_star"], rtol=1e-5, atol=1e-9)
-    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld)
+    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld, fl)
+    check_verify(ld, d["lt"], x, None, d["u_acc"], d["u_res"], wl.T, n, y, flags_gpu=fl)
 
 
 @pytest.mark.parametrize("wl", [inputs.SINGLE_USER, inputs.SINGLE_USER_GREEDY], ids=lambda w: w.name)
 def test_single_user(wl):
     d = inputs.full_inputs(wl)
     x, ld, n, y, c, fl = gpu_round(d, wl)
-    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld)
-    check_verify(ld, d["lt"], x, None, d["u_acc"], d["u_res"], wl.T, n, y)
+    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld, fl)
+    check_verify(ld, d["lt"], x, None, d["u_acc"], d["u_res"], wl.T, n, y, flags_gpu=fl)
     check_labels(ld, d["lt"], wl.T, c)
 
 
@@ -52,8 +53,8 @@ def test_high_concurrency_all_requests():
     wl = inputs.HIGH_CONCURRENCY
     d = inputs.full_inputs(wl)
     x, ld, n, y, c, fl = gpu_round(d, wl)
-    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld)
-    check_verify(ld, d["lt"], x, None, d["u_acc"], d["u_res"], wl.T, n, y)
+    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld, fl)
+    check_verify(ld, d["lt"], x, None, d["u_acc"], d["u_res"], wl.T, n, y, flags_gpu=fl)
     check_labels(ld, d["lt"], wl.T, c)
     # suffix decay of the synthetic target: later positions agree less
     assert c[:, :4].mean() > c[:, -4:].mean()
@@ -68,10 +69,13 @@ def test_scheduled_step():
     if not (r["near_tie"] or host(sfl)[0] & D.FLAG_SCHED_NEAR_TIE):
         assert np.array_equal(Lg, r["L"])
     assert float(host(th)[0]) == pytest.approx(r["theta"], rel=1e-12)
-    x, ld, n, y, c, fl = gpu_round(d, wl, L=Lg, want_c=False)
-    check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld)
-    check_verify(ld, d["lt"], x, Lg, d["u_acc"], d["u_res"], wl.T, n, y)
-    assert np.all(n <= Lg)
+    for want_c in (False, True):   # labels of every position are computed whatever L is
+        x, ld, n, y, c, fl = gpu_round(d, wl, L=Lg, want_c=want_c)
+        check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, x, ld, fl)
+        check_verify(ld, d["lt"], x, Lg, d["u_acc"], d["u_res"], wl.T, n, y, flags_gpu=fl)
+        assert np.all(n <= Lg)
+        if want_c:
+            check_labels(ld, d["lt"], wl.T, c)
 
 
 @pytest.mark.parametrize("B", inputs.SWEEP_B)
@@ -94,8 +98,9 @@ def test_vocabulary_sweep(B, gamma):
     reqs = sorted({0, B - 1, B // 2})
     Uh, lth, ldh = host_rm(U[:, reqs]), host(lt[reqs]), host_rm(ld[:, reqs])
     sub = dict(U=Uh, x0=x0[reqs], u=u_draft[reqs])
-    check_draft(sub["U"], W1h, W2h, sub["x0"], sub["u"], wl.T, xh[reqs], ldh)
-    check_verify(ldh, lth, xh[reqs], None, u_acc[reqs], u_res[reqs], wl.T, nh[reqs], yh[reqs])
+    flh = host(fl)[reqs]
+    check_draft(sub["U"], W1h, W2h, sub["x0"], sub["u"], wl.T, xh[reqs], ldh, flh)
+    check_verify(ldh, lth, xh[reqs], None, u_acc[reqs], u_res[reqs], wl.T, nh[reqs], yh[reqs], flags_gpu=flh)
     check_labels(ldh, lth, wl.T, host(c)[reqs])
     del U, lt, ld
     torch.cuda.empty_cache()
