@@ -736,7 +736,8 @@ __device__ void combine_group(const DraftArgs& a, int k, int b, const Grp& g, do
   float* shf = reinterpret_cast<float*>(sh + 34);     // max scratch (32 floats = 16 doubles)
   int* shi = reinterpret_cast<int*>(sh + 52);         // [0] pick, [1] token, [2] flags
   double* shd = sh + 56;                              // [0] lo of the pick, [1] hi
-  const float u = __ldg(a.u_draft + b * a.gamma + k);  // requested before the first dependent load
+  // requested before the first dependent load; greedy drafting takes no uniforms (u_draft may be null)
+  const float u = a.greedy ? 0.f : __ldg(a.u_draft + b * a.gamma + k);
   if (tid == 0) shi[0] = -1;
 
   if (a.greedy) {
