@@ -82,11 +82,15 @@ const char* dspark_last_error(void);
  *   "draft_fused"     1 (default) tensor-core draft: all gamma positions in one cooperative
  *                     launch with grid barriers (falls back to one launch pair per position
  *                     when the grid cannot be co-resident); 0 always one pair per position
- *   "verify_stream"   1 (default) verification with a workspace and V % 4 == 0 runs the
- *                     streaming kernels; 0 the per-row cluster kernels
+ *   "verify_impl"     verification with a workspace (V % 4 == 0, 16-byte aligned rows):
+ *                     0 (default) the streaming kernels; 1 the column-sliced kernels (every row
+ *                     read from HBM once, rows exchanged through L2; slower at the sizes measured);
+ *                     2 the per-row cluster kernels.  Calls the chosen kernels cannot take fall
+ *                     back to the next ones and finally to the per-row kernels.
  *   "verify_stream_cluster"  CTAs per cluster of the streaming verify, 1..8 (default 3)
  *   "verify_stream_lag"      rows between a row's first and second pass, 1..3 (default 1)
  *   "verify_stream_l2hint"   1 (default) first-pass copies evict-last, second-pass evict-first
+ *   "verify_groups"   column-sliced verify: CTA groups (0: slices of about 16 KB per row)
  *   "verify_cluster"  0 automatic, else the cluster size of the per-row verify kernels (1..16,
  *                     power of 2)
  *   "verify_persistent" 1 (default) per-row sampled verification and labels run on persistent
@@ -94,8 +98,9 @@ const char* dspark_last_error(void);
  *                     cluster per row
  *   "sm_count"        0 query the device, else the SM count used to size persistent grids
  * The environment variables DSPARK_DRAFT_TC_MIN_B, DSPARK_DRAFT_PATH, DSPARK_DRAFT_PDL,
- * DSPARK_DRAFT_FUSED, DSPARK_VERIFY_CLUSTER, DSPARK_VERIFY_PERSISTENT, DSPARK_VERIFY_STREAM and
- * DSPARK_VERIFY_STREAM_CLUSTER set the initial values of the keys of the same names.
+ * DSPARK_DRAFT_FUSED, DSPARK_VERIFY_CLUSTER, DSPARK_VERIFY_PERSISTENT, DSPARK_VERIFY_IMPL,
+ * DSPARK_VERIFY_GROUPS and DSPARK_VERIFY_STREAM_CLUSTER set the initial values of the keys of the
+ * same names.
  * Returns DSPARK_EINVAL for an unknown key. */
 int dspark_set_option(const char* key, long value);
 

@@ -33,7 +33,8 @@ static Options& options_ref() {
     if (const char* e = std::getenv("DSPARK_DRAFT_FUSED")) o.draft_fused = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_CLUSTER")) o.verify_cluster = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_PERSISTENT")) o.verify_persistent = std::atoi(e);
-    if (const char* e = std::getenv("DSPARK_VERIFY_STREAM")) o.verify_stream = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_VERIFY_IMPL")) o.verify_impl = std::atoi(e);
+    if (const char* e = std::getenv("DSPARK_VERIFY_GROUPS")) o.verify_groups = std::atoi(e);
     if (const char* e = std::getenv("DSPARK_VERIFY_STREAM_CLUSTER")) o.verify_stream_cluster = std::atoi(e);
   });
   return o;
@@ -116,7 +117,8 @@ int dspark_set_option(const char* key, long value) {
   else if (!std::strcmp(key, "draft_fused")) o.draft_fused = (int)value;
   else if (!std::strcmp(key, "verify_cluster")) o.verify_cluster = (int)value;
   else if (!std::strcmp(key, "verify_persistent")) o.verify_persistent = (int)value;
-  else if (!std::strcmp(key, "verify_stream")) o.verify_stream = (int)value;
+  else if (!std::strcmp(key, "verify_impl")) o.verify_impl = (int)value;
+  else if (!std::strcmp(key, "verify_groups")) o.verify_groups = (int)value;
   else if (!std::strcmp(key, "verify_stream_cluster")) o.verify_stream_cluster = (int)value;
   else if (!std::strcmp(key, "verify_stream_lag")) o.verify_stream_lag = (int)value;
   else if (!std::strcmp(key, "verify_stream_l2hint")) o.verify_stream_l2hint = (int)value;

@@ -20,7 +20,8 @@ struct Options {
   int draft_fused = 1;           // tensor-core draft: all steps in one cooperative launch
   int verify_cluster = 0;        // 0 auto, else the cluster size (1, 2, 4, 8, 16)
   int verify_persistent = 1;     // sampled verify / labels: persistent double-buffered clusters
-  int verify_stream = 1;         // verify with a workspace: streaming kernels (one HBM read + one L2 read)
+  int verify_impl = 0;           // verify with a workspace: 0 streaming kernels, 1 column-sliced, 2 per-row
+  int verify_groups = 0;         // sliced verify: CTA groups (0: slices of about 16 KB per row)
   int verify_stream_cluster = 3; // CTAs per cluster of the streaming verify (1 to 8)
   int verify_stream_lag = 1;     // rows between a row's first and second pass (1 to 3)
   int verify_stream_l2hint = 1;  // streaming verify: first-pass copies evict-last, second-pass evict-first
@@ -94,6 +95,8 @@ dspark_status launch_draft(const DraftCall& c);
 dspark_status launch_verify(const VerifyCall& c);
 dspark_status launch_verify_stream(const VerifyCall& c);
 size_t stream_verify_workspace_bytes(int B, int gamma, int V);
+dspark_status launch_verify_sliced(const VerifyCall& c);
+size_t sliced_verify_workspace_bytes(int B, int gamma, int V);
 dspark_status launch_schedule(const ScheduleCall& c);
 
 constexpr int kMaxGamma = 64;

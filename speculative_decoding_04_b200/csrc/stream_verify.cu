@@ -1121,7 +1121,7 @@ size_t stream_verify_workspace_bytes(int B, int gamma, int V) { return sv_layout
 // 4, unaligned rows, a workspace sized for the per-row kernels, or no cluster fits).
 dspark_status launch_verify_stream(const VerifyCall& c) {
   const Options opt = options();
-  if (!c.do_verify || !opt.verify_stream) return DSPARK_ENOTIMPL;
+  if (!c.do_verify || c.per_row_only || opt.verify_impl != 0) return DSPARK_ENOTIMPL;
   if (c.V % 4 || (uintptr_t)c.ld % 16 || (uintptr_t)c.lt % 16) return DSPARK_ENOTIMPL;
   const SvLayout Ly = sv_layout(c.B, c.gamma, c.V);
   if (c.ws_bytes < Ly.total) return DSPARK_ENOTIMPL;

@@ -1041,7 +1041,8 @@ size_t verify_rows_workspace_bytes(int B, int gamma) {
 }
 
 size_t verify_workspace_bytes(int B, int gamma, int V) {
-  return std::max(verify_rows_workspace_bytes(B, gamma), stream_verify_workspace_bytes(B, gamma, V));
+  return std::max({verify_rows_workspace_bytes(B, gamma), stream_verify_workspace_bytes(B, gamma, V),
+                   sliced_verify_workspace_bytes(B, gamma, V)});
 }
 
 // Cluster size: the smallest power of two whose per-CTA slices (ℓ_d and ℓ_t, fp32) fit the
@@ -1132,7 +1133,9 @@ static dspark_status launch_verify_persistent(const VerifyArgs& a, int cs, cudaS
 
 dspark_status launch_verify(const VerifyCall& c) {
   if (c.do_verify && !c.per_row_only) {
-    const dspark_status st = launch_verify_stream(c);
+    dspark_status st = launch_verify_stream(c);
+    if (st != DSPARK_ENOTIMPL) return st;
+    st = launch_verify_sliced(c);
     if (st != DSPARK_ENOTIMPL) return st;  // else: the per-row kernels below
   }
   VerifyArgs a{};

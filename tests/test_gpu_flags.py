@@ -18,11 +18,11 @@ from tests.parity import check_draft, check_verify, dev, dev_weights, host, host
 
 pytestmark = pytest.mark.gpu
 
-VERIFY_IMPLS = ["stream", "rows", "noalloc"]
+VERIFY_IMPLS = ["sliced", "stream", "rows", "noalloc"]
 
 
 def run_verify(impl, ld, lt, x, L, u_acc, u_res, T):
-    D.set_option("verify_stream", 0 if impl == "rows" else 1)
+    D.set_option("verify_impl", {"stream": 0, "sliced": 1, "rows": 2, "noalloc": 0}[impl])
     args = (pm(ld), dev(lt), dev(x), None if L is None else dev(L), dev(u_acc), dev(u_res), T)
     if impl == "noalloc":
         n, y, c, fl = D.verify_noalloc(*args, want_c_star=True)

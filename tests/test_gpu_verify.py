@@ -29,16 +29,20 @@ def run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=True):
     return host(n), host(y), (host(c) if c is not None else None), host(fl)
 
 
-# kernels: "stream-C" = streaming kernels with clusters of C CTAs (the default with a
-# workspace); "rows-C" = one cluster of C CTAs per row (0: chosen from V), which serves calls
-# without a workspace, V not a multiple of 4 and the labels entry point.
-IMPLS = ["stream-8", "stream-6", "stream-4", "stream-3", "stream-1", "rows-0", "rows-1", "rows-4", "rows-16"]
+# kernels: "stream-C" = streaming kernels with clusters of C CTAs (the default with a workspace);
+# "sliced-G" = column-sliced kernels with G groups of CTAs (0: slices of about 16 KB);
+# "rows-C" = one cluster of C CTAs per row (0: chosen from V), which serves calls without a
+# workspace, V not a multiple of 4 and the labels entry point.
+IMPLS = ["sliced-0", "sliced-1", "sliced-3", "sliced-16", "stream-8", "stream-3", "stream-1", "rows-0", "rows-1",
+         "rows-4", "rows-16"]
 
 
 def use_impl(impl):
     kind, c = impl.split("-")
-    D.set_option("verify_stream", 1 if kind == "stream" else 0)
-    if kind == "stream":
+    D.set_option("verify_impl", {"stream": 0, "sliced": 1, "rows": 2}[kind])
+    if kind == "sliced":
+        D.set_option("verify_groups", int(c))
+    elif kind == "stream":
         D.set_option("verify_stream_cluster", int(c))
     else:
         D.set_option("verify_cluster", int(c))
@@ -54,8 +58,8 @@ def test_verify_matches_oracle(V, T, scheduled, impl, labels):
     kind, cluster = use_impl(impl)
     if kind == "rows" and cluster and V < 4096 and cluster > 4:
         pytest.skip("slice smaller than the block")
-    if kind == "stream" and V % 4:
-        pytest.skip("the streaming kernels need V % 4 == 0 (other V take the per-row kernels)")
+    if kind in ("stream", "sliced") and V % 4:
+        pytest.skip("the sliced and streaming kernels need V % 4 == 0 (other V take the per-row kernels)")
     B, G = 6, 4
     ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=V + int(T * 10) + cluster)
     # without labels, rows past L_b + 1 are skipped by the kernels
@@ -134,11 +138,13 @@ def test_acceptance_rate_matches_label_statistically():
     assert abs(rate - c1) < 4 * np.sqrt(c1 * (1 - c1) / B)
 
 
-@pytest.mark.parametrize("impl", ["stream-8", "stream-2", "persistent-1", "persistent-0"])
+@pytest.mark.parametrize("impl", ["sliced-0", "sliced-7", "stream-8", "stream-2", "persistent-1", "persistent-0"])
 def test_scheduled_rows_skipped_many_requests(impl):
     kind, v = impl.split("-")
-    D.set_option("verify_stream", 1 if kind == "stream" else 0)
-    if kind == "stream":
+    D.set_option("verify_impl", {"stream": 0, "sliced": 1, "persistent": 2}[kind])
+    if kind == "sliced":
+        D.set_option("verify_groups", int(v))
+    elif kind == "stream":
         D.set_option("verify_stream_cluster", int(v))
     else:
         D.set_option("verify_persistent", int(v))
@@ -152,14 +158,14 @@ def test_scheduled_rows_skipped_many_requests(impl):
 
 @pytest.mark.parametrize("T", [1.0, 0.0])
 def test_stream_vocabulary_beyond_per_row_kernels(T):
-    # V = 500,000: more than one 16-CTA cluster can hold per row; only the streaming kernels
-    # take it (rows of 489 tiles, the last one 288 columns wide)
+    # V = 500,000: more than one 16-CTA cluster can hold per row; the streaming kernels take it
+    # (rows of 489 tiles, the last one 288 columns wide), the per-row kernels refuse it
     B, G, V = 3, 3, 500_000
     ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=91)
     n, y, c, fl = run_verify(ld, lt, x, None, u_acc, u_res, T)
     check_verify(ld, lt, x, None, u_acc, u_res, T, n, y, flags_gpu=fl)
     check_labels(ld, lt, T, c)
-    D.set_option("verify_stream", 0)
+    D.set_option("verify_impl", 2)
     with pytest.raises(D.DsparkError) as e:
         run_verify(ld, lt, x, None, u_acc, u_res, T)
     assert e.value.status == D.ENOTIMPL
@@ -170,6 +176,7 @@ def test_stream_vocabulary_beyond_per_row_kernels(T):
 @pytest.mark.parametrize("T", [1.0, 0.0])
 def test_stream_lag_between_passes(lag, cluster, T):
     # the second pass of a row runs `lag` rows after its first pass; scheduled rows are skipped
+    D.set_option("verify_impl", 0)
     D.set_option("verify_stream_cluster", cluster)
     D.set_option("verify_stream_lag", lag)
     B, G, V = 24, 5, 20000
@@ -180,3 +187,34 @@ def test_stream_lag_between_passes(lag, cluster, T):
         check_verify(ld, lt, x, L, u_acc, u_res, T, n, y, flags_gpu=fl)
         if want_c:
             check_labels(ld, lt, T, c)
+
+
+@pytest.mark.parametrize("groups", [1, 5, 30])
+@pytest.mark.parametrize("T", [0.9, 0.0])
+def test_sliced_many_jobs_per_group(groups, T):
+    D.set_option("verify_impl", 1)
+    # more jobs per group than slots of the partial and decision rings (16) and stages of the
+    # copy ring; scheduled rows skipped; labels on and off
+    D.set_option("verify_groups", groups)
+    B, G, V = 40, 5, 12000
+    ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=400 + groups)
+    L = (np.arange(B) * 5 % (G + 1)).astype(np.int32)
+    for want_c in (True, False):
+        for Lc in (L, None):
+            n, y, c, fl = run_verify(ld, lt, x, Lc, u_acc, u_res, T, want_c=want_c)
+            check_verify(ld, lt, x, Lc, u_acc, u_res, T, n, y, flags_gpu=fl)
+            if want_c:
+                check_labels(ld, lt, T, c)
+
+
+@pytest.mark.parametrize("V", [64, 260, 1024, 4100])
+def test_sliced_narrow_vocabulary(V):
+    # slices of a few quads: tiles of 0 to 2 quads per warp, ragged everywhere
+    D.set_option("verify_impl", 1)
+    D.set_option("verify_groups", 1)
+    B, G = 9, 3
+    for T in (1.0, 0.0):
+        ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=V + int(T))
+        n, y, c, fl = run_verify(ld, lt, x, None, u_acc, u_res, T)
+        check_verify(ld, lt, x, None, u_acc, u_res, T, n, y, flags_gpu=fl)
+        check_labels(ld, lt, T, c)
