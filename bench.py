@@ -1,27 +1,35 @@
 """Benchmark of one DSpark draft/verify round on B200 (one JSON line on rank 0).
 
-Workload (BASELINE metric): high concurrency, B=64 requests, gamma=16, V=151936, r=256,
-T=0.8, bf16 Markov-head weights, fp32 logits (synthetic, seeded; see inputs.py).
+Default workload (the headline): high concurrency, B=64 requests, gamma=16, V=151936, r=256,
+T=0.8, bf16 Markov-head weights, fp32 logits (synthetic, seeded; see inputs.py).  --workload
+selects another of the five cases: single_user (B=1, gamma=7, T=1), single_user_greedy (T=0),
+scheduled_step (B=256, gamma=5, V=129280, the scheduler's verify lengths), sweep_B{B}_g{gamma}
+(V=262144, B in 1/8/32/128/512, gamma in 4/8/16), or profile (B=64, gamma=4: the headline's kernels
+on about 0.6 GB, for ncu captures).
 
 One step = one pass of the whole hot path over one batch:
-  markov_draft (16 x [tensor-core main pass + combine])
-  -> prefix_schedule (prefix survival + greedy scheduler; flat steps/s table, so the whole
-     gamma-block is selected and the verified work is the gamma=16 block)
-  -> verify (acceptance, residual/bonus sample, fused TV labels).
-Inputs live in HBM when the timed region starts; L2 (126 MB) is flushed by writing a
-256 MB buffer before every timed step, outside the timed events.
+  markov_draft (gamma positions in one cooperative launch on the tensor-core path)
+  -> prefix_schedule (prefix survival + greedy scheduler; a flat steps/s table, so the whole
+     gamma-block is verified, except on scheduled_step, which uses its affine-latency table)
+  -> verify (acceptance, residual/bonus sample; TV labels fused in, except on scheduled_step,
+     where only the scheduled rows are read).
+Inputs live in HBM when the timed region starts; L2 (126 MB) is flushed by writing a 256 MB
+buffer before every timed step, outside the timed events ("warm" repeats the timing without it).
+Times are medians of the per-step CUDA-event times on the launching stream.
 
 value       = rounds/s over all ranks (each rank runs its own batch: weak scaling)
-e2e         = the same rounds/s through the public API with pinned host buffers: the
-              per-step inputs are copied host->device and the step's result (n_acc, y)
-              device->host inside the timed region
-roofline    = the draft stage (all of its launches) against measured HBM copy bandwidth,
-              algorithmic bytes B*gamma*V*4 (read U) + gamma*r*V*2 (W2 per step) +
-              B*gamma*V*4 (write l_d); the verify kernel is reported beside it
-              (B*gamma*V*4 + B*(gamma+1)*V*4 bytes)
-cpu_baseline= the CPU oracle on a bounded sample of requests of the same workload
+e2e         = the same rounds/s through the public API with pinned host buffers: the per-step
+              inputs are copied host->device and the step's result (n_acc, y) device->host
+              inside the timed region
+roofline    = the draft stage (its one launch) against measured HBM copy bandwidth, algorithmic
+              bytes B*gamma*V*4 (read U) + gamma*r*V*2 (W2 per position) + B*gamma*V*4 (write l_d);
+              the verify call is reported beside it (rows it must read: every l_d and l_t row
+              with labels, else the scheduled ones)
+cpu_baseline= the CPU oracle on the machine's host cores: its request-independent and per-request
+              costs timed separately on small samples and combined for the whole batch
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+  python bench.py --draft-crossover     # draft time on the GEMV and tensor-core paths over B
 """
 
 import argparse
@@ -43,6 +51,7 @@ METRIC = "draft+verify rounds/s and verified tokens/s at V=151936, γ=16; HBM GB
 UNIT = "rounds/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+HOST_E2E_LIMIT = 6 << 30   # larger per-step inputs (big sweep points) are not staged in pinned memory
 
 
 def peaks():
@@ -70,21 +79,48 @@ def measured_traffic(key, units):
     return t["dram_bytes_per_launch"] * units / t["units_per_launch"]
 
 
-def workload_bytes(wl):
+def workload_of(name):
+    from speculative_decoding_04_b200 import inputs
+
+    if name in inputs.WORKLOADS:
+        return inputs.WORKLOADS[name]
+    if name == "profile":
+        return inputs.HIGH_CONCURRENCY.with_(name="profile", B=64, gamma=4)
+    if name.startswith("sweep_B"):
+        b, g = name[len("sweep_B"):].split("_g")
+        return inputs.sweep_point(int(b), int(g))
+    raise SystemExit(f"unknown workload {name}")
+
+
+def uses_schedule_table(wl):
+    return wl.name == "scheduled_step"
+
+
+def draft_bytes(wl):
     B, G, V, r = wl.B, wl.gamma, wl.V, wl.r
-    draft = B * G * V * 4 + G * r * V * 2 + B * G * V * 4
-    verify = B * G * V * 4 + B * (G + 1) * V * 4
-    flops = 2 * B * r * V * G
-    return draft, verify, flops
+    return B * G * V * 4 + G * r * V * 2 + B * G * V * 4
 
 
-def config_of(wl, n):
+def verify_bytes(wl, L=None, labels=True):
+    """Rows the verification must read: every l_d and l_t row with labels; else l_d rows
+    k < L_b and l_t rows k <= L_b of each request."""
+    B, G, V = wl.B, wl.gamma, wl.V
+    if labels or L is None:
+        return B * G * V * 4 + B * (G + 1) * V * 4
+    L = np.asarray(L, dtype=np.int64)
+    return int((2 * L + 1).sum()) * V * 4
+
+
+def config_of(wl, n, labels):
     return {"workload": f"{wl.name}: B={wl.B} requests, gamma={wl.gamma}, V={wl.V}, r={wl.r}, T={wl.T}, "
-                        f"bf16 W1/W2, fp32 log-Zipf+Gaussian logits",
+                        f"{wl.w_dtype} W1/W2, fp32 {'log-Zipf+Gaussian' if wl.logits == 'logzipf' else 'Gaussian'} "
+                        "logits",
             "B_per_gpu": wl.B, "gamma": wl.gamma, "V": wl.V, "r": wl.r, "T": wl.T,
             "parallelism": f"replicas over {n} GPU(s), no data-path collective",
-            "l2_policy": "256 MB write before every timed step (outside the timed events)",
-            "step": "markov_draft -> prefix_schedule (flat sps, full block) -> verify (+TV labels)"}
+            "l2_policy": "256 MB write before every timed step (outside the timed events); inputs > L2 too",
+            "step": ("markov_draft -> prefix_schedule ("
+                     + ("affine-latency sps, scheduled lengths" if uses_schedule_table(wl) else "flat sps, full block")
+                     + ") -> verify" + (" (+TV labels)" if labels else " (scheduled rows only)"))}
 
 
 class Clocks:
@@ -128,28 +164,44 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_baseline(wl, n_req, d=None):
-    """The oracle on n_req requests of the workload: one full round, scaled to the whole batch."""
+def oracle_round(wl, reqs, labels):
+    """One full oracle round (draft, schedule, verify, labels) on the given requests; seconds."""
     import oracle as O
     from speculative_decoding_04_b200 import inputs
 
-    threads = os.cpu_count() or 1
-    reqs = list(range(n_req))
     U, lt = inputs.logits(wl, reqs)
     W1, W2 = inputs.weights(wl)
     x0 = inputs.tokens(wl)[reqs]
     u_draft, u_acc, u_res = (a[reqs] for a in inputs.uniforms(wl))
     c = inputs.confidences(wl)
+    sps = inputs.sps_table(wl) if uses_schedule_table(wl) else np.ones(wl.D_max + 1)
     t0 = time.perf_counter()
     x, ld, _ = O.markov_draft(U, W1, W2, x0, u_draft, wl.T)
-    sch = O.prefix_schedule(c, np.ones(wl.D_max + 1), wl.D_max)
+    sch = O.prefix_schedule(c, sps, wl.D_max)
     O.verify(ld, lt, x, sch["L"][reqs], u_acc, u_res, wl.T)
-    O.tv_labels(ld, lt[:, :wl.gamma], wl.T)
-    dt = time.perf_counter() - t0
-    per_round = dt * wl.B / n_req
+    if labels:
+        O.tv_labels(ld, lt[:, :wl.gamma], wl.T)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, labels, n1=1, n2=3):
+    """The oracle (as it stands) on the host cores.  A round's cost is a request-independent part
+    (the fp64 copy of W2, the scheduler over the whole batch) plus a per-request part; both come
+    from timing one round on n1 and on n2 requests, and are combined for the whole batch."""
+    threads = os.cpu_count() or 1
+    n1, n2 = min(n1, wl.B), min(n2, wl.B)
+    t1 = oracle_round(wl, list(range(n1)), labels)
+    if n2 <= n1:  # the whole batch is the sample
+        return {"value": 1.0 / t1, "unit": UNIT, "cores": threads, "kind": "oracle",
+                "sample": f"one round on all {wl.B} request(s), {t1:.2f} s"}
+    t2 = oracle_round(wl, list(range(n2)), labels)
+    per_req = max((t2 - t1) / (n2 - n1), 1e-9)
+    fixed = max(t1 - n1 * per_req, 0.0)
+    per_round = fixed + wl.B * per_req
     return {"value": 1.0 / per_round, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n_req} of {wl.B} requests, one full round (draft, schedule, verify, labels), "
-                      f"{dt:.1f} s, scaled by {wl.B}/{n_req} (requests are independent)"}
+            "sample": f"one round on {n1} and on {n2} of {wl.B} requests ({t1:.2f} s, {t2:.2f} s): "
+                      f"{fixed:.2f} s request-independent + {per_req:.2f} s per request, "
+                      f"= {per_round:.1f} s for the whole batch"}
 
 
 def rank_workload(wl, rank):
@@ -170,51 +222,101 @@ def combine_ranks(times, accepted, world, device):
     return vals.tolist(), tot.item()
 
 
-def run_reference(args, wl, rank, world):
-    # the CPU oracle is the reference arm; rank 0 alone runs it
+def run_reference(args, wl, labels, rank):
+    """The reference arm: the CPU oracle as it stands.  Each step is one oracle round on a
+    bounded sample of requests (n_req of B); rounds/s of the whole batch come from the sample's
+    request-independent and per-request costs (timed once, as cpu_baseline does)."""
     if rank != 0:
         return
+    n_req = 1
+    cb = cpu_baseline(wl, labels)
     steps = []
-    n_req = 2
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(wl, n_req)
+        t = oracle_round(wl, list(range(n_req)), labels)
         if i >= args.warmup:
-            steps.append(1.0 / cb["value"])
-    t = statistics.mean(steps)
-    line = {"impl": "reference", "metric": METRIC, "value": 1.0 / t, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            steps.append(t)
+    t_step = statistics.median(steps)
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, see inputs.py)",
-            "config": config_of(wl, args.gpus),
-            "cpu_baseline": {"value": 1.0 / t, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
-                             "sample": cb["sample"]},
-            "e2e": {"value": 1.0 / t, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "config": config_of(wl, args.gpus, labels),
+            "cpu_baseline": dict(cb, sample=cb["sample"] + f"; each timed step: one round on {n_req} request(s)"),
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
+
+
+def median_ms(pairs):
+    return statistics.median(a.elapsed_time(b) for a, b in pairs)
+
+
+def draft_crossover(args):
+    """Draft time (CUDA events, median of 10 after 3 warm-ups, L2 flushed) on the CUDA-core GEMV
+    path and on the tensor-core path for B = 1 .. 32 at gamma = 16, V = 151936, r = 256."""
+    import torch
+
+    from speculative_decoding_04_b200 import build
+    build.build()
+    from speculative_decoding_04_b200 import dspark as D
+    from speculative_decoding_04_b200 import inputs
+
+    dev = torch.device("cuda")
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    base = inputs.HIGH_CONCURRENCY
+    W1h, W2h = inputs.weights(base)
+    W1 = torch.from_numpy(W1h).to(torch.bfloat16).to(dev)
+    W2 = torch.from_numpy(W2h).to(torch.bfloat16).to(dev)
+    for B in (1, 2, 4, 8, 9, 12, 16, 24, 32):
+        wl = base.with_(B=B)
+        U, _ = inputs.device_logits(wl, dev)
+        x0 = torch.from_numpy(inputs.tokens(wl)).to(dev)
+        u = torch.from_numpy(inputs.uniforms(wl)[0]).to(dev)
+        row = {"B": B, "gamma": wl.gamma, "V": wl.V}
+        for path, name in ((1, "gemv_ms"), (2, "tensor_core_ms")):
+            D.set_option("draft_path", path)
+            ev = []
+            for i in range(13):
+                flush.fill_(float(i))
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                D.markov_draft(U, W1, W2, x0, u, wl.T)
+                e1.record()
+                if i >= 3:
+                    ev.append((e0, e1))
+            torch.cuda.synchronize()
+            row[name] = median_ms(ev)
+        D.set_option("draft_path", 0)
+        row["draft_bytes_GB"] = draft_bytes(wl) / 1e9
+        print(json.dumps(row), flush=True)
+        del U
+        torch.cuda.empty_cache()
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dspark", choices=["dspark", "reference"])
-    ap.add_argument("--workload", default="high_concurrency", choices=["high_concurrency", "profile"],
-                    help="profile: B=64, gamma=4 (same kernels as the headline, ~0.6 GB on the device) for ncu captures")
+    ap.add_argument("--workload", default="high_concurrency",
+                    help="high_concurrency (default), single_user, single_user_greedy, scheduled_step, "
+                         "sweep_B{B}_g{gamma}, profile")
+    ap.add_argument("--labels", choices=["auto", "on", "off"], default="auto",
+                    help="TV labels in the verify call (auto: on, except on scheduled_step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle timing (after the GPU timing)")
-    ap.add_argument("--cpu-requests", type=int, default=4)
+    ap.add_argument("--draft-crossover", action="store_true", help="print draft times of both main-pass paths over B")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.draft_crossover:
+        return draft_crossover(args)
 
-    from speculative_decoding_04_b200 import inputs
-
-    wl = inputs.HIGH_CONCURRENCY
-    if args.workload == "profile":
-        wl = wl.with_(name="profile", B=64, gamma=4)
+    wl = workload_of(args.workload)
+    labels = (args.labels == "on") or (args.labels == "auto" and not uses_schedule_table(wl))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
-        return run_reference(args, wl, rank, world)
+        return run_reference(args, wl, labels, rank)
 
     import torch
     import torch.distributed as dist
@@ -222,6 +324,7 @@ def main():
     from speculative_decoding_04_b200 import build
     build.build()
     from speculative_decoding_04_b200 import dspark as D
+    from speculative_decoding_04_b200 import inputs
 
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
@@ -231,15 +334,25 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     # ---------------------------------------------------------------- inputs (each rank its own batch)
-    d = inputs.full_inputs(rank_workload(wl, rank))
-    d["U"] = d["U"].transpose(1, 0, 2)      # the draft's base logits are position-major [gamma, B, V]
-    pin = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
-           for k, v in d.items() if k in ("U", "lt", "x0", "u_draft", "u_acc", "u_res", "c")}
-    W1 = torch.from_numpy(d["W1"]).to(torch.bfloat16).to(dev)
-    W2 = torch.from_numpy(d["W2"]).to(torch.bfloat16).to(dev)
-    dv = {k: v.to(dev) for k, v in pin.items()}
+    wr = rank_workload(wl, rank)
     B, G, V, r = wl.B, wl.gamma, wl.V, wl.r
-    sps = torch.ones(B * G + 1, dtype=torch.float64, device=dev)       # flat: every drafted token is worth verifying
+    wdt = torch.bfloat16 if wl.w_dtype == "bf16" else torch.float32
+    W1h, W2h = inputs.weights(wr)
+    W1 = torch.from_numpy(W1h).to(wdt).to(dev)
+    W2 = torch.from_numpy(W2h).to(wdt).to(dev)
+    u_draft, u_acc, u_res = inputs.uniforms(wr)
+    small = {"x0": inputs.tokens(wr), "u_draft": u_draft, "u_acc": u_acc, "u_res": u_res, "c": inputs.confidences(wr)}
+    dv = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in small.items()}
+    host_logit_bytes = (B * G * V + B * (G + 1) * V) * 4
+    if wl.name.startswith("sweep_B"):
+        dv["U"], dv["lt"] = inputs.device_logits(wr, dev)          # drawn on the device (up to 26 GB)
+    else:
+        U, lt = inputs.logits(wr)
+        dv["U"] = torch.from_numpy(np.ascontiguousarray(U.transpose(1, 0, 2))).to(dev)  # position-major
+        dv["lt"] = torch.from_numpy(lt).to(dev)
+        del U, lt
+    sps_h = inputs.sps_table(wr) if uses_schedule_table(wl) else np.ones(B * G + 1)
+    sps = torch.from_numpy(sps_h).to(dev)
     x = torch.empty((B, G), dtype=torch.int32, device=dev)
     ld = torch.empty((G, B, V), dtype=torch.float32, device=dev)
     fl = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -247,17 +360,21 @@ def main():
     theta = torch.empty(1, dtype=torch.float64, device=dev)
     n_acc = torch.empty(B, dtype=torch.int32, device=dev)
     y = torch.empty((B, G + 1), dtype=torch.int32, device=dev)
-    c_star = torch.empty((B, G), dtype=torch.float32, device=dev)
+    c_star = torch.empty((B, G), dtype=torch.float32, device=dev) if labels else None
     ws_d = D.workspace(D.WS_DRAFT, B, G, V, r, dev)
     ws_v = D.workspace(D.WS_VERIFY, B, G, V, 0, dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    D.set_option("draft_fused", 1)  # the draft's gamma positions in one cooperative launch
-    n_launch = 1 + 1 + 2  # draft; schedule; verify: stream + finalize
+    # draft: one cooperative launch on the tensor-core path, else a main pass and a combine per
+    # position; schedule; verify: main kernel + finalize
+    tc = wl.w_dtype == "bf16" and r % 64 == 0 and r <= 256 and V % 8 == 0
+    n_launch = (1 if tc else 2 * G) + 1 + 2
 
-    def round_(src):
+    def draft(src):
         D.markov_draft(src["U"], W1, W2, src["x0"], src["u_draft"], wl.T, x_out=x, ld_out=ld, flags=fl, ws=ws_d,
                        stream=stream)
+
+    def schedule_and_verify(src):
         D.prefix_schedule(src["c"], sps, B * G, D.SCHED_ARGMAX, L_out=L, theta_out=theta, flags=fl, want_a=False,
                           stream=stream)
         D.verify(ld, src["lt"], x, L, src["u_acc"], src["u_res"], wl.T, n_acc=n_acc, y_out=y, c_star=c_star,
@@ -269,38 +386,39 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    def timed_rounds(nsteps, cold):
+        ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(nsteps)]
+        acc_dev = torch.zeros((), dtype=torch.int64, device=dev)
+        for i in range(nsteps):
+            if cold:
+                flush.fill_(float(i))
+            ev[i][0].record(stream)
+            draft(dv)
+            ev[i][1].record(stream)
+            schedule_and_verify(dv)
+            ev[i][2].record(stream)
+            acc_dev += n_acc.sum() + B
+        barrier()
+        step = statistics.median(a.elapsed_time(c) for a, _, c in ev)
+        dr = statistics.median(a.elapsed_time(b) for a, b, _ in ev)
+        return step, dr, int(acc_dev.item())
+
     clk = Clocks(local)      # sampling starts before the warm-up so that it covers the timed region
     time.sleep(0.5)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush.fill_(1.0)
-            round_(dv)
+            draft(dv)
+            schedule_and_verify(dv)
         barrier()
         tw0 = time.perf_counter()
-        accepted = 0
-        acc_dev = torch.zeros((), dtype=torch.int64, device=dev)
-        for i in range(args.steps):
-            flush.fill_(float(i))
-            ev[i][0].record(stream)
-            D.markov_draft(dv["U"], W1, W2, dv["x0"], dv["u_draft"], wl.T, x_out=x, ld_out=ld, flags=fl, ws=ws_d,
-                           stream=stream)
-            ev[i][1].record(stream)
-            D.prefix_schedule(dv["c"], sps, B * G, D.SCHED_ARGMAX, L_out=L, theta_out=theta, flags=fl, want_a=False,
-                              stream=stream)
-            D.verify(ld, dv["lt"], x, L, dv["u_acc"], dv["u_res"], wl.T, n_acc=n_acc, y_out=y, c_star=c_star,
-                     flags=fl, ws=ws_v, stream=stream)
-            ev[i][2].record(stream)
-            acc_dev += n_acc.sum() + B
-        barrier()
+        step_ms, draft_ms, accepted = timed_rounds(args.steps, cold=True)
         tw1 = time.perf_counter()
         clocks = clk.stop()
-        accepted = int(acc_dev.item())
-        step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(args.steps)]
-        draft_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+        L_h = L.cpu().numpy()
+        warm_step_ms, warm_draft_ms, _ = timed_rounds(args.steps, cold=False)
 
-        # verify alone, timed live around its one launch (same inputs, after a flush)
+        # verify alone (schedule + verify for the scheduled workload), timed live after a flush
         vt = []
         for i in range(args.steps):
             flush.fill_(float(i))
@@ -311,54 +429,85 @@ def main():
             e1.record(stream)
             vt.append((e0, e1))
         barrier()
-        verify_ms = [a.elapsed_time(b) for a, b in vt]
+        verify_ms = median_ms(vt)
+
+        # back-to-back rounds through the API without flushes or syncs: host wall clock per round
+        # against device time (launch overheads of the calls)
+        barrier()
+        tb0 = time.perf_counter()
+        eb0, eb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        eb0.record(stream)
+        for _ in range(args.steps):
+            draft(dv)
+            schedule_and_verify(dv)
+        eb1.record(stream)
+        th = time.perf_counter()
+        barrier()
+        tb1 = time.perf_counter()
+        b2b = {"rounds": args.steps, "host_issue_ms_per_round": (th - tb0) * 1e3 / args.steps,
+               "wall_ms_per_round": (tb1 - tb0) * 1e3 / args.steps,
+               "device_ms_per_round": eb0.elapsed_time(eb1) / args.steps}
 
         # end to end through the public API with pinned host buffers
-        n_out = torch.empty_like(n_acc, device="cpu").pin_memory()
-        y_out = torch.empty_like(y, device="cpu").pin_memory()
-        e2e = []
-        h2d = sum(v.numel() * v.element_size() for v in pin.values())
-        d2h = n_out.numel() * 4 + y_out.numel() * 4
-        stage = {k: torch.empty_like(v) for k, v in dv.items()}
-        for i in range(args.warmup + args.steps):
-            flush.fill_(float(i))
-            barrier()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for k in stage:
-                stage[k].copy_(pin[k], non_blocking=True)
-            round_(stage)
-            n_out.copy_(n_acc, non_blocking=True)
-            y_out.copy_(y, non_blocking=True)
-            e1.record(stream)
-            e1.synchronize()
-            if i >= args.warmup:
-                e2e.append(e0.elapsed_time(e1))
+        e2e = None
+        if host_logit_bytes <= HOST_E2E_LIMIT:
+            pin = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in dv.items()}
+            for k in pin:
+                pin[k].copy_(dv[k])
+            n_out = torch.empty(B, dtype=torch.int32).pin_memory()
+            y_out = torch.empty((B, G + 1), dtype=torch.int32).pin_memory()
+            h2d = sum(v.numel() * v.element_size() for v in pin.values())
+            d2h = n_out.numel() * 4 + y_out.numel() * 4
+            stage = {k: torch.empty_like(v) for k, v in dv.items()}
+            ev = []
+            for i in range(args.warmup + args.steps):
+                flush.fill_(float(i))
+                barrier()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for k in stage:
+                    stage[k].copy_(pin[k], non_blocking=True)
+                draft(stage)
+                schedule_and_verify(stage)
+                n_out.copy_(n_acc, non_blocking=True)
+                y_out.copy_(y, non_blocking=True)
+                e1.record(stream)
+                e1.synchronize()
+                if i >= args.warmup:
+                    ev.append((e0, e1))
+            e2e_ms = median_ms(ev)
+            del stage, pin
 
-    t_step = statistics.mean(step_ms) / 1e3
-    t_e2e = statistics.mean(e2e) / 1e3
-    t_draft = statistics.mean(draft_ms) / 1e3
-    t_verify = statistics.mean(verify_ms) / 1e3
+    t_step, t_draft, t_verify = step_ms / 1e3, draft_ms / 1e3, verify_ms / 1e3
+    t_e2e = e2e_ms / 1e3 if host_logit_bytes <= HOST_E2E_LIMIT else 0.0
     (t_step, t_e2e, t_draft, t_verify), accepted_all = combine_ranks([t_step, t_e2e, t_draft, t_verify], accepted,
                                                                        world, dev)
-
     if rank == 0:
         hbm, bf16, src = peaks()
-        draft_b, verify_b, flops = workload_bytes(wl)
+        draft_b = draft_bytes(wl)
+        verify_b = verify_bytes(wl, L_h, labels)
+        flops = 2 * B * r * V * G
         rounds = world / t_step
+        tokens_per_round = accepted_all / (args.steps * world)          # per rank's batch
+        tau = tokens_per_round / B                                       # tokens emitted per request
         line = {
             "metric": METRIC, "value": rounds, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded log-Zipf + Gaussian logits, bf16 weights)",
-            "config": config_of(wl, world),
+            "vs_baseline": None, "dtype": "f32", "data": f"synthetic (seeded log-Zipf + Gaussian logits, "
+                                                         f"{wl.w_dtype} weights)",
+            "config": config_of(wl, world, labels),
             "verified_tokens_per_s": accepted_all / (args.steps * t_step),
+            "tokens_per_request_per_round": tau,
+            "latency_per_token_us": (t_draft + t_verify) / tau * 1e6,
             "draft_ms": t_draft * 1e3, "verify_ms": t_verify * 1e3,
             "hbm_gbs_round": (draft_b + verify_b) / t_step / 1e9,
-            "roofline": {"kernel": f"markov_draft (draft_main_tc<64>: {G} positions in one cooperative launch, "
-                                   "timed with CUDA events around the call)",
+            "roofline": {"kernel": "markov_draft (draft_main_tc: all positions in one cooperative launch; "
+                                   "CUDA events around the call)" if tc else
+                                   "markov_draft (draft_main_fma + draft_combine per position; CUDA events "
+                                   "around the call)",
                          "bound": "hbm", "achieved": draft_b / t_draft / 1e9, "peak": hbm, "unit": "GB/s",
                          "frac": draft_b / t_draft / 1e9 / hbm,
-                         "traffic": measured_traffic("draft_main_tc", B * G),
+                         "traffic": measured_traffic("draft_main_tc", B * G) if tc else None,
                          "peak_source": src, "algorithmic_bytes": draft_b, "bias_tflops": flops / t_draft / 1e12,
                          "frac_of_nominal_8TBs": draft_b / t_draft / 8e12},
             "roofline_verify": {"kernel": "verify (verify_stream + verify_stream_finalize, timed together)",
@@ -366,13 +515,18 @@ def main():
                                 "frac": verify_b / t_verify / 1e9 / hbm,
                                 "traffic": measured_traffic("verify_stream", verify_b),
                                 "algorithmic_bytes": verify_b},
-            "e2e": {"value": world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "warm_l2": {"ms_per_step": warm_step_ms, "draft_ms": warm_draft_ms, "rounds_per_s": 1e3 / warm_step_ms},
+            "back_to_back": b2b,
+            "e2e": ({"value": world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                    if host_logit_bytes <= HOST_E2E_LIMIT else
+                    {"value": None, "unit": UNIT, "h2d_bytes_per_step": None, "d2h_bytes_per_step": None,
+                     "note": f"inputs of {host_logit_bytes / 1e9:.1f} GB per step are not staged in pinned memory"}),
             "gpu_launches": n_launch * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": tw1 - tw0,
         }
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, args.cpu_requests)
+            line["cpu_baseline"] = cpu_baseline(wl, labels)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -375,6 +375,7 @@ __device__ __forceinline__ bool grid_sync(uint32_t* count, uint32_t nblocks, uin
 }
 
 __device__ void combine_group(const DraftArgs& a, int k, int b, const Grp& g, double* sh);
+__device__ void combine_warp(const DraftArgs& a, int k, int b, uint32_t* gready);
 
 // Steps k0 .. k1-1 of the draft.  With fused = 0 the launch is one step and a separate combine
 // kernel samples its tokens; with fused = 1 (a cooperative launch, all CTAs resident) every step
@@ -408,14 +409,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L.misc + 4);
   const TcSync sy{s_abort, a.status};
-  __shared__ double s_comb[72];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % n_bgroups;
   const int jc = blockIdx.x / n_bgroups;
-  const int t_beg = (int)((long long)jc * a.ntiles / ctas_per_group);
-  const int t_end = (int)((long long)(jc + 1) * a.ntiles / ctas_per_group);
-  const int nt = t_end - t_beg;
+  // This CTA's columns are half-tiles [h_beg, h_end) of 64 columns (a.ntiles of them in V), so
+  // the CTAs' shares differ by at most 64 columns; it runs them as 128-column tiles starting at
+  // h_beg, the last one half when the count is odd.  A half tile still computes, loads and stores
+  // 128 columns (its second half is the next CTA's first, and the values written are the same
+  // bits: the same inputs through the same MMA), but only its own 64 enter the statistics.
+  const int h_beg = (int)((long long)jc * a.ntiles / ctas_per_group);
+  const int h_end = (int)((long long)(jc + 1) * a.ntiles / ctas_per_group);
+  const int nt = (h_end - h_beg + 1) / 2;
+  const bool last_half = ((h_end - h_beg) & 1) != 0;
+  auto tile_col = [&](int i) { return (h_beg + 2 * i) * 64; };  // first column of tile i
   const int b0 = g * NB;
   const int ksteps = a.r / 16;
   const int total = (k1 - k0) * nt;  // tiles of this CTA over the launch
@@ -459,11 +466,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int bb = b0 + h * 32;
   constexpr uint32_t kUStage = (uint32_t)NB * kTcTile;  // floats of one U stage: [NB requests][128 columns]
   // U (an input of the call) for the first two tiles is requested before waiting for the previous
-  // kernel: one 128-column x NB-request box per tile.
+  // kernel: one 128-column x NB-request box per tile.  L2 policies: U and l_d, streamed once per
+  // step, are evict-first; W2, read at every step, is evict-last on half of its lines (the
+  // setting measured fastest at B = 64, gamma = 16: 562 against 595 us without policies; W2
+  // evict-last on every line, 587 us).
   auto load_u = [&](int gi) {
     const int j = gi & 1, ku = k0 + gi / nt, iu = gi % nt;
     mbar_arrive_expect_tx(&u_full[j], kUStage * 4u);
-    tma_load_3d(sU + j * kUStage, &tmU, (t_beg + iu) * kTcTile, b0, ku, &u_full[j]);
+    tma_load_3d_hint(sU + j * kUStage, &tmU, tile_col(iu), b0, ku, &u_full[j], l2_policy_evict_first());
   };
   if (warp == 3 && lane == 0)
     for (int gi = 0; gi < 2 && gi < total; ++gi) load_u(gi);
@@ -475,13 +485,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       int issued = 0;
       for (int gi = 0; gi < total; ++gi) {
-        const int v0 = (t_beg + gi % nt) * kTcTile;
+        // a half tile loads its whole W2 tile too: its upper 64 columns are stored as well
+        const int v0 = tile_col(gi % nt);
         const int s = gi % kTcStages;
         if (!tc_wait(sy, &w_empty[s], ((gi / kTcStages) & 1) ^ 1)) break;
         uint8_t* st = sW + s * L.w2_stage_bytes;
         mbar_arrive_expect_tx(&w_full[s], L.w2_stage_bytes);
-        tma_load_2d(st, &tmW2, v0, 0, &w_full[s]);
-        tma_load_2d(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s]);
+        const uint64_t pol = l2_policy_evict_last_half();
+        tma_load_2d_hint(st, &tmW2, v0, 0, &w_full[s], pol);
+        tma_load_2d_hint(st + L.w2_stage_bytes / 2, &tmW2, v0 + 64, 0, &w_full[s], pol);
         issued = gi + 1;
       }
       if (*s_abort) {
@@ -497,6 +509,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     pdl_wait();
     uint32_t epoch = 0;
     uint32_t* gcount = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.status) + 64);
+    uint32_t* gready = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.status) + 128);
     bool bad = false;
     int last_load[2] = {total > 0 ? 0 : -1, total > 1 ? 1 : -1};  // (warp 3) last tile loaded into each U stage
     for (int k = k0; k < k1; ++k) {
@@ -534,7 +547,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < nt; ++i) {
             const int gi = gbase + i, j = gi & 1;
             if (!tc_wait(sy, &c_done[j], (gi >> 1) & 1)) break;
-            tma_store_3d(&tmLd, sU + j * kUStage, (t_beg + i) * kTcTile, b0, k);
+            tma_store_3d_hint(&tmLd, sU + j * kUStage, tile_col(i), b0, k, l2_policy_evict_first());
             bulk_commit();
             if (gi + 2 < total) {
               if (!tc_wait(sy, &u_empty[j], (gi >> 1) & 1)) break;
@@ -582,7 +595,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ChunkStat run = stat_empty();
         for (int i = 0; i < nt; ++i) {
           const int gi = gbase + i, j = gi & 1, acc = gi & 1;
-          const int v0w = (t_beg + i) * kTcTile + q * 32;  // this warp's 32 columns
+          const int v0w = tile_col(i) + q * 32;  // this warp's 32 columns
+          const bool own = !(last_half && i == nt - 1 && q >= 2);  // columns of this CTA
           const bool ok_u = tc_wait(sy, &u_full[j], (gi >> 1) & 1);
           const bool ok_t = __all_sync(0xffffffffu, tc_wait(sy, &t_full[acc], (gi >> 1) & 1) && ok_u);
           float x[32];
@@ -614,7 +628,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               lv[4 * s4 + 2] = f.z;
               lv[4 * s4 + 3] = f.w;
             }
-            const int nval = min(32, a.V - v0w);  // valid columns of this chunk (multiple of 8)
+            const int nval = own ? min(32, a.V - v0w) : 0;  // valid columns of this chunk (multiple of 8)
             ChunkStat st;
             if (a.greedy) {
               Top2 t{-INFINITY, -1, -INFINITY};
@@ -650,7 +664,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               bad |= isnan(sm) || mx == INFINITY;
               st = ChunkStat{mx, sm, 0, 0.f};
             }
-            if (v0w < a.V) stat_fold(run, st, a.greedy);
+            if (own && v0w < a.V) stat_fold(run, st, a.greedy);
           }
           __syncwarp();  // every lane is done with this stage
           if (lane == 0) mbar_arrive(&u_empty[j]);
@@ -671,16 +685,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (fused) {
         // ---------------------------------------------------------------- sample this step
+        // every CTA's partition records and l_d stores of the step are in place
         named_bar(3, kTcThreads - 32);
         if (warp == 1 && lane == 0) grid_sync(gcount, gridDim.x, epoch, sy);
         named_bar(3, kTcThreads - 32);
-        // one request per CTA at a time, all non-producer warps together
-        // (no test of the abort flag here: every thread of the group must take the same path)
-        for (int rq = blockIdx.x; rq < a.B; rq += gridDim.x)
-          combine_group(a, k, rq, Grp{(int)threadIdx.x - 32, kTcThreads - 32, 4}, s_comb);
-        named_bar(3, kTcThreads - 32);
-        if (warp == 1 && lane == 0) grid_sync(gcount, gridDim.x, epoch, sy);
-        named_bar(3, kTcThreads - 32);
+        // one warp per request, the requests spread over the grid (request blockIdx.x + m*gridDim.x
+        // goes to warp 1 + m % 11 of this CTA): no block barrier inside a combine
+        for (int m = 0;; ++m) {
+          const int rq = (int)blockIdx.x + m * (int)gridDim.x;
+          if (rq >= a.B) break;
+          if (warp == 1 + m % (kTcThreads / 32 - 1)) combine_warp(a, k, rq, gready);
+        }
+        // the next step's B operand needs the W1 rows of all B tokens just drafted: each combine
+        // counts its row in; the MMA warp waits for the step's B rows before it loads them
+        if (k + 1 < k1 && a.gbuf) {
+          if (warp == 1 && lane == 0) {
+            const uint32_t target = (uint32_t)(k - k0 + 1) * (uint32_t)a.B;
+            bool okc = !*s_abort;
+            for (uint32_t i = 0; okc; ++i) {
+              uint32_t v;
+              asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gready) : "memory");
+              if ((int32_t)(v - target) >= 0) break;
+              if (i >= kSpinLimit || ((i & 1023u) == 1023u && *s_abort)) {
+                if (!*s_abort) {
+                  *s_abort = 1;
+                  atomicOr(a.status, (uint32_t)DSPARK_ETIMEOUT);
+                }
+                okc = false;
+              }
+            }
+            // the rows were written with generic stores; the B operand is read by TMA
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+          }
+          named_bar(3, kTcThreads - 32);
+        }
       }
     }
     if (epi) {
@@ -892,6 +930,186 @@ __device__ void combine_group(const DraftArgs& a, int k, int b, const Grp& g, do
   g.sync();
 }
 
+// Combine of one request by one warp (the multi-step launch: the B requests' combines run on B
+// warps spread over the grid, with no block barrier).  The same two levels and arithmetic as
+// combine_group, each lane a contiguous run of records (level 1, np <= 256) or of logits
+// (level 2).  The warp then copies W1[x_k] into row b of gbuf and adds 1 to *gready with
+// release semantics.
+__device__ void combine_warp(const DraftArgs& a, int k, int b, uint32_t* gready) {
+  const size_t B = (size_t)a.B;
+  const int np = a.np, lane = threadIdx.x & 31;
+  constexpr unsigned FULL = 0xffffffffu;
+  // requested before the first dependent load; greedy drafting takes no uniforms (u_draft may be null)
+  const float u = a.greedy ? 0.f : __ldg(a.u_draft + b * a.gamma + k);
+  int x = 0;
+  uint32_t fl = 0;
+  if (a.greedy) {
+    Top2 t{-INFINITY, -1, -INFINITY};
+    for (int p = lane; p < np; p += 32) {
+      const ChunkStat s = ld_stat_cg(a.cpart + p * B + b);
+      t = top2_merge(t, Top2{s.m, s.idx, s.m2});
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t = top2_merge(t, top2_shfl_xor(t, o));
+    x = t.idx;
+    if (x < 0 || x >= a.V) {
+      fl |= DSPARK_FLAG_NONFINITE;
+      x = min(max(x, 0), a.V - 1);
+    }
+    if (t.best - t.second <= 1e-6f * fmaxf(1.f, fabsf(t.best))) fl |= DSPARK_FLAG_DRAFT_NEAR_TIE;
+  } else {
+    // ---- level 1: each lane a contiguous run of at most 8 partition records
+    const int e1 = (np + 31) / 32;
+    const int i0 = min(np, lane * e1), i1 = min(np, i0 + e1);
+    ChunkStat rec[8];
+    float ml = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      rec[j] = (i0 + j < i1) ? ld_stat_cg(a.cpart + (size_t)(i0 + j) * B + b) : stat_empty();
+      ml = fmaxf(ml, rec[j].m);
+    }
+    const float M = warp_max(ml);
+    double w[8], own = 0.0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      w[j] = rec[j].m == -INFINITY ? 0.0 : (double)rec[j].s * (double)ex_shift(rec[j].m, M);
+      own += w[j];
+    }
+    const double incl = warp_incl_scan_d(own);
+    const double S = __shfl_sync(FULL, incl, 31);
+    const double t = (double)u * S;
+    const double excl = incl - own;
+    int pick = -1;
+    double plo = 0.0;
+    if (i0 < i1 && excl <= t && (t < incl || i1 == np)) {
+      double R = excl, lastlo = 0.0;
+      int last = -1;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (pick < 0 && w[j] > 0.0) {
+          last = i0 + j;
+          lastlo = R;
+          if (t < R + w[j]) {
+            pick = i0 + j;
+            plo = R;
+          }
+        }
+        R += w[j];
+      }
+      if (pick < 0) {
+        pick = last;
+        plo = lastlo;
+      }
+    }
+    const unsigned hit = __ballot_sync(FULL, pick >= 0);
+    const int src = hit ? __ffs(hit) - 1 : 0;
+    const int p = hit ? __shfl_sync(FULL, pick, src) : -1;
+    const double lo1 = __shfl_sync(FULL, plo, src);
+    if (p < 0 || !(S > 0.0) || !isfinite(S)) {
+      fl |= DSPARK_FLAG_NONFINITE;
+      x = 0;
+    } else {
+      // ---- level 2: the partition's stored logits in 128-column chunks (lane l holds quad l of
+      // each chunk, so a chunk's lanes are in vocabulary order); every load of a block of 16
+      // chunks is issued before any arithmetic (one L2 latency per 2048 columns)
+      const int t0 = (int)((long long)p * a.ntiles / np), t1 = (int)((long long)(p + 1) * a.ntiles / np);
+      const int tw = a.tile_chunks * kChunk;
+      const int v0 = t0 * tw, n = min(t1 * tw, a.V) - v0;
+      const float4* row4 = reinterpret_cast<const float4*>(a.ld + ((size_t)k * a.B + b) * a.V + v0);  // 16-byte aligned
+      const float inv_T = a.inv_T;
+      const int nq4 = (n + 3) / 4;
+      double base = lo1;  // weight before the current chunk
+      int pk = -1, lastq = -1;
+      double qlo = 0.0, qhi = 0.0;
+      for (int blk = 0; blk < nq4 && pk < 0; blk += 16 * 32) {
+        float4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int q = blk + 32 * i + lane;
+          v[i] = q < nq4 ? __ldcg(row4 + q) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (pk >= 0 || blk + 32 * i >= nq4) break;  // warp-uniform
+          const int e0 = (blk + 32 * i + lane) * 4;   // first column (relative to v0) of this lane's quad
+          const float l4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+          double we[4], wl = 0.0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float z = __fmul_rn(l4[c], inv_T);
+            we[c] = (e0 + c < n && z != -INFINITY) ? (double)ex_shift(z, M) : 0.0;
+            wl += we[c];
+          }
+          const double incl2 = warp_incl_scan_d(wl);
+          const double tot = __shfl_sync(FULL, incl2, 31);
+          const unsigned pos = __ballot_sync(FULL, wl > 0.0);
+          if (pos) lastq = blk + 32 * i + 31 - __clz(pos);  // the last quad with weight so far
+          if (base + tot > t) {
+            // the chunk holds u*S: the first lane whose running sum passes it, then its element
+            const unsigned hit = __ballot_sync(FULL, wl > 0.0 && base + incl2 > t);
+            if (hit) {
+              const int hl = __ffs(hit) - 1;
+              if (lane == hl) {
+                double R = base + incl2 - wl;
+                for (int c = 0; c < 4; ++c) {
+                  if (we[c] > 0.0 && t < R + we[c]) {
+                    pk = e0 + c;
+                    qlo = R;
+                    qhi = R + we[c];
+                    break;
+                  }
+                  R += we[c];
+                }
+                if (pk < 0) {  // rounding inside the quad: its last element with weight
+                  for (int c = 3; c >= 0 && pk < 0; --c)
+                    if (we[c] > 0.0) pk = e0 + c;
+                  qlo = qhi = t;
+                }
+              }
+              pk = __shfl_sync(FULL, pk, hl);
+              qlo = __shfl_sync(FULL, qlo, hl);
+              qhi = __shfl_sync(FULL, qhi, hl);
+            }
+          }
+          base += tot;
+        }
+      }
+      if (pk < 0 && lastq >= 0) {
+        // rounding left u*S past the partition: its last element with weight, flagged as a tie
+        for (int c = 3; c >= 0 && pk < 0; --c) {
+          const int e = lastq * 4 + c;
+          if (e < n) {
+            const float z = __fmul_rn(__ldcg(a.ld + ((size_t)k * a.B + b) * a.V + v0 + e), inv_T);
+            if (z != -INFINITY && ex_shift(z, M) > 0.f) pk = e;
+          }
+        }
+        qlo = qhi = t;
+      }
+      if (pk >= 0) {
+        x = v0 + pk;
+        if ((t - qlo) < 1e-6 * S || (qhi - t) < 1e-6 * S) fl |= DSPARK_FLAG_DRAFT_NEAR_TIE;
+      } else {
+        fl |= DSPARK_FLAG_NONFINITE;
+        x = 0;
+      }
+      x = min(max(x, 0), a.V - 1);
+    }
+  }
+  if (lane == 0) {
+    if (fl) atomicOr(a.flags + b, fl);
+    a.x_out[b * a.gamma + k] = x;
+  }
+  // the next step's B operand row: W1[x_k] (bf16 weights only)
+  if (a.gbuf && k + 1 < a.gamma) {
+    const int cpr = a.r / 8;  // 16-byte chunks per row
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.W1) + (size_t)x * a.r);
+    uint4* dst = reinterpret_cast<uint4*>(a.gbuf + (size_t)b * a.r);
+    for (int c = lane; c < cpr; c += 32) dst[c] = __ldg(src + c);
+    __syncwarp();  // orders the lanes' row stores before lane 0's release
+    if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(gready) : "memory");
+  }
+}
+
 // Combine kernel of the per-step launches: one CTA of kCombThreads per request.
 constexpr int kCombThreads = 512;
 __global__ void __launch_bounds__(kCombThreads) draft_combine(DraftArgs a, int k) {
@@ -1034,8 +1252,8 @@ dspark_status launch_draft(const DraftCall& c) {
   size_t tc_smem = 0;
   if (use_tc) {
     nb = c.B <= 32 ? 32 : 64;
-    a.ntiles = (c.V + kTcTile - 1) / kTcTile;
-    a.tile_chunks = kTcTile / kChunk;
+    a.ntiles = (c.V + 63) / 64;  // half tiles: the unit of the CTAs' column shares
+    a.tile_chunks = 64 / kChunk;
     n_bgroups = (c.B + nb - 1) / nb;
     const int sms = device_sm_count();
     cpg = std::max(1, sms / n_bgroups);
@@ -1083,7 +1301,10 @@ dspark_status launch_draft(const DraftCall& c) {
     a.np = a.ntiles;
   }
 
-  if (use_tc && opt.draft_fused) {
+  // the in-kernel combine takes <= 8 partition records a lane; other shapes run one launch pair
+  // per step
+  const bool fusable = a.np <= 256;
+  if (use_tc && opt.draft_fused && fusable) {
     // all gamma steps in one cooperative launch (every CTA resident; grid barriers between steps)
     const dim3 grid(cpg * n_bgroups), block(kTcThreads);
     if (nb == 32)

@@ -14,7 +14,7 @@ namespace dspark {
 void set_error(const std::string& msg);
 
 struct Options {
-  int draft_tc_min_b = 9;        // bf16 drafts with at least this many requests use the tensor-core path
+  int draft_tc_min_b = 1;        // bf16 drafts with at least this many requests use the tensor-core path
   int draft_force_path = 0;      // 0 auto, 1 CUDA-core GEMV, 2 tensor cores
   int draft_pdl = 1;             // chain the draft kernels with programmatic dependent launch
   int draft_fused = 1;           // tensor-core draft: all steps in one cooperative launch

@@ -23,7 +23,7 @@ def _default_options():
     if torch.cuda.is_available():
         from speculative_decoding_04_b200 import dspark as D
         D.set_option("draft_path", 0)
-        D.set_option("draft_tc_min_b", 9)
+        D.set_option("draft_tc_min_b", 1)
         D.set_option("verify_cluster", 0)
         D.set_option("draft_pdl", 1)
         D.set_option("draft_fused", 1)
