@@ -90,15 +90,19 @@ const char* dspark_last_error(void);
  *                     2 the per-row cluster kernels.  Calls the chosen kernels cannot take fall
  *                     back to the next ones and finally to the per-row kernels.
  *   "verify_stream_cluster"  CTAs per cluster of the streaming verify, 1..8 (default 3)
- *   "verify_stream_lag"      rows between a row's first and second pass, 1..3 (default 1)
  *   "verify_stream_l2hint"   1 (default) first-pass copies evict-last, second-pass evict-first
  *   "verify_groups"   column-sliced verify: CTA groups (0: slices of about 16 KB per row)
  *   "verify_cluster"  0 automatic, else the cluster size of the per-row verify kernels (1..16,
  *                     power of 2)
  *   "verify_persistent" 1 (default) per-row sampled verification and labels run on persistent
- *                     clusters with double-buffered rows; 2 the same single-buffered; 0 one
- *                     cluster per row
+ *                     clusters with double-buffered rows; 0 one cluster per row
  *   "sm_count"        0 query the device, else the SM count used to size persistent grids
+ *   "debug_wait_limit", "debug_unreachable_barrier"  test-only: the first shortens the bounded
+ *                     device waits (draft: polls per wait; streaming verify: nanoseconds; 0: the
+ *                     defaults of about a second and 2 s); the second makes one wait unsatisfiable
+ *                     (1: the fused draft's first grid barrier, 2: the streaming verify's cluster
+ *                     exchange), so that a test can check that the kernel returns with
+ *                     DSPARK_ETIMEOUT in the workspace status and DEVICE_TIMEOUT in the flags
  * The environment variables DSPARK_DRAFT_TC_MIN_B, DSPARK_DRAFT_PATH, DSPARK_DRAFT_PDL,
  * DSPARK_DRAFT_FUSED, DSPARK_VERIFY_CLUSTER, DSPARK_VERIFY_PERSISTENT, DSPARK_VERIFY_IMPL,
  * DSPARK_VERIFY_GROUPS and DSPARK_VERIFY_STREAM_CLUSTER set the initial values of the keys of the

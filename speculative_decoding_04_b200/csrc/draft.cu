@@ -41,6 +41,8 @@ struct DraftArgs {
   ChunkStat* cpart;    // [np][B]: per (main-pass partition, request) statistics
   __nv_bfloat16* gbuf; // [B][r]: W1 rows of the tokens just drafted (next step's B operand), or null
   uint32_t* status;
+  uint32_t spin_limit;   // polls before a bounded wait gives up
+  int barrier_extra;     // test-only: arrivals the first grid barrier expects beyond the grid
   int B, gamma, V, r, nchunk;
   float inv_T;
   int greedy;
@@ -301,12 +303,13 @@ __host__ __device__ inline TcLayout tc_layout(int r, int nb) {
 struct TcSync {
   volatile int* abort;
   uint32_t* status;
+  uint32_t limit;  // polls before a wait gives up
 };
 
 // Bounded mbarrier wait shared by all roles; after any timeout every later wait returns at once.
 __device__ __forceinline__ bool tc_wait(const TcSync& s, uint64_t* bar, uint32_t parity) {
   if (*s.abort) return false;
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  for (uint32_t i = 0; i < s.limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 1023u) == 1023u && *s.abort) return false;
   }
@@ -359,11 +362,12 @@ __device__ __forceinline__ float grp_max_f(float v, float* sh, const Grp& g) {
 // returned value, so the arrivals do not queue on each other) and waits, with acquire loads, for
 // it to reach nblocks times the barrier's number.  Bounded: gives up with the timeout status and
 // the abort flag.
-__device__ __forceinline__ bool grid_sync(uint32_t* count, uint32_t nblocks, uint32_t& epoch, const TcSync& sy) {
+__device__ __forceinline__ bool grid_sync(uint32_t* count, uint32_t nblocks, uint32_t& epoch, const TcSync& sy,
+                                          uint32_t extra = 0) {
   if (*sy.abort) return false;
-  const uint32_t target = ++epoch * nblocks;
+  const uint32_t target = ++epoch * nblocks + extra;
   asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+  for (uint32_t i = 0; i < sy.limit; ++i) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(count) : "memory");
     if ((int32_t)(v - target) >= 0) return true;
@@ -408,7 +412,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* g_full = c_done + 2;    // the B operand arrived by TMA from gbuf
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.misc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L.misc + 4);
-  const TcSync sy{s_abort, a.status};
+  const TcSync sy{s_abort, a.status, a.spin_limit};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x % n_bgroups;
@@ -512,6 +516,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t* gready = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(a.status) + 128);
     bool bad = false;
     int last_load[2] = {total > 0 ? 0 : -1, total > 1 ? 1 : -1};  // (warp 3) last tile loaded into each U stage
+    int g_issued = 0;  // (warp 1) TMA loads of the B operand issued
     for (int k = k0; k < k1; ++k) {
       const int gbase = (k - k0) * nt;
       // ---------------------------------------------------------------- B operand = W1[x_{k-1}] rows
@@ -532,10 +537,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *reinterpret_cast<uint4*>(sG + kb * (NB * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) = val;
         }
         fence_proxy_async_smem();
-      } else if (warp == 1 && lane == 0) {
+      } else if (warp == 1 && lane == 0 && !*s_abort) {  // after a timeout nothing waits for it
         fence_proxy_async_smem();  // earlier generic accesses to the G region come first
         mbar_arrive_expect_tx(g_full, (uint32_t)NB * a.r * 2u);
         for (int kb = 0; kb < a.r / 64; ++kb) tma_load_2d(sG + kb * (NB * 128), &tmG, kb * 64, b0, g_full);
+        ++g_issued;
       }
       named_bar(1, kTcThreads - 32);
       if (warp == 3) {
@@ -687,7 +693,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // ---------------------------------------------------------------- sample this step
         // every CTA's partition records and l_d stores of the step are in place
         named_bar(3, kTcThreads - 32);
-        if (warp == 1 && lane == 0) grid_sync(gcount, gridDim.x, epoch, sy);
+        if (warp == 1 && lane == 0) grid_sync(gcount, gridDim.x, epoch, sy, (uint32_t)a.barrier_extra);
         named_bar(3, kTcThreads - 32);
         // one warp per request, the requests spread over the grid (request blockIdx.x + m*gridDim.x
         // goes to warp 1 + m % 11 of this CTA): no block barrier inside a combine
@@ -706,7 +712,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               uint32_t v;
               asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(gready) : "memory");
               if ((int32_t)(v - target) >= 0) break;
-              if (i >= kSpinLimit || ((i & 1023u) == 1023u && *s_abort)) {
+              if (i >= a.spin_limit || ((i & 1023u) == 1023u && *s_abort)) {
                 if (!*s_abort) {
                   *s_abort = 1;
                   atomicOr(a.status, (uint32_t)DSPARK_ETIMEOUT);
@@ -731,6 +737,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (last_load[j] >= 0)
           for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(&u_full[j], (last_load[j] >> 1) & 1); ++t) {
           }
+    }
+    if (warp == 1 && lane == 0 && *s_abort && g_issued > 0) {
+      // a B-operand copy issued before the timeout that no wait saw land: let it land
+      for (uint32_t t = 0; t < kSpinLimit && !mbar_try_wait(g_full, (uint32_t)(g_issued - 1) & 1u); ++t) {
+      }
     }
     if (warp == 1 && lane == 0) tc_commit(mma_done);
   }
@@ -1212,6 +1223,8 @@ dspark_status launch_draft(const DraftCall& c) {
   a.u_draft = c.u_draft;
   a.flags = c.flags;
   a.status = reinterpret_cast<uint32_t*>(c.ws);
+  a.spin_limit = opt.debug_wait_limit > 0 ? (uint32_t)std::min<long>(opt.debug_wait_limit, kSpinLimit) : kSpinLimit;
+  a.barrier_extra = opt.debug_unreachable_barrier == 1 ? 1 : 0;
   a.B = c.B;
   a.gamma = c.gamma;
   a.V = c.V;

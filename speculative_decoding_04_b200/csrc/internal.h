@@ -19,13 +19,16 @@ struct Options {
   int draft_pdl = 1;             // chain the draft kernels with programmatic dependent launch
   int draft_fused = 1;           // tensor-core draft: all steps in one cooperative launch
   int verify_cluster = 0;        // 0 auto, else the cluster size (1, 2, 4, 8, 16)
-  int verify_persistent = 1;     // sampled verify / labels: persistent double-buffered clusters
+  int verify_persistent = 1;     // sampled verify / labels: persistent clusters with double-buffered rows (0: one cluster per row)
   int verify_impl = 0;           // verify with a workspace: 0 streaming kernels, 1 column-sliced, 2 per-row
   int verify_groups = 0;         // sliced verify: CTA groups (0: slices of about 16 KB per row)
   int verify_stream_cluster = 3; // CTAs per cluster of the streaming verify (1 to 8)
-  int verify_stream_lag = 1;     // rows between a row's first and second pass (1 to 3)
   int verify_stream_l2hint = 1;  // streaming verify: first-pass copies evict-last, second-pass evict-first
   int sm_count = 0;              // 0: query the device
+  // test-only: make the bounded device waits give up sooner and one of them unsatisfiable, so that
+  // a test can check that the kernels return with a timeout status (never on in normal use)
+  long debug_wait_limit = 0;      // draft: polls per wait; streaming verify: nanoseconds (0: defaults)
+  int debug_unreachable_barrier = 0;  // 1: the draft's first grid barrier; 2: the streaming verify's exchange
 };
 // A copy of the process-wide options, taken under their lock (dspark_set_option may run on
 // another thread).

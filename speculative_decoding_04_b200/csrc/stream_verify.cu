@@ -106,6 +106,8 @@ struct SvArgs {
   const float* u_acc;
   const float* u_res;
   int B, gamma, V, lt_rows, njobs, ntile, C, lag, l2hint;
+  uint64_t wait_ns;  // bounded waits give up after this long
+  int xbar_extra;    // test-only: arrivals the exchange barriers expect beyond the cluster
   float zscale;  // log2(e) / T (T > 0)
   int greedy, do_verify;
   float* c_star;
@@ -380,6 +382,7 @@ __device__ __forceinline__ void sv_cluster_sync_all() {
 struct SvSync {
   volatile int* abort;
   uint32_t* status;
+  uint64_t limit_ns;  // a wait gives up after this long
 };
 
 // Bounded wait: gives up (setting the abort flag and the status word) after kSvTimeoutNs, or
@@ -391,7 +394,7 @@ __device__ __forceinline__ bool sv_wait(const SvSync& s, uint64_t* bar, uint32_t
   while (true) {
     if (sv_try_wait_suspend(bar, parity, cluster_scope)) return true;
     if (*s.abort) return false;
-    if (sv_now_ns() - t0 > kSvTimeoutNs) break;
+    if (sv_now_ns() - t0 > s.limit_ns) break;
   }
   *s.abort = 1;
   atomicOr(s.status, (uint32_t)DSPARK_ETIMEOUT);
@@ -405,7 +408,7 @@ __device__ __forceinline__ bool sv_wait_count(const SvSync& s, volatile int* cnt
   const uint64_t t0 = sv_now_ns();
   while (*cnt < target) {
     if (*s.abort) return false;
-    if (sv_now_ns() - t0 > kSvTimeoutNs) {
+    if (sv_now_ns() - t0 > s.limit_ns) {
       *s.abort = 1;
       atomicOr(s.status, (uint32_t)DSPARK_ETIMEOUT);
       return false;
@@ -523,7 +526,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   __shared__ volatile int s_decided;  // rows of this cluster's sequence decided by this CTA
   __shared__ volatile int s_combined;  // passes whose warp partials the combiner has read
 
-  const SvSync sy{&s_abort, a.status};
+  const SvSync sy{&s_abort, a.status, a.wait_ns};
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSvStages; ++i) {
       mbar_init(&full[i], 1);
@@ -531,7 +534,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     }
     for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
     for (int i = 0; i < kSvJobSlots; ++i) {
-      mbar_init(&xbar[i], C);
+      mbar_init(&xbar[i], C + a.xbar_extra);
       mbar_init(&dbar[i], 1);
     }
     s_abort = 0;
@@ -1051,6 +1054,7 @@ __global__ void __launch_bounds__(128) verify_stream_finalize(SvArgs a) {
   const int G = a.gamma, R = G + 1;
   const SvRow* rr = a.rows + (size_t)b * R;
   const int Lb = a.L ? min(max(__ldg(a.L + b), 0), G) : G;
+  const bool timed_out = __ldcg(a.status) != 0u;
   if (a.c_star) {
     for (int k = lane; k < G; k += 32) {
       float cs;
@@ -1088,6 +1092,7 @@ __global__ void __launch_bounds__(128) verify_stream_finalize(SvArgs a) {
   } else {
     tok = sv_sample(a, b, n, n < Lb, rr[n].nm, fl);
   }
+  if (timed_out) fl |= DSPARK_FLAG_DEVICE_TIMEOUT;
   int32_t* y = a.y_out + (size_t)b * R;
   for (int j = lane; j < R; j += 32) y[j] = j < n ? a.x[(size_t)b * G + j] : (j == n ? tok : -1);
   if (lane == 0) {
@@ -1141,8 +1146,10 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.lt_rows = c.lt_rows;
   a.njobs = c.B * (c.gamma + 1);
   a.ntile = (c.V + kSvTile - 1) / kSvTile;
-  a.lag = std::min(std::max(opt.verify_stream_lag, 1), 3);
+  a.lag = 1;  // a row's second pass right after the next row's first (lags of 2 and 3 measured slower)
   a.l2hint = opt.verify_stream_l2hint;
+  a.wait_ns = opt.debug_wait_limit > 0 ? (uint64_t)std::min<long>(opt.debug_wait_limit, (long)kSvTimeoutNs) : kSvTimeoutNs;
+  a.xbar_extra = opt.debug_unreachable_barrier == 2 ? 1 : 0;
   a.greedy = c.T == 0.f ? 1 : 0;
   a.zscale = a.greedy ? 0.f : (float)(1.4426950408889634 / (double)c.T);
   a.do_verify = 1;

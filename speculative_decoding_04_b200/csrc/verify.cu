@@ -1181,7 +1181,7 @@ dspark_status launch_verify(const VerifyCall& c) {
   }
   a.bulk = (c.V % 4 == 0) && ((uintptr_t)c.lt % 16 == 0) && ((uintptr_t)c.ld % 16 == 0);
   if (!a.greedy && a.bulk && opt.verify_persistent) {
-    dspark_status st = launch_verify_persistent(a, cs, c.stream, opt.verify_persistent != 2);
+    dspark_status st = launch_verify_persistent(a, cs, c.stream, true);
     if (st == DSPARK_OK) st = launch_finalize(a, c.stream);
     if (st != DSPARK_ENOTIMPL) return st;  // else: no resident cluster fits; use the one-row-per-cluster kernel
   }

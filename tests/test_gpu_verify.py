@@ -171,16 +171,14 @@ def test_stream_vocabulary_beyond_per_row_kernels(T):
     assert e.value.status == D.ENOTIMPL
 
 
-@pytest.mark.parametrize("lag", [1, 2, 3])
 @pytest.mark.parametrize("cluster", [2, 8])
 @pytest.mark.parametrize("T", [1.0, 0.0])
-def test_stream_lag_between_passes(lag, cluster, T):
-    # the second pass of a row runs `lag` rows after its first pass; scheduled rows are skipped
+def test_stream_scheduled_rows_with_and_without_labels(cluster, T):
+    # rows past L_b + 1 skipped when no labels are asked for; all rows read with labels
     D.set_option("verify_impl", 0)
     D.set_option("verify_stream_cluster", cluster)
-    D.set_option("verify_stream_lag", lag)
     B, G, V = 24, 5, 20000
-    ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=300 + lag + cluster)
+    ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=300 + cluster)
     L = (np.arange(B) * 5 % (G + 1)).astype(np.int32)
     for want_c in (True, False):
         n, y, c, fl = run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=want_c)
