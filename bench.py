@@ -111,8 +111,10 @@ def verify_bytes(wl, L=None, labels=True):
     return int((2 * L + 1).sum()) * V * 4
 
 
-def config_of(wl, n, labels):
-    return {"workload": f"{wl.name}: B={wl.B} requests, gamma={wl.gamma}, V={wl.V}, r={wl.r}, T={wl.T}, "
+def config_of(wl, n, labels, layout="position"):
+    return {"layout": ("position-major [gamma, B, V]" if layout == "position" else "request-major [B, gamma, V]")
+                      + " draft logits U and ld",
+            "workload": f"{wl.name}: B={wl.B} requests, gamma={wl.gamma}, V={wl.V}, r={wl.r}, T={wl.T}, "
                         f"{wl.w_dtype} W1/W2, fp32 {'log-Zipf+Gaussian' if wl.logits == 'logzipf' else 'Gaussian'} "
                         "logits",
             "B_per_gpu": wl.B, "gamma": wl.gamma, "V": wl.V, "r": wl.r, "T": wl.T,
@@ -305,6 +307,9 @@ def main():
                     help="TV labels in the verify call (auto: on, except on scheduled_step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle timing (after the GPU timing)")
     ap.add_argument("--draft-crossover", action="store_true", help="print draft times of both main-pass paths over B")
+    ap.add_argument("--layout", choices=["position", "request"], default="position",
+                    help="layout of the draft logits U and of ld: position-major [gamma, B, V] (default) or "
+                         "request-major [B, gamma, V]")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -346,15 +351,18 @@ def main():
     host_logit_bytes = (B * G * V + B * (G + 1) * V) * 4
     if wl.name.startswith("sweep_B"):
         dv["U"], dv["lt"] = inputs.device_logits(wr, dev)          # drawn on the device (up to 26 GB)
+        if args.layout == "request":
+            dv["U"] = dv["U"].transpose(0, 1).contiguous()
     else:
         U, lt = inputs.logits(wr)
-        dv["U"] = torch.from_numpy(np.ascontiguousarray(U.transpose(1, 0, 2))).to(dev)  # position-major
+        Uh = U.transpose(1, 0, 2) if args.layout == "position" else U
+        dv["U"] = torch.from_numpy(np.ascontiguousarray(Uh)).to(dev)
         dv["lt"] = torch.from_numpy(lt).to(dev)
-        del U, lt
+        del U, lt, Uh
     sps_h = inputs.sps_table(wr) if uses_schedule_table(wl) else np.ones(B * G + 1)
     sps = torch.from_numpy(sps_h).to(dev)
     x = torch.empty((B, G), dtype=torch.int32, device=dev)
-    ld = torch.empty((G, B, V), dtype=torch.float32, device=dev)
+    ld = torch.empty(tuple(dv["U"].shape), dtype=torch.float32, device=dev)
     fl = torch.zeros(B, dtype=torch.int32, device=dev)
     L = torch.empty(B, dtype=torch.int32, device=dev)
     theta = torch.empty(1, dtype=torch.float64, device=dev)
@@ -371,14 +379,14 @@ def main():
     n_launch = (1 if tc else 2 * G) + 1 + 2
 
     def draft(src):
-        D.markov_draft(src["U"], W1, W2, src["x0"], src["u_draft"], wl.T, x_out=x, ld_out=ld, flags=fl, ws=ws_d,
-                       stream=stream)
+        D.markov_draft(src["U"], W1, W2, src["x0"], src["u_draft"], wl.T, layout=args.layout, x_out=x, ld_out=ld,
+                       flags=fl, ws=ws_d, stream=stream)
 
     def schedule_and_verify(src):
         D.prefix_schedule(src["c"], sps, B * G, D.SCHED_ARGMAX, L_out=L, theta_out=theta, flags=fl, want_a=False,
                           stream=stream)
-        D.verify(ld, src["lt"], x, L, src["u_acc"], src["u_res"], wl.T, n_acc=n_acc, y_out=y, c_star=c_star,
-                 flags=fl, ws=ws_v, stream=stream)
+        D.verify(ld, src["lt"], x, L, src["u_acc"], src["u_res"], wl.T, ld_layout=args.layout, n_acc=n_acc, y_out=y,
+                 c_star=c_star, flags=fl, ws=ws_v, stream=stream)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -424,8 +432,8 @@ def main():
             flush.fill_(float(i))
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            D.verify(ld, dv["lt"], x, L, dv["u_acc"], dv["u_res"], wl.T, n_acc=n_acc, y_out=y, c_star=c_star,
-                     flags=fl, ws=ws_v, stream=stream)
+            D.verify(ld, dv["lt"], x, L, dv["u_acc"], dv["u_res"], wl.T, ld_layout=args.layout, n_acc=n_acc, y_out=y,
+                     c_star=c_star, flags=fl, ws=ws_v, stream=stream)
             e1.record(stream)
             vt.append((e0, e1))
         barrier()
@@ -495,7 +503,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": f"synthetic (seeded log-Zipf + Gaussian logits, "
                                                          f"{wl.w_dtype} weights)",
-            "config": config_of(wl, world, labels),
+            "config": config_of(wl, world, labels, args.layout),
             "verified_tokens_per_s": accepted_all / (args.steps * t_step),
             "tokens_per_request_per_round": tau,
             "latency_per_token_us": (t_draft + t_verify) / tau * 1e6,

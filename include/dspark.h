@@ -51,6 +51,13 @@ typedef enum {
 /* weight dtypes */
 enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 };
 
+/* layouts of the draft logits U and l_d (rows of V fp32 values):
+ *   DSPARK_POSITION_MAJOR  [gamma, B, V]: step k of the draft reads and writes one contiguous
+ *                          block of B rows (the fast layout: see dspark_markov_draft)
+ *   DSPARK_REQUEST_MAJOR   [B, gamma, V]: as a backbone that emits all positions of a request
+ *                          together writes them */
+enum { DSPARK_POSITION_MAJOR = 0, DSPARK_REQUEST_MAJOR = 1 };
+
 /* scheduler modes */
 enum { DSPARK_SCHED_ARGMAX = 0, DSPARK_SCHED_EARLY_STOP = 1 };
 
@@ -131,23 +138,23 @@ int dspark_workspace_status(const void* ws, void* stream);
  *                  z = l_d[k,b,:] * (1/T)              (T > 0)
  *     x_k        = argmax_v l_d[k,b,v], lowest index    (T == 0)
  *
- * U        [gamma, B, V] fp32   base logits of the parallel stage, position-major: step k
- *          reads and writes one position of every request, and keeping those B rows in
- *          one contiguous block (rather than B rows gamma*V apart) nearly halves the
- *          time of a step at B = 64, gamma = 16, V = 151936.
+ * U        fp32 base logits of the parallel stage, [gamma, B, V] (layout DSPARK_POSITION_MAJOR)
+ *          or [B, gamma, V] (DSPARK_REQUEST_MAJOR).  Step k reads and writes one position of
+ *          every request; position-major keeps those B rows in one contiguous block.
+ * layout   DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR, for U and ld_out alike.
  * W1       [V, r]  and  W2 [r, V]   Markov-head factors, dtype w_dtype
  *          (DSPARK_BF16 or DSPARK_F32), fp32 accumulation.
  * x0       [B] int32    last committed token of each request (must be in [0, V)).
  * u_draft  [B, gamma] fp32 uniforms in [0, 1) (ignored when T == 0).
  * x_out    [B, gamma] int32   drafted tokens.
- * ld_out   [gamma, B, V] fp32 raw draft logits l_d (U + bias), kept for verify.
+ * ld_out   raw draft logits l_d (U + bias) in the layout of U, kept for verify.
  * flags    [B] uint32   OR'ed with DRAFT_NEAR_TIE / NONFINITE / TOKEN_RANGE.
  * ws       workspace of at least dspark_workspace_size(DSPARK_WS_DRAFT, B, gamma, V, r) bytes.
  * Limits: 1 <= gamma <= 64, B >= 1, V >= 2, r >= 1, T >= 0.
  * -------------------------------------------------------------------------- */
 int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dtype,
                         const int32_t* x0, const float* u_draft,
-                        int B, int gamma, int V, int r, float T,
+                        int B, int gamma, int V, int r, float T, int layout,
                         int32_t* x_out, float* ld_out, uint32_t* flags,
                         void* ws, size_t ws_bytes, void* stream);
 
@@ -167,7 +174,9 @@ int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dt
  *     n == L: y_L ~ p_t,L (the bonus row)       (inverse CDF with u_res[b])
  *     T == 0: accept iff x_k == argmax l_t,k; the resampled/bonus token is argmax l_t,n.
  *
- * ld     [gamma, B, V] fp32 draft logits, position-major (dspark_markov_draft's ld_out).
+ * ld     fp32 draft logits, [gamma, B, V] or [B, gamma, V] as ld_layout says (dspark_markov_draft's
+ *        ld_out).
+ * ld_layout  DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR.
  * lt     [B, gamma+1, V] fp32 target logits (row gamma = bonus position).
  * x      [B, gamma] int32 drafted tokens.
  * L      [B] int32 verify lengths in [0, gamma] (e.g. from dspark_prefix_schedule), or NULL.
@@ -183,7 +192,7 @@ int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dt
  * -------------------------------------------------------------------------- */
 int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int32_t* L,
                   const float* u_acc, const float* u_res,
-                  int B, int gamma, int V, float T,
+                  int B, int gamma, int V, float T, int ld_layout,
                   int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags,
                   void* ws, size_t ws_bytes, void* stream);
 
@@ -209,7 +218,7 @@ int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int3
  * -------------------------------------------------------------------------- */
 int dspark_verify_noalloc(const float* ld, const float* lt, const int32_t* x, const int32_t* L,
                           const float* u_acc, const float* u_res,
-                          int B, int gamma, int V, float T,
+                          int B, int gamma, int V, float T, int ld_layout,
                           int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags, void* stream);
 
 /* --------------------------------------------------------------------------
@@ -220,14 +229,14 @@ int dspark_verify_noalloc(const float* ld, const float* lt, const int32_t* x, co
  * obtained from the total-variation distance.  For every b and k = 0..gamma-1.
  * T == 0: c* = 1 if the argmaxes agree, else 0.
  *
- * ld      [gamma, B, V] fp32, position-major as in dspark_verify.
+ * ld      fp32 draft logits in the layout ld_layout names, as in dspark_verify.
  * lt      [B, lt_rows, V] fp32, lt_rows = gamma or gamma+1 (row stride of lt);
  *         only the first gamma rows of each request are read.
  * c_star  [B, gamma] fp32.
  * No workspace.
  * -------------------------------------------------------------------------- */
 int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, int lt_rows,
-                     float T, float* c_star, void* stream);
+                     float T, int ld_layout, float* c_star, void* stream);
 
 /* --------------------------------------------------------------------------
  * dspark_prefix_schedule -- prefix survival + greedy hardware-aware prefix scheduler.

@@ -151,7 +151,7 @@ int dspark_workspace_status(const void* ws, void* stream) {
 }
 
 int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dtype, const int32_t* x0,
-                        const float* u_draft, int B, int gamma, int V, int r, float T, int32_t* x_out,
+                        const float* u_draft, int B, int gamma, int V, int r, float T, int layout, int32_t* x_out,
                         float* ld_out, uint32_t* flags, void* ws, size_t ws_bytes, void* stream) {
   if (!U || !W1 || !W2 || !x0 || !x_out || !ld_out || !flags || !ws) return einval("dspark_markov_draft: null pointer");
   if (T != 0.f && !u_draft) return einval("dspark_markov_draft: u_draft is required when T > 0");
@@ -159,37 +159,43 @@ int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dt
   if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_markov_draft: gamma must be in [1, 64]");
   if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_markov_draft: T must be finite and >= 0");
   if (w_dtype != DSPARK_BF16 && w_dtype != DSPARK_F32) return einval("dspark_markov_draft: w_dtype must be DSPARK_BF16 or DSPARK_F32");
+  if (layout != DSPARK_POSITION_MAJOR && layout != DSPARK_REQUEST_MAJOR)
+    return einval("dspark_markov_draft: layout must be DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR");
   if ((long long)B * gamma * V >= (1ll << 40)) return einval("dspark_markov_draft: tensor too large");
   if (ws_bytes < draft_workspace_bytes(B, gamma, V, r)) return einval("dspark_markov_draft: workspace too small");
   if ((uintptr_t)ws % 256) return einval("dspark_markov_draft: workspace must be 256-byte aligned");
-  DraftCall c{U, W1, W2, w_dtype, x0, u_draft, B, gamma, V, r, T, x_out, ld_out, flags, ws, ws_bytes,
+  DraftCall c{U, W1, W2, w_dtype, x0, u_draft, B, gamma, V, r, T, layout, x_out, ld_out, flags, ws, ws_bytes,
               (cudaStream_t)stream};
   return launch_draft(c);
 }
 
 int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int32_t* L, const float* u_acc,
-                  const float* u_res, int B, int gamma, int V, float T, int32_t* n_acc, int32_t* y_out,
+                  const float* u_res, int B, int gamma, int V, float T, int ld_layout, int32_t* n_acc, int32_t* y_out,
                   float* c_star, uint32_t* flags, void* ws, size_t ws_bytes, void* stream) {
   if (!ld || !lt || !x || !n_acc || !y_out || !flags || !ws) return einval("dspark_verify: null pointer");
   if (T != 0.f && (!u_acc || !u_res)) return einval("dspark_verify: u_acc and u_res are required when T > 0");
   if (B <= 0 || V < 2) return einval("dspark_verify: B must be >= 1 and V >= 2");
   if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_verify: gamma must be in [1, 64]");
   if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_verify: T must be finite and >= 0");
+  if (ld_layout != DSPARK_POSITION_MAJOR && ld_layout != DSPARK_REQUEST_MAJOR)
+    return einval("dspark_verify: ld_layout must be DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR");
   if (ws_bytes < verify_workspace_bytes(B, gamma, V)) return einval("dspark_verify: workspace too small");
   if ((uintptr_t)ws % 256) return einval("dspark_verify: workspace must be 256-byte aligned");
-  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, 1, 0, n_acc, y_out, c_star, flags, ws, ws_bytes,
+  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, ld_layout, 1, 0, n_acc, y_out, c_star, flags, ws, ws_bytes,
                (cudaStream_t)stream};
   return launch_verify(c);
 }
 
-int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, int lt_rows, float T, float* c_star,
-                     void* stream) {
+int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, int lt_rows, float T, int ld_layout,
+                     float* c_star, void* stream) {
   if (!ld || !lt || !c_star) return einval("dspark_tv_labels: null pointer");
   if (B <= 0 || V < 2) return einval("dspark_tv_labels: B must be >= 1 and V >= 2");
   if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_tv_labels: gamma must be in [1, 64]");
   if (lt_rows != gamma && lt_rows != gamma + 1) return einval("dspark_tv_labels: lt_rows must be gamma or gamma+1");
+  if (ld_layout != DSPARK_POSITION_MAJOR && ld_layout != DSPARK_REQUEST_MAJOR)
+    return einval("dspark_tv_labels: ld_layout must be DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR");
   if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_tv_labels: T must be finite and >= 0");
-  VerifyCall c{ld, lt, nullptr, nullptr, nullptr, nullptr, B, gamma, V, lt_rows, T, 0, 0, nullptr, nullptr, c_star,
+  VerifyCall c{ld, lt, nullptr, nullptr, nullptr, nullptr, B, gamma, V, lt_rows, T, ld_layout, 0, 0, nullptr, nullptr, c_star,
                nullptr, nullptr, 0, (cudaStream_t)stream};
   return launch_verify(c);
 }

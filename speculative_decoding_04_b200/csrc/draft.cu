@@ -41,6 +41,8 @@ struct DraftArgs {
   ChunkStat* cpart;    // [np][B]: per (main-pass partition, request) statistics
   __nv_bfloat16* gbuf; // [B][r]: W1 rows of the tokens just drafted (next step's B operand), or null
   uint32_t* status;
+  size_t sk, sb;         // element strides of the U / l_d row of position k and request b
+  int rm;                // 1: request-major U / l_d ([B][gamma][V]; tensor maps {V, gamma, B})
   uint32_t spin_limit;   // polls before a bounded wait gives up
   int barrier_extra;     // test-only: arrivals the first grid barrier expects beyond the grid
   int B, gamma, V, r, nchunk;
@@ -231,7 +233,7 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
       bias0 += red[(w * BG + bb) * 256 + c];
       bias1 += red[(w * BG + bb) * 256 + c + 1];
     }
-    const size_t row = ((size_t)k * a.B + b) * V;  // position-major [gamma][B][V]
+    const size_t row = (size_t)k * a.sk + (size_t)b * a.sb;
     float l0 = 0.f, l1 = 0.f;
     if (val0) {
       l0 = a.U[row + v] + bias0;
@@ -477,7 +479,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto load_u = [&](int gi) {
     const int j = gi & 1, ku = k0 + gi / nt, iu = gi % nt;
     mbar_arrive_expect_tx(&u_full[j], kUStage * 4u);
-    tma_load_3d_hint(sU + j * kUStage, &tmU, tile_col(iu), b0, ku, &u_full[j], l2_policy_evict_first());
+    tma_load_3d_hint(sU + j * kUStage, &tmU, tile_col(iu), a.rm ? ku : b0, a.rm ? b0 : ku, &u_full[j],
+                     l2_policy_evict_first());
   };
   if (warp == 3 && lane == 0)
     for (int gi = 0; gi < 2 && gi < total; ++gi) load_u(gi);
@@ -553,7 +556,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < nt; ++i) {
             const int gi = gbase + i, j = gi & 1;
             if (!tc_wait(sy, &c_done[j], (gi >> 1) & 1)) break;
-            tma_store_3d_hint(&tmLd, sU + j * kUStage, tile_col(i), b0, k, l2_policy_evict_first());
+            tma_store_3d_hint(&tmLd, sU + j * kUStage, tile_col(i), a.rm ? k : b0, a.rm ? b0 : k,
+                              l2_policy_evict_first());
             bulk_commit();
             if (gi + 2 < total) {
               if (!tc_wait(sy, &u_empty[j], (gi >> 1) & 1)) break;
@@ -875,7 +879,7 @@ __device__ void combine_group(const DraftArgs& a, int k, int b, const Grp& g, do
       const int t0 = (int)((long long)p * a.ntiles / np), t1 = (int)((long long)(p + 1) * a.ntiles / np);
       const int tw = a.tile_chunks * kChunk;
       const int v0 = t0 * tw, n = min(t1 * tw, a.V) - v0;
-      const float* row = a.ld + ((size_t)k * a.B + b) * a.V + v0;
+      const float* row = a.ld + (size_t)k * a.sk + (size_t)b * a.sb + v0;
       const float inv_T = a.inv_T;
       auto w2 = [&](int j) -> double {
         const float z = __fmul_rn(__ldcg(row + j), inv_T);
@@ -1026,7 +1030,7 @@ __device__ void combine_warp(const DraftArgs& a, int k, int b, uint32_t* gready)
       const int t0 = (int)((long long)p * a.ntiles / np), t1 = (int)((long long)(p + 1) * a.ntiles / np);
       const int tw = a.tile_chunks * kChunk;
       const int v0 = t0 * tw, n = min(t1 * tw, a.V) - v0;
-      const float4* row4 = reinterpret_cast<const float4*>(a.ld + ((size_t)k * a.B + b) * a.V + v0);  // 16-byte aligned
+      const float4* row4 = reinterpret_cast<const float4*>(a.ld + (size_t)k * a.sk + (size_t)b * a.sb + v0);  // 16-byte aligned
       const float inv_T = a.inv_T;
       const int nq4 = (n + 3) / 4;
       double base = lo1;  // weight before the current chunk
@@ -1090,7 +1094,7 @@ __device__ void combine_warp(const DraftArgs& a, int k, int b, uint32_t* gready)
         for (int c = 3; c >= 0 && pk < 0; --c) {
           const int e = lastq * 4 + c;
           if (e < n) {
-            const float z = __fmul_rn(__ldcg(a.ld + ((size_t)k * a.B + b) * a.V + v0 + e), inv_T);
+            const float z = __fmul_rn(__ldcg(a.ld + (size_t)k * a.sk + (size_t)b * a.sb + v0 + e), inv_T);
             if (z != -INFINITY && ex_shift(z, M) > 0.f) pk = e;
           }
         }
@@ -1223,6 +1227,8 @@ dspark_status launch_draft(const DraftCall& c) {
   a.u_draft = c.u_draft;
   a.flags = c.flags;
   a.status = reinterpret_cast<uint32_t*>(c.ws);
+  ld_strides(c.layout, c.B, c.gamma, c.V, a.sk, a.sb);
+  a.rm = c.layout == DSPARK_REQUEST_MAJOR ? 1 : 0;
   a.spin_limit = opt.debug_wait_limit > 0 ? (uint32_t)std::min<long>(opt.debug_wait_limit, kSpinLimit) : kSpinLimit;
   a.barrier_extra = opt.debug_unreachable_barrier == 1 ? 1 : 0;
   a.B = c.B;
@@ -1279,12 +1285,21 @@ dspark_status launch_draft(const DraftCall& c) {
       set_error("cuTensorMapEncodeTiled failed for W2");
       return DSPARK_ECUDA;
     }
-    // U and l_d are position-major [gamma][B][V]: a box is one 128-column tile of the nb
-    // requests of a group at one position (32 KB at nb = 64: large copies keep the copy
-    // engine near full bandwidth, where 4 KB copies were measured to stream at under half)
+    // A box is one 128-column tile of the nb requests of a group at one position (32 KB at
+    // nb = 64: large copies keep the copy engine near full bandwidth, where 4 KB copies were
+    // measured to stream at under half); position-major U / l_d [gamma][B][V]: dims {V, B, gamma}
+    // request-major U / l_d: dims {V, gamma, B}, box {128, 1, nb} (the same [nb][128] layout in
+    // shared memory; coordinates (column, k, b0))
     uint64_t udims[3] = {(uint64_t)c.V, (uint64_t)c.B, (uint64_t)c.gamma};
     uint64_t ustrides[2] = {(uint64_t)c.V * 4, (uint64_t)c.B * c.V * 4};
     uint32_t ubox[3] = {(uint32_t)kTcTile, (uint32_t)nb, 1};
+    if (a.rm) {
+      udims[1] = (uint64_t)c.gamma;
+      udims[2] = (uint64_t)c.B;
+      ustrides[1] = (uint64_t)c.gamma * c.V * 4;
+      ubox[1] = 1;
+      ubox[2] = (uint32_t)nb;
+    }
     if (!make_map(&mU, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(c.U), udims, ustrides, ubox, false)) {
       set_error("cuTensorMapEncodeTiled failed for U");
       return DSPARK_ECUDA;

@@ -51,6 +51,7 @@ struct DraftCall {
   const float* u_draft;
   int B, gamma, V, r;
   float T;
+  int layout;  // of U and ld_out: DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR
   int32_t* x_out;
   float* ld_out;
   uint32_t* flags;
@@ -68,6 +69,7 @@ struct VerifyCall {
   const float* u_res;
   int B, gamma, V, lt_rows;
   float T;
+  int ld_layout;     // DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR
   int do_verify;
   int per_row_only;  // 1: the per-row cluster kernels only (their workspace layout), never the streaming ones
   int32_t* n_acc;
@@ -107,5 +109,16 @@ constexpr int kMaxScheduleItems = 16384;
 constexpr size_t kWsHeader = 256;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Element strides of the l_d (or U) row of position k and request b: row = k * sk + b * sb.
+inline void ld_strides(int layout, int B, int gamma, int V, size_t& sk, size_t& sb) {
+  if (layout == DSPARK_REQUEST_MAJOR) {
+    sk = (size_t)V;
+    sb = (size_t)gamma * V;
+  } else {
+    sk = (size_t)B * V;
+    sb = (size_t)V;
+  }
+}
 
 }  // namespace dspark

@@ -113,6 +113,7 @@ struct VsArgs {
   const float* u_res;
   int B, gamma, V, lt_rows;
   int G, P, NS, wmax, nq, njobs;
+  size_t ld_sk, ld_sb;  // element strides of the l_d row of position k and request b
   float zc;  // log2(e) / T (T > 0)
   int greedy;
   float* c_star;
@@ -614,7 +615,7 @@ __global__ void __launch_bounds__(kVsThreads, 1) verify_sliced(VsArgs a) {
         float* st = ring + (size_t)s * 2 * a.wmax;
         mbar_expect_tx(&full[s], bytes ? (J.d ? 2u : 1u) * bytes : 0u);
         if (bytes) {
-          if (J.d) bulk_g2s(st, a.ld + ((size_t)J.k * a.B + J.b) * a.V + (size_t)q0 * 4, bytes, &full[s]);
+          if (J.d) bulk_g2s(st, a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb + (size_t)q0 * 4, bytes, &full[s]);
           bulk_g2s(st + a.wmax, a.lt + ((size_t)J.b * a.lt_rows + J.k) * a.V + (size_t)q0 * 4, bytes, &full[s]);
         }
         mbar_arrive(&full[s]);
@@ -812,7 +813,7 @@ __global__ void __launch_bounds__(kVsThreads, 1) verify_sliced(VsArgs a) {
       const float u_acc = (J.verify && !GREEDY) ? __ldg(a.u_acc + (size_t)J.b * a.gamma + J.k) : 0.f;
       float ldx = 0.f, ltx = 0.f;
       if (!GREEDY && J.verify && (unsigned)xk < (unsigned)a.V) {
-        ldx = __ldg(a.ld + ((size_t)J.k * a.B + J.b) * a.V + xk);
+        ldx = __ldg(a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb + xk);
         ltx = __ldg(a.lt + ((size_t)J.b * a.lt_rows + J.k) * a.V + xk);
       }
       VsRec x;
@@ -935,7 +936,7 @@ __device__ int vs_sample(const VsArgs& a, int b, int k, bool resid, const VsRow&
   const int r = c / kVsTiles, w = c - r * kVsTiles;
   const int q0 = vs_q0(r, a.nq, P), ns = vs_q0(r + 1, a.nq, P) - q0;
   const int v0 = (q0 + vs_t0(w, ns)) * 4, cnt = (vs_t0(w + 1, ns) - vs_t0(w, ns)) * 4;
-  const float* rowd = a.ld + ((size_t)k * a.B + b) * a.V + v0;
+  const float* rowd = a.ld + (size_t)k * a.ld_sk + (size_t)b * a.ld_sb + v0;
   const float* rowt = a.lt + ((size_t)b * a.lt_rows + k) * a.V + v0;
   float md = -INFINITY, mt = -INFINITY;
   for (int e = lane; e < cnt; e += 32) {
@@ -1148,6 +1149,7 @@ dspark_status launch_verify_sliced(const VerifyCall& c) {
   a.gamma = c.gamma;
   a.V = c.V;
   a.lt_rows = c.lt_rows;
+  ld_strides(c.ld_layout, c.B, c.gamma, c.V, a.ld_sk, a.ld_sb);
   a.G = geo.G;
   a.P = geo.P;
   a.NS = NS;

@@ -106,6 +106,7 @@ struct SvArgs {
   const float* u_acc;
   const float* u_res;
   int B, gamma, V, lt_rows, njobs, ntile, C, lag, l2hint;
+  size_t ld_sk, ld_sb;  // element strides of the l_d row of position k and request b
   uint64_t wait_ns;  // bounded waits give up after this long
   int xbar_extra;    // test-only: arrivals the exchange barriers expect beyond the cluster
   float zscale;  // log2(e) / T (T > 0)
@@ -577,7 +578,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           const int c0 = (tb + lo - pbase) * kSvTile, c1 = min((tb + hi - pbase) * kSvTile, a.V);
           const uint32_t bytes = (uint32_t)(c1 - c0) * 4u;
           const bool with_d = ph.second || ph.J.d;
-          const float* rd = a.ld + ((size_t)ph.J.k * a.B + ph.J.b) * a.V;
+          const float* rd = a.ld + (size_t)ph.J.k * a.ld_sk + (size_t)ph.J.b * a.ld_sb;
           const float* rt = a.lt + ((size_t)ph.J.b * a.lt_rows + ph.J.k) * a.V;
           mbar_expect_tx(&full[s], with_d ? 2 * bytes : bytes);
           if (a.l2hint) {
@@ -654,7 +655,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       const float u_acc = (J.verify && !GREEDY) ? __ldg(a.u_acc + (size_t)J.b * a.gamma + J.k) : 0.f;
       float ldx = 0.f, ltx = 0.f;
       if (!GREEDY && J.verify && (unsigned)xk < (unsigned)a.V) {
-        ldx = __ldg(a.ld + ((size_t)J.k * a.B + J.b) * a.V + xk);
+        ldx = __ldg(a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb + xk);
         ltx = __ldg(a.lt + ((size_t)J.b * a.lt_rows + J.k) * a.V + xk);
       }
       ok = sv_wait(sy, &xbar[js], (i / kSvJobSlots) & 1, true);
@@ -927,7 +928,7 @@ __device__ int sv_sample(const SvArgs& a, int b, int k, bool resid, const SvNorm
   const bool has_trec = !resid;  // the bonus row
   const SvP2 k2 = sv_p2_consts(nm);
   const float zc = a.zscale;
-  const float* rowd = a.ld + ((size_t)k * a.B + b) * a.V;
+  const float* rowd = a.ld + (size_t)k * a.ld_sk + (size_t)b * a.ld_sb;
   const float* rowt = a.lt + ((size_t)b * a.lt_rows + k) * a.V;
   const int per = (a.ntile + 31) / 32;
   const int t_lo = min(lane * per, a.ntile), t_hi = min(t_lo + per, a.ntile);
@@ -1144,6 +1145,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.gamma = c.gamma;
   a.V = c.V;
   a.lt_rows = c.lt_rows;
+  ld_strides(c.ld_layout, c.B, c.gamma, c.V, a.ld_sk, a.ld_sb);
   a.njobs = c.B * (c.gamma + 1);
   a.ntile = (c.V + kSvTile - 1) / kSvTile;
   a.lag = 1;  // a row's second pass right after the next row's first (lags of 2 and 3 measured slower)

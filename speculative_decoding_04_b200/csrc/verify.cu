@@ -40,6 +40,7 @@ struct VerifyArgs {
   const float* u_acc;
   const float* u_res;
   int B, gamma, V, lt_rows, rows_per_req;
+  size_t ld_sk, ld_sb;  // element strides of the l_d row of position k and request b
   float inv_T;
   int greedy;
   int do_verify;
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
 
   const int v_beg = rank * a.Vc;
   const int n = max(0, min(a.V, v_beg + a.Vc) - v_beg);
-  const size_t rowd = ((size_t)kk * a.B + b) * a.V + v_beg;  // l_d is [gamma][B][V]
+  const size_t rowd = (size_t)kk * a.ld_sk + (size_t)b * a.ld_sb + v_beg;
   const size_t rowt = ((size_t)b * a.lt_rows + kk) * a.V + v_beg;
   bool timed_out = false;
 
@@ -663,7 +664,7 @@ __global__ void __launch_bounds__(512, 1) verify_rows_pc(VerifyArgs a) {
     if (tid == 0) {
       float* sd = psm + (size_t)j * 2 * a.Vc;
       const uint32_t bytes = (uint32_t)n * 4u;
-      const size_t rowd = ((size_t)rn.kk * a.B + rn.b) * a.V + v_beg;
+      const size_t rowd = (size_t)rn.kk * a.ld_sk + (size_t)rn.b * a.ld_sb + v_beg;
       const size_t rowt = ((size_t)rn.b * a.lt_rows + rn.kk) * a.V + v_beg;
       mbar_arrive_expect_tx(&bar[j], rn.d ? 2u * bytes : bytes);
       if (rn.d) bulk_g2s(sd, a.ld + rowd, bytes, &bar[j]);
@@ -1149,6 +1150,7 @@ dspark_status launch_verify(const VerifyCall& c) {
   a.gamma = c.gamma;
   a.V = c.V;
   a.lt_rows = c.lt_rows;
+  ld_strides(c.ld_layout, c.B, c.gamma, c.V, a.ld_sk, a.ld_sb);
   a.rows_per_req = c.do_verify ? c.gamma + 1 : c.gamma;
   a.greedy = (c.T == 0.f) ? 1 : 0;
   a.inv_T = a.greedy ? 1.f : 1.f / c.T;
@@ -1299,7 +1301,8 @@ static dspark_status verify_scratch(void** ptr) {
 
 extern "C" int dspark_verify_noalloc(const float* ld, const float* lt, const int32_t* x, const int32_t* L,
                                      const float* u_acc, const float* u_res, int B, int gamma, int V, float T,
-                                     int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags, void* stream) {
+                                     int ld_layout, int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags,
+                                     void* stream) {
   using namespace dspark;
   auto einval = [](const char* msg) {
     set_error(msg);
@@ -1310,6 +1313,8 @@ extern "C" int dspark_verify_noalloc(const float* ld, const float* lt, const int
   if (B <= 0 || V < 2) return einval("dspark_verify_noalloc: B must be >= 1 and V >= 2");
   if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_verify_noalloc: gamma must be in [1, 64]");
   if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_verify_noalloc: T must be finite and >= 0");
+  if (ld_layout != DSPARK_POSITION_MAJOR && ld_layout != DSPARK_REQUEST_MAJOR)
+    return einval("dspark_verify_noalloc: ld_layout must be DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR");
   if (B > kNoAllocMaxB || (long long)B * (gamma + 1) > kNoAllocMaxRows)
     return einval("dspark_verify_noalloc: needs B <= 4096 and B*(gamma+1) <= 16384 (fixed scratch); use dspark_verify");
   if (verify_rows_workspace_bytes(B, gamma) > kNoAllocScratchBytes)  // holds within the limits above
@@ -1317,7 +1322,7 @@ extern "C" int dspark_verify_noalloc(const float* ld, const float* lt, const int
   void* ws = nullptr;
   const dspark_status st = verify_scratch(&ws);
   if (st != DSPARK_OK) return st;
-  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, 1, 1, n_acc, y_out, c_star, flags, ws,
+  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, ld_layout, 1, 1, n_acc, y_out, c_star, flags, ws,
                kNoAllocScratchBytes, (cudaStream_t)stream};
   return launch_verify(c);
 }

@@ -20,6 +20,8 @@ from .build import LIB_PATH, ROOT
 
 OK, EINVAL, ECUDA, ENOTIMPL, ETIMEOUT = 0, 1, 2, 3, 4
 F32, BF16 = 0, 1
+POSITION_MAJOR, REQUEST_MAJOR = 0, 1
+_LAYOUTS = {"position": POSITION_MAJOR, "request": REQUEST_MAJOR}
 SCHED_ARGMAX, SCHED_EARLY_STOP = 0, 1
 WS_DRAFT, WS_VERIFY, WS_SCHEDULE = 0, 1, 2
 
@@ -60,13 +62,14 @@ def _load() -> ctypes.CDLL:
     lib.dspark_workspace_status.restype = _i
     lib.dspark_workspace_status.argtypes = [_vp, _vp]
     lib.dspark_markov_draft.restype = _i
-    lib.dspark_markov_draft.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_markov_draft.argtypes = [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _vp, _sz,
+                                        _vp]
     lib.dspark_verify.restype = _i
-    lib.dspark_verify.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_verify.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.dspark_verify_noalloc.restype = _i
-    lib.dspark_verify_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _vp, _vp, _vp]
+    lib.dspark_verify_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, _vp, _vp, _vp, _vp]
     lib.dspark_tv_labels.restype = _i
-    lib.dspark_tv_labels.argtypes = [_vp, _vp, _i, _i, _i, _i, _f, _vp, _vp]
+    lib.dspark_tv_labels.argtypes = [_vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp]
     lib.dspark_prefix_schedule.restype = _i
     lib.dspark_prefix_schedule.argtypes = [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     return lib
@@ -135,13 +138,25 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _bgv(t: torch.Tensor, layout: str):
+    """(B, gamma, V) of a logit tensor in the given layout ("position": [gamma, B, V],
+    "request": [B, gamma, V])."""
+    if layout not in _LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(_LAYOUTS)}")
+    if t.dim() != 3:
+        raise ValueError("logits must be 3-D")
+    a, b, V = t.shape
+    return (b, a, V) if layout == "position" else (a, b, V)
+
+
 def markov_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, x0: torch.Tensor,
-                 u_draft: Optional[torch.Tensor], T: float, *, x_out=None, ld_out=None, flags=None, ws=None,
-                 stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+                 u_draft: Optional[torch.Tensor], T: float, *, layout: str = "position", x_out=None, ld_out=None,
+                 flags=None, ws=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Markov-head draft of gamma tokens per request.
 
-    U is position-major [gamma, B, V]; returns (x [B, gamma], l_d [gamma, B, V], flags [B])."""
-    G, B, V = U.shape
+    U is [gamma, B, V] (layout "position", the fast one) or [B, gamma, V] ("request"); returns
+    (x [B, gamma], l_d in the layout of U, flags [B])."""
+    B, G, V = _bgv(U, layout)
     r = W1.shape[1]
     _need(U, "U", torch.float32)
     if W1.dtype not in (torch.bfloat16, torch.float32) or W2.dtype != W1.dtype:
@@ -153,14 +168,15 @@ def markov_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, x0: torch.
         _need(u_draft, "u_draft", torch.float32, (B, G))
     dev = U.device
     x_out = torch.empty((B, G), dtype=torch.int32, device=dev) if x_out is None else x_out
-    ld_out = torch.empty((G, B, V), dtype=torch.float32, device=dev) if ld_out is None else ld_out
+    ld_out = torch.empty(U.shape, dtype=torch.float32, device=dev) if ld_out is None else ld_out
     flags = torch.zeros(B, dtype=torch.int32, device=dev) if flags is None else flags
     ws = workspace(WS_DRAFT, B, G, V, r, dev) if ws is None else ws
     _need(x_out, "x_out", torch.int32, (B, G))
-    _need(ld_out, "ld_out", torch.float32, (G, B, V))
+    _need(ld_out, "ld_out", torch.float32, tuple(U.shape))
     _need(flags, "flags", torch.int32, (B,))
     st = lib.dspark_markov_draft(_p(U), _p(W1), _p(W2), BF16 if W1.dtype == torch.bfloat16 else F32, _p(x0),
-                                 _p(u_draft), B, G, V, r, float(T), _p(x_out), _p(ld_out), _p(flags), _p(ws),
+                                 _p(u_draft), B, G, V, r, float(T), _LAYOUTS[layout], _p(x_out), _p(ld_out),
+                                 _p(flags), _p(ws),
                                  ws.numel(), _s(stream))
     _check("dspark_markov_draft", st)
     return x_out, ld_out, flags
@@ -168,10 +184,11 @@ def markov_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, x0: torch.
 
 def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torch.Tensor],
            u_acc: Optional[torch.Tensor], u_res: Optional[torch.Tensor], T: float, *, want_c_star: bool = False,
-           n_acc=None, y_out=None, c_star=None, flags=None, ws=None, stream=None):
-    """Rejection-sampling verification of l_d [gamma, B, V] (position-major) against l_t [B, gamma+1, V];
-    returns (n_acc [B], y [B, gamma+1], c_star [B, gamma] or None, flags [B])."""
-    G, B, V = ld.shape
+           ld_layout: str = "position", n_acc=None, y_out=None, c_star=None, flags=None, ws=None, stream=None):
+    """Rejection-sampling verification of l_d ([gamma, B, V], or [B, gamma, V] with ld_layout
+    "request") against l_t [B, gamma+1, V]; returns (n_acc [B], y [B, gamma+1], c_star [B, gamma]
+    or None, flags [B])."""
+    B, G, V = _bgv(ld, ld_layout)
     _need(ld, "ld", torch.float32)
     _need(lt, "lt", torch.float32, (B, G + 1, V))
     _need(x, "x", torch.int32, (B, G))
@@ -193,7 +210,8 @@ def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torc
     _need(flags, "flags", torch.int32, (B,))
     if c_star is not None:
         _need(c_star, "c_star", torch.float32, (B, G))
-    st = lib.dspark_verify(_p(ld), _p(lt), _p(x), _p(L), _p(u_acc), _p(u_res), B, G, V, float(T), _p(n_acc),
+    st = lib.dspark_verify(_p(ld), _p(lt), _p(x), _p(L), _p(u_acc), _p(u_res), B, G, V, float(T),
+                           _LAYOUTS[ld_layout], _p(n_acc),
                            _p(y_out), _p(c_star), _p(flags), _p(ws), ws.numel(), _s(stream))
     _check("dspark_verify", st)
     return n_acc, y_out, c_star, flags
@@ -201,10 +219,11 @@ def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torc
 
 def verify_noalloc(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torch.Tensor],
                    u_acc: Optional[torch.Tensor], u_res: Optional[torch.Tensor], T: float, *,
-                   want_c_star: bool = False, n_acc=None, y_out=None, c_star=None, flags=None, stream=None):
+                   want_c_star: bool = False, ld_layout: str = "position", n_acc=None, y_out=None, c_star=None,
+                   flags=None, stream=None):
     """verify() for callers that cannot provide device scratch: the library uses a fixed array of
     its own (B <= 4096, B*(gamma+1) <= 16384).  Outputs are allocated here only when not passed."""
-    G, B, V = ld.shape
+    B, G, V = _bgv(ld, ld_layout)
     _need(ld, "ld", torch.float32)
     _need(lt, "lt", torch.float32, (B, G + 1, V))
     _need(x, "x", torch.int32, (B, G))
@@ -216,24 +235,26 @@ def verify_noalloc(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optio
     if c_star is None and want_c_star:
         c_star = torch.empty((B, G), dtype=torch.float32, device=dev)
     flags = torch.zeros(B, dtype=torch.int32, device=dev) if flags is None else flags
-    st = lib.dspark_verify_noalloc(_p(ld), _p(lt), _p(x), _p(L), _p(u_acc), _p(u_res), B, G, V, float(T), _p(n_acc),
+    st = lib.dspark_verify_noalloc(_p(ld), _p(lt), _p(x), _p(L), _p(u_acc), _p(u_res), B, G, V, float(T),
+                                   _LAYOUTS[ld_layout], _p(n_acc),
                                    _p(y_out), _p(c_star), _p(flags), _s(stream))
     _check("dspark_verify_noalloc", st)
     return n_acc, y_out, c_star, flags
 
 
-def tv_labels(ld: torch.Tensor, lt: torch.Tensor, T: float, *, c_star=None, stream=None) -> torch.Tensor:
-    """c*_k = 1 - ½‖p_d,k - p_t,k‖₁ for every drafted position; l_d is [gamma, B, V] and l_t
-    [B, gamma or gamma+1, V]."""
-    G, B, V = ld.shape
+def tv_labels(ld: torch.Tensor, lt: torch.Tensor, T: float, *, ld_layout: str = "position", c_star=None,
+              stream=None) -> torch.Tensor:
+    """c*_k = 1 - ½‖p_d,k - p_t,k‖₁ for every drafted position; l_d is [gamma, B, V] (or
+    [B, gamma, V] with ld_layout "request") and l_t [B, gamma or gamma+1, V]."""
+    B, G, V = _bgv(ld, ld_layout)
     _need(ld, "ld", torch.float32)
     _need(lt, "lt", torch.float32)
     if lt.dim() != 3 or lt.shape[0] != B or lt.shape[2] != V or lt.shape[1] not in (G, G + 1):
         raise ValueError("lt must be [B, gamma or gamma+1, V]")
     c_star = torch.empty((B, G), dtype=torch.float32, device=ld.device) if c_star is None else c_star
     _need(c_star, "c_star", torch.float32, (B, G))
-    _check("dspark_tv_labels", lib.dspark_tv_labels(_p(ld), _p(lt), B, G, V, lt.shape[1], float(T), _p(c_star),
-                                                    _s(stream)))
+    _check("dspark_tv_labels", lib.dspark_tv_labels(_p(ld), _p(lt), B, G, V, lt.shape[1], float(T),
+                                                    _LAYOUTS[ld_layout], _p(c_star), _s(stream)))
     return c_star
 
 

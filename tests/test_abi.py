@@ -47,11 +47,13 @@ def test_workspace_sizes():
 
 
 def _draft(**kw):
-    a = dict(U=FAKE, W1=FAKE, W2=FAKE, w=D.BF16, x0=FAKE, u=FAKE, B=4, G=4, V=1024, r=16, T=1.0, x=FAKE, ld=FAKE,
-             flags=FAKE, ws=ctypes.c_void_p(4096 * 256), wsb=1 << 30, stream=None)
+    a = dict(U=FAKE, W1=FAKE, W2=FAKE, w=D.BF16, x0=FAKE, u=FAKE, B=4, G=4, V=1024, r=16, T=1.0,
+             layout=D.POSITION_MAJOR, x=FAKE, ld=FAKE, flags=FAKE, ws=ctypes.c_void_p(4096 * 256), wsb=1 << 30,
+             stream=None)
     a.update(kw)
     return D.lib.dspark_markov_draft(a["U"], a["W1"], a["W2"], a["w"], a["x0"], a["u"], a["B"], a["G"], a["V"],
-                                     a["r"], a["T"], a["x"], a["ld"], a["flags"], a["ws"], a["wsb"], a["stream"])
+                                     a["r"], a["T"], a["layout"], a["x"], a["ld"], a["flags"], a["ws"], a["wsb"],
+                                     a["stream"])
 
 
 @no_gpu
@@ -67,16 +69,18 @@ def test_draft_argument_checks():
     assert _draft(w=7) == D.EINVAL
     assert _draft(wsb=100) == D.EINVAL
     assert _draft(ws=ctypes.c_void_p(4096 * 256 + 16)) == D.EINVAL
+    assert _draft(layout=2) == D.EINVAL
+    assert "layout" in D.last_error()
     assert _draft(u=None) == D.EINVAL           # sampling needs uniforms
     assert "gamma" in D.last_error() or "u_draft" in D.last_error()
 
 
 def _verify(**kw):
-    a = dict(ld=FAKE, lt=FAKE, x=FAKE, L=None, ua=FAKE, ur=FAKE, B=4, G=4, V=1024, T=1.0, n=FAKE, y=FAKE, c=None,
-             flags=FAKE, ws=ctypes.c_void_p(4096 * 256), wsb=1 << 30, stream=None)
+    a = dict(ld=FAKE, lt=FAKE, x=FAKE, L=None, ua=FAKE, ur=FAKE, B=4, G=4, V=1024, T=1.0, layout=D.REQUEST_MAJOR,
+             n=FAKE, y=FAKE, c=None, flags=FAKE, ws=ctypes.c_void_p(4096 * 256), wsb=1 << 30, stream=None)
     a.update(kw)
     return D.lib.dspark_verify(a["ld"], a["lt"], a["x"], a["L"], a["ua"], a["ur"], a["B"], a["G"], a["V"], a["T"],
-                               a["n"], a["y"], a["c"], a["flags"], a["ws"], a["wsb"], a["stream"])
+                               a["layout"], a["n"], a["y"], a["c"], a["flags"], a["ws"], a["wsb"], a["stream"])
 
 
 @no_gpu
@@ -86,9 +90,11 @@ def test_verify_and_labels_argument_checks():
     assert _verify(T=-0.5) == D.EINVAL
     assert _verify(ua=None) == D.EINVAL
     assert _verify(wsb=8) == D.EINVAL
-    assert D.lib.dspark_tv_labels(FAKE, FAKE, 2, 4, 1024, 3, 1.0, FAKE, None) == D.EINVAL   # lt_rows
-    assert D.lib.dspark_tv_labels(None, FAKE, 2, 4, 1024, 4, 1.0, FAKE, None) == D.EINVAL
-    assert D.lib.dspark_tv_labels(FAKE, FAKE, 2, 4, 1, 4, 1.0, FAKE, None) == D.EINVAL
+    assert _verify(layout=-1) == D.EINVAL
+    assert D.lib.dspark_tv_labels(FAKE, FAKE, 2, 4, 1024, 3, 1.0, 0, FAKE, None) == D.EINVAL   # lt_rows
+    assert D.lib.dspark_tv_labels(None, FAKE, 2, 4, 1024, 4, 1.0, 0, FAKE, None) == D.EINVAL
+    assert D.lib.dspark_tv_labels(FAKE, FAKE, 2, 4, 1, 4, 1.0, 0, FAKE, None) == D.EINVAL
+    assert D.lib.dspark_tv_labels(FAKE, FAKE, 2, 4, 1024, 4, 1.0, 3, FAKE, None) == D.EINVAL   # layout
 
 
 @no_gpu
