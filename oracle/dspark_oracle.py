@@ -28,6 +28,10 @@ What each function follows:
                   Θ = τ·SPS(B)); P1 §"硬件感知与置信度自适应调度机制" (sort all
                   candidate tokens by survival, add them one at a time, evaluate
                   expected throughput, stop when it falls; global search on the GPU).
+  * prefix_schedule_t2 -- P1 §"硬件感知与置信度自适应调度机制", last paragraph (the
+                  truncation of step t decided from step t-2's confidence history);
+                  P3 §Confidence-Scheduled Verification, production notes ("asynchronous":
+                  confidences two steps back predict the batch capacity K).
 
 Readings where the pages leave a step open:
   * temperature: p ∝ exp(ℓ/T) on both draft and target; the scaling is an fp32
@@ -49,6 +53,10 @@ Readings where the pages leave a step open:
   * ties in the survival sort: survival descending, then request, then position.
   * ARGMAX mode takes the smallest D attaining max Θ (global search);
     EARLY_STOP takes the first D with Θ(D+1) ≤ Θ(D).
+  * asynchronous (t-2) scheduling: only the capacity K_t (how many drafts step t
+    verifies) comes from step t-2, as the search result D*_{t-2}; which drafts fill it is
+    the first K_t items of step t's own survival order; steps 0 and 1 use a given
+    initial capacity (default D_max).
   * near-ties: a decision closer than 1e-6 (|u - F|, |u - p_t/p_d|, a greedy
     top-2 gap of 1e-6·max(1,|z|)) or than 1e-12 relative (scheduler Θ) is
     reported together with every outcome that is valid within that window.
@@ -339,6 +347,56 @@ def prefix_schedule(c, sps, D_max: int, mode: int = SCHED_ARGMAX, near: float = 
         raise ValueError(mode)
     L = np.bincount(order[:D] // G, minlength=B).astype(np.int32)
     return dict(L=L, a=a, theta=float(theta[D]), D=D, thetas=theta, near_tie=tie)
+
+
+def schedule_at_capacity(c, sps, K: int):
+    """Algorithm 1 with the number of verified drafts fixed at K instead of searched.
+
+    The first K items of the survival order are kept (K clamped to [0, B·γ]); returns
+    (L [B] int32, Θ(K) = (B + S(K))·sps[K])."""
+    a = prefix_survival(c)
+    B, G = a.shape
+    K = int(max(0, min(K, B * G)))
+    order = schedule_order(a)
+    S = float(np.sum(a.reshape(-1)[order[:K]].astype(np.float64)))
+    return np.bincount(order[:K] // G, minlength=B).astype(np.int32), (B + S) * float(np.asarray(sps)[K])
+
+
+def prefix_schedule_t2(c_steps: Sequence, sps, D_max, mode: int = SCHED_ARGMAX, K_init=None,
+                       near: float = THETA_NEAR_TIE):
+    """Asynchronous scheduling: the capacity of step t comes from step t-2's confidences.
+
+    P1 §"硬件感知与置信度自适应调度机制", last paragraph: the truncation decision of step t
+    rests on the confidence history of step t-2, so the global search can run inside the GPU
+    pipeline without a host handshake; P3 §Confidence-Scheduled Verification (production
+    notes, "asynchronous"): confidences from two steps earlier predict the batch capacity K.
+
+    Reading: for each step t, D*_t is the global search of `prefix_schedule` on step t's
+    confidences; the capacity of step t is K_t = D*_{t-2} (K_init for t < 2, default D_max),
+    clamped to [0, min(D_max_t, B_t·γ)]; step t verifies the first K_t items of its own
+    survival order (`schedule_at_capacity`).  c_steps is a sequence of [B_t, γ] arrays (B may
+    change between steps); D_max is an int or one per step.
+
+    Returns one dict per step: L, K (capacity applied), theta (Θ_t(K_t)), D (D*_t, the
+    capacity that step t+2 will apply) and near_tie (whether the decision that gave K_t,
+    made at step t-2, was a near-tie; False for t < 2).
+    """
+    steps = []
+    n = len(c_steps)
+    Dm = [int(D_max)] * n if np.isscalar(D_max) else [int(d) for d in D_max]
+    for t, c in enumerate(c_steps):
+        c = np.asarray(c, dtype=np.float32)
+        B, G = c.shape
+        cap = min(Dm[t], B * G)
+        if t >= 2:
+            K, tie = steps[t - 2]["D"], steps[t - 2]["decision_tie"]
+        else:
+            K, tie = (cap if K_init is None else int(K_init)), False
+        K = int(max(0, min(K, cap)))
+        L, theta = schedule_at_capacity(c, sps, K)
+        d = prefix_schedule(c, sps, cap, mode, near)
+        steps.append(dict(L=L, K=K, theta=theta, D=d["D"], near_tie=tie, decision_tie=d["near_tie"]))
+    return steps
 
 
 def exhaustive_schedule(c, sps, D_max: int):

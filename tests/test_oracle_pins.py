@@ -6,6 +6,7 @@ measurement of the oracle's own u-driven decisions compared with the
 distribution the pages say the round must reproduce.
 """
 
+import itertools
 import math
 
 import numpy as np
@@ -476,3 +477,76 @@ def test_scheduler_ties_by_request_then_position():
     assert order.tolist() == [0, 1, 2, 3]
     r = O.prefix_schedule(c, np.ones(5), 3)
     assert r["L"].tolist() == [2, 1]
+
+
+# --------------------------------------------------------------------------- asynchronous (t-2) scheduling
+
+def _ones_then_zeros(m, G):
+    # request b passes its first m[b] positions for sure and fails the rest: a = 1 ... 1 0 ... 0
+    return np.array([[1.0 if j < mb else 0.0 for j in range(G)] for mb in m], dtype=np.float32)
+
+
+def test_t2_schedule_hand_example():
+    # B = 3, gamma = 4, flat sps: Θ(D) = B + S(D) stops rising after the last positive survival,
+    # so D*_t = sum(m_t).  Capacities: K_0 = K_1 = K_init = 12, then K_t = D*_{t-2}.
+    # The survival order puts the ones first by (request, position), then the zeros likewise.
+    #   t=2: m=[2,2,2], K=D*_0=5: ones (0,0)(0,1)(1,0)(1,1)(2,0)      -> L = [2,2,1]
+    #   t=3: m=[0,0,0], K=D*_1=3: zeros (0,0)(0,1)(0,2)               -> L = [3,0,0]
+    #   t=4: m=[4,4,4], K=D*_2=6: ones (0,0..3)(1,0)(1,1)             -> L = [4,2,0]
+    #   t=5: m=[1,0,3], K=D*_3=0                                      -> L = [0,0,0]
+    # A one-step lag would give K_2 = 3 and L_2 = [2,1,0].
+    ms = [[4, 0, 1], [1, 1, 1], [2, 2, 2], [0, 0, 0], [4, 4, 4], [1, 0, 3]]
+    c = [_ones_then_zeros(m, 4) for m in ms]
+    r = O.prefix_schedule_t2(c, np.ones(13), 12, K_init=12)
+    assert [s["D"] for s in r] == [5, 3, 6, 0, 12, 4]
+    assert [s["K"] for s in r] == [12, 12, 5, 3, 6, 0]
+    assert [s["L"].tolist() for s in r] == [[4, 4, 4], [4, 4, 4], [2, 2, 1], [3, 0, 0], [4, 2, 0], [0, 0, 0]]
+    # Θ_t(K_t) = B + (number of ones among the first K_t items)
+    assert [s["theta"] for s in r] == [8.0, 6.0, 8.0, 3.0, 9.0, 3.0]
+
+
+def _exhaustive_at_capacity(a, K):
+    """Largest Σ_b Σ_{j<L_b} a_{b,j} over prefix lengths with Σ L = K, by brute force."""
+    B, G = a.shape
+    best = -1.0
+    for Ls in itertools.product(range(G + 1), repeat=B):
+        if sum(Ls) == K:
+            best = max(best, sum(float(np.sum(a[b, :Ls[b]], dtype=np.float64)) for b in range(B)))
+    return best
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_capacity_schedule_maximises_expected_accepts(seed):
+    # for a fixed number K of verified drafts, the first K items of the survival order carry
+    # the largest expected number of accepted drafts among all prefix-closed choices
+    rng = np.random.default_rng(300 + seed)
+    B, G = int(rng.integers(1, 4)), int(rng.integers(1, 5))
+    c = rng.beta(3, 2, size=(B, G)).astype(np.float32)
+    a = O.prefix_survival(c).astype(np.float64)
+    for K in range(B * G + 1):
+        L, theta = O.schedule_at_capacity(c, np.ones(B * G + 1), K)
+        assert L.sum() == K and np.all(L <= G)
+        assert theta - B == pytest.approx(_exhaustive_at_capacity(a, K), rel=1e-12)
+
+
+def test_t2_schedule_lag_and_clamp():
+    rng = np.random.default_rng(41)
+    sps = 1.0 / (0.005 + 0.0004 * (6 + np.arange(6 * 5 + 1)))
+    c = [rng.beta(4, 2, size=(6, 5)).astype(np.float32) for _ in range(6)]
+    r = O.prefix_schedule_t2(c, sps, 30)
+    sync = [O.prefix_schedule(ct, sps, 30) for ct in c]
+    assert r[0]["K"] == r[1]["K"] == 30                       # default initial capacity: D_max
+    for t in range(6):
+        assert r[t]["D"] == sync[t]["D"]
+        if t >= 2:
+            assert r[t]["K"] == sync[t - 2]["D"]
+            assert r[t]["near_tie"] == sync[t - 2]["near_tie"]
+    # stationary confidences: from step 2 on, the asynchronous schedule is the synchronous one
+    r = O.prefix_schedule_t2([c[0]] * 4, sps, 30)
+    for t in (2, 3):
+        assert np.array_equal(r[t]["L"], sync[0]["L"]) and r[t]["theta"] == pytest.approx(sync[0]["theta"], rel=1e-15)
+    # the batch shrinks: a capacity from a larger step is clamped to the new B * gamma and D_max
+    c2 = [c[0], c[1], c[2][:2], c[3][:1]]
+    r = O.prefix_schedule_t2(c2, sps, [30, 30, 7, 30])
+    assert r[2]["K"] == min(sync[0]["D"], 7) and r[3]["K"] == min(sync[1]["D"], 5)
+    assert r[3]["L"].sum() == r[3]["K"]
