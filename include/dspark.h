@@ -265,6 +265,41 @@ int dspark_prefix_schedule(const float* c, const double* sps, int B, int gamma, 
                            int32_t* L_out, float* a_out, double* theta_out, uint32_t* flags,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* --------------------------------------------------------------------------
+ * dspark_prefix_schedule_t2 -- asynchronous scheduling: step t's capacity from step t-2.
+ *
+ * [P1 §"硬件感知与置信度自适应调度机制", last paragraph] the truncation of step t is
+ * decided from the confidence history of step t-2, so the global search runs inside the
+ * GPU pipeline, needs no host handshake and is compatible with CUDA-graph replay and
+ * zero-overhead scheduling; [P3 §Confidence-Scheduled Verification, production notes,
+ * "asynchronous"] confidences from two steps earlier predict the batch capacity K.
+ * Reading taken: only the capacity comes from step t-2.  For the step t held in the ring,
+ *     K_t   = D*_{t-2} (the search result of dspark_prefix_schedule on step t-2's c), or
+ *             K_init for t < 2 (K_init < 0: D_max); clamped to [0, D_max]
+ *     L[b]  = number of request b's items among the first K_t of THIS step's survival order
+ *     Θ     = (B + S_t(K_t)) * sps[K_t]  -> theta_out
+ * and the launch also runs the full search on this step's c (mode ARGMAX or EARLY_STOP),
+ * stores D*_t in the ring for step t+2 and advances the ring's step counter.  With c, sps
+ * and the ring in device memory, one captured graph replays the round step after step.
+ *
+ * ring   DSPARK_T2_RING_BYTES of device memory, 8-byte aligned, owned by the caller, zeroed
+ *        (e.g. cudaMemsetAsync) before the first step of a sequence; one ring per sequence,
+ *        calls on it ordered on one stream.  Layout (read it after a step to steer the host):
+ *          offset  0  int64   t          steps taken
+ *          offset  8  int32   D[4]       D*_s of step s at D[s % 4]
+ *          offset 24  uint32  tie[4]     1 if that decision was within 1e-12 of another D
+ *          offset 40  fp64    theta[4]   Θ_s(D*_s)
+ *          offset 72  int32   K[4]       capacity applied at step s
+ *        B may change from step to step (a capacity is clamped to the new D_max).
+ * K_out  [1] int32 or NULL: K_t.   flags: CONF_RANGE as above; SCHED_NEAR_TIE in every
+ *        word when the decision that produced K_t was a near-tie.
+ * Other arguments and limits as dspark_prefix_schedule.  No workspace.
+ * -------------------------------------------------------------------------- */
+#define DSPARK_T2_RING_BYTES 128
+int dspark_prefix_schedule_t2(const float* c, const double* sps, int B, int gamma, int D_max, int mode,
+                              int K_init, void* ring, int32_t* L_out, float* a_out, double* theta_out,
+                              int32_t* K_out, uint32_t* flags, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

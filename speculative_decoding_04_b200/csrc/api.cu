@@ -214,4 +214,21 @@ int dspark_prefix_schedule(const float* c, const double* sps, int B, int gamma, 
   return launch_schedule(s);
 }
 
+int dspark_prefix_schedule_t2(const float* c, const double* sps, int B, int gamma, int D_max, int mode, int K_init,
+                              void* ring, int32_t* L_out, float* a_out, double* theta_out, int32_t* K_out,
+                              uint32_t* flags, void* stream) {
+  if (!c || !sps || !L_out || !theta_out || !ring) return einval("dspark_prefix_schedule_t2: null pointer");
+  if ((uintptr_t)ring % 8 != 0) return einval("dspark_prefix_schedule_t2: ring must be 8-byte aligned");
+  if (B <= 0 || gamma < 1 || gamma > kMaxGamma) return einval("dspark_prefix_schedule_t2: B >= 1, gamma in [1, 64]");
+  if ((long long)B * gamma > kMaxScheduleItems) return einval("dspark_prefix_schedule_t2: B*gamma must be <= 16384");
+  if (D_max < 0 || D_max > B * gamma) return einval("dspark_prefix_schedule_t2: D_max must be in [0, B*gamma]");
+  if (mode != DSPARK_SCHED_ARGMAX && mode != DSPARK_SCHED_EARLY_STOP)
+    return einval("dspark_prefix_schedule_t2: bad mode");
+  ScheduleCall s{c, sps, B, gamma, D_max, mode, L_out, a_out, theta_out, flags, (cudaStream_t)stream};
+  s.ring = static_cast<T2Ring*>(ring);
+  s.K_init = K_init;
+  s.K_out = K_out;
+  return launch_schedule(s);
+}
+
 }  // extern "C"

@@ -81,6 +81,19 @@ struct VerifyCall {
   cudaStream_t stream;
 };
 
+// State of the asynchronous (t-2) scheduler, DSPARK_T2_RING_BYTES of caller-owned device memory;
+// the field offsets are part of the C interface.
+struct T2Ring {
+  long long t;       // steps taken on this ring
+  int D[4];          // D*_s of step s at D[s % 4]
+  unsigned tie[4];   // that decision was a near-tie
+  double theta[4];   // Θ_s(D*_s)
+  int K[4];          // capacity applied at step s
+};
+static_assert(offsetof(T2Ring, D) == 8 && offsetof(T2Ring, tie) == 24 && offsetof(T2Ring, theta) == 40 &&
+                  offsetof(T2Ring, K) == 72 && sizeof(T2Ring) <= DSPARK_T2_RING_BYTES,
+              "T2Ring layout");
+
 struct ScheduleCall {
   const float* c;
   const double* sps;
@@ -90,6 +103,9 @@ struct ScheduleCall {
   double* theta_out;
   uint32_t* flags;
   cudaStream_t stream;
+  T2Ring* ring = nullptr;
+  int K_init = -1;
+  int32_t* K_out = nullptr;
 };
 
 size_t draft_workspace_bytes(int B, int gamma, int V, int r);

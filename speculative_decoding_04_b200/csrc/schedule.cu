@@ -11,6 +11,15 @@
 // warp shuffles for the short strides, an fp64 block scan of the sorted survivals giving
 // Θ(D) = (B + S(D)) * sps[D] for D = 0..D_max, the ARGMAX / EARLY_STOP choice, and per-request
 // counts of the kept items.
+//
+// Asynchronous variant ([P1 §硬件感知与置信度自适应调度机制, last paragraph: the truncation of
+// step t is decided from the confidence history of step t-2, so the global search stays inside
+// the GPU pipeline with no host handshake and survives CUDA-graph replay]; [P3 production notes,
+// "asynchronous": confidences two steps back predict the batch capacity K]): a small device ring
+// carries the step counter and the search results of the last four steps.  The same launch reads
+// the capacity K_t = D*_{t-2} from it, keeps the first K_t items of this step's own survival
+// order, stores this step's D*_t for step t+2 and advances the counter, so a captured graph can
+// replay step after step with the ring as its only state.
 
 #include <algorithm>
 
@@ -30,6 +39,9 @@ struct SchedArgs {
   float* a_out;
   double* theta_out;
   uint32_t* flags;
+  T2Ring* ring;  // asynchronous (t-2) mode when set
+  int K_init;    // capacity of steps 0 and 1 (< 0: D_max)
+  int32_t* K_out;
 };
 
 // Survival descending -> ascending 32-bit key; -0 ranks as +0, NaN ranks last.
@@ -57,8 +69,20 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
   __shared__ int sh_tie[kSchedWarps];
   __shared__ int s_D;
   __shared__ double s_theta;
+  __shared__ int s_K;          // asynchronous mode: capacity applied at this step
+  __shared__ double s_thetaK;  // Θ(s_K) of this step's order
+  __shared__ unsigned s_tieK;  // the decision that gave s_K was a near-tie
+  __shared__ long long s_t;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int B = s.B, G = s.gamma, N = B * G, P = s.P, Dm = s.D_max;
+  if (s.ring && tid == 0) {
+    const long long t = s.ring->t;
+    int K = t >= 2 ? s.ring->D[(t - 2) & 3] : (s.K_init < 0 ? Dm : s.K_init);
+    s_K = max(0, min(K, Dm));
+    s_tieK = t >= 2 ? s.ring->tie[(t - 2) & 3] : 0u;
+    s_t = t;
+    s_thetaK = (double)B * s.sps[0];
+  }
 
   // ---------------------------------------------------------------- survival and keys
   // c is staged in shared memory (the key array's space) with coalesced loads; each request's
@@ -166,6 +190,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
             bestD = i + 1;
           }
           if (th_hi <= th_lo && i < stop) stop = i;
+          if (s.ring && i + 1 == s_K) s_thetaK = th_hi;
         } else if (s.mode == DSPARK_SCHED_ARGMAX) {
           if (i + 1 != Dstar && fabs(th_hi - th_star) <= 1e-12 * fabs(th_star)) tie = 1;
         } else {
@@ -247,15 +272,29 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
   }
 
   // ---------------------------------------------------------------- counts and outputs
-  const int Ds = s_D;
+  // synchronous mode keeps the first D* items; asynchronous mode the first K_t (= D*_{t-2})
+  const int Ds = s.ring ? s_K : s_D;
   for (int i = tid; i < Ds; i += kSchedThreads) atomicAdd(&cnt[(int)(uint32_t)keys[i] / G], 1);
   __syncthreads();
-  const bool near = sh_tie[0] != 0;
+  const bool near = s.ring ? s_tieK != 0 : sh_tie[0] != 0;
   for (int b = tid; b < B; b += kSchedThreads) {
     s.L_out[b] = cnt[b];
     if (near && s.flags) atomicOr(s.flags + b, DSPARK_FLAG_SCHED_NEAR_TIE);
   }
-  if (tid == 0) s.theta_out[0] = s_theta;
+  if (tid == 0) {
+    if (s.ring) {
+      const int slot = (int)(s_t & 3);
+      s.ring->D[slot] = s_D;
+      s.ring->tie[slot] = sh_tie[0] ? 1u : 0u;
+      s.ring->theta[slot] = s_theta;
+      s.ring->K[slot] = s_K;
+      s.ring->t = s_t + 1;
+      s.theta_out[0] = s_thetaK;
+      if (s.K_out) s.K_out[0] = s_K;
+    } else {
+      s.theta_out[0] = s_theta;
+    }
+  }
 }
 
 dspark_status launch_schedule(const ScheduleCall& c) {
@@ -273,6 +312,9 @@ dspark_status launch_schedule(const ScheduleCall& c) {
   s.a_out = c.a_out;
   s.theta_out = c.theta_out;
   s.flags = c.flags;
+  s.ring = c.ring;
+  s.K_init = c.K_init;
+  s.K_out = c.K_out;
   const size_t smem = (size_t)P * 8 + align_up((size_t)c.B * 4, 16);
   cudaError_t rc;
   if (smem > 48 * 1024) {

@@ -14,6 +14,7 @@ import os
 import re
 from typing import Optional, Tuple
 
+import numpy as np
 import torch
 
 from .build import LIB_PATH, ROOT
@@ -24,6 +25,7 @@ POSITION_MAJOR, REQUEST_MAJOR = 0, 1
 _LAYOUTS = {"position": POSITION_MAJOR, "request": REQUEST_MAJOR}
 SCHED_ARGMAX, SCHED_EARLY_STOP = 0, 1
 WS_DRAFT, WS_VERIFY, WS_SCHEDULE = 0, 1, 2
+T2_RING_BYTES = 128
 
 FLAG_DRAFT_NEAR_TIE = 1 << 0
 FLAG_ACCEPT_NEAR_TIE = 1 << 1
@@ -72,6 +74,8 @@ def _load() -> ctypes.CDLL:
     lib.dspark_tv_labels.argtypes = [_vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp]
     lib.dspark_prefix_schedule.restype = _i
     lib.dspark_prefix_schedule.argtypes = [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_prefix_schedule_t2.restype = _i
+    lib.dspark_prefix_schedule_t2.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     return lib
 
 
@@ -276,3 +280,41 @@ def prefix_schedule(c: torch.Tensor, sps: torch.Tensor, D_max: int, mode: int = 
                                     _p(theta_out), _p(flags), None, 0, _s(stream))
     _check("dspark_prefix_schedule", st)
     return L_out, a_out, theta_out, flags
+
+
+def schedule_ring(device=None) -> torch.Tensor:
+    """A zeroed ring for prefix_schedule_t2 (the start of a new sequence of steps)."""
+    return torch.zeros(T2_RING_BYTES // 8, dtype=torch.int64, device=device or "cuda")
+
+
+def ring_state(ring: torch.Tensor) -> dict:
+    """The ring's fields, read back to the host (synchronises)."""
+    raw = ring.cpu().numpy().view(np.uint8)
+    return {"t": int(raw[0:8].view(np.int64)[0]), "D": raw[8:24].view(np.int32).tolist(),
+            "tie": raw[24:40].view(np.uint32).tolist(), "theta": raw[40:72].view(np.float64).tolist(),
+            "K": raw[72:88].view(np.int32).tolist()}
+
+
+def prefix_schedule_t2(c: torch.Tensor, sps: torch.Tensor, D_max: int, ring: torch.Tensor,
+                       mode: int = SCHED_ARGMAX, K_init: int = -1, *, L_out=None, a_out=None, theta_out=None,
+                       K_out=None, flags=None, want_a: bool = False, stream=None):
+    """Asynchronous (t-2) scheduler step on `ring`; returns (L [B], a or None, theta [1] fp64,
+    K [1] int32, flags [B])."""
+    B, G = c.shape
+    _need(c, "c", torch.float32)
+    _need(sps, "sps", torch.float64)
+    if sps.numel() < D_max + 1:
+        raise ValueError("sps must hold D_max + 1 entries")
+    if ring.device != c.device or ring.numel() * ring.element_size() < T2_RING_BYTES or not ring.is_contiguous():
+        raise ValueError("ring must be a contiguous device tensor of T2_RING_BYTES bytes")
+    dev = c.device
+    L_out = torch.empty(B, dtype=torch.int32, device=dev) if L_out is None else L_out
+    if a_out is None and want_a:
+        a_out = torch.empty((B, G), dtype=torch.float32, device=dev)
+    theta_out = torch.empty(1, dtype=torch.float64, device=dev) if theta_out is None else theta_out
+    K_out = torch.empty(1, dtype=torch.int32, device=dev) if K_out is None else K_out
+    flags = torch.zeros(B, dtype=torch.int32, device=dev) if flags is None else flags
+    st = lib.dspark_prefix_schedule_t2(_p(c), _p(sps), B, G, int(D_max), int(mode), int(K_init), _p(ring),
+                                       _p(L_out), _p(a_out), _p(theta_out), _p(K_out), _p(flags), _s(stream))
+    _check("dspark_prefix_schedule_t2", st)
+    return L_out, a_out, theta_out, K_out, flags
