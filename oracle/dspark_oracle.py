@@ -23,6 +23,10 @@ What each function follows:
                   consistent prefix plus a bonus token).
   * tv_labels  -- P3 §Confidence-Scheduled Verification: c*_k = 1 - ½‖p_d - p_t‖₁;
                   P1 §"硬件感知与置信度自适应调度机制" (label = analytic acceptance rate).
+  * ragged_offsets, ragged_tags, pack_ragged, verify_ragged, tv_labels_ragged --
+                  P1 §极致的工程实现与内核优化 (inference: all tokens to verify flattened into one
+                  1-D array with a light token-tag tensor, no padding) and P3 production notes
+                  (variable-length verify over flattened tokens with a marker tensor).
   * prefix_survival -- P3 §Confidence-Scheduled Verification: a_{r,j} = ∏_{i≤j} c_{r,i}.
   * prefix_schedule -- P3 §Confidence-Scheduled Verification (Algorithm 1,
                   Θ = τ·SPS(B)); P1 §"硬件感知与置信度自适应调度机制" (sort all
@@ -53,6 +57,10 @@ Readings where the pages leave a step open:
   * ties in the survival sort: survival descending, then request, then position.
   * ARGMAX mode takes the smallest D attaining max Θ (global search);
     EARLY_STOP takes the first D with Θ(D+1) ≤ Θ(D).
+  * flattened verification: request b owns target rows off[b] .. off[b] + L_b of one
+    packed [Σ(L_b+1), V] array (off = exclusive prefix sum of L_b + 1); its tag is
+    b·(γ+1) + k; it is verified exactly as the padded block; TV labels exist for the
+    positions k <= min(L_b, γ-1) whose target row is present.
   * asynchronous (t-2) scheduling: only the capacity K_t (how many drafts step t
     verifies) comes from step t-2, as the search result D*_{t-2}; which drafts fill it is
     the first K_t items of step t's own survival order; steps 0 and 1 use a given
@@ -291,6 +299,80 @@ def tv_labels(ld, lt, T: float) -> np.ndarray:
                 out[b, k] = 1.0 if int(np.argmax(ld[b, k])) == int(np.argmax(lt[b, k])) else 0.0
             else:
                 out[b, k] = 1.0 - 0.5 * float(np.sum(np.abs(softmax(ld[b, k], T) - softmax(lt[b, k], T))))
+    return out
+
+
+# --------------------------------------------------------------------------- flattened (ragged) verification
+
+def ragged_offsets(L, gamma: int):
+    """Row offsets of the flattened target block: request b owns rows off[b] .. off[b] + L_b
+    (its L_b verified positions and the bonus/resample position), so off[0] = 0 and
+    off[b+1] = off[b] + L_b + 1; off[B] is the number of rows.  P1 §极致的工程实现与内核优化
+    (inference): every token to verify goes into one contiguous 1-D array, no padding.
+    L_b is clamped to [0, gamma] first.  Returns int64 [B+1]."""
+    Lc = np.clip(np.asarray(L, dtype=np.int64), 0, gamma)
+    off = np.zeros(Lc.size + 1, dtype=np.int64)
+    for b in range(Lc.size):
+        off[b + 1] = off[b] + Lc[b] + 1
+    return off
+
+
+def ragged_tags(L, gamma: int):
+    """Token tags of the flattened rows: row off[b] + k carries b*(gamma+1) + k, which names
+    its request and its position (P1 §极致的工程实现与内核优化: a light tag tensor marks
+    which sequence, and where in it, each flattened token belongs).  int32 [off[B]]."""
+    off = ragged_offsets(L, gamma)
+    tags = np.empty(int(off[-1]), dtype=np.int32)
+    for b in range(off.size - 1):
+        for k in range(int(off[b + 1] - off[b])):
+            tags[off[b] + k] = b * (gamma + 1) + k
+    return tags
+
+
+def pack_ragged(lt, L):
+    """Padded target logits [B, γ+1, V] -> the flattened rows [off[B], V] (rows 0..L_b of b)."""
+    lt = np.asarray(lt)
+    B, G1, V = lt.shape
+    off = ragged_offsets(L, G1 - 1)
+    out = np.empty((int(off[-1]), V), dtype=lt.dtype)
+    for b in range(B):
+        n = int(off[b + 1] - off[b])
+        out[off[b]:off[b] + n] = lt[b, :n]
+    return out
+
+
+def verify_ragged(ld, lt_packed, off, x, L, u_acc, u_res, T: float):
+    """Verification over flattened target rows: request b's target row k is lt_packed[off[b] + k]
+    for k = 0..L_b; otherwise exactly `verify` (rows past L_b are never read there either).
+    Returns (n_acc, y, detail) like `verify`."""
+    ld = np.asarray(ld, dtype=np.float32)
+    lt_packed = np.asarray(lt_packed, dtype=np.float32)
+    B, G = np.asarray(x).shape
+    V = lt_packed.shape[1]
+    n_acc = np.zeros(B, dtype=np.int32)
+    y = np.full((B, G + 1), -1, dtype=np.int32)
+    detail = []
+    for b in range(B):
+        Lb = int(L[b])
+        assert int(off[b + 1]) - int(off[b]) == Lb + 1, "offsets must hold L_b + 1 rows per request"
+        rows = np.full((G + 1, V), np.nan, dtype=np.float32)     # rows past L_b do not exist
+        rows[:Lb + 1] = lt_packed[int(off[b]):int(off[b]) + Lb + 1]
+        r = verify_request(ld[b], rows, x[b], Lb, u_acc[b], u_res[b], T)
+        n_acc[b], y[b] = r["n"], r["y"]
+        detail.append(r)
+    return n_acc, y, detail
+
+
+def tv_labels_ragged(ld, lt_packed, off, L, T: float):
+    """TV labels of the positions whose target row exists in the flattened block
+    (k <= min(L_b, γ-1)); NaN at the others."""
+    ld = np.asarray(ld, dtype=np.float32)
+    B, G, V = ld.shape
+    out = np.full((B, G), np.nan, dtype=np.float64)
+    for b in range(B):
+        for k in range(min(int(L[b]) + 1, G)):
+            out[b, k] = tv_labels(ld[b:b + 1, k:k + 1], np.asarray(lt_packed)[None, int(off[b]) + k:int(off[b]) + k + 1],
+                                  T)[0, 0]
     return out
 
 

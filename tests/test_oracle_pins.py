@@ -550,3 +550,44 @@ def test_t2_schedule_lag_and_clamp():
     r = O.prefix_schedule_t2(c2, sps, [30, 30, 7, 30])
     assert r[2]["K"] == min(sync[0]["D"], 7) and r[3]["K"] == min(sync[1]["D"], 5)
     assert r[3]["L"].sum() == r[3]["K"]
+
+
+# --------------------------------------------------------------------------- flattened (ragged) verification
+
+def test_ragged_offsets_and_tags_hand_example():
+    # request b owns L_b + 1 rows: lengths 3, 1, 6, 2 -> offsets 0, 3, 4, 10, 12
+    assert O.ragged_offsets([2, 0, 5, 1], 5).tolist() == [0, 3, 4, 10, 12]
+    # tags b*(gamma+1) + k with gamma = 3: request 0 rows k=0..2, request 1 k=0, request 2 k=0..1
+    assert O.ragged_tags([2, 0, 1], 3).tolist() == [0, 1, 2, 4, 8, 9]
+    # lengths outside [0, gamma] are clamped first
+    assert O.ragged_offsets([7, -1], 5).tolist() == [0, 6, 7]
+    assert O.ragged_offsets([], 4).tolist() == [0]
+
+
+@pytest.mark.parametrize("T", [1.0, 0.7, 0.0])
+def test_ragged_verify_is_the_padded_verify(T):
+    rng = np.random.default_rng(51)
+    B, G, V = 7, 4, 300
+    ld = rng.normal(0, 1.5, (B, G, V)).astype(np.float32)
+    lt = (ld[:, [0, 1, 2, 3, 3]] + rng.normal(0, 0.7, (B, G + 1, V))).astype(np.float32)
+    L = np.array([0, 4, 2, 1, 3, 4, 0], dtype=np.int32)
+    x = np.argmax(ld + rng.gumbel(size=ld.shape).astype(np.float32), axis=2).astype(np.int32)
+    u_acc = rng.random((B, G)).astype(np.float32)
+    u_res = rng.random(B).astype(np.float32)
+    # rows past L_b are NaN in the padded block: neither form may read them
+    lt_pad = lt.copy()
+    for b in range(B):
+        lt_pad[b, L[b] + 1:] = np.nan
+    packed = O.pack_ragged(lt_pad, L)
+    off = O.ragged_offsets(L, G)
+    assert packed.shape == (int(L.sum()) + B, V) and not np.isnan(packed).any()
+    n0, y0, _ = O.verify(ld, lt_pad, x, L, u_acc, u_res, T)
+    n1, y1, _ = O.verify_ragged(ld, packed, off, x, L, u_acc, u_res, T)
+    assert np.array_equal(n0, n1) and np.array_equal(y0, y1)
+    assert np.all(n1 <= L) and np.all(y1[np.arange(B), n1] >= 0)
+    # TV labels where the target row exists, NaN elsewhere
+    c = O.tv_labels_ragged(ld, packed, off, L, T)
+    full = O.tv_labels(ld, lt, T)
+    for b in range(B):
+        k_have = min(int(L[b]) + 1, G)
+        assert np.array_equal(c[b, :k_have], full[b, :k_have]) and np.isnan(c[b, k_have:]).all()
