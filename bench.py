@@ -456,6 +456,36 @@ def main():
                "wall_ms_per_round": (tb1 - tb0) * 1e3 / args.steps,
                "device_ms_per_round": eb0.elapsed_time(eb1) / args.steps}
 
+        # the round captured once as a CUDA graph and replayed, with the asynchronous scheduler
+        # (capacity from step t-2, kept on a device ring), L2 flushed before every replay
+        ring = D.schedule_ring(dev)
+        K_t = torch.empty(1, dtype=torch.int32, device=dev)
+
+        def round_t2(src):
+            draft(src)
+            D.prefix_schedule_t2(src["c"], sps, B * G, ring, L_out=L, theta_out=theta, K_out=K_t, flags=fl,
+                                 stream=stream)
+            D.verify(ld, src["lt"], x, L, src["u_acc"], src["u_res"], wl.T, ld_layout=args.layout, n_acc=n_acc,
+                     y_out=y, c_star=c_star, flags=fl, ws=ws_v, stream=stream)
+
+        round_t2(dv)
+        barrier()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            round_t2(dv)
+        gt = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(float(i))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            if i >= args.warmup:
+                gt.append((e0, e1))
+        barrier()
+        graph_ms = median_ms(gt)
+        del graph
+
         # end to end through the public API with pinned host buffers
         e2e = None
         if host_logit_bytes <= HOST_E2E_LIMIT:
@@ -525,6 +555,9 @@ def main():
                                 "algorithmic_bytes": verify_b},
             "warm_l2": {"ms_per_step": warm_step_ms, "draft_ms": warm_draft_ms, "rounds_per_s": 1e3 / warm_step_ms},
             "back_to_back": b2b,
+            "graph_t2": {"ms_per_round": graph_ms, "rounds_per_s": 1e3 / graph_ms,
+                         "round": "markov_draft -> prefix_schedule_t2 (capacity from step t-2, device ring) -> "
+                                  "verify, captured once as a CUDA graph and replayed; L2 flushed between replays"},
             "e2e": ({"value": world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
                     if host_logit_bytes <= HOST_E2E_LIMIT else
                     {"value": None, "unit": UNIT, "h2d_bytes_per_step": None, "d2h_bytes_per_step": None,

@@ -73,6 +73,7 @@ enum { DSPARK_WS_DRAFT = 0, DSPARK_WS_VERIFY = 1, DSPARK_WS_SCHEDULE = 2 };
 #define DSPARK_FLAG_TOKEN_RANGE       (1u << 5) /* a token id outside [0, V) */
 #define DSPARK_FLAG_CONF_RANGE        (1u << 6) /* a confidence outside [0, 1] */
 #define DSPARK_FLAG_SCHED_NEAR_TIE    (1u << 7) /* the chosen D is within 1e-12 (relative) of another */
+#define DSPARK_FLAG_RAGGED_OFFSETS    (1u << 8) /* flattened l_t: lt_off[b+1] - lt_off[b] != L[b] + 1, or outside [0, lt_nrows] */
 #define DSPARK_FLAG_DEVICE_TIMEOUT    (1u << 31)
 
 /* Human-readable name of a status code. */
@@ -195,6 +196,49 @@ int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int3
                   int B, int gamma, int V, float T, int ld_layout,
                   int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags,
                   void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_ragged_layout -- row offsets and token tags of a flattened verify block.
+ *
+ * [P1 §"极致的工程实现与内核优化", inference paragraph] all tokens a batch verifies are
+ * flattened into one contiguous 1-D array without padding, and a light token-tag tensor
+ * tells which sequence, and where in it, each token belongs; [P3 §Confidence-Scheduled
+ * Verification, production notes] variable-length verify over flattened tokens with a
+ * marker tensor.  Request b (verify length L_b, clamped to [0, gamma]) owns the L_b + 1 rows
+ *     lt_off[b] .. lt_off[b] + L_b,  lt_off[0] = 0,  lt_off[b+1] = lt_off[b] + L_b + 1,
+ * its L_b verified positions and the resample/bonus position; lt_off[B] is the row count.
+ * L       [B] int32 device (e.g. dspark_prefix_schedule's L_out).
+ * lt_off  [B+1] int64 device, written.
+ * tags    [B*(gamma+1)] int32 device or NULL: row lt_off[b] + k gets b*(gamma+1) + k; the
+ *         entries past lt_off[B] get -1.
+ * One CTA; no workspace.
+ * -------------------------------------------------------------------------- */
+int dspark_ragged_layout(const int32_t* L, int B, int gamma, int64_t* lt_off, int32_t* tags, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_verify_ragged -- dspark_verify over a flattened target block.
+ *
+ * The same verification as dspark_verify with L given, reading request b's target row k
+ * (k = 0..L_b) from row lt_off[b] + k of the flattened lt instead of row k of a padded
+ * [B, gamma+1, V] block: the target forward then computes and stores only the
+ * sum over b of (L_b + 1) rows that verification uses (dspark_ragged_layout gives
+ * lt_off).  Results equal dspark_verify's on the padded block holding the same rows.
+ * lt        [lt_nrows, V] fp32 device, the flattened target logits.
+ * lt_off    [B+1] int64 device row offsets.  Offsets that do not give request b exactly
+ *           L_b + 1 rows inside [0, lt_nrows] set RAGGED_OFFSETS in flags[b]; every row
+ *           index is clamped into [0, lt_nrows - 1], so the call never reads outside lt
+ *           (that request's results are then meaningless).
+ * L         [B] int32 verify lengths, required.
+ * c_star    [B, gamma] fp32 or NULL: TV labels at the positions k <= min(L_b, gamma-1) whose
+ *           target row the block holds; NaN at the others.
+ * Other arguments, flags and the workspace as dspark_verify.  The streaming kernels run
+ * (verify_impl 0); with verify_impl 1 or 2 the per-row kernels do.
+ * -------------------------------------------------------------------------- */
+int dspark_verify_ragged(const float* ld, const float* lt, const int64_t* lt_off, int64_t lt_nrows,
+                         const int32_t* x, const int32_t* L, const float* u_acc, const float* u_res,
+                         int B, int gamma, int V, float T, int ld_layout,
+                         int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags,
+                         void* ws, size_t ws_bytes, void* stream);
 
 /* --------------------------------------------------------------------------
  * dspark_verify_noalloc -- dspark_verify without a caller workspace.

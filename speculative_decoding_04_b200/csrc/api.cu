@@ -186,6 +186,34 @@ int dspark_verify(const float* ld, const float* lt, const int32_t* x, const int3
   return launch_verify(c);
 }
 
+int dspark_ragged_layout(const int32_t* L, int B, int gamma, int64_t* lt_off, int32_t* tags, void* stream) {
+  if (!L || !lt_off) return einval("dspark_ragged_layout: null pointer");
+  if (B <= 0 || gamma < 1 || gamma > kMaxGamma) return einval("dspark_ragged_layout: B >= 1, gamma in [1, 64]");
+  return launch_ragged_layout(L, B, gamma, lt_off, tags, (cudaStream_t)stream);
+}
+
+int dspark_verify_ragged(const float* ld, const float* lt, const int64_t* lt_off, int64_t lt_nrows, const int32_t* x,
+                         const int32_t* L, const float* u_acc, const float* u_res, int B, int gamma, int V, float T,
+                         int ld_layout, int32_t* n_acc, int32_t* y_out, float* c_star, uint32_t* flags, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (!ld || !lt || !lt_off || !x || !L || !n_acc || !y_out || !flags || !ws)
+    return einval("dspark_verify_ragged: null pointer");
+  if (T != 0.f && (!u_acc || !u_res)) return einval("dspark_verify_ragged: u_acc and u_res are required when T > 0");
+  if (B <= 0 || V < 2) return einval("dspark_verify_ragged: B must be >= 1 and V >= 2");
+  if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_verify_ragged: gamma must be in [1, 64]");
+  if (lt_nrows < 1) return einval("dspark_verify_ragged: lt_nrows must be >= 1");
+  if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_verify_ragged: T must be finite and >= 0");
+  if (ld_layout != DSPARK_POSITION_MAJOR && ld_layout != DSPARK_REQUEST_MAJOR)
+    return einval("dspark_verify_ragged: ld_layout must be DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR");
+  if (ws_bytes < verify_workspace_bytes(B, gamma, V)) return einval("dspark_verify_ragged: workspace too small");
+  if ((uintptr_t)ws % 256) return einval("dspark_verify_ragged: workspace must be 256-byte aligned");
+  VerifyCall c{ld, lt, x, L, u_acc, u_res, B, gamma, V, gamma + 1, T, ld_layout, 1, 0, n_acc, y_out, c_star, flags, ws, ws_bytes,
+               (cudaStream_t)stream};
+  c.lt_off = lt_off;
+  c.lt_nrows = (long long)lt_nrows;
+  return launch_verify(c);
+}
+
 int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, int lt_rows, float T, int ld_layout,
                      float* c_star, void* stream) {
   if (!ld || !lt || !c_star) return einval("dspark_tv_labels: null pointer");

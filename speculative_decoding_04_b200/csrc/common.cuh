@@ -354,4 +354,20 @@ struct ChunkStat {
   float m2;
 };
 
+// Row of l_t holding position k of request b: row b*lt_rows + k of the padded block, or, when
+// the block is flattened (off = per-request row offsets), row off[b] + k, clamped into the
+// array's nrows rows so that inconsistent offsets never read outside it.
+__device__ __forceinline__ size_t lt_row_index(const int64_t* off, long long nrows, int lt_rows, int b, int k) {
+  if (!off) return (size_t)b * (size_t)lt_rows + (size_t)k;
+  long long r = __ldg(off + b) + k;
+  r = r < 0 ? 0 : (r >= nrows ? nrows - 1 : r);
+  return (size_t)r;
+}
+
+// The flattened block's offsets of request b do not hold exactly L_b + 1 rows inside the array.
+__device__ __forceinline__ bool ragged_mismatch(const int64_t* off, long long nrows, int b, int Lb) {
+  const long long o0 = __ldg(off + b), o1 = __ldg(off + b + 1);
+  return o1 - o0 != (long long)Lb + 1 || o0 < 0 || o1 > nrows;
+}
+
 }  // namespace dspark

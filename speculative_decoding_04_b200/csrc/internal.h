@@ -79,7 +79,12 @@ struct VerifyCall {
   void* ws;
   size_t ws_bytes;
   cudaStream_t stream;
+  const int64_t* lt_off = nullptr;  // flattened l_t: request b's rows start at lt_off[b] (nullptr: padded)
+  long long lt_nrows = 0;           // rows of the flattened l_t
 };
+
+dspark_status launch_ragged_layout(const int32_t* L, int B, int gamma, int64_t* lt_off, int32_t* tags,
+                                   cudaStream_t stream);
 
 // State of the asynchronous (t-2) scheduler, DSPARK_T2_RING_BYTES of caller-owned device memory;
 // the field offsets are part of the C interface.

@@ -1112,6 +1112,7 @@ dspark_status launch_verify_sliced(const VerifyCall& c) {
   const Options opt = options();
   if (!c.do_verify || c.per_row_only || opt.verify_impl != 1) return DSPARK_ENOTIMPL;
   if (c.V % 4 || (uintptr_t)c.ld % 16 || (uintptr_t)c.lt % 16) return DSPARK_ENOTIMPL;
+  if (c.lt_off) return DSPARK_ENOTIMPL;  // the flattened block runs the per-row kernels
   const int sms = device_sm_count();
   const VsGeometry geo = vs_geometry(c.B, c.gamma, c.V, sms, opt.verify_groups);
   // descriptors hold b in 20 bits and k in 7

@@ -107,6 +107,8 @@ struct SvArgs {
   const float* u_res;
   int B, gamma, V, lt_rows, njobs, ntile, C, lag, l2hint;
   size_t ld_sk, ld_sb;  // element strides of the l_d row of position k and request b
+  const int64_t* lt_off;  // flattened l_t: request b's rows start at row lt_off[b] (null: padded)
+  long long lt_nrows;
   uint64_t wait_ns;  // bounded waits give up after this long
   int xbar_extra;    // test-only: arrivals the exchange barriers expect beyond the cluster
   float zscale;  // log2(e) / T (T > 0)
@@ -135,7 +137,8 @@ __device__ __forceinline__ SvJob sv_job(const SvArgs& a, int j) {
   J.rec = J.b * (a.gamma + 1) + J.k;
   int Lb = a.gamma;
   if (a.do_verify && a.L) Lb = min(max(__ldg(a.L + J.b), 0), a.gamma);
-  const bool cstar = a.c_star != nullptr && J.k < a.gamma;
+  // a flattened l_t holds rows 0..L_b of a request only: labels exist there
+  const bool cstar = a.c_star != nullptr && J.k < a.gamma && (!a.lt_off || J.k <= Lb);
   J.verify = a.do_verify && J.k < Lb;
   const bool bonus = a.do_verify && J.k == Lb;
   J.d = cstar || (J.verify && !a.greedy);  // greedy acceptance needs only argmax l_t
@@ -579,7 +582,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           const uint32_t bytes = (uint32_t)(c1 - c0) * 4u;
           const bool with_d = ph.second || ph.J.d;
           const float* rd = a.ld + (size_t)ph.J.k * a.ld_sk + (size_t)ph.J.b * a.ld_sb;
-          const float* rt = a.lt + ((size_t)ph.J.b * a.lt_rows + ph.J.k) * a.V;
+          const float* rt = a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, ph.J.b, ph.J.k) * a.V;
           mbar_expect_tx(&full[s], with_d ? 2 * bytes : bytes);
           if (a.l2hint) {
             // first pass: keep the lines for the second; second pass: they are done with
@@ -656,7 +659,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       float ldx = 0.f, ltx = 0.f;
       if (!GREEDY && J.verify && (unsigned)xk < (unsigned)a.V) {
         ldx = __ldg(a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb + xk);
-        ltx = __ldg(a.lt + ((size_t)J.b * a.lt_rows + J.k) * a.V + xk);
+        ltx = __ldg(a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, J.b, J.k) * a.V + xk);
       }
       ok = sv_wait(sy, &xbar[js], (i / kSvJobSlots) & 1, true);
       if (!ok) break;
@@ -929,7 +932,7 @@ __device__ int sv_sample(const SvArgs& a, int b, int k, bool resid, const SvNorm
   const SvP2 k2 = sv_p2_consts(nm);
   const float zc = a.zscale;
   const float* rowd = a.ld + (size_t)k * a.ld_sk + (size_t)b * a.ld_sb;
-  const float* rowt = a.lt + ((size_t)b * a.lt_rows + k) * a.V;
+  const float* rowt = a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, b, k) * a.V;
   const int per = (a.ntile + 31) / 32;
   const int t_lo = min(lane * per, a.ntile), t_hi = min(t_lo + per, a.ntile);
   auto tile_w = [&](int t, bool use_q) -> double {
@@ -1059,7 +1062,9 @@ __global__ void __launch_bounds__(128) verify_stream_finalize(SvArgs a) {
   if (a.c_star) {
     for (int k = lane; k < G; k += 32) {
       float cs;
-      if (a.greedy) {
+      if (a.lt_off && k > Lb) {
+        cs = __int_as_float(0x7fc00000);  // no target row in the flattened block: NaN
+      } else if (a.greedy) {
         cs = rr[k].cstar;
       } else {
         // sum min(p_d, p_t); exactly 1 when no column has p_t > p_d (then q = 0 everywhere)
@@ -1094,6 +1099,7 @@ __global__ void __launch_bounds__(128) verify_stream_finalize(SvArgs a) {
     tok = sv_sample(a, b, n, n < Lb, rr[n].nm, fl);
   }
   if (timed_out) fl |= DSPARK_FLAG_DEVICE_TIMEOUT;
+  if (a.lt_off && ragged_mismatch(a.lt_off, a.lt_nrows, b, Lb)) fl |= DSPARK_FLAG_RAGGED_OFFSETS;
   int32_t* y = a.y_out + (size_t)b * R;
   for (int j = lane; j < R; j += 32) y[j] = j < n ? a.x[(size_t)b * G + j] : (j == n ? tok : -1);
   if (lane == 0) {
@@ -1145,6 +1151,8 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.gamma = c.gamma;
   a.V = c.V;
   a.lt_rows = c.lt_rows;
+  a.lt_off = c.lt_off;
+  a.lt_nrows = c.lt_nrows;
   ld_strides(c.ld_layout, c.B, c.gamma, c.V, a.ld_sk, a.ld_sb);
   a.njobs = c.B * (c.gamma + 1);
   a.ntile = (c.V + kSvTile - 1) / kSvTile;

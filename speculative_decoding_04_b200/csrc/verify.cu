@@ -41,6 +41,8 @@ struct VerifyArgs {
   const float* u_res;
   int B, gamma, V, lt_rows, rows_per_req;
   size_t ld_sk, ld_sb;  // element strides of the l_d row of position k and request b
+  const int64_t* lt_off;  // flattened l_t: request b's rows start at row lt_off[b] (null: padded)
+  long long lt_nrows;
   float inv_T;
   int greedy;
   int do_verify;
@@ -150,6 +152,11 @@ __global__ void verify_finalize(VerifyArgs a) {
   const int cand = a.row_cand[(size_t)b * R + n];
   for (int j = 0; j < R; ++j) y[j] = (j < n) ? a.x[(size_t)b * a.gamma + j] : (j == n ? cand : -1);
   a.n_acc[b] = n;
+  if (a.lt_off) {
+    if (ragged_mismatch(a.lt_off, a.lt_nrows, b, Lb)) fl |= DSPARK_FLAG_RAGGED_OFFSETS;
+    if (a.c_star)  // no target row in the flattened block: NaN
+      for (int k = Lb + 1; k < a.gamma; ++k) a.c_star[(size_t)b * a.gamma + k] = __int_as_float(0x7fc00000);
+  }
   if (fl && a.flags) atomicOr(a.flags + b, fl);
 }
 
@@ -180,7 +187,8 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
 
   int Lb = a.gamma;
   if (a.do_verify && a.L) Lb = min(max(a.L[b], 0), a.gamma);
-  const bool need_cstar = (a.c_star != nullptr) && kk < a.gamma;
+  // a flattened l_t holds rows 0..L_b of a request only: labels exist there
+  const bool need_cstar = (a.c_star != nullptr) && kk < a.gamma && (!a.lt_off || kk <= Lb);
   const bool need_acc = a.do_verify && kk < Lb;
   const bool need_bonus = a.do_verify && kk == Lb;
   const bool need_d = need_cstar || need_acc;
@@ -191,7 +199,7 @@ __global__ void __launch_bounds__(512) verify_rows(VerifyArgs a) {
   const int v_beg = rank * a.Vc;
   const int n = max(0, min(a.V, v_beg + a.Vc) - v_beg);
   const size_t rowd = (size_t)kk * a.ld_sk + (size_t)b * a.ld_sb + v_beg;
-  const size_t rowt = ((size_t)b * a.lt_rows + kk) * a.V + v_beg;
+  const size_t rowt = lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, b, kk) * a.V + v_beg;
   bool timed_out = false;
 
   if (tid == 0) {
@@ -605,7 +613,7 @@ __device__ __forceinline__ RowNeed row_need(const VerifyArgs& a, long long row) 
   r.kk = (int)(row - (long long)r.b * a.rows_per_req);
   r.Lb = a.gamma;
   if (a.do_verify && a.L) r.Lb = min(max(a.L[r.b], 0), a.gamma);
-  r.cstar = (a.c_star != nullptr) && r.kk < a.gamma;
+  r.cstar = (a.c_star != nullptr) && r.kk < a.gamma && (!a.lt_off || r.kk <= r.Lb);
   r.acc = a.do_verify && r.kk < r.Lb;
   r.bonus = a.do_verify && r.kk == r.Lb;
   r.d = r.cstar || r.acc;
@@ -665,7 +673,7 @@ __global__ void __launch_bounds__(512, 1) verify_rows_pc(VerifyArgs a) {
       float* sd = psm + (size_t)j * 2 * a.Vc;
       const uint32_t bytes = (uint32_t)n * 4u;
       const size_t rowd = (size_t)rn.kk * a.ld_sk + (size_t)rn.b * a.ld_sb + v_beg;
-      const size_t rowt = ((size_t)rn.b * a.lt_rows + rn.kk) * a.V + v_beg;
+      const size_t rowt = lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, rn.b, rn.kk) * a.V + v_beg;
       mbar_arrive_expect_tx(&bar[j], rn.d ? 2u * bytes : bytes);
       if (rn.d) bulk_g2s(sd, a.ld + rowd, bytes, &bar[j]);
       bulk_g2s(sd + a.Vc, a.lt + rowt, bytes, &bar[j]);
@@ -1150,6 +1158,8 @@ dspark_status launch_verify(const VerifyCall& c) {
   a.gamma = c.gamma;
   a.V = c.V;
   a.lt_rows = c.lt_rows;
+  a.lt_off = c.lt_off;
+  a.lt_nrows = c.lt_nrows;
   ld_strides(c.ld_layout, c.B, c.gamma, c.V, a.ld_sk, a.ld_sb);
   a.rows_per_req = c.do_verify ? c.gamma + 1 : c.gamma;
   a.greedy = (c.T == 0.f) ? 1 : 0;
@@ -1326,3 +1336,63 @@ extern "C" int dspark_verify_noalloc(const float* ld, const float* lt, const int
                kNoAllocScratchBytes, (cudaStream_t)stream};
   return launch_verify(c);
 }
+
+// ============================================================================ flattened target block
+//
+// Row offsets and token tags of the flattened verify block (one CTA): request b owns rows
+// off[b] .. off[b] + L_b, off being the exclusive prefix sum of L_b + 1 (L_b clamped to
+// [0, gamma]); row off[b] + k carries the tag b*(gamma+1) + k, and the tags past the last row,
+// up to the capacity B*(gamma+1), are -1.
+
+namespace dspark {
+
+__global__ void __launch_bounds__(1024) ragged_layout_kernel(const int32_t* L, int B, int gamma, int64_t* off,
+                                                             int32_t* tags) {
+  __shared__ long long sh[32];
+  __shared__ long long s_carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    s_carry = 0;
+    off[0] = 0;
+  }
+  __syncthreads();
+  for (int base = 0; base < B; base += 1024) {
+    const int b = base + tid;
+    const long long v = b < B ? (long long)min(max(__ldg(L + b), 0), gamma) + 1 : 0;
+    long long x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) sh[warp] = x;
+    __syncthreads();
+    long long incl = s_carry + x;
+    for (int w = 0; w < warp; ++w) incl += sh[w];
+    if (b < B) {
+      off[b + 1] = incl;
+      if (tags)
+        for (int k = 0; k < (int)v; ++k) tags[incl - v + k] = b * (gamma + 1) + k;
+    }
+    __syncthreads();
+    if (tid == 1023) s_carry = incl;  // the chunk's total plus the carry
+    __syncthreads();
+  }
+  if (tags) {
+    const long long cap = (long long)B * (gamma + 1);
+    for (long long i = s_carry + tid; i < cap; i += 1024) tags[i] = -1;
+  }
+}
+
+dspark_status launch_ragged_layout(const int32_t* L, int B, int gamma, int64_t* lt_off, int32_t* tags,
+                                   cudaStream_t stream) {
+  ragged_layout_kernel<<<1, 1024, 0, stream>>>(L, B, gamma, lt_off, tags);
+  const cudaError_t rc = cudaGetLastError();
+  if (rc != cudaSuccess) {
+    set_error(std::string("ragged layout launch: ") + cudaGetErrorString(rc));
+    return DSPARK_ECUDA;
+  }
+  return DSPARK_OK;
+}
+
+}  // namespace dspark

@@ -35,6 +35,7 @@ FLAG_NONFINITE = 1 << 4
 FLAG_TOKEN_RANGE = 1 << 5
 FLAG_CONF_RANGE = 1 << 6
 FLAG_SCHED_NEAR_TIE = 1 << 7
+FLAG_RAGGED_OFFSETS = 1 << 8
 FLAG_DEVICE_TIMEOUT = 1 << 31
 
 HEADER = os.path.join(ROOT, "include", "dspark.h")
@@ -74,6 +75,11 @@ def _load() -> ctypes.CDLL:
     lib.dspark_tv_labels.argtypes = [_vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp]
     lib.dspark_prefix_schedule.restype = _i
     lib.dspark_prefix_schedule.argtypes = [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_ragged_layout.restype = _i
+    lib.dspark_ragged_layout.argtypes = [_vp, _i, _i, _vp, _vp, _vp]
+    lib.dspark_verify_ragged.restype = _i
+    lib.dspark_verify_ragged.argtypes = [_vp, _vp, _vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp,
+                                         _vp, _vp, _vp, _vp, _sz, _vp]
     lib.dspark_prefix_schedule_t2.restype = _i
     lib.dspark_prefix_schedule_t2.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     return lib
@@ -218,6 +224,56 @@ def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torc
                            _LAYOUTS[ld_layout], _p(n_acc),
                            _p(y_out), _p(c_star), _p(flags), _p(ws), ws.numel(), _s(stream))
     _check("dspark_verify", st)
+    return n_acc, y_out, c_star, flags
+
+
+def ragged_layout(L: torch.Tensor, gamma: int, *, lt_off=None, tags=None, want_tags: bool = True, stream=None):
+    """Row offsets [B+1] int64 (and tags [B*(gamma+1)] int32) of the flattened verify block for the
+    verify lengths L [B]."""
+    _need(L, "L", torch.int32)
+    B = L.shape[0]
+    lt_off = torch.empty(B + 1, dtype=torch.int64, device=L.device) if lt_off is None else lt_off
+    if tags is None and want_tags:
+        tags = torch.empty(B * (gamma + 1), dtype=torch.int32, device=L.device)
+    _need(lt_off, "lt_off", torch.int64, (B + 1,))
+    if tags is not None:
+        _need(tags, "tags", torch.int32, (B * (gamma + 1),))
+    _check("dspark_ragged_layout", lib.dspark_ragged_layout(_p(L), B, int(gamma), _p(lt_off), _p(tags), _s(stream)))
+    return lt_off, tags
+
+
+def verify_ragged(ld: torch.Tensor, lt: torch.Tensor, lt_off: torch.Tensor, x: torch.Tensor, L: torch.Tensor,
+                  u_acc: Optional[torch.Tensor], u_res: Optional[torch.Tensor], T: float, *, want_c_star: bool = False,
+                  ld_layout: str = "position", n_acc=None, y_out=None, c_star=None, flags=None, ws=None, stream=None):
+    """verify() with the target logits flattened: lt [rows, V], request b's rows from lt_off[b]."""
+    B, G, V = _bgv(ld, ld_layout)
+    _need(ld, "ld", torch.float32)
+    _need(lt, "lt", torch.float32)
+    if lt.dim() != 2 or lt.shape[1] != V:
+        raise ValueError("lt must be [rows, V]")
+    _need(lt_off, "lt_off", torch.int64, (B + 1,))
+    _need(x, "x", torch.int32, (B, G))
+    _need(L, "L", torch.int32, (B,))
+    if u_acc is not None:
+        _need(u_acc, "u_acc", torch.float32, (B, G))
+    if u_res is not None:
+        _need(u_res, "u_res", torch.float32, (B,))
+    dev = ld.device
+    n_acc = torch.empty(B, dtype=torch.int32, device=dev) if n_acc is None else n_acc
+    y_out = torch.empty((B, G + 1), dtype=torch.int32, device=dev) if y_out is None else y_out
+    if c_star is None and want_c_star:
+        c_star = torch.empty((B, G), dtype=torch.float32, device=dev)
+    flags = torch.zeros(B, dtype=torch.int32, device=dev) if flags is None else flags
+    ws = workspace(WS_VERIFY, B, G, V, 0, dev) if ws is None else ws
+    _need(n_acc, "n_acc", torch.int32, (B,))
+    _need(y_out, "y_out", torch.int32, (B, G + 1))
+    _need(flags, "flags", torch.int32, (B,))
+    if c_star is not None:
+        _need(c_star, "c_star", torch.float32, (B, G))
+    st = lib.dspark_verify_ragged(_p(ld), _p(lt), _p(lt_off), lt.shape[0], _p(x), _p(L), _p(u_acc), _p(u_res), B, G,
+                                  V, float(T), _LAYOUTS[ld_layout], _p(n_acc), _p(y_out), _p(c_star), _p(flags),
+                                  _p(ws), ws.numel(), _s(stream))
+    _check("dspark_verify_ragged", st)
     return n_acc, y_out, c_star, flags
 
 
