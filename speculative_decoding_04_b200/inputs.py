@@ -26,6 +26,8 @@ shapes and value structure stated below:
 * confidences c ~ Beta(a, b) per (request, position), optionally decayed by
   a geometric factor per position.
 * steps/s tables indexed by D, the number of scheduled draft tokens.
+* calibration sets: true pass probabilities q ~ Beta(a, b), accepted counts drawn from them,
+  and over-confident raw confidences c = 1 - (1 - q)^s (s between 1.1 and 1.3 along the block).
 
 Every tensor is drawn from its own Philox stream keyed by
 (workload seed, tensor id[, request]); logits are keyed per request so that a
@@ -40,7 +42,7 @@ from typing import Optional, Tuple
 import numpy as np
 
 # tensor ids for the Philox key
-_T_UEXT, _T_TNOISE, _T_W1, _T_W2, _T_X0, _T_UDRAFT, _T_UACC, _T_URES, _T_CONF, _T_PERM = range(1, 11)
+_T_UEXT, _T_TNOISE, _T_W1, _T_W2, _T_X0, _T_UDRAFT, _T_UACC, _T_URES, _T_CONF, _T_PERM, _T_CALIB = range(1, 12)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -182,6 +184,27 @@ def confidences(wl: Workload) -> np.ndarray:
     c = _rng(wl.seed, _T_CONF).beta(wl.conf_a, wl.conf_b, size=(wl.B, wl.gamma))
     c = c * wl.conf_decay ** np.arange(wl.gamma)[None, :]
     return c.astype(np.float32)
+
+
+def calibration_set(N: int, gamma: int, seed: int, a: float = 5.0, b: float = 2.0,
+                    over: Tuple[float, float] = (1.1, 1.3)) -> Tuple[np.ndarray, np.ndarray]:
+    """A validation set for confidence calibration: (c [N, gamma] fp32 raw confidences,
+    n [N] int32 accepted counts).
+
+    q ~ Beta(a, b) is the true probability that position k of sample i passes given that the
+    positions before it passed; the sample's count n is its number of leading passes
+    (position k passes when a U[0, 1) draw is below q).  The raw confidence overstates q as an
+    over-confident head would: c = 1 - (1 - q)^s_k, with s_k rising linearly along the block
+    from over[0] to over[1].
+    """
+    rng = _rng(seed, _T_CALIB)
+    q = rng.beta(a, b, size=(N, gamma))
+    u = rng.random((N, gamma))
+    passed = np.cumprod(u < q, axis=1)
+    n = passed.sum(axis=1).astype(np.int32)
+    s = np.linspace(over[0], over[1], gamma)[None, :]
+    c = 1.0 - (1.0 - q) ** s
+    return c.astype(np.float32), n
 
 
 def sps_table(wl: Workload, D_max: Optional[int] = None) -> np.ndarray:

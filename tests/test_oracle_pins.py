@@ -591,3 +591,77 @@ def test_ragged_verify_is_the_padded_verify(T):
     for b in range(B):
         k_have = min(int(L[b]) + 1, G)
         assert np.array_equal(c[b, :k_have], full[b, :k_have]) and np.isnan(c[b, k_have:]).all()
+
+
+# --------------------------------------------------------------------------- calibration (STS, ECE)
+
+def test_ece_closed_forms():
+    # one bin, predictions equal to the bin's frequency: 0
+    assert O.ece([0.75] * 4, [1, 1, 1, 0]) == 0.0
+    # bins 1 and 13 (15 bins): (|1 - 0.1| + |0 - 0.9|) / 2
+    assert O.ece([0.1, 0.9], [1, 0]) == pytest.approx(0.9, rel=1e-15)
+    # p = 1 falls in the last bin together with 0.95: |2 - 1.95| / 2
+    assert O.ece([1.0, 0.95], [1, 1]) == pytest.approx(0.025, rel=1e-12)
+    # two bins of 10 bins: (|3 - 4*0.25| + |1 - 2*0.85|) / 6
+    assert O.ece([0.25] * 4 + [0.85] * 2, [1, 1, 1, 0, 1, 0], n_bins=10) == pytest.approx((2.0 + 0.7) / 6, rel=1e-12)
+
+
+def test_ece_matches_the_library_reliability_curve():
+    from sklearn.calibration import calibration_curve
+    rng = np.random.default_rng(61)
+    p = rng.beta(3, 2, 5000)
+    s = (rng.random(5000) < p ** 1.3).astype(np.int64)
+    frac_pos, mean_pred = calibration_curve(s, p, n_bins=15, strategy="uniform")
+    counts = np.bincount(np.minimum((p * 15).astype(int), 14), minlength=15)
+    w = counts[counts > 0] / p.size
+    assert O.ece(p, s) == pytest.approx(float(np.sum(w * np.abs(frac_pos - mean_pred))), rel=1e-12)
+
+
+def test_temperature_scaling_closed_forms_and_order():
+    # logit(0.8) = ln 4; halved: ln 2 -> 2/3
+    assert float(O.sts_scale(0.8, 2.0)) == pytest.approx(2.0 / 3.0, rel=1e-15)
+    assert float(O.sts_scale(0.2, 0.5)) == pytest.approx(1.0 / 17.0, rel=1e-14)   # logit -ln 4 doubled
+    c = np.array([0.0, 1e-6, 0.3, 0.5, 0.9, 1.0, np.nan, 1.5, -0.2])
+    for tau in (0.3, 1.0, 2.7):
+        out = O.sts_scale(c, tau)
+        assert out[0] == 0.0 and out[5] == 1.0 and out[3] == 0.5 and out[6] == 0.0
+        assert out[7] == 1.0 and out[8] == 0.0                          # clamped into [0, 1]
+        assert np.all(np.diff(out[:6]) > 0)                             # order kept
+    assert np.allclose(O.sts_scale(c[:6], 1.0), c[:6], rtol=1e-15, atol=0)
+
+
+def _logit_overconfident(N, scales, seed):
+    from scipy.special import expit, logit
+    rng = np.random.default_rng(seed)
+    G = len(scales)
+    q = rng.beta(4, 2, size=(N, G))
+    n = np.cumprod(rng.random((N, G)) < q, axis=1).sum(axis=1)
+    c = expit(logit(q) * np.asarray(scales)[None, :])
+    return c, n
+
+
+def test_sts_recovers_known_temperatures_position_by_position():
+    # confidences miscalibrated by a known temperature per position (over-, under-, over-
+    # confident): the fit recovers each one, which it can only do if position k is fitted on
+    # top of the calibrated positions before it
+    scales = [2.0, 0.5, 1.5]
+    c, n = _logit_overconfident(200_000, scales, 62)
+    grid = np.exp(np.linspace(np.log(0.25), np.log(4.0), 81))
+    r = O.sts_fit(c, n, grid)
+    assert np.all(np.abs(np.log(r["tau"]) - np.log(scales)) < 0.08), r["tau"]
+    assert np.all(r["ece_cal"] < 0.01) and np.all(r["ece_cal"] < r["ece_raw"])
+    assert np.all(r["curves"][np.arange(3), r["index"]] == r["ece_cal"])
+    # following a grid value that is not the minimum is refused
+    with pytest.raises(ValueError):
+        O.sts_fit(c, n, grid, follow=[0, 0, 0])
+
+
+def test_sts_on_the_synthetic_validation_set():
+    # the pages: ECE of 3-8 % before calibration, about 1 % after
+    from speculative_decoding_04_b200 import inputs
+    c, n = inputs.calibration_set(40_000, 8, 5)
+    grid = np.exp(np.linspace(np.log(0.25), np.log(4.0), 81))
+    r = O.sts_fit(c, n, grid)
+    assert np.all((r["ece_raw"] > 0.02) & (r["ece_raw"] < 0.08))
+    assert np.all(r["ece_cal"] < 0.02) and np.mean(r["ece_cal"]) < 0.013
+    assert np.all(r["tau"] > 1.0)                                       # over-confident: flattened
