@@ -294,6 +294,65 @@ def draft_crossover(args):
         torch.cuda.empty_cache()
 
 
+def calibration(args):
+    """Sequential temperature scaling: sts_fit on a validation set of N = 1,000,000 samples, gamma = 16,
+    81 grid temperatures, 15 bins (CUDA events, median of --steps after --warmup), the oracle's
+    sts_fit on a 20,000-sample slice of it (one run), and sts_apply on the high-concurrency
+    round's [64, 16] confidences."""
+    import torch
+
+    from speculative_decoding_04_b200 import build
+    build.build()
+    from speculative_decoding_04_b200 import dspark as D
+    from speculative_decoding_04_b200 import inputs
+
+    dev = torch.device("cuda")
+    N, G, M = 1_000_000, 16, 15
+    grid_h = np.exp(np.linspace(np.log(0.25), np.log(4.0), 81))
+    c_h, n_h = inputs.calibration_set(N, G, seed=11)
+    c, n, grid = (torch.from_numpy(v).to(dev) for v in (c_h, n_h, grid_h))
+    ws = torch.empty(D.lib.dspark_sts_workspace_size(N, G, grid.numel(), M), dtype=torch.uint8, device=dev)
+    ev = []
+    for i in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        out = D.sts_fit(c, n, grid, M, ws=ws)
+        e1.record()
+        if i >= args.warmup:
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    fit_ms = median_ms(ev)
+    evals = N * G * (grid.numel() + 1)
+    rc = inputs.confidences(inputs.HIGH_CONCURRENCY)
+    rcd = torch.from_numpy(rc).to(dev)
+    ev = []
+    for i in range(args.warmup + args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        D.sts_apply(rcd, out["tau"])
+        e1.record()
+        if i >= args.warmup:
+            ev.append((e0, e1))
+    torch.cuda.synchronize()
+    apply_ms = median_ms(ev)
+    import oracle as O
+    cpu_n = 20_000
+    t0 = time.perf_counter()
+    O.sts_fit(c_h[:cpu_n], n_h[:cpu_n], grid_h, M)
+    cpu_s = time.perf_counter() - t0
+    line = {"metric": "sts_fit (sample, position, temperature) evaluations/s", "value": evals / (fit_ms * 1e-3),
+            "unit": "evaluations/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": fit_ms,
+            "higher_is_better": True, "dtype": "f64", "data": "synthetic (inputs.calibration_set)",
+            "config": {"workload": f"validation set N={N}, gamma={G}, {grid.numel()} grid temperatures, {M} bins"},
+            "ece_raw_pct": [round(100 * v, 3) for v in out["ece_raw"].tolist()],
+            "ece_cal_pct": [round(100 * v, 3) for v in out["ece_cal"].tolist()],
+            "tau": [round(v, 4) for v in out["tau"].tolist()],
+            "sts_apply_us": apply_ms * 1e3, "gpu_launches": 2 * G + 1,
+            "cpu_baseline": {"value": cpu_n * G * (grid.numel() + 1) / cpu_s, "unit": "evaluations/s", "cores": 1,
+                             "kind": "oracle", "sample": f"oracle sts_fit on the first {cpu_n} samples, one run"}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -307,6 +366,8 @@ def main():
                     help="TV labels in the verify call (auto: on, except on scheduled_step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle timing (after the GPU timing)")
     ap.add_argument("--draft-crossover", action="store_true", help="print draft times of both main-pass paths over B")
+    ap.add_argument("--calibration", action="store_true",
+                    help="time sequential temperature scaling (sts_fit, sts_apply) instead of the round")
     ap.add_argument("--layout", choices=["position", "request"], default="position",
                     help="layout of the draft logits U and of ld: position-major [gamma, B, V] (default) or "
                          "request-major [B, gamma, V]")
@@ -315,6 +376,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     if args.draft_crossover:
         return draft_crossover(args)
+    if args.calibration:
+        return calibration(args)
 
     wl = workload_of(args.workload)
     labels = (args.labels == "on") or (args.labels == "auto" and not uses_schedule_table(wl))

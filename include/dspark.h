@@ -283,6 +283,42 @@ int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, 
                      float T, int ld_layout, float* c_star, void* stream);
 
 /* --------------------------------------------------------------------------
+ * dspark_sts_fit -- sequential temperature scaling of the confidences, fitted on a validation set.
+ *
+ * [P1 §"硬件感知与置信度自适应调度机制"] the raw confidence head is over-confident; on a
+ * validation set a 1-D grid search per candidate position finds the temperature that
+ * calibrates it (expected calibration error from 3-8 % to about 1 %); temperature scaling
+ * keeps the order of the confidences.  [P3 §Confidence-Scheduled Verification] STS
+ * calibrates the cumulative product position by position.  Reading taken:
+ *     scaled(c, tau) = sigma(logit(c) / tau)      (fp64; c clamped to [0, 1], NaN as 0)
+ *     for k = 0 .. gamma-1, in order:
+ *       s_i      = 1 if n_acc[i] >= k + 1 (sample i's positions 0..k all accepted), else 0
+ *       a'_i(t)  = prod_{j<k} scaled(c[i,j], tau[j]) * scaled(c[i,k], t)
+ *       ECE(t)   = sum over M equal-width bins of |sum_{i in bin} (s_i - a'_i(t))| / N
+ *                  (bin of p: min(floor(p M), M - 1))
+ *       tau[k]   = grid[j] for the first j minimising ECE(grid[j])
+ *     ece_raw[k] is the ECE of the raw products prod_{j<=k} c[i,j].
+ * c          [N, gamma] fp32 raw confidences.    n_acc  [N] int32 accepted counts.
+ * grid       [n_grid] fp64 candidate temperatures (> 0).
+ * tau_out    [gamma] fp64 (required);  index_out [gamma] int32, ece_raw / ece_cal [gamma] fp64,
+ *            curve_out [gamma, n_grid] fp64 (ECE of every candidate) -- each may be NULL.
+ * ws         dspark_sts_workspace_size(N, gamma, n_grid, n_bins) bytes, 256-byte aligned.
+ * Limits: gamma <= 64, (n_grid + 1) * n_bins <= 25600.  2 * gamma launches on `stream`.
+ * fp64 sums in atomic order: ECE values agree with a serial sum to about 1e-15.
+ * -------------------------------------------------------------------------- */
+size_t dspark_sts_workspace_size(int64_t N, int gamma, int n_grid, int n_bins);
+int dspark_sts_fit(const float* c, const int32_t* n_acc, int64_t N, int gamma, const double* grid, int n_grid,
+                   int n_bins, double* tau_out, int32_t* index_out, double* ece_raw, double* ece_cal,
+                   double* curve_out, void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_sts_apply -- calibrated confidences of a round: c_out[b,k] = fp32(scaled(c[b,k], tau[k]))
+ * (the scaling of dspark_sts_fit, rounded once to fp32), ready for dspark_prefix_schedule.
+ * c, c_out [B, gamma] fp32 (may be the same array);  tau [gamma] fp64.  No workspace.
+ * -------------------------------------------------------------------------- */
+int dspark_sts_apply(const float* c, const double* tau, int B, int gamma, float* c_out, void* stream);
+
+/* --------------------------------------------------------------------------
  * dspark_prefix_schedule -- prefix survival + greedy hardware-aware prefix scheduler.
  *
  * [P3 §Confidence-Scheduled Verification] a_{b,j} = ∏_{i<=j} c_{b,i} and

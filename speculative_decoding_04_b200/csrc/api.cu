@@ -214,6 +214,32 @@ int dspark_verify_ragged(const float* ld, const float* lt, const int64_t* lt_off
   return launch_verify(c);
 }
 
+size_t dspark_sts_workspace_size(int64_t N, int gamma, int n_grid, int n_bins) {
+  if (N < 1 || gamma < 1 || n_grid < 1 || n_bins < 1) return 0;
+  return sts_workspace_bytes((long long)N, gamma, n_grid, n_bins);
+}
+
+int dspark_sts_fit(const float* c, const int32_t* n_acc, int64_t N, int gamma, const double* grid, int n_grid,
+                   int n_bins, double* tau_out, int32_t* index_out, double* ece_raw, double* ece_cal,
+                   double* curve_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!c || !n_acc || !grid || !tau_out || !ws) return einval("dspark_sts_fit: null pointer");
+  if (N < 1 || gamma < 1 || gamma > kMaxGamma) return einval("dspark_sts_fit: N >= 1, gamma in [1, 64]");
+  if (n_grid < 1 || n_bins < 1) return einval("dspark_sts_fit: n_grid and n_bins must be >= 1");
+  if ((size_t)(n_grid + 1) * (size_t)n_bins * 8 > kStsMaxHistBytes)
+    return einval("dspark_sts_fit: (n_grid + 1) * n_bins must be <= 25600");
+  if (ws_bytes < sts_workspace_bytes((long long)N, gamma, n_grid, n_bins)) return einval("dspark_sts_fit: workspace too small");
+  if ((uintptr_t)ws % 256) return einval("dspark_sts_fit: workspace must be 256-byte aligned");
+  StsCall sc{c, n_acc, (long long)N, gamma, n_grid, n_bins, grid, tau_out, index_out, ece_raw, ece_cal, curve_out, ws,
+             (cudaStream_t)stream};
+  return launch_sts_fit(sc);
+}
+
+int dspark_sts_apply(const float* c, const double* tau, int B, int gamma, float* c_out, void* stream) {
+  if (!c || !tau || !c_out) return einval("dspark_sts_apply: null pointer");
+  if (B < 1 || gamma < 1 || gamma > kMaxGamma) return einval("dspark_sts_apply: B >= 1, gamma in [1, 64]");
+  return launch_sts_apply(c, tau, B, gamma, c_out, (cudaStream_t)stream);
+}
+
 int dspark_tv_labels(const float* ld, const float* lt, int B, int gamma, int V, int lt_rows, float T, int ld_layout,
                      float* c_star, void* stream) {
   if (!ld || !lt || !c_star) return einval("dspark_tv_labels: null pointer");

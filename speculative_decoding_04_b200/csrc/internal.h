@@ -83,6 +83,25 @@ struct VerifyCall {
   long long lt_nrows = 0;           // rows of the flattened l_t
 };
 
+struct StsCall {
+  const float* c;
+  const int32_t* n_acc;
+  long long N;
+  int gamma, n_grid, n_bins;
+  const double* grid;
+  double* tau;
+  int32_t* index;
+  double* ece_raw;
+  double* ece_cal;
+  double* curve;
+  void* ws;
+  cudaStream_t stream;
+};
+size_t sts_workspace_bytes(long long N, int gamma, int n_grid, int n_bins);
+dspark_status launch_sts_fit(const StsCall& c);
+dspark_status launch_sts_apply(const float* c, const double* tau, int B, int gamma, float* out, cudaStream_t stream);
+constexpr size_t kStsMaxHistBytes = 200 * 1024;  // (n_grid + 1) * n_bins fp64 sums in shared memory
+
 dspark_status launch_ragged_layout(const int32_t* L, int B, int gamma, int64_t* lt_off, int32_t* tags,
                                    cudaStream_t stream);
 

@@ -75,6 +75,12 @@ def _load() -> ctypes.CDLL:
     lib.dspark_tv_labels.argtypes = [_vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp]
     lib.dspark_prefix_schedule.restype = _i
     lib.dspark_prefix_schedule.argtypes = [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_sts_workspace_size.restype = _sz
+    lib.dspark_sts_workspace_size.argtypes = [ctypes.c_int64, _i, _i, _i]
+    lib.dspark_sts_fit.restype = _i
+    lib.dspark_sts_fit.argtypes = [_vp, _vp, ctypes.c_int64, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_sts_apply.restype = _i
+    lib.dspark_sts_apply.argtypes = [_vp, _vp, _i, _i, _vp, _vp]
     lib.dspark_ragged_layout.restype = _i
     lib.dspark_ragged_layout.argtypes = [_vp, _i, _i, _vp, _vp, _vp]
     lib.dspark_verify_ragged.restype = _i
@@ -225,6 +231,40 @@ def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torc
                            _p(y_out), _p(c_star), _p(flags), _p(ws), ws.numel(), _s(stream))
     _check("dspark_verify", st)
     return n_acc, y_out, c_star, flags
+
+
+def sts_fit(c: torch.Tensor, n_acc: torch.Tensor, grid: torch.Tensor, n_bins: int = 15, *, want_curve: bool = False,
+            ws=None, stream=None):
+    """Sequential temperature scaling on a validation set (c [N, gamma] fp32, n_acc [N] int32,
+    grid [J] fp64); returns dict(tau, index, ece_raw, ece_cal, curve or None) of device tensors."""
+    N, G = c.shape
+    _need(c, "c", torch.float32)
+    _need(n_acc, "n_acc", torch.int32, (N,))
+    _need(grid, "grid", torch.float64)
+    J = grid.numel()
+    dev = c.device
+    out = {"tau": torch.empty(G, dtype=torch.float64, device=dev),
+           "index": torch.empty(G, dtype=torch.int32, device=dev),
+           "ece_raw": torch.empty(G, dtype=torch.float64, device=dev),
+           "ece_cal": torch.empty(G, dtype=torch.float64, device=dev),
+           "curve": torch.empty((G, J), dtype=torch.float64, device=dev) if want_curve else None}
+    if ws is None:
+        ws = torch.empty(max(1, lib.dspark_sts_workspace_size(N, G, J, n_bins)), dtype=torch.uint8, device=dev)
+    st = lib.dspark_sts_fit(_p(c), _p(n_acc), N, G, _p(grid), J, int(n_bins), _p(out["tau"]), _p(out["index"]),
+                            _p(out["ece_raw"]), _p(out["ece_cal"]), _p(out["curve"]), _p(ws), ws.numel(), _s(stream))
+    _check("dspark_sts_fit", st)
+    return out
+
+
+def sts_apply(c: torch.Tensor, tau: torch.Tensor, *, c_out=None, stream=None) -> torch.Tensor:
+    """Calibrated confidences fp32(sigma(logit(c) / tau[k])) of a [B, gamma] round."""
+    B, G = c.shape
+    _need(c, "c", torch.float32)
+    _need(tau, "tau", torch.float64, (G,))
+    c_out = torch.empty_like(c) if c_out is None else c_out
+    _need(c_out, "c_out", torch.float32, (B, G))
+    _check("dspark_sts_apply", lib.dspark_sts_apply(_p(c), _p(tau), B, G, _p(c_out), _s(stream)))
+    return c_out
 
 
 def ragged_layout(L: torch.Tensor, gamma: int, *, lt_off=None, tags=None, want_tags: bool = True, stream=None):
