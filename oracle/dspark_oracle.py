@@ -17,6 +17,9 @@ What each function follows:
                   Markov head B(x_{k-1}, ·) = W1[x_{k-1}] W2 of low rank r;
                   P1 §"DSpark 架构设计：半自回归生成与马尔可夫修正" (one previous
                   token only, positions filled left to right).
+  * rnn_draft  -- P1 §"DSpark 架构设计：半自回归生成与马尔可夫修正" (the optional RNN head: a
+                  hidden state updated over the drafted prefix); P3 §Semi-Autoregressive
+                  Generation (B_k(x_<k, v); RNN head with a recurrent state in the block).
   * verify     -- P1 §"大模型推理的显存瓶颈与推测解码的演进逻辑" (rejection
                   sampling: accept the longest prefix, resample at the first
                   rejection, drop the rest) and P3 opening paragraph (longest
@@ -61,6 +64,8 @@ Readings where the pages leave a step open:
   * ties in the survival sort: survival descending, then request, then position.
   * ARGMAX mode takes the smallest D attaining max Θ (global search);
     EARLY_STOP takes the first D with Θ(D+1) ≤ Θ(D).
+  * RNN head: the pages give no form; here h_k = tanh(W1[x_{k-1}] + h_{k-1} W_h) (rank r,
+    h_{-1} = 0) and the bias is h_k W2, so that W_h = 0 is the Markov head on tanh(W1).
   * flattened verification: request b owns target rows off[b] .. off[b] + L_b of one
     packed [Σ(L_b+1), V] array (off = exclusive prefix sum of L_b + 1); its tag is
     b·(γ+1) + k; it is verified exactly as the padded block; TV labels exist for the
@@ -160,26 +165,17 @@ def draft_step(U_k, W1, W2, prev, u, T: float, W2_64: Optional[np.ndarray] = Non
     return x, ld32, alts
 
 
-def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None, near: float = NEAR_TIE):
-    """The γ sequential Markov-head steps for every request.
-
-    U [B, γ, V] fp32, x0 [B], u_draft [B, γ].  Step k uses the token chosen at
-    step k-1 (x0 for the first step).  Returns (x [B, γ] int32,
-    ld [B, γ, V] fp32, alts) where alts[(b, k)] lists the valid tokens at a
-    near-tie.  `follow` maps (b, k) to a token that must be one of the valid
-    alternatives at that step; the chain then continues from it (used to
-    follow one branch of a near-tie).  `near` is the near-tie window.
-    """
+def _sequential_draft(U, bias_of, x0, u_draft, T: float, follow: Optional[Dict], near: float):
+    """The γ left-to-right sampling steps shared by both heads: step k stores
+    ℓ_d = fl32(U_k + bias_of(k, previous tokens)) and samples x_k from it."""
     U = np.asarray(U, dtype=np.float32)
     B, G, V = U.shape
-    W1 = np.asarray(W1)
-    W2_64 = np.asarray(W2).astype(np.float64)
     x = np.zeros((B, G), dtype=np.int32)
     ld = np.zeros((B, G, V), dtype=np.float32)
     alts = {}
     prev = np.asarray(x0, dtype=np.int64).copy()
     for k in range(G):
-        bias = markov_bias(W1, W2_64, prev)                      # [B, V] fp64
+        bias = bias_of(k, prev)                                   # [B, V] fp64
         ld[:, k] = (U[:, k].astype(np.float64) + bias).astype(np.float32)
         for b in range(B):
             if T == 0.0:
@@ -196,6 +192,52 @@ def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None
             x[b, k] = xk
         prev = x[:, k].astype(np.int64)
     return x, ld, alts
+
+
+def markov_draft(U, W1, W2, x0, u_draft, T: float, follow: Optional[Dict] = None, near: float = NEAR_TIE):
+    """The γ sequential Markov-head steps for every request.
+
+    U [B, γ, V] fp32, x0 [B], u_draft [B, γ].  Step k uses the token chosen at
+    step k-1 (x0 for the first step).  Returns (x [B, γ] int32,
+    ld [B, γ, V] fp32, alts) where alts[(b, k)] lists the valid tokens at a
+    near-tie.  `follow` maps (b, k) to a token that must be one of the valid
+    alternatives at that step; the chain then continues from it (used to
+    follow one branch of a near-tie).  `near` is the near-tie window.
+    """
+    W1 = np.asarray(W1)
+    W2_64 = np.asarray(W2).astype(np.float64)
+    return _sequential_draft(U, lambda k, prev: markov_bias(W1, W2_64, prev), x0, u_draft, T, follow, near)
+
+
+def rnn_state(W1, Wh, prev, h_prev) -> np.ndarray:
+    """h_k = tanh(W1[x_{k-1}] + h_{k-1} · W_h) in fp64 (row vectors; h before the block is 0)."""
+    return np.tanh(np.asarray(W1)[np.asarray(prev)].astype(np.float64) + h_prev @ np.asarray(Wh).astype(np.float64))
+
+
+def rnn_draft(U, W1, W2, Wh, x0, u_draft, T: float, follow: Optional[Dict] = None, near: float = NEAR_TIE):
+    """The γ sequential steps with the recurrent head instead of the Markov head.
+
+    P1 §DSpark 架构设计：半自回归生成与马尔可夫修正 (the optional RNN head keeps and updates a
+    hidden state over the whole drafted prefix); P3 §Semi-Autoregressive Generation
+    (p_k(v) ∝ exp(U_k(v) + B_k(x_<k, v)), RNN head: a recurrent state inside the block).
+    Reading: a state h_k of the Markov head's rank r, h_k = tanh(W1[x_{k-1}] + h_{k-1} W_h)
+    with h_{-1} = 0 and x_{-1} = x0, and B_k = h_k W2 (the Markov head's projections; W_h = 0
+    gives the Markov head on tanh(W1)).  Returns (x, ld, alts, h [B, γ, r] fp64).
+    """
+    W1 = np.asarray(W1)
+    Wh = np.asarray(Wh)
+    W2_64 = np.asarray(W2).astype(np.float64)
+    B = np.asarray(U).shape[0]
+    hs = []
+    state = {"h": np.zeros((B, W1.shape[1]))}
+
+    def bias_of(k, prev):
+        state["h"] = rnn_state(W1, Wh, prev, state["h"])
+        hs.append(state["h"])
+        return state["h"] @ W2_64
+
+    x, ld, alts = _sequential_draft(U, bias_of, x0, u_draft, T, follow, near)
+    return x, ld, alts, np.stack(hs, axis=1)
 
 
 # --------------------------------------------------------------------------- verification

@@ -665,3 +665,58 @@ def test_sts_on_the_synthetic_validation_set():
     assert np.all((r["ece_raw"] > 0.02) & (r["ece_raw"] < 0.08))
     assert np.all(r["ece_cal"] < 0.02) and np.mean(r["ece_cal"]) < 0.013
     assert np.all(r["tau"] > 1.0)                                       # over-confident: flattened
+
+
+# --------------------------------------------------------------------------- RNN head
+
+def test_rnn_head_hand_example():
+    # V = 2, r = 2, greedy with token 0 far ahead everywhere, so x_k = 0 throughout:
+    #   h_0 = tanh(W1[0]),  h_k = tanh(W1[0] + h_{k-1} Wh)  (row vector times Wh, Wh not symmetric)
+    #   l_d[k] = U[k] + h_k W2
+    W1 = np.array([[0.5, -0.25], [0.1, 0.3]])
+    Wh = np.array([[0.8, -0.4], [0.3, 0.6]])
+    W2 = np.array([[1.0, -1.0], [0.5, 2.0]])
+    U = np.zeros((1, 3, 2), dtype=np.float32)
+    U[0, :, 0] = 10.0
+    x, ld, _, h = O.rnn_draft(U, W1, W2, Wh, np.array([0]), np.zeros((1, 3)), 0.0)
+    assert x.tolist() == [[0, 0, 0]]
+    hk = [math.tanh(0.5), math.tanh(-0.25)]
+    for k in range(3):
+        if k:
+            hk = [math.tanh(0.5 + hk[0] * 0.8 + hk[1] * 0.3), math.tanh(-0.25 + hk[0] * -0.4 + hk[1] * 0.6)]
+        assert h[0, k].tolist() == pytest.approx(hk, rel=1e-15)
+        want = [10.0 + hk[0] * 1.0 + hk[1] * 0.5, hk[0] * -1.0 + hk[1] * 2.0]
+        assert ld[0, k].tolist() == pytest.approx(np.float32(want).tolist(), rel=0, abs=0)
+
+
+def test_rnn_head_without_recurrence_is_the_markov_head_on_tanh_embeddings():
+    rng = np.random.default_rng(71)
+    B, G, V, r = 5, 4, 300, 8
+    U = rng.normal(0, 1.0, (B, G, V)).astype(np.float32)
+    W1 = rng.normal(0, 0.8, (V, r))
+    W2 = rng.normal(0, 0.5, (r, V))
+    x0 = rng.integers(0, V, B)
+    u = rng.random((B, G)).astype(np.float32)
+    for T in (1.0, 0.0):
+        x, ld, _, _ = O.rnn_draft(U, W1, W2, np.zeros((r, r)), x0, u, T)
+        xm, ldm, _ = O.markov_draft(U, np.tanh(W1), W2, x0, u, T)
+        assert np.array_equal(x, xm) and np.array_equal(ld, ldm)
+
+
+def test_rnn_head_sees_the_whole_prefix():
+    # the same token at position 0 after different starting tokens: the Markov head's logits at
+    # position 1 agree, the recurrent head's do not (its state still carries x0)
+    rng = np.random.default_rng(72)
+    V, r = 50, 6
+    W1 = rng.normal(0, 0.8, (V, r))
+    W2 = rng.normal(0, 0.5, (r, V))
+    Wh = rng.normal(0, 0.5, (r, r))
+    U = np.zeros((2, 2, V), dtype=np.float32)
+    U[:, 0, 7] = 50.0                                              # position 0 drafts token 7 in both
+    x0 = np.array([3, 11])
+    u = np.full((2, 2), 0.5, dtype=np.float32)
+    x, ld, _, _ = O.rnn_draft(U, W1, W2, Wh, x0, u, 1.0)
+    assert x[0, 0] == x[1, 0] == 7
+    assert not np.allclose(ld[0, 1], ld[1, 1])
+    xm, ldm, _ = O.markov_draft(U, W1, W2, x0, u, 1.0)
+    assert np.array_equal(ldm[0, 1], ldm[1, 1])
