@@ -62,7 +62,7 @@ enum { DSPARK_POSITION_MAJOR = 0, DSPARK_REQUEST_MAJOR = 1 };
 enum { DSPARK_SCHED_ARGMAX = 0, DSPARK_SCHED_EARLY_STOP = 1 };
 
 /* workspace kinds for dspark_workspace_size */
-enum { DSPARK_WS_DRAFT = 0, DSPARK_WS_VERIFY = 1, DSPARK_WS_SCHEDULE = 2 };
+enum { DSPARK_WS_DRAFT = 0, DSPARK_WS_VERIFY = 1, DSPARK_WS_SCHEDULE = 2, DSPARK_WS_RNN_DRAFT = 3 };
 
 /* bits of flags[b] */
 #define DSPARK_FLAG_DRAFT_NEAR_TIE    (1u << 0) /* |u - F| < 1e-6 at the drafted token, or greedy top-2 gap <= 1e-6*max(1,|z|) */
@@ -158,6 +158,28 @@ int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dt
                         int B, int gamma, int V, int r, float T, int layout,
                         int32_t* x_out, float* ld_out, uint32_t* flags,
                         void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * dspark_rnn_draft -- the draft stage with the recurrent (RNN) head instead of the Markov head.
+ *
+ * [P1 §"DSpark 架构设计：半自回归生成与马尔可夫修正"] the optional RNN head keeps and updates a
+ * hidden state that accumulates the whole drafted prefix (the pages find its small accuracy gain
+ * not worth the cost and keep the Markov head in production); [P3 §Semi-Autoregressive
+ * Generation] p_k(v) ∝ exp(U_k(v) + B_k(x_<k, v)) with a recurrent state inside the block.
+ * The pages give no functional form.  Reading taken (rank r, as the Markov head):
+ *     h_{-1} = 0,  x_{-1} = x0,  h_k = tanh(W1[x_{k-1}] + h_{k-1} W_h),  l_d[k] = U_k + h_k W2
+ * so that W_h = 0 is the Markov head on tanh(W1).  The state is fp32 and the whole stage runs
+ * on the CUDA-core pass (one state kernel, one main pass and one combine per position); the
+ * fused tensor-core launch is not used (it would round the state to bf16).
+ * Wh      [r, r] in w_dtype, row i multiplies h[i].
+ * h_out   [B, gamma, r] fp32 device or NULL: the states h_k.
+ * ws      dspark_workspace_size(DSPARK_WS_RNN_DRAFT, B, gamma, V, r) bytes.
+ * Other arguments, outputs, flags and limits as dspark_markov_draft; r <= 1024.
+ * -------------------------------------------------------------------------- */
+int dspark_rnn_draft(const float* U, const void* W1, const void* W2, const void* Wh, int w_dtype,
+                     const int32_t* x0, const float* u_draft, int B, int gamma, int V, int r, float T, int layout,
+                     int32_t* x_out, float* ld_out, float* h_out, uint32_t* flags,
+                     void* ws, size_t ws_bytes, void* stream);
 
 /* --------------------------------------------------------------------------
  * dspark_verify -- lossless rejection-sampling verification of the drafted block.

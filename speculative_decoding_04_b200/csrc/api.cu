@@ -134,6 +134,7 @@ size_t dspark_workspace_size(int which, int B, int gamma, int V, int r) {
     case DSPARK_WS_DRAFT: return draft_workspace_bytes(B, gamma, V, r);
     case DSPARK_WS_VERIFY: return verify_workspace_bytes(B, gamma, V);
     case DSPARK_WS_SCHEDULE: return 0;
+    case DSPARK_WS_RNN_DRAFT: return rnn_draft_workspace_bytes(B, gamma, V, r);
     default: return 0;
   }
 }
@@ -166,6 +167,28 @@ int dspark_markov_draft(const float* U, const void* W1, const void* W2, int w_dt
   if ((uintptr_t)ws % 256) return einval("dspark_markov_draft: workspace must be 256-byte aligned");
   DraftCall c{U, W1, W2, w_dtype, x0, u_draft, B, gamma, V, r, T, layout, x_out, ld_out, flags, ws, ws_bytes,
               (cudaStream_t)stream};
+  return launch_draft(c);
+}
+
+int dspark_rnn_draft(const float* U, const void* W1, const void* W2, const void* Wh, int w_dtype, const int32_t* x0,
+                     const float* u_draft, int B, int gamma, int V, int r, float T, int layout, int32_t* x_out,
+                     float* ld_out, float* h_out, uint32_t* flags, void* ws, size_t ws_bytes, void* stream) {
+  if (!U || !W1 || !W2 || !Wh || !x0 || !x_out || !ld_out || !flags || !ws) return einval("dspark_rnn_draft: null pointer");
+  if (T != 0.f && !u_draft) return einval("dspark_rnn_draft: u_draft is required when T > 0");
+  if (B <= 0 || V < 2 || r <= 0) return einval("dspark_rnn_draft: B, r must be >= 1 and V >= 2");
+  if (r > 1024) return einval("dspark_rnn_draft: r must be <= 1024");
+  if (gamma < 1 || gamma > kMaxGamma) return einval("dspark_rnn_draft: gamma must be in [1, 64]");
+  if (!(T >= 0.f) || std::isinf(T)) return einval("dspark_rnn_draft: T must be finite and >= 0");
+  if (w_dtype != DSPARK_BF16 && w_dtype != DSPARK_F32) return einval("dspark_rnn_draft: w_dtype must be DSPARK_BF16 or DSPARK_F32");
+  if (layout != DSPARK_POSITION_MAJOR && layout != DSPARK_REQUEST_MAJOR)
+    return einval("dspark_rnn_draft: layout must be DSPARK_POSITION_MAJOR or DSPARK_REQUEST_MAJOR");
+  if ((long long)B * gamma * V >= (1ll << 40)) return einval("dspark_rnn_draft: tensor too large");
+  if (ws_bytes < rnn_draft_workspace_bytes(B, gamma, V, r)) return einval("dspark_rnn_draft: workspace too small");
+  if ((uintptr_t)ws % 256) return einval("dspark_rnn_draft: workspace must be 256-byte aligned");
+  DraftCall c{U, W1, W2, w_dtype, x0, u_draft, B, gamma, V, r, T, layout, x_out, ld_out, flags, ws, ws_bytes,
+              (cudaStream_t)stream};
+  c.Wh = Wh;
+  c.h_out = h_out;
   return launch_draft(c);
 }
 

@@ -45,6 +45,9 @@ struct DraftArgs {
   int rm;                // 1: request-major U / l_d ([B][gamma][V]; tensor maps {V, gamma, B})
   uint32_t spin_limit;   // polls before a bounded wait gives up
   int barrier_extra;     // test-only: arrivals the first grid barrier expects beyond the grid
+  const void* Wh;        // recurrent head: [r][r] state matrix, or null (Markov head)
+  float* hstate;         // recurrent head: [B][r] fp32 state h_k of the step being drafted
+  float* h_out;          // recurrent head: [B][gamma][r] copy of every state, or null
   int B, gamma, V, r, nchunk;
   float inv_T;
   int greedy;
@@ -176,7 +179,9 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
   for (int i = tid; i < BG * r; i += blockDim.x) {
     const int bb = i / r, kk = i - bb * r;
     float g = 0.f;
-    if (bb < nb) g = wload<WT>(a.W1, (size_t)prev_token(a, b0 + bb, k, kk == 0) * r + kk);
+    if (bb < nb)
+      g = a.hstate ? a.hstate[(size_t)(b0 + bb) * r + kk]  // recurrent head: the state h_k
+                   : wload<WT>(a.W1, (size_t)prev_token(a, b0 + bb, k, kk == 0) * r + kk);
     G[i] = g;
   }
   __syncthreads();
@@ -253,6 +258,34 @@ __global__ void __launch_bounds__(128) draft_main_fma(DraftArgs a, int k, int ve
     ChunkStat acc = s_stat[0][tid];
     for (int q = 1; q < 8; ++q) stat_fold(acc, s_stat[q][tid], a.greedy);
     a.cpart[(size_t)blockIdx.x * a.B + b0 + tid] = acc;
+  }
+}
+
+// ============================================================================ recurrent head state
+//
+// [P1 §DSpark 架构设计：半自回归生成与马尔可夫修正: the optional RNN head keeps a hidden state over
+//  the whole drafted prefix; P3 §Semi-Autoregressive Generation: B_k(x_<k, v) from a recurrent
+//  state inside the block]  The pages give no form; the state here has the Markov head's rank r:
+//      h_k = tanh(W1[x_{k-1}] + h_{k-1} W_h),  h_{-1} = 0,  x_{-1} = x0,   bias_k = h_k W2,
+// in fp32 (the contraction over W_h sums i = 0..r-1 in order with fused multiply-adds).  One CTA
+// per request, one thread per state element; the main pass then reads h_k where the Markov head
+// reads W1[x_{k-1}].  The state stays fp32 on the CUDA-core pass (the tensor-core pass would
+// have to round it to bf16 for its operand).
+
+template <typename WT>
+__global__ void __launch_bounds__(256) rnn_state_kernel(DraftArgs a, int k) {
+  extern __shared__ float hp[];  // [r]: h_{k-1}
+  const int b = blockIdx.x, r = a.r;
+  float* h = a.hstate + (size_t)b * r;
+  for (int j = threadIdx.x; j < r; j += blockDim.x) hp[j] = k == 0 ? 0.f : h[j];
+  __syncthreads();  // every read of this request's state precedes the writes below
+  const int prev = prev_token(a, b, k, threadIdx.x == 0);
+  for (int j = threadIdx.x; j < r; j += blockDim.x) {
+    float pre = wload<WT>(a.W1, (size_t)prev * r + j);
+    for (int i = 0; i < r; ++i) pre = fmaf(hp[i], wload<WT>(a.Wh, (size_t)i * r + j), pre);
+    const float hj = tanhf(pre);
+    h[j] = hj;
+    if (a.h_out) a.h_out[((size_t)b * a.gamma + k) * r + j] = hj;
   }
 }
 
@@ -1142,6 +1175,10 @@ size_t draft_workspace_bytes(int B, int gamma, int V, int r) {
   return kWsHeader + align_up((size_t)B * np_max * sizeof(ChunkStat), 256) + align_up((size_t)B * r * 2, 256);
 }
 
+size_t rnn_draft_workspace_bytes(int B, int gamma, int V, int r) {
+  return draft_workspace_bytes(B, gamma, V, r) + align_up((size_t)B * r * 4, 256);
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -1244,14 +1281,21 @@ dspark_status launch_draft(const DraftCall& c) {
   }
   a.greedy = (c.T == 0.f) ? 1 : 0;
   a.inv_T = a.greedy ? 1.f : 1.f / c.T;
-  const bool pdl = opt.draft_pdl != 0;
+  const bool rnn = c.Wh != nullptr;
+  if (rnn) {  // the recurrent head: CUDA-core pass, one state kernel before each step
+    a.Wh = c.Wh;
+    a.hstate = reinterpret_cast<float*>(static_cast<uint8_t*>(c.ws) + draft_workspace_bytes(c.B, c.gamma, c.V, c.r));
+    a.h_out = c.h_out;
+    a.gbuf = nullptr;
+  }
+  const bool pdl = opt.draft_pdl != 0 && !rnn;
 
   const bool aligned16 = ((uintptr_t)c.W1 % 16 == 0) && ((uintptr_t)c.W2 % 16 == 0) && ((uintptr_t)c.U % 16 == 0) &&
                          ((uintptr_t)c.ld_out % 16 == 0);
   const bool tc_ok = c.w_dtype == DSPARK_BF16 && c.r % 64 == 0 && c.r <= 256 && c.V % 8 == 0 && aligned16;
-  bool use_tc = tc_ok && c.B >= opt.draft_tc_min_b;
+  bool use_tc = tc_ok && c.B >= opt.draft_tc_min_b && !rnn;
   if (opt.draft_force_path == 1) use_tc = false;
-  if (opt.draft_force_path == 2) {
+  if (opt.draft_force_path == 2 && !rnn) {
     if (!tc_ok) {
       set_error("tensor-core draft path forced but the shape or dtype does not allow it");
       return DSPARK_ENOTIMPL;
@@ -1348,6 +1392,18 @@ dspark_status launch_draft(const DraftCall& c) {
     // The first main pass waits for everything before the call in full: its producers read U
     // and W2 before the grid-dependency wait, which is only safe behind this call's own kernels.
     const bool pdl_k = pdl && k > 0;
+    if (rnn) {
+      const int thr = std::min(256, (c.r + 31) / 32 * 32);
+      if (c.w_dtype == DSPARK_BF16)
+        rnn_state_kernel<__nv_bfloat16><<<c.B, thr, (size_t)c.r * 4, c.stream>>>(a, k);
+      else
+        rnn_state_kernel<float><<<c.B, thr, (size_t)c.r * 4, c.stream>>>(a, k);
+      rc = cudaGetLastError();
+      if (rc != cudaSuccess) {
+        set_error(std::string("recurrent state launch: ") + cudaGetErrorString(rc));
+        return DSPARK_ECUDA;
+      }
+    }
     if (use_tc) {
       const dim3 grid(cpg * n_bgroups), block(kTcThreads);
       if (nb == 32)

@@ -58,6 +58,8 @@ struct DraftCall {
   void* ws;
   size_t ws_bytes;
   cudaStream_t stream;
+  const void* Wh = nullptr;  // recurrent head: [r][r] state matrix (null: the Markov head)
+  float* h_out = nullptr;    // recurrent head: [B][gamma][r] fp32 states, or null
 };
 
 struct VerifyCall {
@@ -133,6 +135,7 @@ struct ScheduleCall {
 };
 
 size_t draft_workspace_bytes(int B, int gamma, int V, int r);
+size_t rnn_draft_workspace_bytes(int B, int gamma, int V, int r);
 size_t verify_workspace_bytes(int B, int gamma, int V);
 size_t verify_rows_workspace_bytes(int B, int gamma);
 

@@ -24,7 +24,7 @@ F32, BF16 = 0, 1
 POSITION_MAJOR, REQUEST_MAJOR = 0, 1
 _LAYOUTS = {"position": POSITION_MAJOR, "request": REQUEST_MAJOR}
 SCHED_ARGMAX, SCHED_EARLY_STOP = 0, 1
-WS_DRAFT, WS_VERIFY, WS_SCHEDULE = 0, 1, 2
+WS_DRAFT, WS_VERIFY, WS_SCHEDULE, WS_RNN_DRAFT = 0, 1, 2, 3
 T2_RING_BYTES = 128
 
 FLAG_DRAFT_NEAR_TIE = 1 << 0
@@ -75,6 +75,9 @@ def _load() -> ctypes.CDLL:
     lib.dspark_tv_labels.argtypes = [_vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp]
     lib.dspark_prefix_schedule.restype = _i
     lib.dspark_prefix_schedule.argtypes = [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.dspark_rnn_draft.restype = _i
+    lib.dspark_rnn_draft.argtypes = [_vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp, _vp, _vp, _vp, _vp,
+                                     _sz, _vp]
     lib.dspark_sts_workspace_size.restype = _sz
     lib.dspark_sts_workspace_size.argtypes = [ctypes.c_int64, _i, _i, _i]
     lib.dspark_sts_fit.restype = _i
@@ -196,6 +199,42 @@ def markov_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, x0: torch.
                                  ws.numel(), _s(stream))
     _check("dspark_markov_draft", st)
     return x_out, ld_out, flags
+
+
+def rnn_draft(U: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, Wh: torch.Tensor, x0: torch.Tensor,
+              u_draft: Optional[torch.Tensor], T: float, *, layout: str = "position", want_h: bool = False,
+              x_out=None, ld_out=None, h_out=None, flags=None, ws=None, stream=None):
+    """Draft with the recurrent head; returns (x [B, gamma], l_d in the layout of U, h [B, gamma, r]
+    or None, flags [B])."""
+    B, G, V = _bgv(U, layout)
+    r = W1.shape[1]
+    _need(U, "U", torch.float32)
+    if W1.dtype not in (torch.bfloat16, torch.float32) or W2.dtype != W1.dtype or Wh.dtype != W1.dtype:
+        raise ValueError("W1, W2 and Wh must all be bf16 or all fp32")
+    _need(W1, "W1", W1.dtype, (V, r))
+    _need(W2, "W2", W1.dtype, (r, V))
+    _need(Wh, "Wh", W1.dtype, (r, r))
+    _need(x0, "x0", torch.int32, (B,))
+    if u_draft is not None:
+        _need(u_draft, "u_draft", torch.float32, (B, G))
+    dev = U.device
+    x_out = torch.empty((B, G), dtype=torch.int32, device=dev) if x_out is None else x_out
+    ld_out = torch.empty(U.shape, dtype=torch.float32, device=dev) if ld_out is None else ld_out
+    if h_out is None and want_h:
+        h_out = torch.empty((B, G, r), dtype=torch.float32, device=dev)
+    flags = torch.zeros(B, dtype=torch.int32, device=dev) if flags is None else flags
+    ws = workspace(WS_RNN_DRAFT, B, G, V, r, dev) if ws is None else ws
+    _need(x_out, "x_out", torch.int32, (B, G))
+    _need(ld_out, "ld_out", torch.float32, tuple(U.shape))
+    _need(flags, "flags", torch.int32, (B,))
+    if h_out is not None:
+        _need(h_out, "h_out", torch.float32, (B, G, r))
+    wdt = BF16 if W1.dtype == torch.bfloat16 else F32
+    st = lib.dspark_rnn_draft(_p(U), _p(W1), _p(W2), _p(Wh), wdt, _p(x0), _p(u_draft), B, G, V, r, float(T),
+                              _LAYOUTS[layout], _p(x_out), _p(ld_out), _p(h_out), _p(flags), _p(ws), ws.numel(),
+                              _s(stream))
+    _check("dspark_rnn_draft", st)
+    return x_out, ld_out, h_out, flags
 
 
 def verify(ld: torch.Tensor, lt: torch.Tensor, x: torch.Tensor, L: Optional[torch.Tensor],
