@@ -28,8 +28,13 @@ roofline    = the draft stage (its one launch) against measured HBM copy bandwid
 cpu_baseline= the CPU oracle on the machine's host cores: its request-independent and per-request
               costs timed separately on small samples and combined for the whole batch
 
+graph_t2    = the round captured once as a CUDA graph with the asynchronous (t-2) scheduler and
+              replayed, L2 flushed between replays
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+                  [--layout position|request] [--labels auto|on|off]
   python bench.py --draft-crossover     # draft time on the GEMV and tensor-core paths over B
+  python bench.py --calibration         # sequential temperature scaling: fit and apply timings
 """
 
 import argparse

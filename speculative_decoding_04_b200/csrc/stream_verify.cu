@@ -1137,8 +1137,12 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   if (c.V % 4 || (uintptr_t)c.ld % 16 || (uintptr_t)c.lt % 16) return DSPARK_ENOTIMPL;
   const SvLayout Ly = sv_layout(c.B, c.gamma, c.V);
   if (c.ws_bytes < Ly.total) return DSPARK_ENOTIMPL;
+  // clusters of 3 (45 clusters on 148 SMs) stream many rows best; with fewer than about 1.3 rows
+  // per cluster, clusters of 6 spread each row over more SMs (measured on a B200: 39.0 -> 32.8 us
+  // at B = 1, gamma = 7; 129.1 -> 122.9 us at B = 32, gamma = 4; 341 -> 388 us at B = 64,
+  // gamma = 16, where 3 stays)
   int C = opt.verify_stream_cluster;
-  if (C < 1 || C > kSvMaxCluster) C = 3;
+  if (C < 1 || C > kSvMaxCluster) C = ((long long)c.B * (c.gamma + 1) * 3 < (long long)device_sm_count() * 4) ? 6 : 3;
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   SvArgs a{};
   a.ld = c.ld;

@@ -32,5 +32,5 @@ def _default_options():
         D.set_option("debug_wait_limit", 0)
         D.set_option("debug_unreachable_barrier", 0)
         D.set_option("verify_groups", 0)
-        D.set_option("verify_stream_cluster", 3)
+        D.set_option("verify_stream_cluster", 0)
         D.set_option("verify_stream_l2hint", 1)
