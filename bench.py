@@ -371,6 +371,9 @@ def main():
                     help="TV labels in the verify call (auto: on, except on scheduled_step)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle timing (after the GPU timing)")
     ap.add_argument("--draft-crossover", action="store_true", help="print draft times of both main-pass paths over B")
+    ap.add_argument("--ragged", action="store_true",
+                    help="target logits as a flattened block of the scheduled rows (sum of L_b + 1 rows) and the "
+                         "flattened verify")
     ap.add_argument("--calibration", action="store_true",
                     help="time sequential temperature scaling (sts_fit, sts_apply) instead of the round")
     ap.add_argument("--layout", choices=["position", "request"], default="position",
@@ -429,6 +432,18 @@ def main():
         del U, lt, Uh
     sps_h = inputs.sps_table(wr) if uses_schedule_table(wl) else np.ones(B * G + 1)
     sps = torch.from_numpy(sps_h).to(dev)
+    lt_off = None
+    if args.ragged:
+        # the target block as a target forward over the scheduled tokens would emit it: rows
+        # 0..L_b of each request, flattened (the schedule is deterministic for these inputs)
+        L0 = torch.empty(B, dtype=torch.int32, device=dev)
+        D.prefix_schedule(dv["c"], sps, B * G, L_out=L0, want_a=False)
+        L0h = L0.cpu().numpy()
+        rows = np.concatenate([b * (G + 1) + np.arange(int(l) + 1) for b, l in enumerate(L0h)])
+        dv["lt"] = dv["lt"].view(B * (G + 1), V).index_select(0, torch.from_numpy(rows).to(dev)).contiguous()
+        host_logit_bytes = (B * G * V + dv["lt"].shape[0] * V) * 4
+        lt_off = torch.empty(B + 1, dtype=torch.int64, device=dev)
+        torch.cuda.synchronize(dev)
     x = torch.empty((B, G), dtype=torch.int32, device=dev)
     ld = torch.empty(tuple(dv["U"].shape), dtype=torch.float32, device=dev)
     fl = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -444,17 +459,25 @@ def main():
     # draft: one cooperative launch on the tensor-core path, else a main pass and a combine per
     # position; schedule; verify: main kernel + finalize
     tc = wl.w_dtype == "bf16" and r % 64 == 0 and r <= 256 and V % 8 == 0
-    n_launch = (1 if tc else 2 * G) + 1 + 2
+    n_launch = (1 if tc else 2 * G) + 1 + 2 + (1 if args.ragged else 0)
 
     def draft(src):
         D.markov_draft(src["U"], W1, W2, src["x0"], src["u_draft"], wl.T, layout=args.layout, x_out=x, ld_out=ld,
                        flags=fl, ws=ws_d, stream=stream)
 
+    def verify_call(src):
+        if args.ragged:
+            D.ragged_layout(L, G, lt_off=lt_off, want_tags=False, stream=stream)
+            D.verify_ragged(ld, src["lt"], lt_off, x, L, src["u_acc"], src["u_res"], wl.T, ld_layout=args.layout,
+                            n_acc=n_acc, y_out=y, c_star=c_star, flags=fl, ws=ws_v, stream=stream)
+        else:
+            D.verify(ld, src["lt"], x, L, src["u_acc"], src["u_res"], wl.T, ld_layout=args.layout, n_acc=n_acc,
+                     y_out=y, c_star=c_star, flags=fl, ws=ws_v, stream=stream)
+
     def schedule_and_verify(src):
         D.prefix_schedule(src["c"], sps, B * G, D.SCHED_ARGMAX, L_out=L, theta_out=theta, flags=fl, want_a=False,
                           stream=stream)
-        D.verify(ld, src["lt"], x, L, src["u_acc"], src["u_res"], wl.T, ld_layout=args.layout, n_acc=n_acc, y_out=y,
-                 c_star=c_star, flags=fl, ws=ws_v, stream=stream)
+        verify_call(src)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -500,8 +523,7 @@ def main():
             flush.fill_(float(i))
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            D.verify(ld, dv["lt"], x, L, dv["u_acc"], dv["u_res"], wl.T, ld_layout=args.layout, n_acc=n_acc, y_out=y,
-                     c_star=c_star, flags=fl, ws=ws_v, stream=stream)
+            verify_call(dv)
             e1.record(stream)
             vt.append((e0, e1))
         barrier()
@@ -536,23 +558,25 @@ def main():
             D.verify(ld, src["lt"], x, L, src["u_acc"], src["u_res"], wl.T, ld_layout=args.layout, n_acc=n_acc,
                      y_out=y, c_star=c_star, flags=fl, ws=ws_v, stream=stream)
 
-        round_t2(dv)
-        barrier()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=stream):
+        graph_ms = None
+        if not args.ragged:   # (the t-2 schedule's lengths are not the ones the flattened block holds)
             round_t2(dv)
-        gt = []
-        for i in range(args.warmup + args.steps):
-            flush.fill_(float(i))
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            graph.replay()
-            e1.record(stream)
-            if i >= args.warmup:
-                gt.append((e0, e1))
-        barrier()
-        graph_ms = median_ms(gt)
-        del graph
+            barrier()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                round_t2(dv)
+            gt = []
+            for i in range(args.warmup + args.steps):
+                flush.fill_(float(i))
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                if i >= args.warmup:
+                    gt.append((e0, e1))
+            barrier()
+            graph_ms = median_ms(gt)
+            del graph
 
         # end to end through the public API with pinned host buffers
         e2e = None
@@ -601,7 +625,9 @@ def main():
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": f"synthetic (seeded log-Zipf + Gaussian logits, "
                                                          f"{wl.w_dtype} weights)",
-            "config": config_of(wl, world, labels, args.layout),
+            "config": dict(config_of(wl, world, labels, args.layout),
+                           lt_layout=("flattened [sum(L_b + 1), V] with row offsets" if args.ragged
+                                      else "padded [B, gamma + 1, V]")),
             "verified_tokens_per_s": accepted_all / (args.steps * t_step),
             "tokens_per_request_per_round": tau,
             "latency_per_token_us": (t_draft + t_verify) / tau * 1e6,
@@ -623,7 +649,7 @@ def main():
                                 "algorithmic_bytes": verify_b},
             "warm_l2": {"ms_per_step": warm_step_ms, "draft_ms": warm_draft_ms, "rounds_per_s": 1e3 / warm_step_ms},
             "back_to_back": b2b,
-            "graph_t2": {"ms_per_round": graph_ms, "rounds_per_s": 1e3 / graph_ms,
+            "graph_t2": None if graph_ms is None else {"ms_per_round": graph_ms, "rounds_per_s": 1e3 / graph_ms,
                          "round": "markov_draft -> prefix_schedule_t2 (capacity from step t-2, device ring) -> "
                                   "verify, captured once as a CUDA graph and replayed; L2 flushed between replays"},
             "e2e": ({"value": world / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
