@@ -7,10 +7,11 @@
 //  accepted tokens x hardware speed keeps rising; the global search runs on the GPU]
 //
 // One CTA of 1024 threads: running products per request (fp32, left to right), 64-bit keys
-// (survival descending, then flat index b*gamma + j) sorted bitonically in shared memory with
-// warp shuffles for the short strides, an fp64 block scan of the sorted survivals giving
-// Θ(D) = (B + S(D)) * sps[D] for D = 0..D_max, the ARGMAX / EARLY_STOP choice, and per-request
-// counts of the kept items.
+// (survival descending, then flat index b*gamma + j), sorted in shared memory -- by a bottom-up
+// merge of the requests' runs when every confidence lies in [0, 1] (each run is then already
+// sorted), else bitonically with warp shuffles for the short strides --, an fp64 block scan of
+// the sorted survivals giving Θ(D) = (B + S(D)) * sps[D] for D = 0..D_max, the ARGMAX /
+// EARLY_STOP choice, and per-request counts of the kept items.
 //
 // Asynchronous variant ([P1 §硬件感知与置信度自适应调度机制, last paragraph: the truncation of
 // step t is decided from the confidence history of step t-2, so the global search stays inside
@@ -30,11 +31,13 @@ namespace dspark {
 
 constexpr int kSchedThreads = 1024;
 constexpr int kSchedWarps = kSchedThreads / 32;
+constexpr int kMergeMaxKeys = 8192;  // two key buffers of 64 KB
 
 struct SchedArgs {
   const float* c;
   const double* sps;
   int B, gamma, D_max, mode, P;
+  int P2;  // second key buffer for the merge sort (0: bitonic sort only)
   int32_t* L_out;
   float* a_out;
   double* theta_out;
@@ -61,7 +64,10 @@ __device__ __forceinline__ float key_value(uint64_t key) {
 
 __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s) {
   extern __shared__ __align__(16) uint64_t keys[];
-  int* cnt = reinterpret_cast<int*>(keys + s.P);
+  uint64_t* keys2 = keys + s.P;  // [P2]
+  int* cnt = reinterpret_cast<int*>(keys + s.P + s.P2);
+  __shared__ double sh_pre[kSchedWarps];
+  __shared__ double sh_tot;
   __shared__ double sh_w[kSchedWarps];
   __shared__ double sh_best[kSchedWarps];
   __shared__ int sh_bestD[kSchedWarps];
@@ -90,6 +96,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
   float* cs = reinterpret_cast<float*>(keys);  // N floats fit in the first N/2 keys
   for (int i = tid; i < N; i += kSchedThreads) cs[i] = s.c[i];
   __syncthreads();
+  int any_bad = 0;
   for (int b = tid; b < B; b += kSchedThreads) {
     float prod = 1.f;
     bool bad = false;
@@ -100,9 +107,12 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
       cs[b * G + j] = prod;
     }
     if (bad && s.flags) atomicOr(s.flags + b, DSPARK_FLAG_CONF_RANGE);
+    any_bad |= bad ? 1 : 0;
     cnt[b] = 0;
   }
-  __syncthreads();
+  // with every confidence in [0, 1] each request's survivals are non-increasing (an fp32 product
+  // with a factor <= 1 never exceeds the other factor), so its keys already form a sorted run
+  const bool runs_sorted = __syncthreads_or(any_bad) == 0;
   constexpr int kMaxPer = kMaxScheduleItems / kSchedThreads;
   float av[kMaxPer];
 #pragma unroll
@@ -119,38 +129,68 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
   }
   __syncthreads();
 
-  // ---------------------------------------------------------------- bitonic sort (ascending)
-  for (int k = 2; k <= P; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      if (j >= 32 || P < 64) {
-        for (int i = tid; i < P; i += kSchedThreads) {
-          const int ixj = i ^ j;
-          if (ixj > i) {
-            const uint64_t x = keys[i], y = keys[ixj];
-            const bool up = (i & k) == 0;
-            if ((x > y) == up) {
-              keys[i] = y;
-              keys[ixj] = x;
+  // ---------------------------------------------------------------- sort (ascending keys)
+  // Sorted runs (every confidence in [0, 1]) and room for a second buffer: a bottom-up merge of
+  // the B runs of gamma keys, each key placed at its run position plus its rank in the partner
+  // run (a binary search; keys are distinct, so the merge keeps b ascending on equal survivals).
+  // Otherwise a bitonic sort of all P keys in place.
+  const uint64_t* ks = keys;
+  if (runs_sorted && s.P2 > 0) {
+    uint64_t* src = keys;
+    uint64_t* dst = keys2;
+    for (int w = G; w < N; w <<= 1) {
+      for (int e = tid; e < N; e += kSchedThreads) {
+        const int r = e / w, pos = e - r * w;
+        const int pstart = (r ^ 1) * w;
+        const int plen = max(0, min(pstart + w, N) - pstart);
+        const uint64_t x = src[e];
+        int lo = 0, hi = plen;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (src[pstart + mid] < x) lo = mid + 1;
+          else hi = mid;
+        }
+        dst[(r & ~1) * w + pos + lo] = x;
+      }
+      __syncthreads();
+      uint64_t* t = src;
+      src = dst;
+      dst = t;
+    }
+    ks = src;
+  } else {
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        if (j >= 32 || P < 64) {
+          for (int i = tid; i < P; i += kSchedThreads) {
+            const int ixj = i ^ j;
+            if (ixj > i) {
+              const uint64_t x = keys[i], y = keys[ixj];
+              const bool up = (i & k) == 0;
+              if ((x > y) == up) {
+                keys[i] = y;
+                keys[ixj] = x;
+              }
             }
           }
-        }
-        __syncthreads();
-      } else {
-        // strides 16..1 stay inside a warp: 32 consecutive keys per warp pass
-        for (int base = warp * 32; base < P; base += kSchedThreads) {
-          const int i = base + lane;
-          uint64_t x = keys[i];
-          for (int jj = j; jj > 0; jj >>= 1) {
-            const uint64_t y = __shfl_xor_sync(0xffffffffu, x, jj);
-            const bool up = (i & k) == 0;
-            const bool lower = (lane & jj) == 0;
-            const uint64_t mn = x < y ? x : y, mx = x < y ? y : x;
-            x = (lower == up) ? mn : mx;
+          __syncthreads();
+        } else {
+          // strides 16..1 stay inside a warp: 32 consecutive keys per warp pass
+          for (int base = warp * 32; base < P; base += kSchedThreads) {
+            const int i = base + lane;
+            uint64_t x = keys[i];
+            for (int jj = j; jj > 0; jj >>= 1) {
+              const uint64_t y = __shfl_xor_sync(0xffffffffu, x, jj);
+              const bool up = (i & k) == 0;
+              const bool lower = (lane & jj) == 0;
+              const uint64_t mn = x < y ? x : y, mx = x < y ? y : x;
+              x = (lower == up) ? mn : mx;
+            }
+            keys[i] = x;
           }
-          keys[i] = x;
+          __syncthreads();
+          break;  // all strides below 32 handled
         }
-        __syncthreads();
-        break;  // all strides below 32 handled
       }
     }
   }
@@ -158,6 +198,24 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
   // ---------------------------------------------------------------- Θ pass (twice: choose, then tie check)
   // The sorted survivals are scanned in chunks of kSchedThreads items; item i moves D from
   // i to i+1, so the thread owning it sees Θ(i) and Θ(i+1).
+  // Block-wide scan step: the sum of the earlier warps' totals (plus the carry of earlier
+  // chunks) for this thread's warp; the carry grows by the chunk's total.
+  auto block_prefix = [&](double incl, double& carry_io) -> double {
+    if (lane == 31) sh_w[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const double v = sh_w[lane];
+      const double inc = warp_incl_scan_d(v);
+      double ex = __shfl_up_sync(0xffffffffu, inc, 1);
+      if (lane == 0) ex = 0.0;
+      sh_pre[lane] = ex;
+      if (lane == 31) sh_tot = inc;
+    }
+    __syncthreads();
+    const double wpre = carry_io + sh_pre[warp];
+    carry_io += sh_tot;
+    return wpre;
+  };
   const double theta0 = (double)B * s.sps[0];
   double best = theta0;
   int bestD = 0;
@@ -169,18 +227,11 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
     const double th_star = pass ? s_theta : 0.0;
     for (int base = 0; base < Dm; base += kSchedThreads) {
       const int i = base + tid;
-      const double ai = (i < Dm) ? (double)key_value(keys[i]) : 0.0;
+      const double ai = (i < Dm) ? (double)key_value(ks[i]) : 0.0;
       const double incl = warp_incl_scan_d(ai);
       double excl = __shfl_up_sync(0xffffffffu, incl, 1);
       if (lane == 0) excl = 0.0;
-      if (lane == 31) sh_w[warp] = incl;
-      __syncthreads();
-      double wpre = carry;
-      for (int w = 0; w < warp; ++w) wpre += sh_w[w];
-      double tot = carry;
-      for (int w = 0; w < kSchedWarps; ++w) tot += sh_w[w];
-      __syncthreads();
-      carry = tot;
+      const double wpre = block_prefix(incl, carry);
       if (i < Dm) {
         const double th_lo = ((double)B + (wpre + excl)) * s.sps[i];      // Θ(i)
         const double th_hi = ((double)B + (wpre + incl)) * s.sps[i + 1];  // Θ(i+1)
@@ -242,16 +293,9 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
         double carry2 = 0.0;
         for (int base = 0; base < max(Ds, 1); base += kSchedThreads) {
           const int i = base + tid;
-          const double ai = (i < Ds) ? (double)key_value(keys[i]) : 0.0;
+          const double ai = (i < Ds) ? (double)key_value(ks[i]) : 0.0;
           const double incl = warp_incl_scan_d(ai);
-          if (lane == 31) sh_w[warp] = incl;
-          __syncthreads();
-          double wpre = carry2;
-          for (int w = 0; w < warp; ++w) wpre += sh_w[w];
-          double tot = carry2;
-          for (int w = 0; w < kSchedWarps; ++w) tot += sh_w[w];
-          __syncthreads();
-          carry2 = tot;
+          const double wpre = block_prefix(incl, carry2);
           if (i == Ds - 1) s_theta = ((double)B + (wpre + incl)) * s.sps[Ds];
         }
         if (Ds == 0 && tid == 0) s_theta = theta0;
@@ -274,7 +318,7 @@ __global__ void __launch_bounds__(kSchedThreads, 1) schedule_kernel(SchedArgs s)
   // ---------------------------------------------------------------- counts and outputs
   // synchronous mode keeps the first D* items; asynchronous mode the first K_t (= D*_{t-2})
   const int Ds = s.ring ? s_K : s_D;
-  for (int i = tid; i < Ds; i += kSchedThreads) atomicAdd(&cnt[(int)(uint32_t)keys[i] / G], 1);
+  for (int i = tid; i < Ds; i += kSchedThreads) atomicAdd(&cnt[(int)(uint32_t)ks[i] / G], 1);
   __syncthreads();
   const bool near = s.ring ? s_tieK != 0 : sh_tie[0] != 0;
   for (int b = tid; b < B; b += kSchedThreads) {
@@ -308,6 +352,7 @@ dspark_status launch_schedule(const ScheduleCall& c) {
   int P = 64;
   while (P < c.B * c.gamma) P <<= 1;
   s.P = P;
+  s.P2 = P <= kMergeMaxKeys ? P : 0;  // a second key buffer fits in shared memory
   s.L_out = c.L_out;
   s.a_out = c.a_out;
   s.theta_out = c.theta_out;
@@ -315,7 +360,7 @@ dspark_status launch_schedule(const ScheduleCall& c) {
   s.ring = c.ring;
   s.K_init = c.K_init;
   s.K_out = c.K_out;
-  const size_t smem = (size_t)P * 8 + align_up((size_t)c.B * 4, 16);
+  const size_t smem = (size_t)(P + s.P2) * 8 + align_up((size_t)c.B * 4, 16);
   cudaError_t rc;
   if (smem > 48 * 1024) {
     rc = ensure_smem_attr((const void*)schedule_kernel, smem);
