@@ -89,3 +89,29 @@ def test_confidence_out_of_range_is_flagged():
     c = np.array([[0.5, 1.5], [0.2, 0.3], [-0.1, 0.9]], dtype=np.float32)
     L, a, th, fl = run(c, np.ones(7), 6)
     assert [bool(f & D.FLAG_CONF_RANGE) for f in fl] == [True, False, True]
+
+
+@pytest.mark.parametrize("B,G", [(512, 16), (300, 7), (1, 9)])
+def test_merged_runs_with_ties(B, G):
+    # every confidence in [0, 1]: the kernel merges the requests' sorted runs (up to 8192 keys);
+    # identical rows and exact 1.0 / 0.0 confidences make equal survivals across requests
+    rng = np.random.default_rng(B + G)
+    c = rng.beta(5, 2, size=(B, G)).astype(np.float32)
+    c[::5] = 0.75
+    c[1::9, 0] = 1.0
+    c[2::11, G // 2] = 0.0
+    sps = 1.0 / (0.005 + 0.00004 * (B + np.arange(B * G + 1)))
+    check(c, sps, B * G)
+    check(c, sps, (B * G) // 4, 1)
+
+
+def test_unsorted_runs_take_the_bitonic_sort():
+    # confidences above 1 make survivals rise along a request: the order must still be the
+    # oracle's (survival descending, then request, then position)
+    rng = np.random.default_rng(9)
+    B, G = 64, 16
+    c = rng.uniform(0.2, 1.3, size=(B, G)).astype(np.float32)
+    sps = 1.0 / (0.005 + 0.00004 * (B + np.arange(B * G + 1)))
+    L, th, r = check(c, sps, B * G)
+    fl = run(c, sps, B * G)[3]
+    assert np.any(fl & D.FLAG_CONF_RANGE)
