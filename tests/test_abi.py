@@ -112,3 +112,45 @@ def test_binding_refuses_cpu_tensors():
     W = torch.zeros(8, 2)
     with pytest.raises(ValueError):
         D.markov_draft(U, W, W.t().contiguous(), torch.zeros(1, dtype=torch.int32), None, 0.0)
+
+
+@no_gpu
+def test_new_entry_points_argument_checks():
+    # asynchronous (t-2) scheduler: ring required and 8-byte aligned; the same limits as the
+    # synchronous scheduler
+    t2 = D.lib.dspark_prefix_schedule_t2
+    assert t2(FAKE, FAKE, 2, 4, 8, 0, -1, None, FAKE, None, FAKE, None, None, None) == D.EINVAL
+    assert t2(FAKE, FAKE, 2, 4, 8, 0, -1, ctypes.c_void_p(4100), FAKE, None, FAKE, None, None, None) == D.EINVAL
+    assert "aligned" in D.last_error()
+    assert t2(FAKE, FAKE, 2, 4, 9, 0, -1, FAKE, FAKE, None, FAKE, None, None, None) == D.EINVAL
+    assert t2(FAKE, FAKE, 2, 4, 8, 3, -1, FAKE, FAKE, None, FAKE, None, None, None) == D.EINVAL
+    # flattened verify: lengths and offsets required, at least one row
+    vr = D.lib.dspark_verify_ragged
+    ws = ctypes.c_void_p(4096 * 256)
+    args = [FAKE, FAKE, FAKE, 10, FAKE, FAKE, FAKE, FAKE, 4, 4, 1024, 1.0, 0, FAKE, FAKE, None, FAKE, ws, 1 << 30, None]
+    for i, bad in ((5, None), (2, None), (3, 0), (12, 2), (11, -1.0)):
+        a = list(args)
+        a[i] = bad
+        assert vr(*a) == D.EINVAL, i
+    assert D.lib.dspark_ragged_layout(None, 4, 4, FAKE, None, None) == D.EINVAL
+    assert D.lib.dspark_ragged_layout(FAKE, 4, 65, FAKE, None, None) == D.EINVAL
+    # calibration
+    assert D.lib.dspark_sts_workspace_size(0, 4, 8, 15) == 0
+    assert D.lib.dspark_sts_workspace_size(100, 4, 8, 15) >= 2 * 100 * 8 + 4 * 9 * 15 * 8
+    fit = D.lib.dspark_sts_fit
+    big = ctypes.c_void_p(4096 * 256)
+    assert fit(FAKE, FAKE, 100, 4, FAKE, 8, 15, None, None, None, None, None, big, 1 << 30, None) == D.EINVAL
+    assert fit(FAKE, FAKE, 100, 4, FAKE, 2000, 15, FAKE, None, None, None, None, big, 1 << 30, None) == D.EINVAL
+    assert "25600" in D.last_error()
+    assert fit(FAKE, FAKE, 100, 4, FAKE, 8, 15, FAKE, None, None, None, None, big, 16, None) == D.EINVAL
+    assert D.lib.dspark_sts_apply(FAKE, None, 4, 4, FAKE, None) == D.EINVAL
+    assert D.lib.dspark_sts_apply(FAKE, FAKE, 4, 65, FAKE, None) == D.EINVAL
+    # recurrent draft head: state matrix required, rank <= 1024
+    rd = D.lib.dspark_rnn_draft
+    a = [FAKE, FAKE, FAKE, FAKE, D.BF16, FAKE, FAKE, 4, 4, 1024, 16, 1.0, 0, FAKE, FAKE, None, FAKE,
+         ctypes.c_void_p(4096 * 256), 1 << 30, None]
+    for i, bad in ((3, None), (10, 1025), (4, 7), (12, 5), (18, 64)):
+        b = list(a)
+        b[i] = bad
+        assert rd(*b) == D.EINVAL, i
+    assert D.workspace_size(D.WS_RNN_DRAFT, 4, 4, 1024, 16) == D.workspace_size(D.WS_DRAFT, 4, 4, 1024, 16) + 256
