@@ -1076,31 +1076,67 @@ __device__ void combine_warp(const DraftArgs& a, int k, int b, uint32_t* gready)
           const int q = blk + 32 * i + lane;
           v[i] = q < nq4 ? __ldcg(row4 + q) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (pk >= 0 || blk + 32 * i >= nq4) break;  // warp-uniform
-          const int e0 = (blk + 32 * i + lane) * 4;   // first column (relative to v0) of this lane's quad
-          const float l4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-          double we[4], wl = 0.0;
+        // weights of this lane's quads: element weight exp(z - M), 0 outside the partition
+        auto quad_w = [&](const float4& q4, int e0, double (&we)[4]) -> double {
+          const float l4[4] = {q4.x, q4.y, q4.z, q4.w};
+          double wl = 0.0;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const float z = __fmul_rn(l4[c], inv_T);
             we[c] = (e0 + c < n && z != -INFINITY) ? (double)ex_shift(z, M) : 0.0;
             wl += we[c];
           }
-          const double incl2 = warp_incl_scan_d(wl);
-          const double tot = __shfl_sync(FULL, incl2, 31);
-          const unsigned pos = __ballot_sync(FULL, wl > 0.0);
-          if (pos) lastq = blk + 32 * i + 31 - __clz(pos);  // the last quad with weight so far
-          if (base + tot > t) {
+          return wl;
+        };
+        // chunk totals eight at a time: the eight butterflies interleave, and the chunk holding
+        // u*S is found from the totals before any scan inside a chunk
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (pk >= 0 || blk + 32 * 8 * h >= nq4) break;  // warp-uniform
+          double T[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            double we[4];
+            T[i] = quad_w(v[8 * h + i], (blk + 32 * (8 * h + i) + lane) * 4, we);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) T[i] += __shfl_xor_sync(FULL, T[i], o);
+          int cs = -1;
+          double cbase = base;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (T[i] > 0.0) lastq = blk + 32 * (8 * h + i);  // a chunk with weight (refined below)
+            if (cs < 0 && base + T[i] > t && T[i] > 0.0) {
+              cs = i;
+              cbase = base;
+            }
+            base += T[i];
+          }
+          if (cs >= 0) {
             // the chunk holds u*S: the first lane whose running sum passes it, then its element
-            const unsigned hit = __ballot_sync(FULL, wl > 0.0 && base + incl2 > t);
-            if (hit) {
-              const int hl = __ffs(hit) - 1;
+            float4 vc = v[8 * h];
+#pragma unroll
+            for (int i = 1; i < 8; ++i)
+              if (i == cs) vc = v[8 * h + i];
+            const int e0 = (blk + 32 * (8 * h + cs) + lane) * 4;
+            double we[4];
+            const double wl = quad_w(vc, e0, we);
+            const double incl2 = warp_incl_scan_d(wl);
+            unsigned hitl = __ballot_sync(FULL, wl > 0.0 && cbase + incl2 > t);
+            bool edge = false;
+            if (!hitl) {  // the totals and the scan round differently: the chunk's last weight
+              hitl = __ballot_sync(FULL, wl > 0.0);
+              hitl = hitl ? (1u << (31 - __clz(hitl))) : 0u;
+              edge = true;
+            }
+            if (hitl) {
+              const int hl = __ffs(hitl) - 1;
               if (lane == hl) {
-                double R = base + incl2 - wl;
+                double R = cbase + incl2 - wl;
                 for (int c = 0; c < 4; ++c) {
-                  if (we[c] > 0.0 && t < R + we[c]) {
+                  if (!edge && we[c] > 0.0 && t < R + we[c]) {
                     pk = e0 + c;
                     qlo = R;
                     qhi = R + we[c];
@@ -1119,8 +1155,25 @@ __device__ void combine_warp(const DraftArgs& a, int k, int b, uint32_t* gready)
               qhi = __shfl_sync(FULL, qhi, hl);
             }
           }
-          base += tot;
         }
+      }
+      if (pk < 0 && lastq >= 0) {
+        // rounding left u*S past the partition: the last quad with weight in the last chunk that
+        // has any (one warp-wide pass over that chunk)
+        const int q = lastq + lane;
+        const float4 q4 = q < nq4 ? __ldcg(row4 + q) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        double we[4];
+        const unsigned pos = __ballot_sync(FULL, [&] {
+          const float l4[4] = {q4.x, q4.y, q4.z, q4.w};
+          bool any = false;
+          for (int c = 0; c < 4; ++c) {
+            const float z = __fmul_rn(l4[c], inv_T);
+            we[c] = (q * 4 + c < n && z != -INFINITY) ? (double)ex_shift(z, M) : 0.0;
+            any |= we[c] > 0.0;
+          }
+          return any;
+        }());
+        lastq = pos ? lastq + 31 - __clz(pos) : -1;
       }
       if (pk < 0 && lastq >= 0) {
         // rounding left u*S past the partition: its last element with weight, flagged as a tie
