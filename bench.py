@@ -116,9 +116,10 @@ def verify_bytes(wl, L=None, labels=True):
     return int((2 * L + 1).sum()) * V * 4
 
 
-def config_of(wl, n, labels, layout="position"):
+def config_of(wl, n, labels, layout="position", ragged=False):
     return {"layout": ("position-major [gamma, B, V]" if layout == "position" else "request-major [B, gamma, V]")
                       + " draft logits U and ld",
+            "lt_layout": "flattened [sum(L_b + 1), V] with row offsets" if ragged else "padded [B, gamma + 1, V]",
             "workload": f"{wl.name}: B={wl.B} requests, gamma={wl.gamma}, V={wl.V}, r={wl.r}, T={wl.T}, "
                         f"{wl.w_dtype} W1/W2, fp32 {'log-Zipf+Gaussian' if wl.logits == 'logzipf' else 'Gaussian'} "
                         "logits",
@@ -246,7 +247,7 @@ def run_reference(args, wl, labels, rank):
     line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, see inputs.py)",
-            "config": config_of(wl, args.gpus, labels),
+            "config": config_of(wl, args.gpus, labels, args.layout, args.ragged),
             "cpu_baseline": dict(cb, sample=cb["sample"] + f"; each timed step: one round on {n_req} request(s)"),
             "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -625,9 +626,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": f"synthetic (seeded log-Zipf + Gaussian logits, "
                                                          f"{wl.w_dtype} weights)",
-            "config": dict(config_of(wl, world, labels, args.layout),
-                           lt_layout=("flattened [sum(L_b + 1), V] with row offsets" if args.ragged
-                                      else "padded [B, gamma + 1, V]")),
+            "config": config_of(wl, world, labels, args.layout, args.ragged),
             "verified_tokens_per_s": accepted_all / (args.steps * t_step),
             "tokens_per_request_per_round": tau,
             "latency_per_token_us": (t_draft + t_verify) / tau * 1e6,
