@@ -11,7 +11,8 @@
  *
  * Conventions shared by every entry point
  *   - Every tensor pointer is a DEVICE pointer owned by the caller; the library
- *     never allocates, frees or keeps device memory between calls.
+ *     never allocates, frees or keeps device memory between calls (the one fixed
+ *     scratch array of dspark_verify_noalloc is part of the library image).
  *   - All tensors are dense and row-major (C order), with the shapes given.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL means the legacy default stream).  Outputs are valid once the stream
