@@ -22,8 +22,9 @@ struct Options {
   int verify_persistent = 1;     // sampled verify / labels: persistent clusters with double-buffered rows (0: one cluster per row)
   int verify_impl = 0;           // verify with a workspace: 0 streaming kernels, 1 column-sliced, 2 per-row
   int verify_groups = 0;         // sliced verify: CTA groups (0: slices of about 16 KB per row)
-  int verify_stream_cluster = 0; // CTAs per cluster of the streaming verify (1 to 8; 0: 3, or 6 for few rows)
+  int verify_stream_cluster = 0; // CTAs per cluster of the streaming verify (1 to 16; 0: automatic)
   int verify_stream_l2hint = 1;  // streaming verify: first-pass copies evict-last, second-pass evict-first
+  int verify_stream_pass2 = 0;   // streaming verify, T > 0: 0 automatic, 1 both passes through the ring, 2 resident rows
   int sm_count = 0;              // 0: query the device
   // test-only: make the bounded device waits give up sooner and one of them unsatisfiable, so that
   // a test can check that the kernels return with a timeout status (never on in normal use)

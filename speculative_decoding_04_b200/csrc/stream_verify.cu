@@ -12,9 +12,10 @@
 // exponent is a = fma(l, c, -ref) in fp32 (l·c exact inside the fma).  Per row each CTA runs
 //   P1  (tiles from HBM)  per-lane maxima and sums of 2^a against an integer reference, so that
 //       every later rescaling is an exact power of two;
-//   --  the CTA's (R, S) pairs go to every CTA of the cluster (distributed shared memory and a
-//       remote mbarrier arrive); each CTA folds them in rank order into the row's normalisers
-//       log2 p = l c - K - lam (K an integer, lam in [0, 1)) and decides the acceptance;
+//   --  the CTA's (R, S) pairs go to every CTA of the cluster (st.async stores into distributed
+//       shared memory that complete on the receiver's mbarrier); each CTA folds them into the
+//       row's normalisers log2 p = l c - K - lam (K an integer, lam in [0, 1)) and decides the
+//       acceptance;
 //   P2  (the same tiles again, now from L2)  sum min(p_d, p_t), taken as one 2^x per column
 //       with x = min(a_d - (lam_d - lam_t), a_t) and the factor 2^-lam_t applied per tile, and
 //       whether any column has p_t > p_d (without one, q = 0 everywhere and the label is exactly
@@ -66,7 +67,7 @@ constexpr int kSvCombiner = kSvWarps + 1;
 constexpr int kSvDecider = kSvWarps + 2;
 constexpr int kSvPhaseSlots = 16;
 constexpr int kSvJobSlots = 4;
-constexpr int kSvMaxCluster = 8;
+constexpr int kSvMaxCluster = 16;
 constexpr uint32_t kSvSuspendNs = 100000;            // longest single suspension of a waiting warp
 constexpr uint64_t kSvTimeoutNs = 2000000000ull;     // a wait gives up after 2 s
 constexpr int kRNone = -(1 << 28);  // reference of an empty sum
@@ -110,7 +111,7 @@ struct SvArgs {
   const int64_t* lt_off;  // flattened l_t: request b's rows start at row lt_off[b] (null: padded)
   long long lt_nrows;
   uint64_t wait_ns;  // bounded waits give up after this long
-  int xbar_extra;    // test-only: arrivals the exchange barriers expect beyond the cluster
+  int xbar_extra;    // test-only: partials the exchange barriers expect beyond the cluster
   float zscale;  // log2(e) / T (T > 0)
   int greedy, do_verify;
   float* c_star;
@@ -165,7 +166,7 @@ struct SvPhase {
   int i;  // index of the row among this cluster's rows (exchange / decision slots)
 };
 
-// The phase sequence of a cluster with a lag of L rows (a.lag, 1 to 3): P1(row i) then
+// The phase sequence of a cluster with a lag of L rows (a.lag, 0 to 3): P1(row i) then
 // P2(row i-L), for i = 0, 1, ..., until both have run out.  Every role walks the same sequence.
 struct SvGen {
   int j, ncl, i, step, nrows, lag;
@@ -200,7 +201,7 @@ struct SvGen {
         step = 2;
         const int q = i - lag;
         if (q >= 0 && q < nrows) {
-          const SvJob J = sv_job(a, lag == 1 ? r1 : (lag == 2 ? r2 : r3));
+          const SvJob J = sv_job(a, lag == 0 ? r0 : (lag == 1 ? r1 : (lag == 2 ? r2 : r3)));
           if (sv_p2(a, J)) {
             ph.J = J;
             ph.second = true;
@@ -368,17 +369,6 @@ __device__ __forceinline__ uint64_t sv_now_ns() {
   return t;
 }
 
-// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster; the
-// release orders this thread's earlier stores into that CTA's shared memory before it.
-__device__ __forceinline__ void sv_remote_arrive(uint64_t* bar, int rank) {
-  asm volatile(
-      "{\n\t.reg .b32 ra;\n\t"
-      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
-      "r"(rank)
-      : "memory");
-}
-
 __device__ __forceinline__ void sv_cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -504,12 +494,266 @@ __device__ __forceinline__ float sv_lane_acc(const float4 (&v)[kSvVec], float c,
   return s;
 }
 
+// One consumer warp's tile of a stage (kSvTile columns of each row; `cnt` of them are real):
+// lane l holds columns 4 (32 jj + l) .. + 3 of the tile in fd[jj] (l_d) and ft[jj] (l_t), -inf
+// past `cnt`; without l_d, fd repeats ft.
+__device__ __forceinline__ void sv_load_tile(const float* sd, const float* st, bool with_d, int cnt,
+                                             float4 (&fd)[kSvVec], float4 (&ft)[kSvVec]) {
+  const int lane = threadIdx.x & 31;
+  if (cnt == kSvTile) {
+#pragma unroll
+    for (int jj = 0; jj < kSvVec; ++jj) {
+      const int idx = (jj * 32 + lane) * 4;
+      ft[jj] = *reinterpret_cast<const float4*>(st + idx);
+      fd[jj] = with_d ? *reinterpret_cast<const float4*>(sd + idx) : ft[jj];
+    }
+  } else {
+    const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+#pragma unroll
+    for (int jj = 0; jj < kSvVec; ++jj) {
+      const int idx = (jj * 32 + lane) * 4;
+      const bool v = idx < cnt;
+      ft[jj] = v ? *reinterpret_cast<const float4*>(st + idx) : ninf;
+      fd[jj] = (v && with_d) ? *reinterpret_cast<const float4*>(sd + idx) : ninf;
+    }
+  }
+}
+
+// First pass over one tile (T > 0): the lane sums of both rows against their references; for
+// the bonus row (trec non-null) also the tile's l_t weight (R, s) for the bonus sample.
+__device__ __forceinline__ void sv_p1_tile(const float4 (&fd)[kSvVec], const float4 (&ft)[kSvVec], float zc,
+                                           bool with_d, float2* trec, int& Rd, float& Sd, float& nRd, int& Rt,
+                                           float& St, float& nRt) {
+  int rt;
+  const float stl = sv_lane_acc(ft, zc, Rt, nRt, St, rt);
+  if (trec) {
+    const int R = __reduce_max_sync(0xffffffffu, rt);
+    const float sw = warp_sum_f(stl * sv_pow2f(rt - R));
+    if ((threadIdx.x & 31) == 0) *trec = make_float2((float)R, sw);
+  }
+  if (with_d) {
+    int rd;
+    sv_lane_acc(fd, zc, Rd, nRd, Sd, rd);
+  }
+}
+
+// Second pass over one tile: 2^min(x_d, x_t) per column, unscaled, into smin and the max of
+// x_t - x_d into dqmax (labels); a rejected row (needq) also stores its tile's sum of
+// q = 2^x_t - 2^min(x_d, x_t), scaled, at *qrec.
+__device__ __forceinline__ void sv_p2_tile(const float4 (&fd)[kSvVec], const float4 (&ft)[kSvVec], float zc,
+                                           const SvP2& k2, bool needq, bool labels, float* qrec, float& smin,
+                                           float& dqmax) {
+  const float2 c2 = make_float2(zc, zc);
+  const float2 nkd = make_float2(k2.nkd, k2.nkd), nkt = make_float2(k2.nkt, k2.nkt);
+  const float2 ndl = make_float2(k2.ndl, k2.ndl), mone = make_float2(-1.f, -1.f);
+  float2 sm2 = make_float2(0.f, 0.f);
+  if (!needq) {
+    if (labels) {
+#pragma unroll
+      for (int jj = 0; jj < kSvVec; ++jj) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
+          const float2 xd = f2add(f2fma(ld2, c2, nkd), ndl), xt = f2fma(lt2, c2, nkt);
+          sm2 = f2add(sm2, make_float2(sv_ex2(fminf(xd.x, xt.x)), sv_ex2(fminf(xd.y, xt.y))));
+          const float2 df = f2fma(xd, mone, xt);
+          dqmax = fmax3(dqmax, df.x, df.y);
+        }
+      }
+    }
+  } else {
+    float2 q2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int jj = 0; jj < kSvVec; ++jj) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
+        const float2 xd = f2add(f2fma(ld2, c2, nkd), ndl), xt = f2fma(lt2, c2, nkt);
+        const float2 mn = make_float2(sv_ex2(fminf(xd.x, xt.x)), sv_ex2(fminf(xd.y, xt.y)));
+        const float2 pt = make_float2(sv_ex2(xt.x), sv_ex2(xt.y));
+        sm2 = f2add(sm2, mn);
+        q2 = f2add(q2, f2fma(mn, mone, pt));
+        const float2 df = f2fma(xd, mone, xt);
+        dqmax = fmax3(dqmax, df.x, df.y);
+      }
+    }
+    const float qw = warp_sum_f(q2.x + q2.y);
+    if ((threadIdx.x & 31) == 0) *qrec = qw * k2.scale;
+  }
+  smin += sm2.x + sm2.y;
+}
+
 // Decision of a row for its second pass.
 struct __align__(16) SvDec {
   SvNorm nm;
   int needq;  // rejected: the second pass also sums the residual weights q
   int pad0, pad1, pad2;
 };
+
+static_assert(sizeof(SvPart) == 64, "a partial is four 16-byte stores");
+
+// Store a partial into the same shared-memory slot of CTA `rank` of the cluster with st.async,
+// whose bytes count toward the transaction count of that CTA's mbarrier `bar` on arrival: the
+// receiver's wait on the barrier then sees the data, and the sender needs no release fence
+// (which would also wait for its earlier global stores).
+__device__ __forceinline__ void sv_push_part(const SvPart& w, SvPart* slot, uint64_t* bar, int rank) {
+  uint32_t ra, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(slot)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(smem_u32(bar)), "r"(rank));
+  const uint4* v = reinterpret_cast<const uint4*>(&w);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 x = v[q];
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     ra + 16u * q),
+                 "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w), "r"(rb)
+                 : "memory");
+  }
+}
+
+// Shared state of the combine and decide roles.
+struct SvRoles {
+  uint64_t* phbar;              // [kSvPhaseSlots]: the consumer warps' partials of a pass are in
+  SvPart (*wpart)[kSvWarps];    // [kSvPhaseSlots][kSvWarps]
+  SvPart (*xs)[kSvMaxCluster];  // [kSvJobSlots][C]: the cluster's partials of a row's first pass
+  uint64_t* xbar;               // [kSvJobSlots]: all C partials of the row have arrived
+  uint64_t* nbar;               // [kSvJobSlots]: the row's normalisers are in dec[].nm
+  uint64_t* dbar;               // [kSvJobSlots]: the row is decided (dec[] complete)
+  SvDec* dec;                   // [kSvJobSlots]
+  volatile int* decided;        // rows of this cluster's sequence decided by this CTA
+  volatile int* combined;       // passes whose warp partials the combiner has read
+};
+
+template <bool GREEDY>
+__device__ __forceinline__ void sv_combine_role(const SvArgs& a, const SvSync& sy, const SvRoles& r, int C, int rank,
+                                                int cid, int ncl) {
+  const int lane = threadIdx.x & 31;
+  // ------------------------------------------------------------------ combine and exchange
+  // Per first pass: fold the warps' partials and push the CTA's into slot [i % 4][rank] of
+  // every CTA of the cluster.  Per second pass: the CTA's label partials to global memory.
+  // A push for row i waits until this CTA has decided row i-2: a peer that has decided row
+  // i-2 has then seen this CTA's push of row i-2, so every peer has decided row i-4, the
+  // previous user of the slot (the second passes give the same order when T > 0; greedy
+  // verification has none).
+  SvGen gen;
+  gen.init(a, cid, ncl);
+  SvPhase ph;
+  int p = 0;
+  bool ok = true;
+  while (ok && gen.next(a, ph)) {
+    const int ps = p % kSvPhaseSlots;
+    ok = sv_wait(sy, &r.phbar[ps], (p / kSvPhaseSlots) & 1);
+    ++p;
+    if (!ok) break;
+    SvPart w = lane < kSvWarps ? r.wpart[ps][lane] : sv_empty_part();
+    // The count that frees the slot is stored after the shuffles that consume the slot's
+    // values, so those reads are complete.  No fence here: one would also wait for this
+    // warp's global stores of the previous pass, microseconds while the copies load HBM.
+    if (!ph.second) {
+      w = sv_fold<GREEDY>(w);
+      if (lane == 0) *r.combined = p;
+      const int i = ph.i;
+      ok = sv_wait_count(sy, r.decided, i - 1);  // r.decided counts rows, so row i-2 is decided
+      if (!ok) break;
+      if (lane < C) sv_push_part(w, &r.xs[i % kSvJobSlots][rank], &r.xbar[i % kSvJobSlots], lane);
+    } else {
+      const double sm = warp_sum_d(w.sd), nq = warp_sum_d(w.st);
+      if (lane == 0) *r.combined = p;
+      if (lane == 0 && ph.J.k < a.gamma)
+        a.part[((size_t)ph.J.b * a.gamma + ph.J.k) * C + rank] = make_double2(sm, nq);
+    }
+  }
+}
+
+template <bool GREEDY>
+__device__ __forceinline__ void sv_decide_role(const SvArgs& a, const SvSync& sy, const SvRoles& r, int C, int rank,
+                                               int cid, int ncl) {
+  const int lane = threadIdx.x & 31;
+  // ------------------------------------------------------------------ decide, row by row
+  SvJob J;
+  int j = sv_next(a, cid, ncl, J);
+  bool ok = true;
+  for (int i = 0; ok && j >= 0; ++i) {
+    const int js = i % kSvJobSlots;
+    // the drafted token and its uniform are requested before the wait for the peers
+    // (and, for T > 0, the two logits at the drafted token)
+    const int xk = J.verify ? __ldg(a.x + (size_t)J.b * a.gamma + J.k) : -1;
+    const float u_acc = (J.verify && !GREEDY) ? __ldg(a.u_acc + (size_t)J.b * a.gamma + J.k) : 0.f;
+    float ldx = 0.f, ltx = 0.f;
+    if (!GREEDY && J.verify && (unsigned)xk < (unsigned)a.V) {
+      ldx = __ldg(a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb + xk);
+      ltx = __ldg(a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, J.b, J.k) * a.V + xk);
+    }
+    // the rejection record only grows: read before the wait, it can only ask for more residual
+    // weights than needed, never fewer
+    const int rej_seen = (!GREEDY && J.verify) ? __ldcg(a.rej + J.b) : 0;
+    // the phase ends when this arrival is in and the cluster's C partials have landed
+    if (lane == 0) mbar_arrive_expect_tx(&r.xbar[js], (uint32_t)((C + a.xbar_extra) * sizeof(SvPart)));
+    ok = sv_wait(sy, &r.xbar[js], (i / kSvJobSlots) & 1, true);
+    if (!ok) break;
+    SvPart x = lane < C ? r.xs[js][lane] : sv_empty_part();
+    x = sv_fold<GREEDY>(x);
+    SvRow row;
+    row.acc = 0;
+    row.fl = 0;
+    row.cand = 0;
+    row.cstar = 0.f;
+    uint32_t dfl = x.fl;
+    if (GREEDY) {
+      row.nm = SvNorm{0.f, 0.f, 0.f, 0.f};
+      const bool ttie = x.gt.best - x.gt.second <= 1e-6f * fmaxf(1.f, fabsf(x.gt.best));
+      row.cand = min(max(x.gt.idx, 0), a.V - 1);
+      if (x.gt.idx < 0) dfl |= DSPARK_FLAG_NONFINITE;
+      row.cstar = (x.gd.idx == x.gt.idx) ? 1.f : 0.f;
+      row.fl = ttie ? (DSPARK_FLAG_ACCEPT_NEAR_TIE | DSPARK_FLAG_SAMPLE_NEAR_TIE) : 0u;
+      if (J.verify) {
+        if ((unsigned)xk >= (unsigned)a.V) dfl |= DSPARK_FLAG_TOKEN_RANGE;
+        row.acc = (xk == x.gt.idx) ? 1 : 0;
+      }
+    } else {
+      SvNorm nm;
+      bool good = sv_norm(x.rt, x.st, nm.Kt, nm.lamt);
+      if (J.d) good &= sv_norm(x.rd, x.sd, nm.Kd, nm.lamd);
+      else nm.Kd = nm.lamd = 0.f;
+      if (!good) dfl |= DSPARK_FLAG_NONFINITE;
+      row.nm = nm;
+      if (lane == 0) {
+        r.dec[js].nm = nm;
+        mbar_arrive(&r.nbar[js]);  // a second pass that needs only the normalisers may start
+      }
+      if (J.verify) {
+        if ((unsigned)xk >= (unsigned)a.V) {
+          dfl |= DSPARK_FLAG_TOKEN_RANGE;
+        } else {
+          // u p_d(x) < p_t(x) with p = 2^(l c - R) / S, in fp64 (l c is exact there)
+          const double pd = exp2((double)ldx * (double)a.zscale - (double)x.rd) / x.sd;
+          const double pt = exp2((double)ltx * (double)a.zscale - (double)x.rt) / x.st;
+          const double u = (double)u_acc;
+          row.acc = (u * pd < pt) ? 1 : 0;
+          if (pd > 0.0 && fabs(u - pt / pd) < 1e-6) row.fl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
+        }
+      }
+      // residual weights only for a rejection that may be the request's first (the others are
+      // never sampled); a rejection is published for the deciders of later rows
+      const int enc = a.gamma + 1 - J.k;
+      const bool rej = J.verify && !row.acc;
+      const bool needq = rej && rej_seen <= enc;
+      if (lane == 0) r.dec[js].needq = needq ? 1 : 0;
+      if (rej && rank == 0 && lane == 0) atomicMax(a.rej + J.b, enc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&r.dbar[js]);  // the second pass of this row may start
+    }
+    if (rank == 0 && lane == 0) {
+      a.rows[J.rec] = row;
+      if (dfl && a.flags) atomicOr(a.flags + J.b, dfl);
+    }
+    // the count that frees this row's slots follows the shuffles that consumed them (no fence:
+    // it would wait for the row's global stores above)
+    __syncwarp();
+    if (lane == 0) *r.decided = i + 1;
+    j = sv_next(a, j + ncl, ncl, J);
+  }
+}
 
 template <bool GREEDY>
 __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
@@ -522,7 +766,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   extern __shared__ __align__(128) float ring[];  // [kSvStages][2][kSvBig]: l_d columns, l_t columns
   __shared__ __align__(8) uint64_t full[kSvStages], empty[kSvStages];
   __shared__ __align__(8) uint64_t phbar[kSvPhaseSlots];
-  __shared__ __align__(8) uint64_t xbar[kSvJobSlots], dbar[kSvJobSlots];
+  __shared__ __align__(8) uint64_t xbar[kSvJobSlots], nbar[kSvJobSlots], dbar[kSvJobSlots];
   __shared__ SvPart wpart[kSvPhaseSlots][kSvWarps];
   __shared__ SvPart xs[kSvJobSlots][kSvMaxCluster];
   __shared__ SvDec dec[kSvJobSlots];
@@ -531,6 +775,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   __shared__ volatile int s_combined;  // passes whose warp partials the combiner has read
 
   const SvSync sy{&s_abort, a.status, a.wait_ns};
+  const SvRoles roles{phbar, wpart, xs, xbar, nbar, dbar, dec, &s_decided, &s_combined};
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSvStages; ++i) {
       mbar_init(&full[i], 1);
@@ -538,7 +783,8 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     }
     for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
     for (int i = 0; i < kSvJobSlots; ++i) {
-      mbar_init(&xbar[i], C + a.xbar_extra);
+      mbar_init(&xbar[i], 1);  // the decider's arrival; the partials count as transaction bytes
+      mbar_init(&nbar[i], 1);
       mbar_init(&dbar[i], 1);
     }
     s_abort = 0;
@@ -608,124 +854,14 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       }
     }
   } else if (warp == kSvCombiner) {
-    // ------------------------------------------------------------------ combine and exchange
-    // Per first pass: fold the warps' partials and push the CTA's into slot [i % 4][rank] of
-    // every CTA of the cluster.  Per second pass: the CTA's label partials to global memory.
-    // A push for row i waits until this CTA has decided row i-2: a peer that has decided row
-    // i-2 has then seen this CTA's push of row i-2, so every peer has decided row i-4, the
-    // previous user of the slot (the second passes give the same order when T > 0; greedy
-    // verification has none).
-    SvGen gen;
-    gen.init(a, cid, ncl);
-    SvPhase ph;
-    int p = 0;
-    bool ok = true;
-    while (ok && gen.next(a, ph)) {
-      const int ps = p % kSvPhaseSlots;
-      ok = sv_wait(sy, &phbar[ps], (p / kSvPhaseSlots) & 1);
-      ++p;
-      if (!ok) break;
-      SvPart w = lane < kSvWarps ? wpart[ps][lane] : sv_empty_part();
-      __syncwarp();
-      __threadfence_block();  // the slot's reads come before the count that frees it
-      if (lane == 0) s_combined = p;
-      if (!ph.second) {
-        w = sv_fold<GREEDY>(w);
-        const int i = ph.i;
-        ok = sv_wait_count(sy, &s_decided, i - 1);  // s_decided counts rows, so row i-2 is decided
-        if (!ok) break;
-        if (lane < C) {
-          SvPart* dst = cluster.map_shared_rank(&xs[i % kSvJobSlots][rank], lane);
-          *dst = w;
-          sv_remote_arrive(&xbar[i % kSvJobSlots], lane);
-        }
-      } else {
-        const double sm = warp_sum_d(w.sd), nq = warp_sum_d(w.st);
-        if (lane == 0 && ph.J.k < a.gamma)
-          a.part[((size_t)ph.J.b * a.gamma + ph.J.k) * C + rank] = make_double2(sm, nq);
-      }
-    }
+    sv_combine_role<GREEDY>(a, sy, roles, C, rank, cid, ncl);
   } else if (warp == kSvDecider) {
-    // ------------------------------------------------------------------ decide, row by row
-    SvJob J;
-    int j = sv_next(a, cid, ncl, J);
-    bool ok = true;
-    for (int i = 0; ok && j >= 0; ++i) {
-      const int js = i % kSvJobSlots;
-      // the drafted token and its uniform are requested before the wait for the peers
-      // (and, for T > 0, the two logits at the drafted token)
-      const int xk = J.verify ? __ldg(a.x + (size_t)J.b * a.gamma + J.k) : -1;
-      const float u_acc = (J.verify && !GREEDY) ? __ldg(a.u_acc + (size_t)J.b * a.gamma + J.k) : 0.f;
-      float ldx = 0.f, ltx = 0.f;
-      if (!GREEDY && J.verify && (unsigned)xk < (unsigned)a.V) {
-        ldx = __ldg(a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb + xk);
-        ltx = __ldg(a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, J.b, J.k) * a.V + xk);
-      }
-      ok = sv_wait(sy, &xbar[js], (i / kSvJobSlots) & 1, true);
-      if (!ok) break;
-      SvPart x = lane < C ? xs[js][lane] : sv_empty_part();
-      x = sv_fold<GREEDY>(x);
-      SvRow row;
-      row.acc = 0;
-      row.fl = 0;
-      row.cand = 0;
-      row.cstar = 0.f;
-      uint32_t dfl = x.fl;
-      if (GREEDY) {
-        row.nm = SvNorm{0.f, 0.f, 0.f, 0.f};
-        const bool ttie = x.gt.best - x.gt.second <= 1e-6f * fmaxf(1.f, fabsf(x.gt.best));
-        row.cand = min(max(x.gt.idx, 0), a.V - 1);
-        if (x.gt.idx < 0) dfl |= DSPARK_FLAG_NONFINITE;
-        row.cstar = (x.gd.idx == x.gt.idx) ? 1.f : 0.f;
-        row.fl = ttie ? (DSPARK_FLAG_ACCEPT_NEAR_TIE | DSPARK_FLAG_SAMPLE_NEAR_TIE) : 0u;
-        if (J.verify) {
-          if ((unsigned)xk >= (unsigned)a.V) dfl |= DSPARK_FLAG_TOKEN_RANGE;
-          row.acc = (xk == x.gt.idx) ? 1 : 0;
-        }
-      } else {
-        SvNorm nm;
-        bool good = sv_norm(x.rt, x.st, nm.Kt, nm.lamt);
-        if (J.d) good &= sv_norm(x.rd, x.sd, nm.Kd, nm.lamd);
-        else nm.Kd = nm.lamd = 0.f;
-        if (!good) dfl |= DSPARK_FLAG_NONFINITE;
-        row.nm = nm;
-        if (J.verify) {
-          if ((unsigned)xk >= (unsigned)a.V) {
-            dfl |= DSPARK_FLAG_TOKEN_RANGE;
-          } else {
-            // u p_d(x) < p_t(x) with p = 2^(l c - R) / S, in fp64 (l c is exact there)
-            const double pd = exp2((double)ldx * (double)zc - (double)x.rd) / x.sd;
-            const double pt = exp2((double)ltx * (double)zc - (double)x.rt) / x.st;
-            const double u = (double)u_acc;
-            row.acc = (u * pd < pt) ? 1 : 0;
-            if (pd > 0.0 && fabs(u - pt / pd) < 1e-6) row.fl |= DSPARK_FLAG_ACCEPT_NEAR_TIE;
-          }
-        }
-        // residual weights only for a rejection that may be the request's first (the others are
-        // never sampled); a rejection is published for the deciders of later rows
-        const int enc = a.gamma + 1 - J.k;
-        const bool rej = J.verify && !row.acc;
-        const bool needq = rej && __ldcg(a.rej + J.b) <= enc;
-        if (lane == 0) dec[js] = SvDec{nm, needq ? 1 : 0, 0, 0, 0};
-        if (rej && rank == 0 && lane == 0) atomicMax(a.rej + J.b, enc);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dbar[js]);  // the second pass of this row may start
-      }
-      if (rank == 0 && lane == 0) {
-        a.rows[J.rec] = row;
-        if (dfl && a.flags) atomicOr(a.flags + J.b, dfl);
-      }
-      __syncwarp();
-      __threadfence_block();  // this row's slot reads come before the count that frees the slot
-      if (lane == 0) s_decided = i + 1;
-      j = sv_next(a, j + ncl, ncl, J);
-    }
+    sv_decide_role<GREEDY>(a, sy, roles, C, rank, cid, ncl);
   } else {
     // ------------------------------------------------------------------ tile consumers
     const int w = warp;
     const int last_tile = a.ntile - 1 - tb;  // the segment's ragged tile, if it has it
     const int last_cnt = a.V - (a.ntile - 1) * kSvTile;
-    const float2 c2 = make_float2(zc, zc);
     bool ok = true;
     int p = 0;  // passes finished by this warp (slot of the partials)
     // state of the current pass
@@ -824,23 +960,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
       const float* st = sd + kSvBig;
       const bool with_d = ph.second || ph.J.d;
       float4 fd[kSvVec], ft[kSvVec];
-      if (t != last_tile) {
-#pragma unroll
-        for (int jj = 0; jj < kSvVec; ++jj) {
-          const int idx = (jj * 32 + lane) * 4;
-          ft[jj] = *reinterpret_cast<const float4*>(st + idx);
-          fd[jj] = with_d ? *reinterpret_cast<const float4*>(sd + idx) : ft[jj];
-        }
-      } else {
-        const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-#pragma unroll
-        for (int jj = 0; jj < kSvVec; ++jj) {
-          const int idx = (jj * 32 + lane) * 4;
-          const bool v = idx < last_cnt;
-          ft[jj] = v ? *reinterpret_cast<const float4*>(st + idx) : ninf;
-          fd[jj] = (v && with_d) ? *reinterpret_cast<const float4*>(sd + idx) : ninf;
-        }
-      }
+      sv_load_tile(sd, st, with_d, t == last_tile ? last_cnt : kSvTile, fd, ft);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);  // the values are in registers
       if (!ph.second) {
@@ -857,60 +977,226 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
             }
           }
         } else {
-          int rt;
-          const float stl = sv_lane_acc(ft, zc, Rt, nRt, St, rt);
-          if (ph.J.bonus) {
-            // l_t weight of the tile for the bonus sample
-            const int R = __reduce_max_sync(0xffffffffu, rt);
-            const float sw = warp_sum_f(stl * sv_pow2f(rt - R));
-            if (lane == 0) a.trec[(size_t)ph.J.rec * a.ntile + tb + t] = make_float2((float)R, sw);
-          }
-          if (with_d) {
-            int rd;
-            sv_lane_acc(fd, zc, Rd, nRd, Sd, rd);
-          }
+          sv_p1_tile(fd, ft, zc, with_d, ph.J.bonus ? a.trec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr, Rd, Sd,
+                     nRd, Rt, St, nRt);
         }
       } else {
-        // 2^min(x_d, x_t) per column, unscaled, and the max of x_t - x_d; a rejected row also
-        // keeps its tile's sum of q = 2^x_t - 2^min(x_d, x_t)
-        const float2 nkd = make_float2(k2.nkd, k2.nkd), nkt = make_float2(k2.nkt, k2.nkt);
-        const float2 ndl = make_float2(k2.ndl, k2.ndl), mone = make_float2(-1.f, -1.f);
-        float2 sm2 = make_float2(0.f, 0.f);
-        if (!needq) {
-          if (a.c_star) {
-#pragma unroll
-            for (int jj = 0; jj < kSvVec; ++jj) {
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
-                const float2 xd = f2add(f2fma(ld2, c2, nkd), ndl), xt = f2fma(lt2, c2, nkt);
-                sm2 = f2add(sm2, make_float2(sv_ex2(fminf(xd.x, xt.x)), sv_ex2(fminf(xd.y, xt.y))));
-                const float2 df = f2fma(xd, mone, xt);
-                dqmax = fmax3(dqmax, df.x, df.y);
-              }
-            }
-          }
-        } else {
-          float2 q2 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int jj = 0; jj < kSvVec; ++jj) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float2 ld2 = h ? hi2(fd[jj]) : lo2(fd[jj]), lt2 = h ? hi2(ft[jj]) : lo2(ft[jj]);
-              const float2 xd = f2add(f2fma(ld2, c2, nkd), ndl), xt = f2fma(lt2, c2, nkt);
-              const float2 mn = make_float2(sv_ex2(fminf(xd.x, xt.x)), sv_ex2(fminf(xd.y, xt.y)));
-              const float2 pt = make_float2(sv_ex2(xt.x), sv_ex2(xt.y));
-              sm2 = f2add(sm2, mn);
-              q2 = f2add(q2, f2fma(mn, mone, pt));
-              const float2 df = f2fma(xd, mone, xt);
-              dqmax = fmax3(dqmax, df.x, df.y);
-            }
-          }
-          const float qw = warp_sum_f(q2.x + q2.y);
-          if (lane == 0) a.qrec[(size_t)ph.J.rec * a.ntile + tb + t] = qw * k2.scale;
-        }
-        smin += sm2.x + sm2.y;
+        sv_p2_tile(fd, ft, zc, k2, needq, a.c_star != nullptr, needq ? a.qrec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr,
+                   smin, dqmax);
       }
+    }
+  }
+
+  __syncwarp();
+  sv_cluster_sync_all();  // no CTA leaves while a peer may still write into its shared memory
+}
+
+// ---------------------------------------------------------------------------------------------
+// Resident rows (T > 0): every row of l_d and l_t read from HBM once.
+//
+// The same cluster layout, roles and records as verify_stream, but a CTA keeps its whole
+// segment of a row pair in shared memory from the first pass to the second, so the second pass
+// reads shared memory instead of copying the tiles again.  The ring is cut into chunks of
+// kRvChunkTiles tiles (one bulk copy per row and chunk); a row starts on a chunk boundary and
+// holds ceil(nt / kRvChunkTiles) chunks until its second pass ends (or its first, for a row
+// without one), when each tile's warp arrives on its chunk.  With a lag of 1 (two rows'
+// chunks and one spare fit) the consumers run P1(row i) before P2(row i-1), as verify_stream
+// does; with a lag of 0 (one row and a spare fit) P2(row i) follows P1(row i) and the copies of
+// row i+1 go on into the spare chunks while the row is decided.  Every copy carries the
+// evict-first policy: nothing is read twice from L2.
+constexpr int kRvChunkTiles = 4;                        // tiles per chunk: copies of 8 KB per row
+constexpr int kRvChunkCols = kRvChunkTiles * kSvTile;
+constexpr int kRvChunks = 12;                           // 12 chunks of (l_d, l_t): 192 KB
+constexpr size_t kRvRingBytes = (size_t)kRvChunks * 2 * kRvChunkCols * sizeof(float);
+
+__global__ void __launch_bounds__(kSvThreads, 1) verify_resident(SvArgs a) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int cid = blockIdx.x / C, ncl = gridDim.x / C;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  extern __shared__ __align__(128) float ring[];  // [2][kRvChunks][kRvChunkCols]: l_d chunks, then l_t chunks
+  __shared__ __align__(8) uint64_t full[kRvChunks], empty[kRvChunks];
+  __shared__ __align__(8) uint64_t phbar[kSvPhaseSlots];
+  __shared__ __align__(8) uint64_t xbar[kSvJobSlots], nbar[kSvJobSlots], dbar[kSvJobSlots];
+  __shared__ SvPart wpart[kSvPhaseSlots][kSvWarps];
+  __shared__ SvPart xs[kSvJobSlots][kSvMaxCluster];
+  __shared__ SvDec dec[kSvJobSlots];
+  __shared__ int s_abort;
+  __shared__ volatile int s_decided;
+  __shared__ volatile int s_combined;
+
+  const SvSync sy{&s_abort, a.status, a.wait_ns};
+  const SvRoles roles{phbar, wpart, xs, xbar, nbar, dbar, dec, &s_decided, &s_combined};
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRvChunks; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kRvChunkTiles);  // one arrival per tile
+    }
+    for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
+    for (int i = 0; i < kSvJobSlots; ++i) {
+      mbar_init(&xbar[i], 1);  // the decider's arrival; the partials count as transaction bytes
+      mbar_init(&nbar[i], 1);
+      mbar_init(&dbar[i], 1);
+    }
+    s_abort = 0;
+    s_decided = 0;
+    s_combined = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  sv_cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+
+  // This CTA's segment of every row: tiles tb .. tb + nt - 1, in nch chunks; row number i of
+  // the cluster's sequence occupies stream chunks i*nch .. i*nch + nch - 1.
+  const int tb = (int)((long long)rank * a.ntile / C);
+  const int nt = (int)((long long)(rank + 1) * a.ntile / C) - tb;  // may be 0
+  const int nch = (nt + kRvChunkTiles - 1) / kRvChunkTiles;
+  const float zc = a.zscale;
+
+  if (warp == kSvProducer) {
+    // ------------------------------------------------------------------ bulk copies
+    if (lane == 0 && nt > 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      uint32_t g = 0;  // stream chunk
+      bool ok = true;
+      SvJob J;
+      for (int j = sv_next(a, cid, ncl, J); ok && j >= 0; j = sv_next(a, j + ncl, ncl, J)) {
+        const float* rd = a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb;
+        const float* rt = a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, J.b, J.k) * a.V;
+        for (int h = 0; h < nch; ++h, ++g) {
+          const int s = (int)(g % kRvChunks);
+          if (!sv_wait(sy, &empty[s], ((g / kRvChunks) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          const int c0 = (tb + h * kRvChunkTiles) * kSvTile;
+          const int c1 = min((tb + min((h + 1) * kRvChunkTiles, nt)) * kSvTile, a.V);
+          const uint32_t bytes = (uint32_t)(c1 - c0) * 4u;
+          float* dd = ring + (size_t)s * kRvChunkCols;
+          float* dt = ring + (size_t)(kRvChunks + s) * kRvChunkCols;
+          mbar_expect_tx(&full[s], J.d ? 2 * bytes : bytes);
+          if (a.l2hint) {
+            if (J.d) bulk_g2s_hint(dd, rd + c0, bytes, &full[s], pol);
+            bulk_g2s_hint(dt, rt + c0, bytes, &full[s], pol);
+          } else {
+            if (J.d) bulk_g2s(dd, rd + c0, bytes, &full[s]);
+            bulk_g2s(dt, rt + c0, bytes, &full[s]);
+          }
+          mbar_arrive(&full[s]);
+        }
+      }
+      if (!ok) {
+        // let the copies still in flight land before the CTA can exit
+        const uint32_t lo = g > (uint32_t)kRvChunks ? g - kRvChunks : 0u;
+        for (uint32_t gb = lo; gb < g; ++gb)
+          for (uint32_t i = 0; i < kSpinLimit && !mbar_try_wait(&full[gb % kRvChunks], (gb / kRvChunks) & 1); ++i) {
+          }
+      }
+    }
+  } else if (warp == kSvCombiner) {
+    sv_combine_role<false>(a, sy, roles, C, rank, cid, ncl);
+  } else if (warp == kSvDecider) {
+    sv_decide_role<false>(a, sy, roles, C, rank, cid, ncl);
+  } else {
+    // ------------------------------------------------------------------ tile consumers
+    // Tile t of row i goes to warp (i nt + t) mod 16 in both passes, so a warp's second pass
+    // reads only tiles whose chunks it saw land in its first.
+    const int w = warp;
+    const int last_tile = a.ntile - 1 - tb;
+    const int last_cnt = a.V - (a.ntile - 1) * kSvTile;
+    int p = 0;  // passes finished by this warp (slot of the partials)
+    bool ok = true;
+    SvGen gen;
+    gen.init(a, cid, ncl);
+    SvPhase ph;
+    while (ok && gen.next(a, ph)) {
+      const uint32_t gbase = (uint32_t)ph.i * (uint32_t)nch;
+      const int t0 = (w - (int)(((long long)ph.i * nt) % kSvWarps) + kSvWarps) % kSvWarps;
+      SvPart out = sv_empty_part();
+      if (!ph.second) {
+        int Rd = kRNone, Rt = kRNone;
+        float Sd = 0.f, St = 0.f, nRd = 0.f, nRt = 0.f;
+        // every warp waits for every chunk of the row in order, its own tiles' or not: a wait on
+        // a slot's use u then always follows the landing of use u - 1, so its parity cannot
+        // match an older phase
+        int hw = 0;  // chunks of the row waited for
+        auto wait_to = [&](int h_end) {
+          for (; hw < h_end; ++hw) {
+            const uint32_t gc = gbase + (uint32_t)hw;
+            if (!__all_sync(0xffffffffu, sv_wait(sy, &full[gc % kRvChunks], (gc / kRvChunks) & 1))) return false;
+          }
+          return true;
+        };
+        for (int t = t0; t < nt; t += kSvWarps) {
+          if (!wait_to(t / kRvChunkTiles + 1)) {
+            ok = false;
+            break;
+          }
+          const int s = (int)((gbase + (uint32_t)(t / kRvChunkTiles)) % kRvChunks);
+          const int o = (t % kRvChunkTiles) * kSvTile;
+          float4 fd[kSvVec], ft[kSvVec];
+          sv_load_tile(ring + (size_t)s * kRvChunkCols + o, ring + (size_t)(kRvChunks + s) * kRvChunkCols + o, ph.J.d,
+                       t == last_tile ? last_cnt : kSvTile, fd, ft);
+          sv_p1_tile(fd, ft, zc, ph.J.d, ph.J.bonus ? a.trec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr, Rd, Sd,
+                     nRd, Rt, St, nRt);
+        }
+        if (!ok || !wait_to(nch)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bad = (St <= FLT_MAX && Sd <= FLT_MAX) ? 0u : 1u;  // a non-finite logit of the pass
+        sv_warp_ref_sum_f(Rd, Sd);
+        sv_warp_ref_sum_f(Rt, St);
+        out.rd = Rd;
+        out.sd = (double)Sd;
+        out.rt = Rt;
+        out.st = (double)St;
+        out.fl = __any_sync(0xffffffffu, bad != 0) ? (uint32_t)DSPARK_FLAG_NONFINITE : 0u;
+      } else {
+        const int js = ph.i % kSvJobSlots;
+        // the normalisers suffice: the residual weights are kept for every verified row, so the
+        // pass need not wait for the acceptance decision
+        ok = __all_sync(0xffffffffu, sv_wait(sy, &nbar[js], (ph.i / kSvJobSlots) & 1));
+        if (!ok) break;
+        const SvP2 k2 = sv_p2_consts(dec[js].nm);
+        const bool needq = ph.J.verify;
+        float smin = 0.f, dqmax = -INFINITY;
+        if (needq || a.c_star) {
+          for (int t = t0; t < nt; t += kSvWarps) {
+            const int s = (int)((gbase + (uint32_t)(t / kRvChunkTiles)) % kRvChunks);
+            const int o = (t % kRvChunkTiles) * kSvTile;
+            float4 fd[kSvVec], ft[kSvVec];
+            sv_load_tile(ring + (size_t)s * kRvChunkCols + o, ring + (size_t)(kRvChunks + s) * kRvChunkCols + o, true,
+                         t == last_tile ? last_cnt : kSvTile, fd, ft);
+            sv_p2_tile(fd, ft, zc, k2, needq, a.c_star != nullptr,
+                       needq ? a.qrec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr, smin, dqmax);
+          }
+        }
+        out.sd = (double)warp_sum_f(smin) * (double)k2.scale;
+        out.st = __any_sync(0xffffffffu, dqmax > 0.f) ? 1.0 : 0.0;
+      }
+      // after the row's last pass, one arrival per tile on its chunk's empty barrier (the
+      // partial last chunk's last tile also stands in for the missing ones); a warp arrives only
+      // for tiles whose landing it waited for, so no arrival can count toward an earlier use
+      if (ph.second || !sv_p2(a, ph.J)) {
+        __syncwarp();
+        if (lane == 0) {
+          for (int t = t0; t < nt; t += kSvWarps) {
+            const uint32_t n = t == nt - 1 ? (uint32_t)(kRvChunkTiles - t % kRvChunkTiles) : 1u;
+            mbar_arrive_n(&empty[(gbase + (uint32_t)(t / kRvChunkTiles)) % kRvChunks], n);
+          }
+        }
+      }
+      const int ps = p % kSvPhaseSlots;
+      ok = __all_sync(0xffffffffu, sv_wait_count(sy, &s_combined, p - kSvPhaseSlots + 1));
+      if (!ok) break;
+      if (lane == 0) {
+        wpart[ps][w] = out;
+        mbar_arrive(&phbar[ps]);
+      }
+      ++p;
     }
   }
 
@@ -1137,12 +1423,37 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   if (c.V % 4 || (uintptr_t)c.ld % 16 || (uintptr_t)c.lt % 16) return DSPARK_ENOTIMPL;
   const SvLayout Ly = sv_layout(c.B, c.gamma, c.V);
   if (c.ws_bytes < Ly.total) return DSPARK_ENOTIMPL;
-  // clusters of 3 (45 clusters on 148 SMs) stream many rows best; with fewer than about 1.3 rows
-  // per cluster, clusters of 6 spread each row over more SMs (measured on a B200: 39.0 -> 32.8 us
-  // at B = 1, gamma = 7; 129.1 -> 122.9 us at B = 32, gamma = 4; 341 -> 388 us at B = 64,
-  // gamma = 16, where 3 stays)
+  const bool greedy = c.T == 0.f;
+  const int ntile = (c.V + kSvTile - 1) / kSvTile;
+  const int rows = c.B * (c.gamma + 1);
+  // How the second pass (T > 0) reads its rows: 1 through the ring again, 2 from the row segment
+  // kept in shared memory (needs ceil(ntile / C) tiles in at most kRvChunks chunks).  Automatic:
+  // resident rows when every row has a cluster of its own (no row waits behind another's
+  // exchange: 30.7 against 32.8 us at B = 1, gamma = 7 on a B200), else the ring (at B = 64,
+  // gamma = 16 the resident kernel is held to one row per cluster at a time by the shared
+  // memory and took 588 us against 343 us).  Greedy verification has no second pass.
+  auto chunks_of = [&](int Cc) { return ((ntile + Cc - 1) / Cc + kRvChunkTiles - 1) / kRvChunkTiles; };
   int C = opt.verify_stream_cluster;
-  if (C < 1 || C > kSvMaxCluster) C = ((long long)c.B * (c.gamma + 1) * 3 < (long long)device_sm_count() * 4) ? 6 : 3;
+  int mode = greedy ? 1 : opt.verify_stream_pass2;
+  if (mode < 1 || mode > 2) {
+    const int Cr = (C >= 1 && C <= kSvMaxCluster) ? C : 8;
+    mode = ((long long)rows * Cr <= (long long)device_sm_count() && chunks_of(Cr) <= kRvChunks - 2) ? 2 : 1;
+  }
+  if (mode == 2) {
+    if (C < 1 || C > kSvMaxCluster) {
+      C = 8;  // the smallest cluster from 8 up that leaves two spare chunks
+      while (C < kSvMaxCluster && chunks_of(C) > kRvChunks - 2) ++C;
+    }
+    if (chunks_of(C) > kRvChunks) mode = 1;
+  }
+  if (mode == 1 && (C < 1 || C > kSvMaxCluster)) {
+    // clusters of 3 (45 clusters on 148 SMs) stream many rows best; with fewer than about 1.3
+    // rows per cluster, clusters of 6 spread each row over more SMs (measured on a B200: 39.0 ->
+    // 32.8 us at B = 1, gamma = 7; 129.1 -> 122.9 us at B = 32, gamma = 4; 341 -> 388 us at
+    // B = 64, gamma = 16, where 3 stays)
+    C = ((long long)rows * 3 < (long long)device_sm_count() * 4) ? 6 : 3;
+  }
+  const bool resident = mode == 2;
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   SvArgs a{};
   a.ld = c.ld;
@@ -1159,12 +1470,14 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.lt_nrows = c.lt_nrows;
   ld_strides(c.ld_layout, c.B, c.gamma, c.V, a.ld_sk, a.ld_sb);
   a.njobs = c.B * (c.gamma + 1);
-  a.ntile = (c.V + kSvTile - 1) / kSvTile;
-  a.lag = 1;  // a row's second pass right after the next row's first (lags of 2 and 3 measured slower)
+  a.ntile = ntile;
+  // streaming: a row's second pass right after the next row's first (lags of 2 and 3 measured
+  // slower); resident: the same when two rows and a spare chunk fit, else right after its own
+  a.lag = (!resident || 2 * chunks_of(C) + 1 <= kRvChunks) ? 1 : 0;
   a.l2hint = opt.verify_stream_l2hint;
   a.wait_ns = opt.debug_wait_limit > 0 ? (uint64_t)std::min<long>(opt.debug_wait_limit, (long)kSvTimeoutNs) : kSvTimeoutNs;
   a.xbar_extra = opt.debug_unreachable_barrier == 2 ? 1 : 0;
-  a.greedy = c.T == 0.f ? 1 : 0;
+  a.greedy = greedy ? 1 : 0;
   a.zscale = a.greedy ? 0.f : (float)(1.4426950408889634 / (double)c.T);
   a.do_verify = 1;
   a.c_star = c.c_star;
@@ -1177,9 +1490,11 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.part = reinterpret_cast<double2*>(ws + Ly.part);
   a.trec = reinterpret_cast<float2*>(ws + Ly.trec);
   a.qrec = reinterpret_cast<float*>(ws + Ly.qrec);
-  auto kern = a.greedy ? verify_stream<true> : verify_stream<false>;
+  auto kern = resident ? verify_resident : (a.greedy ? verify_stream<true> : verify_stream<false>);
+  const size_t smem = resident ? kRvRingBytes : kSvRingBytes;
   cudaError_t rc;
-  rc = ensure_smem_attr((const void*)kern, kSvRingBytes);
+  rc = ensure_smem_attr((const void*)kern, smem);
+  if (rc == cudaSuccess && C > 8) rc = ensure_nonportable_cluster((const void*)kern);
   if (rc != cudaSuccess) {
     set_error(std::string("cudaFuncSetAttribute(verify_stream): ") + cudaGetErrorString(rc));
     return DSPARK_ECUDA;
@@ -1191,7 +1506,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kSvThreads);
-  cfg.dynamicSmemBytes = kSvRingBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = c.stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1201,13 +1516,20 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int ncl = 0;
-  for (; C >= 1; --C) {
+  // a cluster size the device cannot hold: smaller streaming clusters, larger resident ones
+  for (; C >= 1 && C <= kSvMaxCluster; C += resident ? 1 : -1) {
+    if (C > 8 && ensure_nonportable_cluster((const void*)kern) != cudaSuccess) {
+      (void)cudaGetLastError();
+      break;
+    }
     attr[0].val.clusterDim.x = C;
     cfg.gridDim = dim3((unsigned)C);
     if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) == cudaSuccess && ncl > 0) break;
     (void)cudaGetLastError();
+    ncl = 0;
   }
-  if (C < 1 || ncl <= 0) return DSPARK_ENOTIMPL;
+  if (C < 1 || C > kSvMaxCluster || ncl <= 0) return DSPARK_ENOTIMPL;
+  if (resident) a.lag = 2 * chunks_of(C) + 1 <= kRvChunks ? 1 : 0;
   a.C = C;
   ncl = std::min(ncl, a.njobs);
   cfg.gridDim = dim3((unsigned)(ncl * C));
