@@ -98,14 +98,8 @@ const char* dspark_last_error(void);
  *                     read from HBM once, rows exchanged through L2; slower at the sizes measured);
  *                     2 the per-row cluster kernels.  Calls the chosen kernels cannot take fall
  *                     back to the next ones and finally to the per-row kernels.
- *   "verify_stream_cluster"  CTAs per cluster of the streaming verify, 1..16; 0 (default): 3, or
- *                     6 when B*(gamma+1) is below 4/3 of the SM count (few rows per cluster); for
- *                     resident rows the smallest size from 8 up whose row segment fits
- *   "verify_stream_pass2"    streaming verify with T > 0, where the second pass reads a row:
- *                     1 through the copy ring again (from L2); 2 from the CTA's row segment kept
- *                     in shared memory since the first pass (every row read from HBM once; rows
- *                     whose segment does not fit take 1); 0 (default) 2 when every row has a
- *                     cluster of its own (B*(gamma+1)*8 <= SM count), else 1
+ *   "verify_stream_cluster"  CTAs per cluster of the streaming verify, 1..16; 0 (default) picks 3,
+ *                     or 6 when B*(gamma+1) is below 4/3 of the SM count (few rows per cluster)
  *   "verify_stream_l2hint"   1 (default) first-pass copies evict-last, second-pass evict-first
  *   "verify_groups"   column-sliced verify: CTA groups (0: slices of about 16 KB per row)
  *   "verify_cluster"  0 automatic, else the cluster size of the per-row verify kernels (1..16,

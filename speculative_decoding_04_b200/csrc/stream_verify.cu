@@ -617,7 +617,6 @@ struct SvRoles {
   SvPart (*wpart)[kSvWarps];    // [kSvPhaseSlots][kSvWarps]
   SvPart (*xs)[kSvMaxCluster];  // [kSvJobSlots][C]: the cluster's partials of a row's first pass
   uint64_t* xbar;               // [kSvJobSlots]: all C partials of the row have arrived
-  uint64_t* nbar;               // [kSvJobSlots]: the row's normalisers are in dec[].nm
   uint64_t* dbar;               // [kSvJobSlots]: the row is decided (dec[] complete)
   SvDec* dec;                   // [kSvJobSlots]
   volatile int* decided;        // rows of this cluster's sequence decided by this CTA
@@ -717,10 +716,6 @@ __device__ __forceinline__ void sv_decide_role(const SvArgs& a, const SvSync& sy
       else nm.Kd = nm.lamd = 0.f;
       if (!good) dfl |= DSPARK_FLAG_NONFINITE;
       row.nm = nm;
-      if (lane == 0) {
-        r.dec[js].nm = nm;
-        mbar_arrive(&r.nbar[js]);  // a second pass that needs only the normalisers may start
-      }
       if (J.verify) {
         if ((unsigned)xk >= (unsigned)a.V) {
           dfl |= DSPARK_FLAG_TOKEN_RANGE;
@@ -738,7 +733,7 @@ __device__ __forceinline__ void sv_decide_role(const SvArgs& a, const SvSync& sy
       const int enc = a.gamma + 1 - J.k;
       const bool rej = J.verify && !row.acc;
       const bool needq = rej && rej_seen <= enc;
-      if (lane == 0) r.dec[js].needq = needq ? 1 : 0;
+      if (lane == 0) r.dec[js] = SvDec{nm, needq ? 1 : 0, 0, 0, 0};
       if (rej && rank == 0 && lane == 0) atomicMax(a.rej + J.b, enc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&r.dbar[js]);  // the second pass of this row may start
@@ -766,7 +761,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   extern __shared__ __align__(128) float ring[];  // [kSvStages][2][kSvBig]: l_d columns, l_t columns
   __shared__ __align__(8) uint64_t full[kSvStages], empty[kSvStages];
   __shared__ __align__(8) uint64_t phbar[kSvPhaseSlots];
-  __shared__ __align__(8) uint64_t xbar[kSvJobSlots], nbar[kSvJobSlots], dbar[kSvJobSlots];
+  __shared__ __align__(8) uint64_t xbar[kSvJobSlots], dbar[kSvJobSlots];
   __shared__ SvPart wpart[kSvPhaseSlots][kSvWarps];
   __shared__ SvPart xs[kSvJobSlots][kSvMaxCluster];
   __shared__ SvDec dec[kSvJobSlots];
@@ -775,7 +770,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   __shared__ volatile int s_combined;  // passes whose warp partials the combiner has read
 
   const SvSync sy{&s_abort, a.status, a.wait_ns};
-  const SvRoles roles{phbar, wpart, xs, xbar, nbar, dbar, dec, &s_decided, &s_combined};
+  const SvRoles roles{phbar, wpart, xs, xbar, dbar, dec, &s_decided, &s_combined};
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSvStages; ++i) {
       mbar_init(&full[i], 1);
@@ -784,7 +779,6 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
     for (int i = 0; i < kSvJobSlots; ++i) {
       mbar_init(&xbar[i], 1);  // the decider's arrival; the partials count as transaction bytes
-      mbar_init(&nbar[i], 1);
       mbar_init(&dbar[i], 1);
     }
     s_abort = 0;
@@ -984,219 +978,6 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
         sv_p2_tile(fd, ft, zc, k2, needq, a.c_star != nullptr, needq ? a.qrec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr,
                    smin, dqmax);
       }
-    }
-  }
-
-  __syncwarp();
-  sv_cluster_sync_all();  // no CTA leaves while a peer may still write into its shared memory
-}
-
-// ---------------------------------------------------------------------------------------------
-// Resident rows (T > 0): every row of l_d and l_t read from HBM once.
-//
-// The same cluster layout, roles and records as verify_stream, but a CTA keeps its whole
-// segment of a row pair in shared memory from the first pass to the second, so the second pass
-// reads shared memory instead of copying the tiles again.  The ring is cut into chunks of
-// kRvChunkTiles tiles (one bulk copy per row and chunk); a row starts on a chunk boundary and
-// holds ceil(nt / kRvChunkTiles) chunks until its second pass ends (or its first, for a row
-// without one), when each tile's warp arrives on its chunk.  With a lag of 1 (two rows'
-// chunks and one spare fit) the consumers run P1(row i) before P2(row i-1), as verify_stream
-// does; with a lag of 0 (one row and a spare fit) P2(row i) follows P1(row i) and the copies of
-// row i+1 go on into the spare chunks while the row is decided.  Every copy carries the
-// evict-first policy: nothing is read twice from L2.
-constexpr int kRvChunkTiles = 4;                        // tiles per chunk: copies of 8 KB per row
-constexpr int kRvChunkCols = kRvChunkTiles * kSvTile;
-constexpr int kRvChunks = 12;                           // 12 chunks of (l_d, l_t): 192 KB
-constexpr size_t kRvRingBytes = (size_t)kRvChunks * 2 * kRvChunkCols * sizeof(float);
-
-__global__ void __launch_bounds__(kSvThreads, 1) verify_resident(SvArgs a) {
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int cid = blockIdx.x / C, ncl = gridDim.x / C;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  extern __shared__ __align__(128) float ring[];  // [2][kRvChunks][kRvChunkCols]: l_d chunks, then l_t chunks
-  __shared__ __align__(8) uint64_t full[kRvChunks], empty[kRvChunks];
-  __shared__ __align__(8) uint64_t phbar[kSvPhaseSlots];
-  __shared__ __align__(8) uint64_t xbar[kSvJobSlots], nbar[kSvJobSlots], dbar[kSvJobSlots];
-  __shared__ SvPart wpart[kSvPhaseSlots][kSvWarps];
-  __shared__ SvPart xs[kSvJobSlots][kSvMaxCluster];
-  __shared__ SvDec dec[kSvJobSlots];
-  __shared__ int s_abort;
-  __shared__ volatile int s_decided;
-  __shared__ volatile int s_combined;
-
-  const SvSync sy{&s_abort, a.status, a.wait_ns};
-  const SvRoles roles{phbar, wpart, xs, xbar, nbar, dbar, dec, &s_decided, &s_combined};
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kRvChunks; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kRvChunkTiles);  // one arrival per tile
-    }
-    for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
-    for (int i = 0; i < kSvJobSlots; ++i) {
-      mbar_init(&xbar[i], 1);  // the decider's arrival; the partials count as transaction bytes
-      mbar_init(&nbar[i], 1);
-      mbar_init(&dbar[i], 1);
-    }
-    s_abort = 0;
-    s_decided = 0;
-    s_combined = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  sv_cluster_sync_all();  // peers' barriers are initialised before any remote arrive
-
-  // This CTA's segment of every row: tiles tb .. tb + nt - 1, in nch chunks; row number i of
-  // the cluster's sequence occupies stream chunks i*nch .. i*nch + nch - 1.
-  const int tb = (int)((long long)rank * a.ntile / C);
-  const int nt = (int)((long long)(rank + 1) * a.ntile / C) - tb;  // may be 0
-  const int nch = (nt + kRvChunkTiles - 1) / kRvChunkTiles;
-  const float zc = a.zscale;
-
-  if (warp == kSvProducer) {
-    // ------------------------------------------------------------------ bulk copies
-    if (lane == 0 && nt > 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      uint32_t g = 0;  // stream chunk
-      bool ok = true;
-      SvJob J;
-      for (int j = sv_next(a, cid, ncl, J); ok && j >= 0; j = sv_next(a, j + ncl, ncl, J)) {
-        const float* rd = a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb;
-        const float* rt = a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, J.b, J.k) * a.V;
-        for (int h = 0; h < nch; ++h, ++g) {
-          const int s = (int)(g % kRvChunks);
-          if (!sv_wait(sy, &empty[s], ((g / kRvChunks) & 1) ^ 1)) {
-            ok = false;
-            break;
-          }
-          const int c0 = (tb + h * kRvChunkTiles) * kSvTile;
-          const int c1 = min((tb + min((h + 1) * kRvChunkTiles, nt)) * kSvTile, a.V);
-          const uint32_t bytes = (uint32_t)(c1 - c0) * 4u;
-          float* dd = ring + (size_t)s * kRvChunkCols;
-          float* dt = ring + (size_t)(kRvChunks + s) * kRvChunkCols;
-          mbar_expect_tx(&full[s], J.d ? 2 * bytes : bytes);
-          if (a.l2hint) {
-            if (J.d) bulk_g2s_hint(dd, rd + c0, bytes, &full[s], pol);
-            bulk_g2s_hint(dt, rt + c0, bytes, &full[s], pol);
-          } else {
-            if (J.d) bulk_g2s(dd, rd + c0, bytes, &full[s]);
-            bulk_g2s(dt, rt + c0, bytes, &full[s]);
-          }
-          mbar_arrive(&full[s]);
-        }
-      }
-      if (!ok) {
-        // let the copies still in flight land before the CTA can exit
-        const uint32_t lo = g > (uint32_t)kRvChunks ? g - kRvChunks : 0u;
-        for (uint32_t gb = lo; gb < g; ++gb)
-          for (uint32_t i = 0; i < kSpinLimit && !mbar_try_wait(&full[gb % kRvChunks], (gb / kRvChunks) & 1); ++i) {
-          }
-      }
-    }
-  } else if (warp == kSvCombiner) {
-    sv_combine_role<false>(a, sy, roles, C, rank, cid, ncl);
-  } else if (warp == kSvDecider) {
-    sv_decide_role<false>(a, sy, roles, C, rank, cid, ncl);
-  } else {
-    // ------------------------------------------------------------------ tile consumers
-    // Tile t of row i goes to warp (i nt + t) mod 16 in both passes, so a warp's second pass
-    // reads only tiles whose chunks it saw land in its first.
-    const int w = warp;
-    const int last_tile = a.ntile - 1 - tb;
-    const int last_cnt = a.V - (a.ntile - 1) * kSvTile;
-    int p = 0;  // passes finished by this warp (slot of the partials)
-    bool ok = true;
-    SvGen gen;
-    gen.init(a, cid, ncl);
-    SvPhase ph;
-    while (ok && gen.next(a, ph)) {
-      const uint32_t gbase = (uint32_t)ph.i * (uint32_t)nch;
-      const int t0 = (w - (int)(((long long)ph.i * nt) % kSvWarps) + kSvWarps) % kSvWarps;
-      SvPart out = sv_empty_part();
-      if (!ph.second) {
-        int Rd = kRNone, Rt = kRNone;
-        float Sd = 0.f, St = 0.f, nRd = 0.f, nRt = 0.f;
-        // every warp waits for every chunk of the row in order, its own tiles' or not: a wait on
-        // a slot's use u then always follows the landing of use u - 1, so its parity cannot
-        // match an older phase
-        int hw = 0;  // chunks of the row waited for
-        auto wait_to = [&](int h_end) {
-          for (; hw < h_end; ++hw) {
-            const uint32_t gc = gbase + (uint32_t)hw;
-            if (!__all_sync(0xffffffffu, sv_wait(sy, &full[gc % kRvChunks], (gc / kRvChunks) & 1))) return false;
-          }
-          return true;
-        };
-        for (int t = t0; t < nt; t += kSvWarps) {
-          if (!wait_to(t / kRvChunkTiles + 1)) {
-            ok = false;
-            break;
-          }
-          const int s = (int)((gbase + (uint32_t)(t / kRvChunkTiles)) % kRvChunks);
-          const int o = (t % kRvChunkTiles) * kSvTile;
-          float4 fd[kSvVec], ft[kSvVec];
-          sv_load_tile(ring + (size_t)s * kRvChunkCols + o, ring + (size_t)(kRvChunks + s) * kRvChunkCols + o, ph.J.d,
-                       t == last_tile ? last_cnt : kSvTile, fd, ft);
-          sv_p1_tile(fd, ft, zc, ph.J.d, ph.J.bonus ? a.trec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr, Rd, Sd,
-                     nRd, Rt, St, nRt);
-        }
-        if (!ok || !wait_to(nch)) {
-          ok = false;
-          break;
-        }
-        const uint32_t bad = (St <= FLT_MAX && Sd <= FLT_MAX) ? 0u : 1u;  // a non-finite logit of the pass
-        sv_warp_ref_sum_f(Rd, Sd);
-        sv_warp_ref_sum_f(Rt, St);
-        out.rd = Rd;
-        out.sd = (double)Sd;
-        out.rt = Rt;
-        out.st = (double)St;
-        out.fl = __any_sync(0xffffffffu, bad != 0) ? (uint32_t)DSPARK_FLAG_NONFINITE : 0u;
-      } else {
-        const int js = ph.i % kSvJobSlots;
-        // the normalisers suffice: the residual weights are kept for every verified row, so the
-        // pass need not wait for the acceptance decision
-        ok = __all_sync(0xffffffffu, sv_wait(sy, &nbar[js], (ph.i / kSvJobSlots) & 1));
-        if (!ok) break;
-        const SvP2 k2 = sv_p2_consts(dec[js].nm);
-        const bool needq = ph.J.verify;
-        float smin = 0.f, dqmax = -INFINITY;
-        if (needq || a.c_star) {
-          for (int t = t0; t < nt; t += kSvWarps) {
-            const int s = (int)((gbase + (uint32_t)(t / kRvChunkTiles)) % kRvChunks);
-            const int o = (t % kRvChunkTiles) * kSvTile;
-            float4 fd[kSvVec], ft[kSvVec];
-            sv_load_tile(ring + (size_t)s * kRvChunkCols + o, ring + (size_t)(kRvChunks + s) * kRvChunkCols + o, true,
-                         t == last_tile ? last_cnt : kSvTile, fd, ft);
-            sv_p2_tile(fd, ft, zc, k2, needq, a.c_star != nullptr,
-                       needq ? a.qrec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr, smin, dqmax);
-          }
-        }
-        out.sd = (double)warp_sum_f(smin) * (double)k2.scale;
-        out.st = __any_sync(0xffffffffu, dqmax > 0.f) ? 1.0 : 0.0;
-      }
-      // after the row's last pass, one arrival per tile on its chunk's empty barrier (the
-      // partial last chunk's last tile also stands in for the missing ones); a warp arrives only
-      // for tiles whose landing it waited for, so no arrival can count toward an earlier use
-      if (ph.second || !sv_p2(a, ph.J)) {
-        __syncwarp();
-        if (lane == 0) {
-          for (int t = t0; t < nt; t += kSvWarps) {
-            const uint32_t n = t == nt - 1 ? (uint32_t)(kRvChunkTiles - t % kRvChunkTiles) : 1u;
-            mbar_arrive_n(&empty[(gbase + (uint32_t)(t / kRvChunkTiles)) % kRvChunks], n);
-          }
-        }
-      }
-      const int ps = p % kSvPhaseSlots;
-      ok = __all_sync(0xffffffffu, sv_wait_count(sy, &s_combined, p - kSvPhaseSlots + 1));
-      if (!ok) break;
-      if (lane == 0) {
-        wpart[ps][w] = out;
-        mbar_arrive(&phbar[ps]);
-      }
-      ++p;
     }
   }
 
@@ -1426,34 +1207,12 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   const bool greedy = c.T == 0.f;
   const int ntile = (c.V + kSvTile - 1) / kSvTile;
   const int rows = c.B * (c.gamma + 1);
-  // How the second pass (T > 0) reads its rows: 1 through the ring again, 2 from the row segment
-  // kept in shared memory (needs ceil(ntile / C) tiles in at most kRvChunks chunks).  Automatic:
-  // resident rows when every row has a cluster of its own (no row waits behind another's
-  // exchange: 30.7 against 32.8 us at B = 1, gamma = 7 on a B200), else the ring (at B = 64,
-  // gamma = 16 the resident kernel is held to one row per cluster at a time by the shared
-  // memory and took 588 us against 343 us).  Greedy verification has no second pass.
-  auto chunks_of = [&](int Cc) { return ((ntile + Cc - 1) / Cc + kRvChunkTiles - 1) / kRvChunkTiles; };
+  // clusters of 3 (45 clusters on 148 SMs) stream many rows best; with fewer than about 1.3 rows
+  // per cluster, clusters of 6 spread each row over more SMs (measured on a B200: 39.0 -> 32.8 us
+  // at B = 1, gamma = 7; 129.1 -> 122.9 us at B = 32, gamma = 4; 341 -> 388 us at B = 64,
+  // gamma = 16, where 3 stays)
   int C = opt.verify_stream_cluster;
-  int mode = greedy ? 1 : opt.verify_stream_pass2;
-  if (mode < 1 || mode > 2) {
-    const int Cr = (C >= 1 && C <= kSvMaxCluster) ? C : 8;
-    mode = ((long long)rows * Cr <= (long long)device_sm_count() && chunks_of(Cr) <= kRvChunks - 2) ? 2 : 1;
-  }
-  if (mode == 2) {
-    if (C < 1 || C > kSvMaxCluster) {
-      C = 8;  // the smallest cluster from 8 up that leaves two spare chunks
-      while (C < kSvMaxCluster && chunks_of(C) > kRvChunks - 2) ++C;
-    }
-    if (chunks_of(C) > kRvChunks) mode = 1;
-  }
-  if (mode == 1 && (C < 1 || C > kSvMaxCluster)) {
-    // clusters of 3 (45 clusters on 148 SMs) stream many rows best; with fewer than about 1.3
-    // rows per cluster, clusters of 6 spread each row over more SMs (measured on a B200: 39.0 ->
-    // 32.8 us at B = 1, gamma = 7; 129.1 -> 122.9 us at B = 32, gamma = 4; 341 -> 388 us at
-    // B = 64, gamma = 16, where 3 stays)
-    C = ((long long)rows * 3 < (long long)device_sm_count() * 4) ? 6 : 3;
-  }
-  const bool resident = mode == 2;
+  if (C < 1 || C > kSvMaxCluster) C = ((long long)rows * 3 < (long long)device_sm_count() * 4) ? 6 : 3;
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   SvArgs a{};
   a.ld = c.ld;
@@ -1471,9 +1230,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   ld_strides(c.ld_layout, c.B, c.gamma, c.V, a.ld_sk, a.ld_sb);
   a.njobs = c.B * (c.gamma + 1);
   a.ntile = ntile;
-  // streaming: a row's second pass right after the next row's first (lags of 2 and 3 measured
-  // slower); resident: the same when two rows and a spare chunk fit, else right after its own
-  a.lag = (!resident || 2 * chunks_of(C) + 1 <= kRvChunks) ? 1 : 0;
+  a.lag = 1;  // a row's second pass right after the next row's first (lags of 0, 2 and 3 measured slower)
   a.l2hint = opt.verify_stream_l2hint;
   a.wait_ns = opt.debug_wait_limit > 0 ? (uint64_t)std::min<long>(opt.debug_wait_limit, (long)kSvTimeoutNs) : kSvTimeoutNs;
   a.xbar_extra = opt.debug_unreachable_barrier == 2 ? 1 : 0;
@@ -1490,8 +1247,8 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.part = reinterpret_cast<double2*>(ws + Ly.part);
   a.trec = reinterpret_cast<float2*>(ws + Ly.trec);
   a.qrec = reinterpret_cast<float*>(ws + Ly.qrec);
-  auto kern = resident ? verify_resident : (a.greedy ? verify_stream<true> : verify_stream<false>);
-  const size_t smem = resident ? kRvRingBytes : kSvRingBytes;
+  auto kern = a.greedy ? verify_stream<true> : verify_stream<false>;
+  const size_t smem = kSvRingBytes;
   cudaError_t rc;
   rc = ensure_smem_attr((const void*)kern, smem);
   if (rc == cudaSuccess && C > 8) rc = ensure_nonportable_cluster((const void*)kern);
@@ -1516,8 +1273,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int ncl = 0;
-  // a cluster size the device cannot hold: smaller streaming clusters, larger resident ones
-  for (; C >= 1 && C <= kSvMaxCluster; C += resident ? 1 : -1) {
+  for (; C >= 1; --C) {  // a cluster size the device cannot hold: try smaller ones
     if (C > 8 && ensure_nonportable_cluster((const void*)kern) != cudaSuccess) {
       (void)cudaGetLastError();
       break;
@@ -1528,8 +1284,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
     (void)cudaGetLastError();
     ncl = 0;
   }
-  if (C < 1 || C > kSvMaxCluster || ncl <= 0) return DSPARK_ENOTIMPL;
-  if (resident) a.lag = 2 * chunks_of(C) + 1 <= kRvChunks ? 1 : 0;
+  if (C < 1 || ncl <= 0) return DSPARK_ENOTIMPL;
   a.C = C;
   ncl = std::min(ncl, a.njobs);
   cfg.gridDim = dim3((unsigned)(ncl * C));
