@@ -57,9 +57,7 @@ namespace {
 constexpr int kSvTile = 512;    // columns per tile (one consumer warp's piece of a stage)
 constexpr int kSvWarps = 16;    // consumer warps (four per scheduler: the passes are latency-bound)
 constexpr int kSvVec = kSvTile / 128;  // float4s per lane and row in a piece
-constexpr int kSvGroups = 1;                       // consumer groups; stage g goes to group g mod kSvGroups
-constexpr int kSvGroupWarps = kSvWarps / kSvGroups;  // warps per group, one piece each
-constexpr int kSvBig = kSvGroupWarps * kSvTile;      // columns per ring stage: one 32 KB copy per row
+constexpr int kSvBig = kSvWarps * kSvTile;          // columns per ring stage: one 32 KB copy per row
 constexpr int kSvStages = 3;                         // ring stages of (l_d 8192 columns, l_t 8192 columns)
 constexpr int kSvThreads = (kSvWarps + 3) * 32;
 constexpr int kSvProducer = kSvWarps;
@@ -774,7 +772,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSvStages; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kSvGroupWarps);
+      mbar_init(&empty[i], kSvWarps);
     }
     for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
     for (int i = 0; i < kSvJobSlots; ++i) {
@@ -813,7 +811,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
           ok = false;
           break;
         }
-        const int T0 = (int)g * kSvGroupWarps, T1 = T0 + kSvGroupWarps;
+        const int T0 = (int)g * kSvWarps, T1 = T0 + kSvWarps;
         float* stg = ring + (size_t)s * 2 * kSvBig;
         // one copy per row for each pass that has tiles in this stage
         while (have && pbase < T1) {
@@ -931,8 +929,8 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     if (have) start();
     int pbase = 0;
     for (uint32_t g = 0; ok && have; ++g) {
-      const int q = (w + (int)g) & (kSvGroupWarps - 1);  // slot of this warp in stage g
-      const int T = (int)g * kSvGroupWarps + q;
+      const int q = (w + (int)g) & (kSvWarps - 1);  // slot of this warp in stage g
+      const int T = (int)g * kSvWarps + q;
       while (T >= pbase + nt) {  // passes that end before this tile
         finish();
         if (!ok) break;
