@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
     fence_mbar_init();
   }
   __syncthreads();
-  sv_cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+  sv_cluster_sync_all();  // peers' barriers are initialised before any remote store completes on them
 
   // This CTA's segment of every row: tiles tb .. tb + nt - 1.  Pass number p of the CTA's
   // sequence covers tiles p*nt .. p*nt + nt - 1 of the CTA's tile stream; stage g of the ring
