@@ -414,13 +414,6 @@ __device__ __forceinline__ float f4c(const float4& v, int c) { return c == 0 ? v
 
 // Packed fp32 pairs (sm_100): per element the same correctly rounded results as the scalar
 // instructions, at half the instruction count.
-__device__ __forceinline__ float2 f2mul(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
 __device__ __forceinline__ float2 f2add(float2 a, float2 b) {
   float2 d;
   asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -868,7 +861,7 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
 
     SvGen cgen;
     cgen.init(a, cid, ncl);
-    SvPhase ph;
+    SvPhase ph{};
     auto start = [&]() {
       Rd = Rt = kRNone;
       Sd = St = 0.f;
