@@ -121,7 +121,6 @@ int dspark_set_option(const char* key, long value) {
   else if (!std::strcmp(key, "verify_groups")) o.verify_groups = (int)value;
   else if (!std::strcmp(key, "verify_stream_cluster")) o.verify_stream_cluster = (int)value;
   else if (!std::strcmp(key, "verify_stream_l2hint")) o.verify_stream_l2hint = (int)value;
-  else if (!std::strcmp(key, "verify_stream_tmem")) o.verify_stream_tmem = (int)value;
   else if (!std::strcmp(key, "sm_count")) o.sm_count = (int)value;
   else if (!std::strcmp(key, "debug_wait_limit")) o.debug_wait_limit = value;
   else if (!std::strcmp(key, "debug_unreachable_barrier")) o.debug_unreachable_barrier = (int)value;

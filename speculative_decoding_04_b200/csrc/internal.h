@@ -24,7 +24,6 @@ struct Options {
   int verify_groups = 0;         // sliced verify: CTA groups (0: slices of about 16 KB per row)
   int verify_stream_cluster = 0; // CTAs per cluster of the streaming verify (1 to 16; 0: automatic)
   int verify_stream_l2hint = 1;  // streaming verify: first-pass copies evict-last, second-pass evict-first
-  int verify_stream_tmem = 1;    // streaming verify, T > 0: the second pass from tensor memory where a row segment fits
   int sm_count = 0;              // 0: query the device
   // test-only: make the bounded device waits give up sooner and one of them unsatisfiable, so that
   // a test can check that the kernels return with a timeout status (never on in normal use)

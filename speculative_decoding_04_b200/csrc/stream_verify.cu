@@ -976,230 +976,6 @@ __global__ void __launch_bounds__(kSvThreads, 1) verify_stream(SvArgs a) {
   sv_cluster_sync_all();  // no CTA leaves while a peer may still write into its shared memory
 }
 
-// ---------------------------------------------------------------------------------------------
-// Second pass from tensor memory (T > 0).
-//
-// verify_stream sends every row through the SM's copy engine twice, and with the 192 KB ring in
-// flight the copy engine moves about 70 GB/s per SM, which bounds that kernel per CTA.  Here the
-// producer copies each row once (the first pass, evict-first) and each consumer warp, once it has
-// read a first-pass tile from the ring, writes the tile's 32 values per lane into tensor memory
-// (tcgen05.st; 256 KB per SM, otherwise idle here) and frees the stage; the row's second pass
-// reads its tiles back with tcgen05.ld.  Tile T of the CTA's first-pass stream goes to warp
-// T mod 16, one tile per warp in every stage, and is kept in one of the warp's four 32-column
-// slots of its lane quadrant.  A row segment of at most 32 tiles leaves room for two rows: slot
-// 2 (row mod 2) + (the tile's index among the warp's tiles of the row), and the lag-1 order
-// P1(i), P2(i-1) of the combine and decide roles.  A segment of 33 to 64 tiles fills the four
-// slots alone: lag 0, P1(i), P2(i), where the ring, already free, streams row i + 1 in while row
-// i is exchanged and decided.  The second pass reads tensor memory alone.
-constexpr int kTmCols = 512;      // tensor-memory columns: per lane quadrant, 4 warps x 128
-constexpr int kTmMaxTiles = 64;   // tiles of a CTA's row segment that fit (four per warp)
-constexpr int kTmLag1Tiles = 32;  // ... and two rows of them
-static_assert(kSvWarps == 16, "four consumer warps per lane quadrant");
-
-__global__ void __launch_bounds__(kSvThreads, 1) verify_stream_tm(SvArgs a) {
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int cid = blockIdx.x / C, ncl = gridDim.x / C;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  extern __shared__ __align__(128) float ring[];  // [kSvStages][2][kSvBig]: l_d columns, l_t columns
-  __shared__ __align__(8) uint64_t full[kSvStages], empty[kSvStages];
-  __shared__ __align__(8) uint64_t phbar[kSvPhaseSlots];
-  __shared__ __align__(8) uint64_t xbar[kSvJobSlots], dbar[kSvJobSlots];
-  __shared__ SvPart wpart[kSvPhaseSlots][kSvWarps];
-  __shared__ SvPart xs[kSvJobSlots][kSvMaxCluster];
-  __shared__ SvDec dec[kSvJobSlots];
-  __shared__ int s_abort;
-  __shared__ volatile int s_decided;
-  __shared__ volatile int s_combined;
-  __shared__ uint32_t s_tmem;
-
-  const SvSync sy{&s_abort, a.status, a.wait_ns};
-  const SvRoles roles{phbar, wpart, xs, xbar, dbar, dec, &s_decided, &s_combined};
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kSvStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kSvWarps);
-    }
-    for (int i = 0; i < kSvPhaseSlots; ++i) mbar_init(&phbar[i], kSvWarps);
-    for (int i = 0; i < kSvJobSlots; ++i) {
-      mbar_init(&xbar[i], 1);  // the decider's arrival; the partials count as transaction bytes
-      mbar_init(&dbar[i], 1);
-    }
-    s_abort = 0;
-    s_decided = 0;
-    s_combined = 0;
-    fence_mbar_init();
-  }
-  if (warp == kSvProducer) {
-    tmem_alloc(&s_tmem, kTmCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_tmem;
-  sv_cluster_sync_all();  // peers' barriers are initialised before any remote store completes on them
-
-  const int tb = (int)((long long)rank * a.ntile / C);
-  const int nt = (int)((long long)(rank + 1) * a.ntile / C) - tb;  // 0 .. kTmMaxTiles (.. kTmLag1Tiles at lag 1)
-  const float zc = a.zscale;
-
-  if (warp == kSvProducer) {
-    // ------------------------------------------------------------------ bulk copies (first pass)
-    if (lane == 0 && nt > 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      SvJob J;
-      int j = sv_next(a, cid, ncl, J);
-      int rbase = 0;  // first stream tile of row j
-      uint32_t g = 0;
-      bool ok = true;
-      for (; j >= 0; ++g) {
-        const int s = (int)(g % kSvStages);
-        if (!sv_wait(sy, &empty[s], ((g / kSvStages) & 1) ^ 1)) {
-          ok = false;
-          break;
-        }
-        const int T0 = (int)g * kSvWarps, T1 = T0 + kSvWarps;
-        float* stg = ring + (size_t)s * 2 * kSvBig;
-        while (j >= 0 && rbase < T1) {
-          const int lo = max(T0, rbase), hi = min(T1, rbase + nt);
-          const int c0 = (tb + lo - rbase) * kSvTile, c1 = min((tb + hi - rbase) * kSvTile, a.V);
-          const uint32_t bytes = (uint32_t)(c1 - c0) * 4u;
-          const float* rd = a.ld + (size_t)J.k * a.ld_sk + (size_t)J.b * a.ld_sb;
-          const float* rt = a.lt + lt_row_index(a.lt_off, a.lt_nrows, a.lt_rows, J.b, J.k) * a.V;
-          mbar_expect_tx(&full[s], J.d ? 2 * bytes : bytes);
-          if (a.l2hint) {
-            if (J.d) bulk_g2s_hint(stg + (lo - T0) * kSvTile, rd + c0, bytes, &full[s], pol);
-            bulk_g2s_hint(stg + kSvBig + (lo - T0) * kSvTile, rt + c0, bytes, &full[s], pol);
-          } else {
-            if (J.d) bulk_g2s(stg + (lo - T0) * kSvTile, rd + c0, bytes, &full[s]);
-            bulk_g2s(stg + kSvBig + (lo - T0) * kSvTile, rt + c0, bytes, &full[s]);
-          }
-          if (hi < rbase + nt) break;  // the row goes on in the next stage
-          j = sv_next(a, j + ncl, ncl, J);
-          rbase += nt;
-        }
-        mbar_arrive(&full[s]);
-      }
-      if (!ok) {
-        // let the copies still in flight land before the CTA can exit
-        const uint32_t lo = g > (uint32_t)kSvStages ? g - kSvStages : 0u;
-        for (uint32_t gb = lo; gb < g; ++gb)
-          for (uint32_t i = 0; i < kSpinLimit && !mbar_try_wait(&full[gb % kSvStages], (gb / kSvStages) & 1); ++i) {
-          }
-      }
-    }
-  } else if (warp == kSvCombiner) {
-    sv_combine_role<false>(a, sy, roles, C, rank, cid, ncl);
-  } else if (warp == kSvDecider) {
-    sv_decide_role<false>(a, sy, roles, C, rank, cid, ncl);
-  } else {
-    // ------------------------------------------------------------------ tile consumers
-    const int w = warp;
-    // this warp's 128 columns of its lane quadrant (lanes 32 (w mod 4) .. + 31)
-    const uint32_t tw = tmem + ((uint32_t)(32 * (w & 3)) << 16) + (uint32_t)((w >> 2) * 128);
-    const int last_tile = a.ntile - 1 - tb;  // the segment's ragged tile, if it has it
-    const int last_cnt = a.V - (a.ntile - 1) * kSvTile;
-    int p = 0;  // passes published by this warp
-    bool ok = true;
-    SvGen gen;
-    gen.init(a, cid, ncl);
-    SvPhase ph{};
-    while (ok && gen.next(a, ph)) {
-      // the warp's tiles of the row are t0 and t0 + 16 (stream tile i nt + t is warp (i nt + t) mod 16's)
-      const int t0 = (int)((((long long)w - (long long)ph.i * nt) % kSvWarps + kSvWarps) % kSvWarps);
-      const uint32_t slot0 = tw + (uint32_t)((a.lag ? (ph.i & 1) * 2 : 0) * 32);
-      SvPart out = sv_empty_part();
-      if (!ph.second) {
-        int Rd = kRNone, Rt = kRNone;
-        float Sd = 0.f, St = 0.f, nRd = 0.f, nRt = 0.f;
-        for (int t = t0; t < nt; t += kSvWarps) {
-          // stage g holds stream tiles 16 g .. 16 g + 15; this warp's is 16 g + w
-          const uint32_t g = (uint32_t)(((long long)ph.i * nt + t - w) / kSvWarps);
-          const int s = (int)(g % kSvStages);
-          if (!__all_sync(0xffffffffu, sv_wait(sy, &full[s], (g / kSvStages) & 1))) {
-            ok = false;
-            break;
-          }
-          const float* sd = ring + (size_t)s * 2 * kSvBig + w * kSvTile;
-          float4 fd[kSvVec], ft[kSvVec];
-          sv_load_tile(sd, sd + kSvBig, ph.J.d, t == last_tile ? last_cnt : kSvTile, fd, ft);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[s]);  // the values are in registers
-          float v[32];
-#pragma unroll
-          for (int jj = 0; jj < kSvVec; ++jj) {
-            v[4 * jj + 0] = fd[jj].x;
-            v[4 * jj + 1] = fd[jj].y;
-            v[4 * jj + 2] = fd[jj].z;
-            v[4 * jj + 3] = fd[jj].w;
-            v[16 + 4 * jj + 0] = ft[jj].x;
-            v[16 + 4 * jj + 1] = ft[jj].y;
-            v[16 + 4 * jj + 2] = ft[jj].z;
-            v[16 + 4 * jj + 3] = ft[jj].w;
-          }
-          tmem_st_32x32b_x32(slot0 + (uint32_t)((t / kSvWarps) * 32), v);  // kept for the second pass
-          sv_p1_tile(fd, ft, zc, ph.J.d, ph.J.bonus ? a.trec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr, Rd, Sd,
-                     nRd, Rt, St, nRt);
-        }
-        if (!ok) break;
-        const uint32_t bad = (St <= FLT_MAX && Sd <= FLT_MAX) ? 0u : 1u;  // a non-finite logit of the pass
-        sv_warp_ref_sum_f(Rd, Sd);
-        sv_warp_ref_sum_f(Rt, St);
-        out.rd = Rd;
-        out.sd = (double)Sd;
-        out.rt = Rt;
-        out.st = (double)St;
-        out.fl = __any_sync(0xffffffffu, bad != 0) ? (uint32_t)DSPARK_FLAG_NONFINITE : 0u;
-      } else {
-        const int js = ph.i % kSvJobSlots;
-        ok = __all_sync(0xffffffffu, sv_wait(sy, &dbar[js], (ph.i / kSvJobSlots) & 1));
-        if (!ok) break;
-        const SvDec dd = dec[js];
-        const SvP2 k2 = sv_p2_consts(dd.nm);
-        const bool needq = dd.needq != 0;
-        float smin = 0.f, dqmax = -INFINITY;
-        if (needq || a.c_star) {
-          tmem_wait_st();  // this warp's stores of the row's tiles have completed
-          for (int t = t0; t < nt; t += kSvWarps) {
-            float v[32];
-            tmem_ld_32x32b_x32(slot0 + (uint32_t)((t / kSvWarps) * 32), v);
-            float4 fd[kSvVec], ft[kSvVec];
-#pragma unroll
-            for (int jj = 0; jj < kSvVec; ++jj) {
-              fd[jj] = make_float4(v[4 * jj], v[4 * jj + 1], v[4 * jj + 2], v[4 * jj + 3]);
-              ft[jj] = make_float4(v[16 + 4 * jj], v[16 + 4 * jj + 1], v[16 + 4 * jj + 2], v[16 + 4 * jj + 3]);
-            }
-            sv_p2_tile(fd, ft, zc, k2, needq, a.c_star != nullptr,
-                       needq ? a.qrec + (size_t)ph.J.rec * a.ntile + tb + t : nullptr, smin, dqmax);
-          }
-        }
-        out.sd = (double)warp_sum_f(smin) * (double)k2.scale;
-        out.st = __any_sync(0xffffffffu, dqmax > 0.f) ? 1.0 : 0.0;
-      }
-      const int ps = p % kSvPhaseSlots;
-      ok = __all_sync(0xffffffffu, sv_wait_count(sy, &s_combined, p - kSvPhaseSlots + 1));
-      if (!ok) break;
-      if (lane == 0) {
-        wpart[ps][w] = out;
-        mbar_arrive(&phbar[ps]);
-      }
-      ++p;
-    }
-    tmem_wait_st();  // stores of tiles whose second pass never came (rows without one, a timeout)
-  }
-
-  // tensor memory is released once every warp's accesses have completed
-  __syncwarp();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == kSvProducer) tmem_dealloc(tmem, kTmCols);
-  sv_cluster_sync_all();  // no CTA leaves while a peer may still write into its shared memory
-}
-
 // Inverse-CDF sample of row `rec` (one warp): weights q = max(0, p_t - p_d) when `resid`
 // (falling back to p_t when their sum is 0), else p_t.  Tile weights come from the records of
 // the main kernel (q of a rejected row, p_t of the bonus row); the p_t fallback of a rejected
@@ -1426,20 +1202,8 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   // per cluster, clusters of 6 spread each row over more SMs (measured on a B200: 39.0 -> 32.8 us
   // at B = 1, gamma = 7; 129.1 -> 122.9 us at B = 32, gamma = 4; 341 -> 388 us at B = 64,
   // gamma = 16, where 3 stays)
-  const int C_ring = ((long long)rows * 3 < (long long)device_sm_count() * 4) ? 6 : 3;
   int C = opt.verify_stream_cluster;
-  // T > 0: the second pass from tensor memory when a CTA's row segment fits there (at most
-  // kTmMaxTiles tiles: the smallest such cluster from the ring's size up; lag 1 when two rows fit)
-  auto tiles_of = [&](int Cc) { return (ntile + Cc - 1) / Cc; };
-  bool tm = !greedy && opt.verify_stream_tmem != 0;
-  if (tm) {
-    if (C < 1 || C > kSvMaxCluster) {
-      C = C_ring;
-      while (C < kSvMaxCluster && tiles_of(C) > kTmMaxTiles) ++C;
-    }
-    if (tiles_of(C) > kTmMaxTiles) tm = false;
-  }
-  if (C < 1 || C > kSvMaxCluster) C = C_ring;
+  if (C < 1 || C > kSvMaxCluster) C = ((long long)rows * 3 < (long long)device_sm_count() * 4) ? 6 : 3;
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   SvArgs a{};
   a.ld = c.ld;
@@ -1474,7 +1238,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   a.part = reinterpret_cast<double2*>(ws + Ly.part);
   a.trec = reinterpret_cast<float2*>(ws + Ly.trec);
   a.qrec = reinterpret_cast<float*>(ws + Ly.qrec);
-  auto kern = tm ? verify_stream_tm : (a.greedy ? verify_stream<true> : verify_stream<false>);
+  auto kern = a.greedy ? verify_stream<true> : verify_stream<false>;
   const size_t smem = kSvRingBytes;
   cudaError_t rc;
   rc = ensure_smem_attr((const void*)kern, smem);
@@ -1500,9 +1264,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int ncl = 0;
-  // a cluster size the device cannot hold: smaller ones for the ring, larger ones for tensor
-  // memory (whose row segments only shrink)
-  for (; C >= 1 && C <= kSvMaxCluster; C += tm ? 1 : -1) {
+  for (; C >= 1; --C) {  // a cluster size the device cannot hold: try smaller ones
     if (C > 8 && ensure_nonportable_cluster((const void*)kern) != cudaSuccess) {
       (void)cudaGetLastError();
       break;
@@ -1513,8 +1275,7 @@ dspark_status launch_verify_stream(const VerifyCall& c) {
     (void)cudaGetLastError();
     ncl = 0;
   }
-  if (C < 1 || C > kSvMaxCluster || ncl <= 0) return DSPARK_ENOTIMPL;
-  if (tm) a.lag = tiles_of(C) <= kTmLag1Tiles ? 1 : 0;
+  if (C < 1 || ncl <= 0) return DSPARK_ENOTIMPL;
   a.C = C;
   ncl = std::min(ncl, a.njobs);
   cfg.gridDim = dim3((unsigned)(ncl * C));

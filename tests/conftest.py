@@ -34,4 +34,3 @@ def _default_options():
         D.set_option("verify_groups", 0)
         D.set_option("verify_stream_cluster", 0)
         D.set_option("verify_stream_l2hint", 1)
-        D.set_option("verify_stream_tmem", 1)

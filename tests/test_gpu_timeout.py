@@ -48,8 +48,8 @@ def test_fused_draft_grid_barrier_times_out_and_returns():
     check_draft(d["U"], d["W1"], d["W2"], d["x0"], d["u_draft"], wl.T, host(x), host_rm(ld), host(fl))
 
 
-@pytest.mark.parametrize("T,tmem", [(1.0, 1), (1.0, 0), (0.0, 1)])
-def test_stream_verify_exchange_times_out_and_returns(T, tmem):
+@pytest.mark.parametrize("T", [1.0, 0.0])
+def test_stream_verify_exchange_times_out_and_returns(T):
     wl = inputs.SINGLE_USER.with_(name="timeout_v", B=10, gamma=4, V=20000, T=T, seed=72)
     ld, lt = inputs.logits(wl)
     u_draft, u_acc, u_res = inputs.uniforms(wl)
@@ -57,7 +57,6 @@ def test_stream_verify_exchange_times_out_and_returns(T, tmem):
     ws = D.workspace(D.WS_VERIFY, wl.B, wl.gamma, wl.V)
     args = (pm(ld), dev(lt), dev(x), None, dev(u_acc), dev(u_res), T)
     D.set_option("verify_impl", 0)                    # the streaming kernels
-    D.set_option("verify_stream_tmem", tmem)          # T > 0: the second pass from tensor memory or the ring
     D.set_option("debug_wait_limit", 20_000_000)      # nanoseconds per wait
     D.set_option("debug_unreachable_barrier", 2)      # the cluster exchange expects one CTA more
     n, y, c, fl = D.verify(*args, want_c_star=True, ws=ws)

@@ -29,23 +29,20 @@ def run_verify(ld, lt, x, L, u_acc, u_res, T, want_c=True):
     return host(n), host(y), (host(c) if c is not None else None), host(fl)
 
 
-# kernels: "stream-C" = streaming kernels with clusters of C CTAs, both passes through the copy
-# ring (C = 0: automatic, C > 8: non-portable cluster sizes); "tmem-C" = the same with the second
-# pass read back from tensor memory (the default with a workspace for T > 0 where a CTA's row
-# segment fits; greedy calls and wider segments take the ring); "sliced-G" = column-sliced kernels with G groups of CTAs (0: slices of about 16 KB);
+# kernels: "stream-C" = streaming kernels with clusters of C CTAs (the default with a workspace;
+# C = 0: automatic, C > 8: non-portable cluster sizes); "sliced-G" = column-sliced kernels with G groups of CTAs (0: slices of about 16 KB);
 # "rows-C" = one cluster of C CTAs per row (0: chosen from V), which serves calls without a
 # workspace, V not a multiple of 4 and the labels entry point.
 IMPLS = ["sliced-0", "sliced-1", "sliced-3", "sliced-16", "stream-0", "stream-16", "stream-8", "stream-3", "stream-1",
-         "tmem-0", "tmem-2", "tmem-3", "tmem-7", "tmem-16", "rows-0", "rows-1", "rows-4", "rows-16"]
+         "rows-0", "rows-1", "rows-4", "rows-16"]
 
 
 def use_impl(impl):
     kind, c = impl.split("-")
-    D.set_option("verify_impl", {"stream": 0, "tmem": 0, "sliced": 1, "rows": 2}[kind])
+    D.set_option("verify_impl", {"stream": 0, "sliced": 1, "rows": 2}[kind])
     if kind == "sliced":
         D.set_option("verify_groups", int(c))
-    elif kind in ("stream", "tmem"):
-        D.set_option("verify_stream_tmem", 1 if kind == "tmem" else 0)
+    elif kind == "stream":
         D.set_option("verify_stream_cluster", int(c))
     else:
         D.set_option("verify_cluster", int(c))
@@ -61,7 +58,7 @@ def test_verify_matches_oracle(V, T, scheduled, impl, labels):
     kind, cluster = use_impl(impl)
     if kind == "rows" and cluster and V < 4096 and cluster > 4:
         pytest.skip("slice smaller than the block")
-    if kind in ("stream", "tmem", "sliced") and V % 4:
+    if kind in ("stream", "sliced") and V % 4:
         pytest.skip("the sliced and streaming kernels need V % 4 == 0 (other V take the per-row kernels)")
     B, G = 6, 4
     ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=V + int(T * 10) + cluster)
@@ -125,13 +122,11 @@ def test_bad_token_and_nonfinite_are_flagged():
     check_verify(ld, lt, x, None, u_acc, u_res, 1.0, n, y, requests=[1])
 
 
-@pytest.mark.parametrize("tmem", [1, 0])
 @pytest.mark.parametrize("cluster", [0, 16])
-def test_acceptance_rate_matches_label_statistically(cluster, tmem):
+def test_acceptance_rate_matches_label_statistically(cluster):
     # P(accept position 1) = c*_1 = sum min(p_d, p_t): many requests sharing the same rows, so that
     # hundreds of rows per cluster pass through the exchange slots (clusters of 16: CTAs without tiles)
     D.set_option("verify_stream_cluster", cluster)
-    D.set_option("verify_stream_tmem", tmem)
     B, G, V = 4000, 1, 512
     rng = np.random.default_rng(0)
     ld1 = (rng.normal(size=V) * 2).astype(np.float32)
@@ -146,15 +141,13 @@ def test_acceptance_rate_matches_label_statistically(cluster, tmem):
     assert abs(rate - c1) < 4 * np.sqrt(c1 * (1 - c1) / B)
 
 
-@pytest.mark.parametrize("impl", ["sliced-0", "sliced-7", "stream-8", "stream-2", "tmem-2", "tmem-8", "persistent-1",
-                                  "persistent-0"])
+@pytest.mark.parametrize("impl", ["sliced-0", "sliced-7", "stream-8", "stream-2", "persistent-1", "persistent-0"])
 def test_scheduled_rows_skipped_many_requests(impl):
     kind, v = impl.split("-")
-    D.set_option("verify_impl", {"stream": 0, "tmem": 0, "sliced": 1, "persistent": 2}[kind])
+    D.set_option("verify_impl", {"stream": 0, "sliced": 1, "persistent": 2}[kind])
     if kind == "sliced":
         D.set_option("verify_groups", int(v))
-    elif kind in ("stream", "tmem"):
-        D.set_option("verify_stream_tmem", 1 if kind == "tmem" else 0)
+    elif kind == "stream":
         D.set_option("verify_stream_cluster", int(v))
     else:
         D.set_option("verify_persistent", int(v))
@@ -181,13 +174,11 @@ def test_stream_vocabulary_beyond_per_row_kernels(T):
     assert e.value.status == D.ENOTIMPL
 
 
-@pytest.mark.parametrize("tmem", [1, 0])
 @pytest.mark.parametrize("cluster", [2, 8, 12])
 @pytest.mark.parametrize("T", [1.0, 0.0])
-def test_stream_scheduled_rows_with_and_without_labels(cluster, T, tmem):
+def test_stream_scheduled_rows_with_and_without_labels(cluster, T):
     # rows past L_b + 1 skipped when no labels are asked for; all rows read with labels
     D.set_option("verify_impl", 0)
-    D.set_option("verify_stream_tmem", tmem)
     D.set_option("verify_stream_cluster", cluster)
     B, G, V = 24, 5, 20000
     ld, lt, x, u_acc, u_res = case(B, G, V, T, seed=300 + cluster)
